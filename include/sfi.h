@@ -1,0 +1,272 @@
+/*
+ * sfi.h — C ABI of the Slow-Fast Inference (SFI) decode hot path on B200.
+ *
+ * Slow-Fast Inference ("Slow-Fast Inference: Training-Free Inference
+ * Acceleration via Within-Sentence Support Stability", arXiv 2603.12038)
+ * splits decoding into frequent cheap "fast" steps, which attend only to a
+ * small sparse memory (sink tokens, Selector-chosen tokens packed into a
+ * contiguous buffer, and a recent window read from the paged KV cache), and
+ * occasional dense "slow" steps, whose attention distribution refreshes that
+ * memory through the Selector.  Page sections cited below:
+ *   [ES] gist.science/es "2. Metodología", "3. Optimización del Sistema"
+ *   [FR] gist.science/fr "B. Le Sélecteur", "C. Optimisations Système"
+ *   [NL] gist.science/nl "De Selector", "Systeemontwerp en Kernel-optimalisatie"
+ *   [ZH] gist.science/zh "2.1", "2.2", "2.3"
+ *
+ * Conventions for every call:
+ *  - Tensors are caller-owned device pointers; nothing is allocated on the
+ *    decode path.  bf16 values are passed as raw 16-bit patterns (sfi_bf16).
+ *  - Calls are asynchronous on the given CUDA stream (cudaStream_t passed as
+ *    void*; NULL = legacy default stream) and return an sfi_status at once.
+ *    Argument errors are reported before anything is enqueued.  Errors found
+ *    on the device (an out-of-range page-table entry or index, a pipeline
+ *    wait that timed out) skip the offending access and are latched into
+ *    sfi_paged_kv.err (if non-NULL): low byte = sfi_status, next byte = the
+ *    kernel site.  Read and clear it with sfi_poll_error().
+ *  - Shapes: G = Hq / Hkv must be an integer in [1, 16]; D in {64, 128};
+ *    page_size == 16.  The context length L (new token included) is passed
+ *    by value and is the same for every sequence of the batch.
+ *  - Device pointers handed to TMA (k_pool, v_pool, packed k/v) must be
+ *    16-byte aligned.  Nothing here ever aborts or exits the process.
+ */
+#ifndef SFI_H_
+#define SFI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SFI_OK = 0,
+  SFI_ERR_INVALID_ARG = 1,  /* NULL pointer, misaligned pointer, bad scalar */
+  SFI_ERR_SHAPE = 2,        /* inconsistent or out-of-range sizes */
+  SFI_ERR_UNSUPPORTED = 3,  /* valid but not built (e.g. D not in {64,128}) */
+  SFI_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  SFI_ERR_DEVICE_CHECK = 5, /* a device-side bounds check fired */
+  SFI_ERR_TIMEOUT = 6,      /* a device-side bounded wait expired */
+  SFI_ERR_WORKSPACE = 7     /* workspace missing or too small */
+} sfi_status;
+
+typedef uint16_t sfi_bf16; /* raw bfloat16 bits */
+typedef void* sfi_stream;  /* cudaStream_t */
+
+/* Sizes of one attention layer.  B sequences, Hq query heads sharing Hkv KV
+ * heads (G = Hq/Hkv query heads per KV group), head dim D.  The paged cache
+ * has num_pages pages of page_size (=16) tokens per KV head; each sequence
+ * owns max_pages entries of the page table. */
+typedef struct {
+  int32_t B, Hq, Hkv, D;
+  int32_t page_size;
+  int32_t max_pages;
+  int32_t num_pages;
+} sfi_shape;
+
+/* Method constants (readings of the pages where they are silent):
+ *  n_sink     sink tokens [0, n_sink), always attended        ([ES] §2)
+ *  n_recent   recent window [L-n_recent, L), read from pages   ([ES] §2, [NL])
+ *  k_fixed    >0: K per query head; else floor(budget_frac*L) ([ES] §4)
+ *  lambda, lambda_clip   s = (1-l) f~ + l r, l = clamp(lambda, 0, lambda_clip)
+ *                         ([NL] "De Selector", [ZH] §2.2, §4 ablations)
+ *  alpha_soft, nms_window  soft-NMS strength and full window width (w = window/2)
+ *  alpha_cross             cross-head exclusivity penalty      ([FR] §2.B)
+ *  refresh_budget          M: a slow step at least every M steps ([ES] §2) */
+typedef struct {
+  int32_t n_sink, n_recent, k_fixed;
+  double budget_frac;   /* K = floor(budget_frac * L) in double precision */
+  float lambda, lambda_clip, alpha_soft, alpha_cross;
+  int32_t nms_window, refresh_budget;
+} sfi_params;
+
+/* The paged KV cache of one layer ([NL] "Systeemontwerp": the recent window is
+ * read straight from it; [ZH] §2.3).
+ *  k_pool, v_pool  bf16 [num_pages, Hkv, 16, D]; token j of sequence b, KV head
+ *                  h is row j%16 of page page_table[b, j/16], head h.
+ *  page_table      int32 [B, max_pages]
+ *  key_norms       fp32  [B, Hkv, max_pages*16]: ||k_j||_2 of the stored bf16
+ *                  key, the cache statistic the Selector's prior reads.
+ *  err             int32 device word for latched device-side errors, or NULL. */
+typedef struct {
+  sfi_bf16* k_pool;
+  sfi_bf16* v_pool;
+  const int32_t* page_table;
+  float* key_norms;
+  int32_t* err;
+} sfi_paged_kv;
+
+/* Contiguous packed buffer of one layer ([ES] §3 item 2, [NL] Memory-Coalesced
+ * Kernel, [ZH] §2.3): per (sequence, KV head) the sink rows, then the union of
+ * the group's selected positions in ascending order, then zero rows up to a
+ * multiple of 16.
+ *  k, v      bf16  [B, Hkv, p_max, D]
+ *  pos       int32 [B, Hkv, p_max]   cache position of each row
+ *  headmask  uint32[B, Hkv, p_max]   bit h set: query head h of the group
+ *                                     attends to this row (sinks: all bits)
+ *  n_rows    int32 [B, Hkv]          rows in use (sinks included)
+ *  p_max     row capacity, a multiple of 64 (see sfi_packed_rows). */
+typedef struct {
+  sfi_bf16* k;
+  sfi_bf16* v;
+  int32_t* pos;
+  uint32_t* headmask;
+  int32_t* n_rows;
+  int32_t p_max;
+} sfi_packed;
+
+/* Optional outputs of the dense (slow-step) attention.  Any pointer may be
+ * NULL.  Rows are [B, Hq, ld] with ld >= L (elements).
+ *  lse        [B, Hq]  log sum_j exp(z_j), natural log, over [0, L)
+ *  logits     z_j = q.k_j / sqrt(D) for j < L                ([ES] §2 "logits")
+ *  probs      f_j = exp(z_j - lse) for j < L (may equal logits: in place;
+ *             needs lse non-NULL)
+ *  lse_cand   [B, Hq]  log sum_{j in [cand_lo, cand_hi)} exp(z_j); the
+ *             Selector's evidence is f~_j = exp(z_j - lse_cand). */
+typedef struct {
+  float* lse;
+  float* logits;
+  float* probs;
+  int64_t ld;
+  float* lse_cand;
+  int32_t cand_lo, cand_hi;
+} sfi_dense_extras;
+
+const char* sfi_status_str(sfi_status s);
+
+/* Library version string (static storage). */
+const char* sfi_version(void);
+
+/* Bytes of scratch the per-op calls below need for contexts up to
+ * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes.
+ * Ownership stays with the caller; contents need no initialisation. */
+sfi_status sfi_workspace_size(const sfi_shape* shape, const sfi_params* params, size_t* bytes);
+
+/* Packed-buffer row capacity p_max needed for contexts up to max_pages*16:
+ * n_sink + min(G*K_max, |C|_max), rounded up to a multiple of 64. */
+sfi_status sfi_packed_rows(const sfi_shape* shape, const sfi_params* params, int32_t* p_max);
+
+/* Selection size K for a slow step at context L: k_fixed or
+ * floor(budget_frac * L), clamped to |C| = L - n_recent - n_sink.
+ * Fails with SFI_ERR_SHAPE when |C| < 1. */
+sfi_status sfi_budget(const sfi_params* params, int32_t L, int32_t* K);
+
+/* Append one token per (sequence, KV head) at position L-1 and record its key
+ * norm.  k_new, v_new: bf16 [B, Hkv, D]. */
+sfi_status sfi_append_kv(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                         const sfi_bf16* k_new, const sfi_bf16* v_new, sfi_stream stream);
+
+/* Recompute key_norms for positions [pos_lo, pos_hi) (e.g. after a prefill). */
+sfi_status sfi_key_norms(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t pos_lo,
+                         int32_t pos_hi, sfi_stream stream);
+
+/* Slow-step dense decode attention over [0, L) ([ES] §2 Pasos Lentos; [FR] §2.A;
+ * [ZH] §2.1), also the in-house full-KV baseline when extras == NULL.
+ *  q    bf16 [B, Hq, D]; query head hq uses KV head hq / G.
+ *  out  fp32 [B, Hq, D] = sum_j softmax(z)_j v_j.
+ * Persistent split-K kernel: TMA page tiles -> shared memory, mma.sync for
+ * the group's QK^T / PV tiles, online softmax, then a combine kernel. */
+sfi_status sfi_dense_attn(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                          const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
+                          void* ws, size_t ws_bytes, sfi_stream stream);
+
+/* f = exp(logits - lse) over j < L for every (b, hq) row. */
+sfi_status sfi_attn_probs(const sfi_shape* shape, int32_t L, const float* logits, int64_t ld,
+                          const float* lse, float* probs, sfi_stream stream);
+
+/* Fast-step sparse attention ([ES] §2 Pasos Rápidos; [NL] Methodologie):
+ * query head h attends to the packed rows whose headmask has bit h (sinks +
+ * its selection) and to the recent window [L - n_recent, L) read from pages.
+ *  out fp32 [B, Hq, D]; lse fp32 [B, Hq] or NULL. */
+sfi_status sfi_fast_attn(const sfi_shape* shape, const sfi_params* params,
+                         const sfi_paged_kv* kv, int32_t L, const sfi_bf16* q,
+                         const sfi_packed* packed, float* out, float* lse, void* ws,
+                         size_t ws_bytes, sfi_stream stream);
+
+/* Selector scores ([FR] "B. Le Sélecteur"; [NL] "De Selector"; [ZH] §2.2):
+ * for the candidates C = [n_sink, L - n_recent) of a slow step at context L,
+ * evidence f~ = exp(z - lse_cand), prior r from key norms and positions,
+ * s = (1-l) f~ + l r, log-score, soft-NMS, cross-head exclusivity.
+ *  logits    fp32 [B, Hq, ld] from sfi_dense_attn;  lse_cand fp32 [B, Hq]
+ *  scores    fp32 [B, Hq, |C|] refined log-scores l''. */
+sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
+                             const sfi_paged_kv* kv, int32_t L, const float* logits, int64_t ld,
+                             const float* lse_cand, float* scores, void* ws, size_t ws_bytes,
+                             sfi_stream stream);
+
+/* Per-row top-K: the K largest of scores[r, 0:n] (ties -> lower index),
+ * written ascending as idx[r, 0:K] = offset + column.  rows = number of rows;
+ * scores row stride ld_s, idx row stride ld_i (elements). */
+sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
+                    int32_t offset, int32_t* idx, int64_t ld_i, sfi_stream stream);
+
+/* Full Selector = sfi_select_scores + sfi_topk.  sel_idx int32 [B, Hq, sel_ld]
+ * receives K ascending absolute positions per query head; *K_out = K. */
+sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
+                      int32_t L, const float* logits, int64_t ld, const float* lse_cand,
+                      int32_t* sel_idx, int32_t sel_ld, int32_t* K_out, void* ws,
+                      size_t ws_bytes, sfi_stream stream);
+
+/* Compaction ([ES] §3 item 2; [FR] §2.C "réorganisation"): build the packed
+ * buffer of every (sequence, KV head) from the group's selections (K ascending
+ * positions per query head, rows of sel_idx with stride sel_ld, all inside
+ * the candidate range [n_sink, L - n_recent) of the slow step at context L)
+ * by gathering K/V rows from the pages.  Bit-exact copies.  Rows beyond
+ * p_max are dropped and reported as SFI_ERR_DEVICE_CHECK. */
+sfi_status sfi_compact(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
+                       int32_t L, const int32_t* sel_idx, int32_t sel_ld, int32_t K,
+                       sfi_packed* packed, void* ws, size_t ws_bytes, sfi_stream stream);
+
+/* Read the latched device error word of kv (synchronous), then clear it. */
+sfi_status sfi_poll_error(const sfi_paged_kv* kv, int32_t* code);
+
+/* ------------------------------------------------------------------------
+ * Decode-step driver ([ES] §2 trigger, §3 item 1 asynchronous pipeline;
+ * [ZH] §2.3 双 CUDA 流).  A context owns one side stream and per-layer events;
+ * the caller owns every tensor and the context workspace.
+ */
+typedef struct sfi_ctx sfi_ctx;
+
+/* L_max = shape->max_pages * 16 bounds every context length used with ctx. */
+sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int32_t n_layers,
+                          int32_t overlap, sfi_ctx** out);
+sfi_status sfi_ctx_destroy(sfi_ctx* ctx);
+sfi_status sfi_ctx_workspace_size(const sfi_ctx* ctx, size_t* bytes);
+sfi_status sfi_ctx_set_workspace(sfi_ctx* ctx, void* ws, size_t bytes);
+
+/* Trigger ([ES] §2 Pasos Lentos; [ZH] §2.1 触发机制): step t is slow when
+ * t == 0, or the previous step emitted a boundary token (boundary_prev != 0),
+ * or t - last_slow >= refresh_budget.  Evaluated when layer == 0; the other
+ * layers of the step reuse the decision.
+ *
+ * One layer of one decode step, enqueued on `stream` (the main stream):
+ *  1. append k_new/v_new at position L-1 (key norm included);
+ *  2. slow step: dense attention (+logits, lse_cand) -> out; then, on the
+ *     side stream after an event, the Selector and compaction refresh this
+ *     layer's packed buffer while the main stream moves on to layer+1;
+ *     fast step: wait for this layer's pending refresh, then sparse attention
+ *     over packed + recent -> out.
+ *  q bf16 [B,Hq,D]; k_new, v_new bf16 [B,Hkv,D]; out fp32 [B,Hq,D].
+ *  *was_slow (may be NULL) receives the step's decision. */
+sfi_status sfi_decode_step(sfi_ctx* ctx, int32_t layer, int32_t step, int32_t boundary_prev,
+                           int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
+                           const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
+                           float* out, sfi_stream stream, int32_t* was_slow);
+
+/* Make `stream` wait for every outstanding side-stream refresh of ctx. */
+sfi_status sfi_ctx_join(sfi_ctx* ctx, sfi_stream stream);
+
+/* Per-kernel CUDA-event timing of the attention kernels launched by
+ * sfi_decode_step (kind 0 = fast-attention main kernel, 1 = dense main
+ * kernel).  Enabled with sfi_ctx_set_timing; sfi_ctx_timing synchronises on
+ * the recorded events and returns total milliseconds and launch count since
+ * the last reset. */
+sfi_status sfi_ctx_set_timing(sfi_ctx* ctx, int32_t enable);
+sfi_status sfi_ctx_timing(sfi_ctx* ctx, int32_t kind, double* total_ms, int64_t* launches,
+                          int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFI_H_ */

@@ -1,0 +1,298 @@
+// Decode-step driver: the slow/fast trigger and the asynchronous two-stream
+// pipeline of Slow-Fast Inference ([ES] "2. Metodología", Pasos Lentos;
+// "3. Optimización del Sistema", item 1; [FR] "C. Optimisations Système",
+// Pipeline Asynchrone; [ZH] "2.3" 异步流水线).
+//
+// On a slow step the main stream runs dense attention for layer i (also
+// writing the logits and the candidate log-sum-exp into one of two ping-pong
+// buffers) and moves on to layer i+1; the Selector and the compaction of
+// layer i run on the context's side stream after an event.  The next step of
+// layer i waits for that refresh before it touches the layer's cache or
+// packed buffer.  A logits buffer is rewritten only after the side stream has
+// finished reading it.
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+struct sfi_ctx {
+  sfi_shape s;
+  sfi_params p;
+  int n_layers;
+  int overlap;
+  int device;
+  int p_max_ws;
+  cudaStream_t side = nullptr;
+  std::vector<cudaEvent_t> ev_dense, ev_sel;
+  std::vector<uint8_t> pending;
+  cudaEvent_t ev_buf_free[2] = {nullptr, nullptr};
+  int cur_step = -1, cur_slow = 0, last_slow = 0;
+  // workspace carving
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  float* part = nullptr;
+  size_t part_bytes = 0;
+  float* logits[2] = {nullptr, nullptr};
+  float* lse_cand[2] = {nullptr, nullptr};
+  int64_t ld = 0;
+  void* stats = nullptr;
+  float* scores = nullptr;
+  int32_t* sel_idx = nullptr;
+  int sel_ld = 0;
+  int32_t* tile_counts = nullptr;
+  size_t tc_bytes = 0;
+  // timing of the attention kernels (kind 0 fast, 1 dense)
+  bool timing = false;
+  std::vector<cudaEvent_t> tev[2];
+  size_t tused[2] = {0, 0};
+};
+
+namespace sfi {
+namespace {
+
+struct CtxLayout {
+  size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, stat_off, stat_bytes, score_off,
+      score_bytes, sel_off, sel_bytes, tc_off, tc_bytes, total;
+};
+
+CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
+  const WsLayout w = ws_layout(s, p);
+  CtxLayout c{};
+  const int Lmax = s.max_pages * kPage;
+  size_t off = 256;
+  c.part_off = off;
+  c.part_bytes = w.part_bytes;
+  off += c.part_bytes;
+  c.logit_off = off;
+  c.logit_bytes = align_up((size_t)s.B * s.Hq * Lmax * sizeof(float), 256);
+  off += 2 * c.logit_bytes;
+  c.lsec_off = off;
+  off += 2 * align_up((size_t)s.B * s.Hq * sizeof(float), 256);
+  c.stat_off = off;
+  c.stat_bytes = w.stat_bytes;
+  off += c.stat_bytes;
+  c.score_off = off;
+  c.score_bytes = w.sel_bytes;
+  off += c.score_bytes;
+  const long kmax = std::max(budget_k(p, Lmax), 1);
+  c.sel_off = off;
+  c.sel_bytes = align_up((size_t)s.B * s.Hq * kmax * sizeof(int32_t), 256);
+  off += c.sel_bytes;
+  c.tc_off = off;
+  c.tc_bytes = w.cmp_bytes;
+  off += c.tc_bytes;
+  c.total = off;
+  return c;
+}
+
+#define SFI_TRY(x)               \
+  do {                           \
+    sfi_status _r = (x);         \
+    if (_r != SFI_OK) return _r; \
+  } while (0)
+
+sfi_status cu(cudaError_t e) { return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA; }
+
+// Event pair for one timed launch, or nulls when timing is off.
+void timing_events(sfi_ctx* c, int kind, cudaEvent_t* b, cudaEvent_t* e) {
+  *b = *e = nullptr;
+  if (!c->timing) return;
+  auto& v = c->tev[kind];
+  if (c->tused[kind] + 2 > v.size()) {
+    for (int i = 0; i < 256; ++i) {
+      cudaEvent_t ev;
+      if (cudaEventCreate(&ev) != cudaSuccess) return;
+      v.push_back(ev);
+    }
+  }
+  *b = v[c->tused[kind]];
+  *e = v[c->tused[kind] + 1];
+  c->tused[kind] += 2;
+}
+
+}  // namespace
+}  // namespace sfi
+
+using namespace sfi;
+
+extern "C" {
+
+sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int32_t n_layers,
+                          int32_t overlap, sfi_ctx** out) {
+  if (!out) return SFI_ERR_INVALID_ARG;
+  *out = nullptr;
+  size_t probe = 0;
+  SFI_TRY(sfi_workspace_size(shape, params, &probe));
+  if (n_layers < 1) return SFI_ERR_INVALID_ARG;
+  auto* c = new sfi_ctx();
+  c->s = *shape;
+  c->p = *params;
+  c->n_layers = n_layers;
+  c->overlap = overlap ? 1 : 0;
+  cudaGetDevice(&c->device);
+  bool ok = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) == cudaSuccess;
+  c->ev_dense.resize(n_layers, nullptr);
+  c->ev_sel.resize(n_layers, nullptr);
+  c->pending.assign(n_layers, 0);
+  for (int i = 0; i < n_layers && ok; ++i)
+    ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; i < 2 && ok; ++i)
+    ok = cudaEventCreateWithFlags(&c->ev_buf_free[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    sfi_ctx_destroy(c);
+    return SFI_ERR_CUDA;
+  }
+  *out = c;
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_destroy(sfi_ctx* c) {
+  if (!c) return SFI_OK;
+  if (c->side) cudaStreamSynchronize(c->side);
+  for (auto e : c->ev_dense) if (e) cudaEventDestroy(e);
+  for (auto e : c->ev_sel) if (e) cudaEventDestroy(e);
+  for (auto e : c->ev_buf_free) if (e) cudaEventDestroy(e);
+  for (int k = 0; k < 2; ++k)
+    for (auto e : c->tev[k]) cudaEventDestroy(e);
+  if (c->side) cudaStreamDestroy(c->side);
+  delete c;
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_workspace_size(const sfi_ctx* c, size_t* bytes) {
+  if (!c || !bytes) return SFI_ERR_INVALID_ARG;
+  *bytes = ctx_layout(c->s, c->p).total;
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
+  if (!c || !ws) return SFI_ERR_INVALID_ARG;
+  const CtxLayout l = ctx_layout(c->s, c->p);
+  if (bytes < l.total) return SFI_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  c->ws = w;
+  c->ws_bytes = bytes;
+  c->part = reinterpret_cast<float*>(w + l.part_off);
+  c->part_bytes = l.part_bytes;
+  c->ld = (int64_t)c->s.max_pages * kPage;
+  for (int i = 0; i < 2; ++i) {
+    c->logits[i] = reinterpret_cast<float*>(w + l.logit_off + i * l.logit_bytes);
+    c->lse_cand[i] =
+        reinterpret_cast<float*>(w + l.lsec_off + i * align_up((size_t)c->s.B * c->s.Hq * sizeof(float), 256));
+  }
+  c->stats = w + l.stat_off;
+  c->scores = reinterpret_cast<float*>(w + l.score_off);
+  c->sel_ld = std::max(budget_k(c->p, c->s.max_pages * kPage), 1);
+  c->sel_idx = reinterpret_cast<int32_t*>(w + l.sel_off);
+  c->tile_counts = reinterpret_cast<int32_t*>(w + l.tc_off);
+  c->tc_bytes = l.tc_bytes;
+  return SFI_OK;
+}
+
+sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boundary_prev,
+                           int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
+                           const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
+                           float* out, sfi_stream stream, int32_t* was_slow) {
+  if (!c || !c->ws) return SFI_ERR_WORKSPACE;
+  if (layer < 0 || layer >= c->n_layers || step < 0) return SFI_ERR_INVALID_ARG;
+  if (!kv || !packed || !q || !k_new || !v_new || !out || !kv->key_norms) return SFI_ERR_INVALID_ARG;
+  if (L < c->p.n_sink + c->p.n_recent + 1 || L > c->s.max_pages * kPage) return SFI_ERR_SHAPE;
+  if (packed->p_max < packed_rows_capacity(c->s, c->p)) return SFI_ERR_SHAPE;
+  const sfi_shape& s = c->s;
+  const sfi_params& p = c->p;
+  cudaStream_t main = (cudaStream_t)stream;
+
+  if (layer == 0) {
+    const bool slow = step == 0 || boundary_prev != 0 || (step - c->last_slow) >= p.refresh_budget;
+    if (slow) c->last_slow = step;
+    c->cur_step = step;
+    c->cur_slow = slow ? 1 : 0;
+  } else if (step != c->cur_step) {
+    return SFI_ERR_INVALID_ARG;   // layer 0 decides the step
+  }
+  if (was_slow) *was_slow = c->cur_slow;
+
+  // this layer's previous refresh must land before its cache or packed buffer is touched
+  if (c->pending[layer]) {
+    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
+    c->pending[layer] = 0;
+  }
+  SFI_TRY(run_append(s, *kv, L, k_new, v_new, main));
+
+  if (!c->cur_slow) {
+    cudaEvent_t b, e;
+    timing_events(c, 0, &b, &e);
+    return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, c->part, c->part_bytes, main, b, e);
+  }
+
+  const int buf = layer & 1;
+  SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
+  sfi_dense_extras ex{};
+  ex.logits = c->logits[buf];
+  ex.ld = c->ld;
+  ex.lse_cand = c->lse_cand[buf];
+  ex.cand_lo = p.n_sink;
+  ex.cand_hi = L - p.n_recent;
+  {
+    cudaEvent_t b, e;
+    timing_events(c, 1, &b, &e);
+    SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, c->part, c->part_bytes, main, b, e));
+  }
+  SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
+  cudaStream_t side = c->side;
+  SFI_TRY(cu(cudaStreamWaitEvent(side, c->ev_dense[layer], 0)));
+  const int nC = L - p.n_recent - p.n_sink;
+  const int K = budget_k(p, L);
+  if (K < 1) return SFI_ERR_SHAPE;
+  SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, nC,
+                            c->stats, side));
+  SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
+  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, nC, K, p.n_sink, c->sel_idx, c->sel_ld, side));
+  SFI_TRY(run_compact(s, p, *kv, c->sel_idx, c->sel_ld, K, *packed, c->tile_counts, c->tc_bytes, L,
+                      side));
+  SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
+  if (c->overlap) {
+    c->pending[layer] = 1;
+  } else {
+    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
+  }
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_join(sfi_ctx* c, sfi_stream stream) {
+  if (!c) return SFI_ERR_INVALID_ARG;
+  for (int i = 0; i < c->n_layers; ++i) {
+    if (c->pending[i]) {
+      SFI_TRY(cu(cudaStreamWaitEvent((cudaStream_t)stream, c->ev_sel[i], 0)));
+      c->pending[i] = 0;
+    }
+  }
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_set_timing(sfi_ctx* c, int32_t enable) {
+  if (!c) return SFI_ERR_INVALID_ARG;
+  c->timing = enable != 0;
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_timing(sfi_ctx* c, int32_t kind, double* total_ms, int64_t* launches,
+                          int32_t reset) {
+  if (!c || kind < 0 || kind > 1 || !total_ms || !launches) return SFI_ERR_INVALID_ARG;
+  double tot = 0.0;
+  const size_t n = c->tused[kind] / 2;
+  for (size_t i = 0; i < n; ++i) {
+    cudaEvent_t b = c->tev[kind][2 * i], e = c->tev[kind][2 * i + 1];
+    if (cudaEventSynchronize(e) != cudaSuccess) return SFI_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, b, e) != cudaSuccess) return SFI_ERR_CUDA;
+    tot += ms;
+  }
+  *total_ms = tot;
+  *launches = (int64_t)n;
+  if (reset) c->tused[kind] = 0;
+  return SFI_OK;
+}
+
+}  // extern "C"

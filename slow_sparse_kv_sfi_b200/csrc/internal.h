@@ -1,0 +1,78 @@
+// Internal host-side interfaces shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/sfi.h"
+
+namespace sfi {
+
+// Streaming-multiprocessor count of the current device (cached per device).
+int num_sms();
+
+// Per-device one-time flag (up to 64 devices).
+struct DeviceOnce {
+  std::atomic<uint64_t> bits{0};
+  bool done() const {
+    int d = 0;
+    cudaGetDevice(&d);
+    return (bits.load() >> (d & 63)) & 1u;
+  }
+  bool mark(cudaError_t e) {
+    if (e != cudaSuccess) return false;
+    int d = 0;
+    cudaGetDevice(&d);
+    bits.fetch_or(uint64_t(1) << (d & 63));
+    return true;
+  }
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace carving: the per-op calls take one caller-provided buffer.
+struct WsLayout {
+  size_t part_off, part_bytes;      // attention split-K partials
+  size_t sel_off, sel_bytes;        // Selector: per-(b,kv) stats + scores
+  size_t stat_off, stat_bytes;
+  size_t cmp_off, cmp_bytes;        // compaction tile counts
+  size_t total;
+};
+WsLayout ws_layout(const sfi_shape& s, const sfi_params& p);
+
+int dense_chunk_tiles(const sfi_shape& s, int L);
+int fast_chunks(const sfi_shape& s, int p_max, int n_recent);
+size_t attn_part_bytes(int n_items, int G, int D);
+int packed_rows_capacity(const sfi_shape& s, const sfi_params& p);
+int budget_k(const sfi_params& p, int L);   // -1 if |C| < 1
+
+sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
+                          float* out, const sfi_dense_extras* ex, float* part, size_t part_bytes,
+                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
+sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
+                         const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse,
+                         float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
+                         cudaEvent_t ev_end);
+sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld,
+                          const float* lse, float* probs, cudaStream_t st);
+
+sfi_status run_append(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* k_new,
+                      const sfi_bf16* v_new, cudaStream_t st);
+sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int hi,
+                         cudaStream_t st);
+
+sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
+                             int L, const float* logits, int64_t ld, const float* lse_cand,
+                             float* scores, int64_t ld_s, void* stat_ws, cudaStream_t st);
+sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset,
+                    int32_t* idx, int64_t ld_i, cudaStream_t st);
+sfi_status run_compact(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
+                       const int32_t* sel_idx, int sel_ld, int K, const sfi_packed& pk,
+                       int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st);
+int compact_tiles(int nC);
+int score_tile(int G);
+
+}  // namespace sfi

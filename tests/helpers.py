@@ -1,0 +1,122 @@
+"""Test-side glue: runs the oracle on the same inputs the CUDA path received
+and compares the two with the tolerances of the hot path:
+
+* attention outputs: per (b, h) row, max_d |o - o_ref| / max(max_d |o_ref|, 1e-6) <= 2e-3
+* probabilities f and lse: absolute 1e-4; key norms: relative 1e-6
+* page-table indexing, gathers and compaction: bit-exact
+* selections: identical except at elements whose deciding comparisons are
+  near-ties (relative gap below NEAR_TIE) in the oracle's float64 values,
+  and >= 99.9 % overlap.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import sfi_oracle as O
+
+ATTN_RTOL = 2e-3
+PROB_ATOL = 1e-4
+NORM_RTOL = 1e-6
+NEAR_TIE = 1e-5
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def group_kv(k_pool: np.ndarray, v_pool: np.ndarray, pt: np.ndarray, b: int, g: int, L: int):
+    """Logical K, V rows [0, L) of (b, g) read through the page table."""
+    pages = pt[b, : (L + 15) // 16]
+    K = k_pool[pages, g].reshape(-1, k_pool.shape[-1])[:L]
+    V = v_pool[pages, g].reshape(-1, v_pool.shape[-1])[:L]
+    return np.asarray(K, np.float64), np.asarray(V, np.float64)
+
+
+def group_kv_device(layer, b: int, g: int, L: int):
+    """Copies only the pages of (b, g) from device pools to host float64."""
+    pages = layer.page_table[b, : (L + 15) // 16].long()
+    K = layer.k_pool[pages, g].reshape(-1, layer.k_pool.shape[-1])[:L]
+    V = layer.v_pool[pages, g].reshape(-1, layer.v_pool.shape[-1])[:L]
+    return to64(K), to64(V)
+
+
+def attn_row_err(o: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """Per-row max relative error, rows on the leading axes."""
+    num = np.abs(o - ref).max(axis=-1)
+    den = np.maximum(np.abs(ref).max(axis=-1), 1e-6)
+    return num / den
+
+
+def assert_attn_close(o, ref, what=""):
+    e = attn_row_err(np.asarray(o, np.float64), np.asarray(ref, np.float64))
+    assert e.max() <= ATTN_RTOL, f"{what}: max row rel err {e.max():.3e}"
+    return float(e.max())
+
+
+def ambiguous_positions(ell: np.ndarray, ell1: np.ndarray, window: int, G: int) -> np.ndarray:
+    """bool [G, nC]: elements whose soft-NMS or cross-head decision rests on a
+    near-tie (relative gap < NEAR_TIE) in the oracle's float64 scores."""
+    w = window // 2
+    Gh, n = ell.shape
+    amb = np.zeros((Gh, n), bool)
+    scale = np.maximum(np.abs(ell), 1e-30)
+    for d in range(1, w + 1):
+        diff = np.abs(ell[:, d:] - ell[:, :-d])
+        near = diff < NEAR_TIE * np.maximum(scale[:, d:], scale[:, :-d])
+        amb[:, d:] |= near
+        amb[:, :-d] |= near
+    if G > 1:
+        s = np.sort(ell1, axis=0)
+        top, second = s[-1], s[-2]
+        near_owner = np.abs(top - second) < NEAR_TIE * np.maximum(np.abs(top), 1e-30)
+        amb |= near_owner[None, :]
+    return amb
+
+
+def oracle_selector_detail(f: np.ndarray, norms: np.ndarray, L: int, cfg):
+    """Oracle scores of one group plus the intermediate ell, ell' (float64)."""
+    lo, hi = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
+    ft = O.evidence(f, lo, hi)
+    r = O.prior(norms, L, lo, hi)
+    s = O.fuse(ft, r, cfg.lam, cfg.lam_clip)
+    ell = O.log_score(s)
+    ell1 = O.soft_nms(ell, cfg.alpha_soft, cfg.nms_window)
+    ell2 = O.cross_head(ell1, cfg.alpha_cross)
+    return ell, ell1, ell2
+
+
+def assert_selection_close(gpu_sel: np.ndarray, ora_sel: np.ndarray, ell2: np.ndarray,
+                           amb: np.ndarray, lo: int, what=""):
+    """gpu_sel, ora_sel: [G, K] absolute positions.  Differences are allowed
+    only at ambiguous elements or at scores within NEAR_TIE of the K-th."""
+    G, K = ora_sel.shape
+    worst = 1.0
+    for h in range(G):
+        a = set(gpu_sel[h].tolist())
+        b = set(ora_sel[h].tolist())
+        assert len(a) == K, f"{what}: head {h} has duplicate picks"
+        sym = a ^ b
+        if sym:
+            s = np.sort(ell2[h])[::-1]
+            kth = s[K - 1]
+            for j in sym:
+                c = j - lo
+                near = abs(ell2[h, c] - kth) <= NEAR_TIE * max(abs(kth), 1e-30)
+                assert amb[h, c] or near, (
+                    f"{what}: head {h} position {j} differs and is not a near-tie "
+                    f"(score {ell2[h, c]!r}, K-th {kth!r})")
+        worst = min(worst, len(a & b) / K)
+    assert worst >= 0.999, f"{what}: overlap {worst:.5f}"
+    return worst
+
+
+def packed_sets(pos: np.ndarray, hm: np.ndarray, n_rows: int, n_sink: int, G: int):
+    """Per-head selected positions recorded in a packed buffer (sinks removed)."""
+    p = pos[:n_rows]
+    m = hm[:n_rows].astype(np.int64) & 0xFFFFFFFF
+    out = []
+    for h in range(G):
+        sel = p[(m >> h) & 1 == 1]
+        out.append(np.asarray(sel[sel >= n_sink], np.int64))
+    return out

@@ -1,0 +1,100 @@
+"""The C-ABI library loads and exports every entry point include/sfi.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "sfi.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sfi_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def S():
+    from slow_sparse_kv_sfi_b200 import build, sfi
+    build.build()
+    return sfi
+
+
+def test_every_declared_symbol_is_exported(S):
+    lib = S.lib()
+    names = _declared()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(S.EXPORTED)
+
+
+def test_version_and_status_strings(S):
+    assert "sm_100a" in S.sfi_version()
+    lib = S.lib()
+    for code in range(8):
+        assert lib.sfi_status_str(code)
+    assert lib.sfi_status_str(99) == b"unknown status"
+
+
+def test_budget_rule_host(S):
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8)
+    assert S.sfi_budget(p, 1025) == 128
+    p = S.make_params(4, 128, 0, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 32)
+    assert S.sfi_budget(p, 8193) == int(0.2 * 8193)
+    assert S.sfi_budget(p, 200) == 40
+    p = S.make_params(4, 128, 0, 0.9, 0.2, 0.5, 0.5, 0.5, 32, 32)
+    assert S.sfi_budget(p, 200) == 200 - 128 - 4          # clamped to |C|
+    with pytest.raises(S.SFIError):
+        S.sfi_budget(p, 132)          # |C| = 0
+
+
+def test_packed_rows_capacity(S):
+    from slow_sparse_kv_sfi_b200.state import shape_of, params_of
+    from slow_sparse_kv_sfi_b200 import workload as W
+    cfg = W.CONFIGS[0]
+    rows = S.sfi_packed_rows(shape_of(cfg), params_of(cfg))
+    nC = cfg.capacity - cfg.n_recent - cfg.n_sink
+    assert rows % 64 == 0
+    assert rows >= cfg.n_sink + min(cfg.G * 128, nC)
+    assert rows - 64 < cfg.n_sink + min(cfg.G * 128, nC)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("D", 96, 3), ("Hkv", 3, 2), ("page_size", 32, 3), ("B", 0, 2), ("Hq", 64, 3)])
+def test_shape_validation(S, field, value, code):
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    setattr(sh, field, value)
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8)
+    n = C.c_size_t()
+    assert S.lib().sfi_workspace_size(C.byref(sh), C.byref(p), C.byref(n)) == code
+
+
+def test_null_pointers_rejected_before_any_launch(S):
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8)
+    kv = S.PagedKV(None, None, None, None, None)
+    lib = S.lib()
+    assert lib.sfi_dense_attn(C.byref(sh), C.byref(kv), 100, None, None, None, None, 0, None) == 1
+    assert lib.sfi_append_kv(C.byref(sh), C.byref(kv), 100, None, None, None) == 1
+    assert lib.sfi_topk(4, 10, None, 10, 3, 0, None, 3, None) == 1
+    # misaligned pool pointer
+    kv = S.PagedKV(8, 16, 16, 16, None)
+    assert lib.sfi_key_norms(C.byref(sh), C.byref(kv), 0, 10, None) == 1
+    # context longer than the cache
+    kv = S.PagedKV(16, 16, 16, 16, None)
+    assert lib.sfi_append_kv(C.byref(sh), C.byref(kv), 161, 16, 16, None) == 2
+    assert lib.sfi_topk(4, 10, 16, 10, 11, 0, 16, 11, None) == 2   # K > n
+    assert lib.sfi_ctx_set_workspace(None, None, 0) == 1
+
+
+def test_context_rejects_bad_calls(S):
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8)
+    h = C.c_void_p()
+    st = S.lib().sfi_ctx_create(C.byref(sh), C.byref(p), 0, 1, C.byref(h))
+    assert st == 1
