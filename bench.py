@@ -1,0 +1,470 @@
+"""Benchmark of the SFI decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl sfi|reference]
+
+One bench *step* is one complete decode run of the workload: every decode
+step of the configured trigger schedule (slow and fast) through every layer,
+i.e. all rows of the hot path (append + key norm, trigger, dense slow-step
+attention with logits, Selector scoring and top-K, compaction, fast
+attention over packed + recent, side-stream overlap).  The default workload is
+the 128K-context, 36-layer Qwen3-4B-shaped configuration: B=2, 32 query / 8
+KV heads, D=128, 131072 cached tokens, 256 decode steps, budget 15 %, sink 4,
+recent 256, Bernoulli(1/16) boundary trigger with refresh budget 32.
+
+value = decode tok/s per attention layer = B * decode_steps * layers / time,
+inputs resident in HBM (the 38.7 GB cache is far larger than L2, so no L2
+flush is needed).  Also reported: the same run through host buffers (e2e),
+the in-house dense full-KV decode on the same cache, the roofline of the
+dominant kernel, and the CPU oracle on a bounded sample.
+
+--impl reference times the CPU oracle on the same workload (the reference
+arm of this repository).  With N > 1 GPUs (torchrun) every rank runs an
+independent replica; the decode path has no cross-GPU exchange.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from slow_sparse_kv_sfi_b200 import sfi as S                      # noqa: E402
+from slow_sparse_kv_sfi_b200 import workload as W                 # noqa: E402
+from slow_sparse_kv_sfi_b200.state import alloc_layer, params_of, shape_of   # noqa: E402
+
+METRIC = "decode tok/s per attn layer (fast/slow mix) vs dense full-KV; % of HBM roofline"
+UNIT = "tok/s per attn layer"
+DEFAULT_CONFIG = "qwen3-4b-128k-36l"
+
+
+# ---------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_traffic(kind: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    src = open(os.path.join(ROOT, "slow_sparse_kv_sfi_b200", "csrc", "attn.cu"), "rb").read()
+    if d.get("attn_cu_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    e = d.get(kind)
+    return None if e is None else float(e)
+
+
+class Clocks:
+    """nvidia-smi sampler for the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the workload on the device
+class Bench:
+    def __init__(self, cfg: W.SFIConfig, device):
+        self.cfg = cfg
+        self.dev = device
+        self.shape, self.params = shape_of(cfg), params_of(cfg)
+        self.boundary = W.boundary_stream(cfg)
+        self.layers, self.inputs = [], []
+        for l in range(cfg.n_layers):
+            li = W.make_layer(cfg, l, device, boundary=self.boundary)
+            self.layers.append(alloc_layer(cfg, li, device))
+            self.inputs.append(li)
+        # per-step inputs stacked by step: [T, layers, ...]
+        self.q = torch.stack([li.q for li in self.inputs], dim=1).contiguous()
+        self.kn = torch.stack([li.k_new for li in self.inputs], dim=1).contiguous()
+        self.vn = torch.stack([li.v_new for li in self.inputs], dim=1).contiguous()
+        for li in self.inputs:
+            li.q = li.k_new = li.v_new = None
+        self.out = torch.empty(cfg.n_layers, cfg.B, cfg.Hq, cfg.D, device=device)
+        self.ctx = S.Context(self.shape, self.params, cfg.n_layers, overlap=True, device=device)
+        self.ws = torch.empty(S.sfi_workspace_size(self.shape, self.params), dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+
+    def run_sfi(self, step_events=None, probe=None, q=None, kn=None, vn=None, out=None):
+        cfg = self.cfg
+        q = self.q if q is None else q
+        kn = self.kn if kn is None else kn
+        vn = self.vn if vn is None else vn
+        out = self.out if out is None else out
+        slows = []
+        for t in range(cfg.steps):
+            L = cfg.seq_len(t)
+            bprev = int(self.boundary[t - 1]) if t > 0 else 0
+            slow = False
+            for l, layer in enumerate(self.layers):
+                slow = self.ctx.decode_step(l, t, bprev, L, layer.kv, layer.packed, q[t, l], kn[t, l],
+                                            vn[t, l], out[l])
+            slows.append(slow)
+            if step_events is not None:
+                step_events[t].record()
+            if probe is not None and slow:
+                self.ctx.join()
+                probe[t] = [layer.n_rows.clone() for layer in self.layers]
+        self.ctx.join()
+        return slows
+
+    def run_dense(self):
+        cfg = self.cfg
+        for t in range(cfg.steps):
+            L = cfg.seq_len(t)
+            for l, layer in enumerate(self.layers):
+                S.sfi_append_kv(self.shape, layer.kv, L, self.kn[t, l], self.vn[t, l])
+                S.sfi_dense_attn(self.shape, layer.kv, L, self.q[t, l], self.out[l], self.ws)
+
+    def run_e2e(self, host_q, host_k, host_v, host_out, dq, dk, dv):
+        """Every decode step copies that step's inputs (all layers) from pinned
+        host memory and reads all layers' outputs back."""
+        cfg = self.cfg
+        for t in range(cfg.steps):
+            dq.copy_(host_q[t], non_blocking=True)
+            dk.copy_(host_k[t], non_blocking=True)
+            dv.copy_(host_v[t], non_blocking=True)
+            L = cfg.seq_len(t)
+            bprev = int(self.boundary[t - 1]) if t > 0 else 0
+            for l, layer in enumerate(self.layers):
+                self.ctx.decode_step(l, t, bprev, L, layer.kv, layer.packed, dq[l], dk[l], dv[l], self.out[l])
+            host_out[t].copy_(self.out, non_blocking=True)
+        self.ctx.join()
+
+
+def _sync_barrier(dist_on):
+    torch.cuda.synchronize()
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def _max_over_ranks(x, dist_on):
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _timed(fn, K, dist_on):
+    _sync_barrier(dist_on)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        fn()
+    e1.record()
+    _sync_barrier(dist_on)
+    return _max_over_ranks(e0.elapsed_time(e1) / 1000.0, dist_on)
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def _group_rows(layer_or_li, b, g, L, device_tensors=True):
+    pool_k, pool_v, pt = layer_or_li.k_pool, layer_or_li.v_pool, layer_or_li.page_table
+    pages = pt[b, : (L + 15) // 16].long()
+    sub_k = pool_k[pages][:, g:g + 1].float().cpu().numpy()
+    sub_v = pool_v[pages][:, g:g + 1].float().cpu().numpy()
+    sub_pt = np.arange(len(pages), dtype=np.int64)[None, :]
+    return sub_k, sub_v, sub_pt
+
+
+def oracle_sample(cfg, layer, q_t, slow_frac):
+    """Times the CPU oracle, as it stands, on one slow and one fast layer-step
+    of one layer (all (sequence, KV head) groups); returns tok/s per attention
+    layer for the run's slow/fast mix, seconds spent and the BLAS threads."""
+    from oracle import sfi_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    G = cfg.G
+    L = cfg.seq_len(0)
+    groups = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    subs = {bg: _group_rows(layer, bg[0], bg[1], L) for bg in groups}
+    qh = q_t.float().cpu().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    sels = {}
+    for (b, g) in groups:
+        sk, sv, spt = subs[(b, g)]
+        K = O.gather_cache(sk, spt, 0, 0, L)
+        V = O.gather_cache(sv, spt, 0, 0, L)
+        o, f, _, _ = O.dense_attention(qh[b, g * G:(g + 1) * G], K, V)
+        sels[(b, g)] = O.select(f, O.key_norms(K), L, cfg.n_sink, cfg.n_recent, cfg.k_fixed,
+                                cfg.budget_frac, cfg.lam, cfg.lam_clip, cfg.alpha_soft,
+                                cfg.alpha_cross, cfg.nms_window)
+    t_slow = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for (b, g) in groups:
+        sk, sv, spt = subs[(b, g)]
+        K = O.gather_cache(sk, spt, 0, 0, L)
+        V = O.gather_cache(sv, spt, 0, 0, L)
+        sets = O.sparse_sets(L, cfg.n_sink, cfg.n_recent, list(sels[(b, g)]))
+        O.sparse_attention(qh[b, g * G:(g + 1) * G], K, V, sets)
+    t_fast = time.perf_counter() - t0
+    per_layer_step = slow_frac * t_slow + (1 - slow_frac) * t_fast
+    return cfg.B / per_layer_step, t_slow + t_fast, cores, t_slow, t_fast
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    li = W.make_layer(cfg.replace(n_layers=1), 0, dev)
+    slow_frac = float(np.mean(__import__("oracle.sfi_oracle", fromlist=["trigger"]).trigger(
+        W.boundary_stream(cfg), cfg.refresh_budget)))
+    vals, secs = [], []
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        v, s, cores, _, _ = oracle_sample(cfg, li, li.q[0], slow_frac)
+        if i >= args.warmup:
+            vals.append(v)
+            secs.append(s)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * float(np.mean(secs)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
+                   "context": cfg.context, "layers": cfg.n_layers, "decode_steps": cfg.steps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "per step: one slow and one fast layer-step of layer 0, all "
+                                   f"{cfg.B * cfg.Hkv} (sequence, KV head) groups, weighted by the "
+                                   f"run's slow fraction {slow_frac:.3f}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_sfi(args, cfg, rank, world, dist_on):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    bench = Bench(cfg, dev)
+    T, NL, B = cfg.steps, cfg.n_layers, cfg.B
+    tokens = B * T * NL
+    # warm-up, then a probe run recording the packed row counts of every slow step
+    for _ in range(args.warmup):
+        bench.run_sfi()
+    probe = {}
+    slows = bench.run_sfi(probe=probe)
+    torch.cuda.synchronize()
+    n_slow = sum(slows)
+    D = cfg.D
+    row_bytes = 4 * D
+    R = cfg.n_recent
+    fast_bytes = 0.0
+    union_rows = []
+    cur = None
+    for t in range(T):
+        if slows[t]:
+            cur = [x.cpu().numpy() for x in probe[t]]
+            union_rows.extend([float(x.mean()) for x in cur])
+        else:
+            for l in range(NL):
+                fast_bytes += float((cur[l].astype(np.float64) + R).sum()) * row_bytes + B * cfg.Hq * D * 2
+    dense_bytes_slow = sum(float(B * cfg.Hkv * cfg.seq_len(t) * row_bytes + B * cfg.Hq * cfg.seq_len(t) * 4)
+                           for t in range(T) if slows[t]) * NL
+    # timed region: SFI mixed decode, with kernel and step events
+    clocks = Clocks(torch.cuda.current_device())
+    bench.ctx.set_timing(True)
+    bench.ctx.timing(0, reset=True)
+    bench.ctx.timing(1, reset=True)
+    step_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(T)] for _ in range(args.steps)]
+    start_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks.start()
+    _sync_barrier(dist_on)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(args.steps):
+        start_ev[k].record()
+        bench.run_sfi(step_events=step_ev[k])
+    e1.record()
+    _sync_barrier(dist_on)
+    clk = clocks.stop()
+    t_sfi = _max_over_ranks(e0.elapsed_time(e1) / 1000.0, dist_on)
+    fast_ms, fast_n = bench.ctx.timing(0, reset=True)
+    dense_ms, dense_n = bench.ctx.timing(1, reset=True)
+    bench.ctx.set_timing(False)
+    # step-type breakdown from main-stream step events
+    st_fast, st_slow = [], []
+    for k in range(args.steps):
+        prev = start_ev[k]
+        for t in range(T):
+            ms = prev.elapsed_time(step_ev[k][t])
+            (st_slow if slows[t] else st_fast).append(ms)
+            prev = step_ev[k][t]
+    # dense full-KV baseline on the same cache
+    bench.run_dense()
+    t_dense = _timed(bench.run_dense, args.steps, dist_on)
+    # end to end through host buffers
+    hq = bench.q.cpu().pin_memory()
+    hk = bench.kn.cpu().pin_memory()
+    hv = bench.vn.cpu().pin_memory()
+    hout = torch.empty((T,) + tuple(bench.out.shape), dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(bench.q[0]), torch.empty_like(bench.kn[0]), torch.empty_like(bench.vn[0])
+    bench.run_e2e(hq, hk, hv, hout, dq, dk, dv)
+    t_e2e = _timed(lambda: bench.run_e2e(hq, hk, hv, hout, dq, dk, dv), args.steps, dist_on)
+    h2d = (hq[0].numel() * 2 + hk[0].numel() * 2 + hv[0].numel() * 2) * T
+    d2h = hout[0].numel() * 4 * T
+    # roofline of the dominant kernel, with launches measured in the timed region
+    peak, peak_kind = peaks()
+    k = args.steps
+    ach_fast = (fast_bytes * k / 1e9) / (fast_ms / 1e3) if fast_ms > 0 else 0.0
+    ach_dense = (dense_bytes_slow * k / 1e9) / (dense_ms / 1e3) if dense_ms > 0 else 0.0
+    dominant = "fast" if fast_ms >= dense_ms else "dense"
+    if dominant == "fast":
+        roof = {"kernel": "attn_kernel<128,1,kFast> (fast step)", "bound": "hbm", "achieved": ach_fast,
+                "peak": peak, "unit": "GB/s", "frac": ach_fast / peak,
+                "traffic": kernel_traffic("fast_attn_bytes_per_launch"),
+                "algorithmic_bytes_per_launch": fast_bytes / max(fast_n / k, 1),
+                "launches": fast_n, "avg_launch_us": 1000 * fast_ms / max(fast_n, 1),
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    else:
+        roof = {"kernel": "attn_kernel<128,1,kDenseExtras> (slow step)", "bound": "hbm", "achieved": ach_dense,
+                "peak": peak, "unit": "GB/s", "frac": ach_dense / peak,
+                "traffic": kernel_traffic("dense_attn_bytes_per_launch"),
+                "algorithmic_bytes_per_launch": dense_bytes_slow / max(dense_n / k, 1),
+                "launches": dense_n, "avg_launch_us": 1000 * dense_ms / max(dense_n, 1),
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    value = world * tokens / t_sfi * args.steps
+    launches_per_run = NL * (n_slow * 8 + (T - n_slow) * 3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * t_sfi / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": D,
+                   "context": cfg.context, "layers": NL, "decode_steps": T, "budget": cfg.budget_frac,
+                   "sink": cfg.n_sink, "recent": R, "trigger": f"bernoulli(1/16), M={cfg.refresh_budget}",
+                   "slow_steps": n_slow, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (KV cache %.1f GB)" %
+                         (NL * 2 * cfg.num_pages * cfg.Hkv * 16 * D * 2 / 1e9)},
+        "roofline": roof,
+        "e2e": {"value": world * tokens / t_e2e * args.steps, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_run * args.steps,
+        "clocks": clk,
+        "breakdown": {
+            "dense_full_kv_tok_s": world * tokens / t_dense * args.steps,
+            "speedup_vs_dense": t_dense / t_sfi,
+            "fast_step_tok_s": B * NL / (statistics.mean(st_fast) / 1e3) if st_fast else None,
+            "slow_step_tok_s": B * NL / (statistics.mean(st_slow) / 1e3) if st_slow else None,
+            "fast_attn_GBps": ach_fast, "dense_attn_GBps": ach_dense,
+            "fast_attn_ms_total": fast_ms, "dense_attn_ms_total": dense_ms,
+            "mean_packed_rows": float(np.mean(union_rows)) if union_rows else None,
+            "fast_frac_of_dense_bytes": None if not union_rows else
+            (float(np.mean(union_rows)) + R) / cfg.seq_len(T // 2),
+        },
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        li0 = bench.layers[0]
+        slow_frac = n_slow / T
+        v, secs, cores, ts, tf = oracle_sample(cfg, li0, bench.q[0, 0], slow_frac)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"one slow ({ts:.1f} s) and one fast ({tf:.1f} s) layer-step of "
+                                          f"layer 0, all {B * cfg.Hkv} (sequence, KV head) groups, "
+                                          f"weighted by the run's slow fraction {slow_frac:.3f}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    bench.ctx.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="sfi", choices=["sfi", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=0, help="override the workload's decode steps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = W.CONFIG_BY_NAME[args.config]
+    if args.decode_steps:
+        cfg = cfg.replace(steps=args.decode_steps)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+    else:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py --impl sfi needs a CUDA device")
+        S.lib()
+        run_sfi(args, cfg, rank, world, dist_on)
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -5,8 +5,8 @@ and compares the two with the tolerances of the hot path:
 * probabilities f and lse: absolute 1e-4; key norms: relative 1e-6
 * page-table indexing, gathers and compaction: bit-exact
 * selections: identical except at elements whose deciding comparisons are
-  near-ties (relative gap below NEAR_TIE) in the oracle's float64 values,
-  and >= 99.9 % overlap.
+  near-ties (relative gap below NEAR_TIE) in the oracle's float64 values
+  (see assert_selection_close).
 """
 from __future__ import annotations
 
@@ -87,27 +87,40 @@ def oracle_selector_detail(f: np.ndarray, norms: np.ndarray, L: int, cfg):
 
 
 def assert_selection_close(gpu_sel: np.ndarray, ora_sel: np.ndarray, ell2: np.ndarray,
-                           amb: np.ndarray, lo: int, what=""):
-    """gpu_sel, ora_sel: [G, K] absolute positions.  Differences are allowed
-    only at ambiguous elements or at scores within NEAR_TIE of the K-th."""
+                           amb: np.ndarray, lo: int, what="", min_overlap=0.98):
+    """gpu_sel, ora_sel: [G, K] absolute positions; ell2: oracle scores.
+
+    Elements whose own soft-NMS dominance or cross-head owner rests on a
+    near-tie (amb) may fall either way: a flipped dominance or owner moves a
+    score by up to alpha.  Every other element must be decided as the oracle
+    decides it: the non-ambiguous part of the GPU's set must be exactly the
+    best non-ambiguous candidates by the oracle's scores (ties to the lower
+    position), as many as the GPU chose, except for scores within NEAR_TIE of
+    that cut.  Also at least `min_overlap` of each set must agree."""
     G, K = ora_sel.shape
     worst = 1.0
     for h in range(G):
-        a = set(gpu_sel[h].tolist())
-        b = set(ora_sel[h].tolist())
-        assert len(a) == K, f"{what}: head {h} has duplicate picks"
-        sym = a ^ b
-        if sym:
-            s = np.sort(ell2[h])[::-1]
-            kth = s[K - 1]
-            for j in sym:
-                c = j - lo
-                near = abs(ell2[h, c] - kth) <= NEAR_TIE * max(abs(kth), 1e-30)
-                assert amb[h, c] or near, (
-                    f"{what}: head {h} position {j} differs and is not a near-tie "
-                    f"(score {ell2[h, c]!r}, K-th {kth!r})")
-        worst = min(worst, len(a & b) / K)
-    assert worst >= 0.999, f"{what}: overlap {worst:.5f}"
+        g = np.asarray(gpu_sel[h], np.int64) - lo
+        assert len(set(g.tolist())) == K, f"{what}: head {h} has duplicate picks"
+        assert g.min() >= 0 and g.max() < ell2.shape[1], f"{what}: head {h} picks outside C"
+        in_amb = amb[h, g]
+        n_amb = int(in_amb.sum())
+        got = set(g[~in_amb].tolist())
+        cand = np.flatnonzero(~amb[h])
+        v32 = ell2[h, cand].astype(np.float32)
+        order = cand[np.lexsort((cand, -v32))]
+        m = K - n_amb
+        want = set(order[:m].tolist())
+        diff = got ^ want
+        if diff:
+            cut = ell2[h, order[m - 1]] if m > 0 else ell2[h, order[0]]
+            for c in diff:
+                assert abs(ell2[h, c] - cut) <= NEAR_TIE * max(abs(cut), 1e-30), (
+                    f"{what}: head {h} position {c + lo} decided differently from the oracle "
+                    f"(score {ell2[h, c]!r}, cut {cut!r}, {n_amb} ambiguous picks)")
+        ov = len(set(gpu_sel[h].tolist()) & set(ora_sel[h].tolist())) / K
+        worst = min(worst, ov)
+    assert worst >= min_overlap, f"{what}: overlap {worst:.5f}"
     return worst
 
 
