@@ -143,7 +143,7 @@ class Bench:
             li.q = li.k_new = li.v_new = None
         self.out = torch.empty(cfg.n_layers, cfg.B, cfg.Hq, cfg.D, device=device)
         self.ctx = S.Context(self.shape, self.params, cfg.n_layers, overlap=True, device=device)
-        self.ws = torch.empty(S.sfi_workspace_size(self.shape, self.params), dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(S.sfi_workspace_size(self.shape, self.params), dtype=torch.uint8, device=device)
         torch.cuda.synchronize()
 
     def run_sfi(self, step_events=None, probe=None, q=None, kn=None, vn=None, out=None):

@@ -138,8 +138,11 @@ const char* sfi_status_str(sfi_status s);
 const char* sfi_version(void);
 
 /* Bytes of scratch the per-op calls below need for contexts up to
- * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes.
- * Ownership stays with the caller; contents need no initialisation. */
+ * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes
+ * (16-byte aligned).  Ownership stays with the caller.  The first 256 bytes
+ * hold a work counter of the attention kernels: they must be zero before the
+ * first call, and every call leaves them zero.  Calls that share one ws must
+ * not run concurrently. */
 sfi_status sfi_workspace_size(const sfi_shape* shape, const sfi_params* params, size_t* bytes);
 
 /* Packed-buffer row capacity p_max needed for contexts up to max_pages*16:

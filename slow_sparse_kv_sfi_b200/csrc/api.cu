@@ -48,20 +48,20 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   const int G = s.Hq / s.Hkv;
   const long bh = (long)s.B * s.Hkv;
   const int Lmax = s.max_pages * kPage;
-  const long T = (Lmax + kPage - 1) / kPage;
-  const long dense_chunks = std::min<long>((T + 7) / 8, (8L * num_sms() + bh - 1) / bh + 1);
-  const long fast_items = bh * fast_chunks(s, packed_rows_capacity(s, p), p.n_recent);
+  const long dense_chunks = dense_chunks_bound(s);
+  const int kmax = std::max(budget_k(p, Lmax), 0);
+  const long fast_items = bh * fast_chunks(s, packed_rows_capacity(s, p), p.n_recent, kmax + p.n_sink);
   const long items = std::max(bh * dense_chunks, fast_items);
   size_t off = 256;   // first 256 bytes reserved
   w.part_off = off;
   w.part_bytes = align_up(attn_part_bytes((int)items, G, s.D), 256);
   off += w.part_bytes;
-  w.stat_off = off;
-  w.stat_bytes = align_up((size_t)bh * 2 * sizeof(float), 256);
-  off += w.stat_bytes;
   const long nC = std::max<long>(Lmax - p.n_recent - p.n_sink, 1);
+  w.stat_off = off;
+  w.stat_bytes = align_up((size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double), 256);
+  off += w.stat_bytes;
   w.sel_off = off;
-  w.sel_bytes = align_up((size_t)s.B * s.Hq * nC * sizeof(float), 256);
+  w.sel_bytes = align_up((size_t)s.B * s.Hq * ((nC + 3) / 4 * 4) * sizeof(float), 256);
   off += w.sel_bytes;
   w.cmp_off = off;
   w.cmp_bytes = align_up((size_t)bh * compact_tiles((int)nC) * sizeof(int32_t), 256);
@@ -211,9 +211,10 @@ sfi_status sfi_dense_attn(const sfi_shape* shape, const sfi_paged_kv* kv, int32_
     if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
       return SFI_ERR_SHAPE;
   }
-  if (!ws) return SFI_ERR_WORKSPACE;
+  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
+  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
   const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
-  return run_dense_attn(*shape, *kv, L, q, out, extras,
+  return run_dense_attn(*shape, *kv, L, q, out, extras, static_cast<int*>(ws),
                         reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
                         (cudaStream_t)stream, nullptr, nullptr);
 }
@@ -237,9 +238,10 @@ sfi_status sfi_fast_attn(const sfi_shape* shape, const sfi_params* params,
   SFI_TRY(check_sparse_L(shape, params, L));
   SFI_TRY(check_packed(shape, params, packed));
   if (!q || !out) return SFI_ERR_INVALID_ARG;
-  if (!ws) return SFI_ERR_WORKSPACE;
+  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
+  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
   const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
-  return run_fast_attn(*shape, *params, *kv, L, q, *packed, out, lse,
+  return run_fast_attn(*shape, *params, *kv, L, q, *packed, out, lse, static_cast<int*>(ws),
                        reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
                        (cudaStream_t)stream, nullptr, nullptr);
 }
@@ -283,10 +285,11 @@ sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sf
   if (!ws || ws_bytes < w.total) return SFI_ERR_WORKSPACE;
   const int nC = L - params->n_recent - params->n_sink;
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + w.sel_off);
+  const int ld_s = (nC + 3) / 4 * 4;
   cudaStream_t st = (cudaStream_t)stream;
-  SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, nC,
+  SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s,
                             static_cast<char*>(ws) + w.stat_off, st));
-  SFI_TRY(run_topk(shape->B * shape->Hq, nC, scores, nC, K, params->n_sink, sel_idx, sel_ld, st));
+  SFI_TRY(run_topk(shape->B * shape->Hq, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, st));
   if (K_out) *K_out = K;
   return SFI_OK;
 }

@@ -36,8 +36,8 @@ namespace sfi {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
-constexpr int kTilesPerStage = 4;
-constexpr int kBoxBytes = 16 * 128;   // one 16-row x 64-col bf16 box
+constexpr int kBoxBytes = 16 * 128;   // 16 rows x 128 bytes: one column block of a tile
+constexpr int kChunkAlign = 8;        // chunk lengths are multiples of the largest stage
 
 enum AttnMode : int { kDense = 0, kDenseExtras = 1, kFast = 2 };
 
@@ -47,8 +47,9 @@ struct AttnArgs {
   const int32_t* page_table;
   const __nv_bfloat16* q;
   float* part;          // [n_items][G][D + 4]
+  int* ctr;             // work counter (zero on entry; the combine kernel re-zeroes it)
   int n_chunks;         // chunks per (b, kv head)
-  int chunk_tiles;      // dense: tiles per chunk (multiple of 4)
+  int chunk_tiles;      // dense: tiles per chunk (multiple of kChunkAlign, <= kMaxChunkTiles)
   int n_items;
   float scale_log2;     // log2(e) / sqrt(D)
   float scale;          // 1 / sqrt(D)
@@ -64,40 +65,61 @@ struct AttnArgs {
   int* err;
 };
 
-template <int D>
-struct Layout {
+constexpr int kMaxChunkTiles = 256;
+constexpr int kMaxBH = 512;
+
+// Shared-memory plan.  A tile is 16 rows of K (or V): one TMA box of
+// [D/64 column blocks][16 rows][128 B], 128B-swizzled.  Each consumer warp
+// takes TT tiles of every stage, so a stage holds 4 * TT tiles of K and V.
+template <int D, int NT>
+struct Plan {
+  static constexpr int TT = (NT == 1) ? 2 : 1;
+  static constexpr int kTPS = 4 * TT;
   static constexpr int kHalves = D / 64;
-  static constexpr int kTileBytes = kHalves * kBoxBytes;          // one 16-row tile of K (or V)
-  static constexpr int kKBytes = kTilesPerStage * kTileBytes;     // K part of a stage
-  static constexpr int kStageBytes = 2 * kKBytes;                 // K + V
+  static constexpr int kTileBytes = kHalves * kBoxBytes;
+  static constexpr int kKBytes = kTPS * kTileBytes;
+  static constexpr int kStageBytes = 2 * kKBytes;
+  static constexpr int kStages = (D == 128) ? (NT == 1 ? 3 : 6) : (NT == 1 ? 6 : 12);
+  static constexpr int kHeads = NT * 8;
+  static constexpr int kQBytes = kHeads * D * 2;
 };
+
+struct StageMeta {
+  int item;        // work item, or -1: no more work
+  int b, g;
+  int flags;       // bit 0: first stage of the item, bit 1: last stage of the item
+  int ntiles;      // tiles in this stage
+  int kinds;       // 2 bits per tile: 0 page, 1 packed, 2 skipped (bad page-table entry)
+  int pos0[8];     // page tiles: cache position of row 0; packed: packed row
+  int pad[2];
+};
+static_assert(sizeof(StageMeta) == 64, "meta size");
 
 template <int D, int NT>
 struct Smem {
-  static constexpr int kStages = (D == 128) ? (NT == 1 ? 5 : 4) : 8;
-  static constexpr int kHeads = NT * 8;
-  static constexpr int kStageBytes = Layout<D>::kStageBytes;
-  static constexpr int kMaskOff = kStages * kStageBytes;
-  static constexpr int kMaskBytes = kStages * kTilesPerStage * 16 * 4;
-  static constexpr int kBarOff = kMaskOff + kMaskBytes;
-  static constexpr int kStatOff = kBarOff + 2 * kStages * 8 + 64;
-  static constexpr int kStatBytes = kConsumerWarps * kHeads * 3 * 4;
-  static constexpr int kOOff = (kStatOff + kStatBytes + 15) / 16 * 16;
-  static constexpr int kOBytes = kConsumerWarps * kHeads * D * 4;
-  static constexpr int kTotal = kOOff + kOBytes + 1024;   // + alignment slack
+  using P = Plan<D, NT>;
+  static constexpr int kStages = P::kStages;
+  static constexpr int kMaskOff = kStages * P::kStageBytes;
+  static constexpr int kMaskBytes = kStages * P::kTPS * 16 * 4;
+  static constexpr int kQOff = kMaskOff + kMaskBytes;
+  static constexpr int kMetaOff = kQOff + kStages * P::kQBytes;
+  static constexpr int kPtOff = kMetaOff + kStages * (int)sizeof(StageMeta);
+  static constexpr int kNrOff = kPtOff + kMaxChunkTiles * 4;
+  static constexpr int kBarOff = kNrOff + kMaxBH * 4;
+  static constexpr int kTotal = kBarOff + 2 * kStages * 8 + 64 + 1024;   // + alignment slack
   static_assert(kTotal <= 227 * 1024, "shared memory budget");
 };
 
+// Tile range and page range of one work item.
 struct Item {
   int bg, b, g;
-  int t_begin, t_end;
-  int n_packed_tiles;
-  int rec_first_page;
-  int n_rows;
+  int t_begin, t_end;     // tiles of the item
+  int n_packed_tiles;     // tiles before this index are packed-buffer tiles
+  int first_page;         // page number of tile n_packed_tiles (fast) or tile 0 (dense)
 };
 
 template <int MODE>
-__device__ __forceinline__ Item decode_item(const AttnArgs& a, int item) {
+__device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const int* nrows_s) {
   Item it;
   it.bg = item / a.n_chunks;
   const int c = item - it.bg * a.n_chunks;
@@ -108,50 +130,24 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item) {
     it.t_begin = min(T, c * a.chunk_tiles);
     it.t_end = min(T, it.t_begin + a.chunk_tiles);
     it.n_packed_tiles = 0;
-    it.rec_first_page = 0;
-    it.n_rows = 0;
+    it.first_page = 0;
   } else {
-    int nr = a.n_rows[it.bg];
-    if (nr < 0 || nr > a.p_max) nr = nr < 0 ? 0 : a.p_max;   // reported by the combine check
-    it.n_rows = nr;
+    int nr = nrows_s[it.bg];
+    if (nr < 0 || nr > a.p_max) nr = nr < 0 ? 0 : a.p_max;   // reported by the combine kernel
     it.n_packed_tiles = (nr + kPage - 1) / kPage;
-    it.rec_first_page = a.rec_lo / kPage;
-    const int rec_last_page = (a.L - 1) / kPage;
-    const int T = it.n_packed_tiles + (rec_last_page - it.rec_first_page + 1);
+    it.first_page = a.rec_lo / kPage;
+    const int T = it.n_packed_tiles + ((a.L - 1) / kPage - it.first_page + 1);
     int ct = (T + a.n_chunks - 1) / a.n_chunks;
-    ct = (ct + kTilesPerStage - 1) / kTilesPerStage * kTilesPerStage;
+    ct = (ct + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
     it.t_begin = min(T, c * ct);
     it.t_end = min(T, it.t_begin + ct);
   }
   return it;
 }
 
-struct TileRef {
-  int kind;   // 0 page, 1 packed, -1 skip (bad page-table entry)
-  int y;      // TMA row coordinate
-  int pos0;   // page tiles: cache position of row 0; packed: packed row of row 0
-};
-
-template <int MODE>
-__device__ __forceinline__ TileRef resolve_tile(const AttnArgs& a, const Item& it, int tile) {
-  TileRef r;
-  if (MODE == kFast && tile < it.n_packed_tiles) {
-    r.kind = 1;
-    r.pos0 = tile * kPage;
-    r.y = it.bg * a.p_max + r.pos0;
-    return r;
-  }
-  const int page_no = (MODE == kFast) ? it.rec_first_page + (tile - it.n_packed_tiles) : tile;
-  const int page = __ldg(a.page_table + (size_t)it.b * a.max_pages + page_no);
-  r.pos0 = page_no * kPage;
-  if ((unsigned)page >= (unsigned)a.num_pages) {
-    r.kind = -1;
-    r.y = 0;
-  } else {
-    r.kind = 0;
-    r.y = (page * a.Hkv + it.g) * kPage;
-  }
-  return r;
+// Page number of page tile `t` of the item (t >= n_packed_tiles).
+__device__ __forceinline__ int item_page(const Item& it, int t) {
+  return it.first_page + (t - it.n_packed_tiles);
 }
 
 // Address of 16-byte chunk `ci` (0 .. D/8-1) of row `row` in a 128B-swizzled tile.
@@ -165,18 +161,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const __grid_constant__ CUtensorMap tpk, const __grid_constant__ CUtensorMap tpv,
                 const AttnArgs a) {
   using S = Smem<D, NT>;
-  using Lay = Layout<D>;
+  using P = Plan<D, NT>;
   constexpr int kStages = S::kStages;
+  constexpr int TT = P::TT;
+  constexpr int kTPS = P::kTPS;
   constexpr int kMT = D / 16;   // 16-wide slices of D
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* smask = reinterpret_cast<uint32_t*>(smem + S::kMaskOff);
+  uint8_t* sq = smem + S::kQOff;
+  StageMeta* smeta = reinterpret_cast<StageMeta*>(smem + S::kMetaOff);
+  int* ptbuf = reinterpret_cast<int*>(smem + S::kPtOff);
+  int* nrows_s = reinterpret_cast<int*>(smem + S::kNrOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
-  float* sstat = reinterpret_cast<float*>(smem + S::kStatOff);
-  float* so = reinterpret_cast<float*>(smem + S::kOOff);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -191,51 +191,148 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   __syncthreads();
 
-  // ------------------------------------------------------------ producer
+  // ------------------------------------------------------------ producer warp
   if (warp == kConsumerWarps) {
-    if (lane != 0) return;
-    prefetch_tensormap(&tk);
-    prefetch_tensormap(&tv);
+    if (lane == 0) {
+      prefetch_tensormap(&tk);
+      prefetch_tensormap(&tv);
+      if (MODE == kFast) {
+        prefetch_tensormap(&tpk);
+        prefetch_tensormap(&tpv);
+      }
+    }
+    const int BH = a.B * a.Hkv;
     if (MODE == kFast) {
-      prefetch_tensormap(&tpk);
-      prefetch_tensormap(&tpv);
+      for (int i = lane; i < BH; i += 32) nrows_s[i] = __ldg(a.n_rows + i);
+      __syncwarp();
     }
     const uint64_t policy = l2_policy_evict_first();
+    const int G = a.G;
+    // Work items come from a global counter; the next item's index and page
+    // table entries are fetched one item ahead so their latency overlaps the
+    // current item's copies.
+    int nxt = 0;
+    if (lane == 0) nxt = atomicAdd(a.ctr, 1);
+    nxt = __shfl_sync(0xffffffffu, nxt, 0);
+    int pf[kMaxChunkTiles / 32];
+    auto prefetch = [&](int item, int* regs) {
+#pragma unroll
+      for (int j = 0; j < kMaxChunkTiles / 32; ++j) regs[j] = 0;
+      if (item >= a.n_items) return;
+      const Item it = decode_item<MODE>(a, item, nrows_s);
+      const int p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
+      const int p_hi = item_page(it, max(it.t_end, it.n_packed_tiles));
+      const int32_t* row = a.page_table + (size_t)it.b * a.max_pages;
+#pragma unroll
+      for (int j = 0; j < kMaxChunkTiles / 32; ++j) {
+        const int p = p_lo + j * 32 + lane;
+        if (p < p_hi) regs[j] = __ldg(row + p);
+      }
+    };
+    prefetch(nxt, pf);
     int slot = 0;
     uint32_t phase = 0;
     int inflight = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < a.n_items && ok; item += gridDim.x) {
-      const Item it = decode_item<MODE>(a, item);
-      for (int t0 = it.t_begin; t0 < it.t_end; t0 += kTilesPerStage) {
-        if (*abort_flag || !mbar_wait(&empty[slot], phase ^ 1, a.err, kSiteAttnProducer)) {
-          ok = false;
-          *abort_flag = 1;
-          break;
-        }
-        const int nt = min(kTilesPerStage, it.t_end - t0);
-        TileRef refs[kTilesPerStage];
-        uint32_t bytes = 0;
-        for (int i = 0; i < nt; ++i) {
-          refs[i] = resolve_tile<MODE>(a, it, t0 + i);
-          if (refs[i].kind >= 0) bytes += 2 * Lay::kTileBytes + (refs[i].kind == 1 ? 64 : 0);
-          else latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteAttnPage);
-        }
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        uint8_t* sk = smem + slot * S::kStageBytes;
-        uint8_t* sv = sk + Lay::kKBytes;
-        for (int i = 0; i < nt; ++i) {
-          if (refs[i].kind < 0) continue;
-          const CUtensorMap* mk = refs[i].kind == 1 ? &tpk : &tk;
-          const CUtensorMap* mv = refs[i].kind == 1 ? &tpv : &tv;
+    int nxt2 = 0;
+    if (lane == 0) nxt2 = atomicAdd(a.ctr, 1);
+    while (ok) {
+      const int item = nxt;
+      // publish this item's page entries, then start fetching the next item's
+      __syncwarp();
 #pragma unroll
-          for (int h = 0; h < Lay::kHalves; ++h) {
-            tma_load_2d(sk + i * Lay::kTileBytes + h * kBoxBytes, mk, h * 64, refs[i].y, &full[slot], policy);
-            tma_load_2d(sv + i * Lay::kTileBytes + h * kBoxBytes, mv, h * 64, refs[i].y, &full[slot], policy);
+      for (int j = 0; j < kMaxChunkTiles / 32; ++j) ptbuf[j * 32 + lane] = pf[j];
+      __syncwarp();
+      nxt = __shfl_sync(0xffffffffu, nxt2, 0);
+      if (item < a.n_items) {
+        prefetch(nxt, pf);
+        if (lane == 0) nxt2 = (nxt < a.n_items) ? atomicAdd(a.ctr, 1) : a.n_items;
+      }
+      // one stage per kTPS tiles; an item without tiles still sends one
+      // (empty) stage so the consumers write its partial; item == n_items: stop.
+      Item it{};
+      int nst = 1;
+      int p_lo = 0;
+      if (item < a.n_items) {
+        it = decode_item<MODE>(a, item, nrows_s);
+        nst = max(1, (it.t_end - it.t_begin + kTPS - 1) / kTPS);
+        p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
+      }
+      for (int st = 0; st < nst; ++st) {
+        bool good = true;
+        if (lane == 0) {
+          good = !*abort_flag && mbar_wait(&empty[slot], phase ^ 1, a.err, kSiteAttnProducer);
+          if (good) {
+            StageMeta& m = smeta[slot];
+            if (item >= a.n_items) {
+              m.item = -1;
+              m.ntiles = 0;
+              mbar_arrive_expect_tx(&full[slot], 0);
+            } else {
+              uint32_t bytes = 0;
+              const int t0 = it.t_begin + st * kTPS;
+              const int nt = max(0, min(kTPS, it.t_end - t0));
+              int kinds = 0;
+              m.item = item;
+              m.b = it.b;
+              m.g = it.g;
+              m.flags = (st == 0 ? 1 : 0) | (st == nst - 1 ? 2 : 0);
+              m.ntiles = nt;
+              uint8_t* sk = smem + slot * P::kStageBytes;
+              uint8_t* sv = sk + P::kKBytes;
+              if (st == 0) bytes += G * D * 2;
+              int ys[kTPS];
+              for (int i = 0; i < nt; ++i) {
+                const int t = t0 + i;
+                int kind, y, pos0;
+                if (MODE == kFast && t < it.n_packed_tiles) {
+                  kind = 1;
+                  pos0 = t * kPage;
+                  y = it.bg * a.p_max + pos0;
+                  bytes += 2 * P::kTileBytes + 64;
+                } else {
+                  const int pg = item_page(it, t);
+                  const int page = ptbuf[pg - p_lo];
+                  pos0 = pg * kPage;
+                  if ((unsigned)page >= (unsigned)a.num_pages) {
+                    kind = 2;
+                    y = 0;
+                    latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteAttnPage);
+                  } else {
+                    kind = 0;
+                    y = (page * a.Hkv + it.g) * kPage;
+                    bytes += 2 * P::kTileBytes;
+                  }
+                }
+                kinds |= kind << (2 * i);
+                m.pos0[i] = pos0;
+                ys[i] = y;
+              }
+              m.kinds = kinds;
+              mbar_arrive_expect_tx(&full[slot], bytes);
+              if (st == 0)
+                bulk_load(sq + slot * P::kQBytes, a.q + ((size_t)it.b * a.Hq + it.g * G) * D, G * D * 2,
+                          &full[slot]);
+              for (int i = 0; i < nt; ++i) {
+                const int kind = (kinds >> (2 * i)) & 3;
+                if (kind == 2) continue;
+                const CUtensorMap* mk = kind == 1 ? &tpk : &tk;
+                const CUtensorMap* mv = kind == 1 ? &tpv : &tv;
+                tma_load_3d(sk + i * P::kTileBytes, mk, 0, ys[i], 0, &full[slot], policy);
+                tma_load_3d(sv + i * P::kTileBytes, mv, 0, ys[i], 0, &full[slot], policy);
+                if (kind == 1)
+                  bulk_load(smask + (slot * kTPS + i) * 16,
+                            a.headmask + (size_t)it.bg * a.p_max + m.pos0[i], 64, &full[slot]);
+              }
+            }
+          } else {
+            *abort_flag = 1;
           }
-          if (refs[i].kind == 1)
-            bulk_load(smask + (slot * kTilesPerStage + i) * 16,
-                      a.headmask + (size_t)it.bg * a.p_max + refs[i].pos0, 64, &full[slot]);
+        }
+        good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+        if (!good) {
+          ok = false;
+          break;
         }
         inflight = min(inflight + 1, kStages);
         if (++slot == kStages) {
@@ -243,8 +340,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           phase ^= 1;
         }
       }
+      if (item >= a.n_items) break;
     }
-    if (!ok) {
+    if (!ok && lane == 0) {
       // Drain: wait (bounded) for the copies of stages still in flight so no
       // TMA write lands after this CTA has left the SM.
       for (int k = 0; k < inflight; ++k) {
@@ -267,180 +365,223 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int rowV = (lane & 7) + ((lane >> 4) & 1) * 8;
   const int chV = (lane >> 3) & 1;
   const float NEG_INF = -INFINITY;
+  constexpr int H8 = P::kHeads;
 
   int slot = 0;
   uint32_t phase = 0;
-  bool dead = false;   // set once any wait of this CTA failed: keep only the barrier protocol
-  for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-    const Item it = decode_item<MODE>(a, item);
-
-    // Q^T fragments (B operand): head nt*8 + r0, dims ks*16 + cq (+8).
-    uint32_t qb[NT][kMT][2];
+  uint32_t qb[NT][kMT][2];
+  float o[NT][kMT][4];
+  float mrun[NT][2], lrun[NT][2], lcand[NT][2];
+  int cur_b = 0, cur_g = 0;
+  for (;;) {
+    if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer)) {
+      *abort_flag = 1;
+      break;
+    }
+    const StageMeta& m = smeta[slot];
+    const int item = m.item;
+    if (item < 0) break;
+    const int flags = m.flags;
+    if (flags & 1) {
+      // first stage of an item: the group's queries (B operand of S^T) and a fresh state
+      cur_b = m.b;
+      cur_g = m.g;
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(sq + slot * P::kQBytes);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int hh = nt * 8 + r0;
-      const bool hv = hh < a.G;
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          a.q + ((size_t)it.b * a.Hq + it.g * a.G + (hv ? hh : 0)) * D);
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hh = nt * 8 + r0;
+        const bool hv = hh < a.G;
 #pragma unroll
-      for (int ks = 0; ks < kMT; ++ks) {
-        qb[nt][ks][0] = hv ? __ldg(qrow + (ks * 16 + cq) / 2) : 0u;
-        qb[nt][ks][1] = hv ? __ldg(qrow + (ks * 16 + 8 + cq) / 2) : 0u;
+        for (int ks = 0; ks < kMT; ++ks) {
+          qb[nt][ks][0] = hv ? q32[(hh * D + ks * 16 + cq) / 2] : 0u;
+          qb[nt][ks][1] = hv ? q32[(hh * D + ks * 16 + 8 + cq) / 2] : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          mrun[nt][j] = NEG_INF;
+          lrun[nt][j] = 0.f;
+          lcand[nt][j] = 0.f;
+        }
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[nt][mt][i] = 0.f;
       }
     }
-    float o[NT][kMT][4];
-    float mrun[NT][2], lrun[NT][2], lcand[NT][2];
+    // this warp's tiles: warp + 4 * tt
+    bool act[TT];
+    int kind_[TT], pos0_[TT];
+    uint32_t kb_[TT], vb_[TT];
+    uint32_t rmask[TT][2];
+    bool any = false;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int tt = 0; tt < TT; ++tt) {
+      const int ti = warp + 4 * tt;
+      kind_[tt] = (m.kinds >> (2 * ti)) & 3;
+      act[tt] = ti < m.ntiles && kind_[tt] != 2;
+      any |= act[tt];
+      pos0_[tt] = m.pos0[ti];
+      uint8_t* sk = smem + slot * P::kStageBytes + ti * P::kTileBytes;
+      uint8_t* sv = sk + P::kKBytes;
+      kb_[tt] = smem_u32(sk);
+      vb_[tt] = smem_u32(sv);
+      rmask[tt][0] = rmask[tt][1] = 0u;
+      if (!act[tt]) continue;
+      if (kind_[tt] == 0) {
+        const int lo = (MODE == kFast) ? a.rec_lo : 0;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        mrun[nt][j] = NEG_INF;
-        lrun[nt][j] = 0.f;
-        lcand[nt][j] = 0.f;
+        for (int j = 0; j < 2; ++j) {
+          const int pos = pos0_[tt] + r0 + 8 * j;
+          rmask[tt][j] = (pos < a.L && pos >= lo) ? 0xffffffffu : 0u;
+        }
+        if (pos0_[tt] + kPage > a.L) {
+          // Rows at or beyond L may hold anything: zero their V rows so
+          // 0 * garbage cannot poison the PV product.
+          const int first_bad = a.L - pos0_[tt];
+          const int nchunks = (kPage - first_bad) * (D / 8);
+          for (int c = lane; c < nchunks; c += 32) {
+            const int row = first_bad + c / (D / 8);
+            const int ci = c % (D / 8);
+            *reinterpret_cast<uint4*>(sv + (ci >> 3) * kBoxBytes + row * 128 + (ci & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      } else {
+        const uint32_t* mk = smask + (slot * kTPS + ti) * 16;
+        rmask[tt][0] = mk[r0];
+        rmask[tt][1] = mk[r0 + 8];
       }
-#pragma unroll
-      for (int mt = 0; mt < kMT; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o[nt][mt][i] = 0.f;
     }
 
-    for (int t0 = it.t_begin; t0 < it.t_end; t0 += kTilesPerStage) {
-      if (!dead && (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer))) {
-        *abort_flag = 1;
-        dead = true;
-      }
-      const int tile = t0 + warp;
-      if (!dead && tile < it.t_end) {
-        const TileRef ref = resolve_tile<MODE>(a, it, tile);
-        if (ref.kind >= 0) {
-          uint8_t* sk = smem + slot * S::kStageBytes + warp * Lay::kTileBytes;
-          uint8_t* sv = sk + Lay::kKBytes;
-          const uint32_t kb = smem_u32(sk);
-          const uint32_t vb = smem_u32(sv);
-          // Row validity.  Page tiles: positions in range (and inside the
-          // recent window for the fast step).  Packed tiles: per-head mask.
-          uint32_t rmask[2];
-          if (ref.kind == 0) {
-            const int lo = (MODE == kFast) ? a.rec_lo : 0;
+    if (any) {
+      // S^T = K . Q^T per tile, two independent accumulator chains over D
+      float s[TT][NT][4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int pos = ref.pos0 + r0 + 8 * j;
-              rmask[j] = (pos < a.L && pos >= lo) ? 0xffffffffu : 0u;
-            }
-            if (ref.pos0 + kPage > a.L) {
-              // Rows at or beyond L may hold anything: zero their V rows so
-              // 0 * garbage cannot poison the PV product.
-              const int first_bad = a.L - ref.pos0;
-              const int nchunks = (kPage - first_bad) * (D / 8);
-              for (int c = lane; c < nchunks; c += 32) {
-                const int row = first_bad + c / (D / 8);
-                const int ci = c % (D / 8);
-                *reinterpret_cast<uint4*>(sv + (ci >> 3) * kBoxBytes + row * 128 + (ci & 7) * 16) =
-                    make_uint4(0, 0, 0, 0);
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
-            }
-          } else {
-            const uint32_t* mk = smask + (slot * kTilesPerStage + warp) * 16;
-            rmask[0] = mk[r0];
-            rmask[1] = mk[r0 + 8];
-          }
-
-          // S^T = K . Q^T
-          float s[NT][4];
+      for (int tt = 0; tt < TT; ++tt) {
+        float s2[NT][4];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+          for (int i = 0; i < 4; ++i) s[tt][nt][i] = s2[nt][i] = 0.f;
+        if (act[tt]) {
 #pragma unroll
-          for (int ks = 0; ks < kMT; ++ks) {
-            uint32_t af[4];
-            ldmatrix_x4(af, swz(kb, rowA, ks * 2 + chA));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], af, qb[nt][ks][0], qb[nt][ks][1]);
-          }
-
-          // mask, scale, online softmax
-          uint32_t pb_hi[NT][2], pb_lo[NT][2];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            float x[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int hh = nt * 8 + cq + (i & 1);
-              const bool v = (rmask[i >> 1] >> hh) & 1u;
-              x[i] = (v && hh < a.G) ? s[nt][i] * a.scale_log2 : NEG_INF;
-            }
-            if (MODE == kDenseExtras && ref.kind == 0 && a.logits) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int hh = nt * 8 + cq + (i & 1);
-                const int pos = ref.pos0 + r0 + 8 * (i >> 1);
-                if (hh < a.G && pos < a.L)
-                  a.logits[((size_t)it.b * a.Hq + it.g * a.G + hh) * a.ld + pos] = s[nt][i] * a.scale;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              float tm = fmaxf(x[j], x[j + 2]);
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
-              tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
-              const float mnew = fmaxf(mrun[nt][j], tm);
-              const float mref = (mnew == NEG_INF) ? 0.f : mnew;
-              const float alpha = fast_exp2(mrun[nt][j] - mref);
-              mrun[nt][j] = mnew;
-              lrun[nt][j] *= alpha;
-              if (MODE == kDenseExtras) lcand[nt][j] *= alpha;
-#pragma unroll
-              for (int mt = 0; mt < kMT; ++mt) {
-                o[nt][mt][j] *= alpha;
-                o[nt][mt][j + 2] *= alpha;
-              }
-              x[j] = fast_exp2(x[j] - mref);
-              x[j + 2] = fast_exp2(x[j + 2] - mref);
-              lrun[nt][j] += x[j] + x[j + 2];
-              if (MODE == kDenseExtras && ref.kind == 0) {
-                const int p0 = ref.pos0 + r0, p1 = p0 + 8;
-                if (p0 >= a.cand_lo && p0 < a.cand_hi) lcand[nt][j] += x[j];
-                if (p1 >= a.cand_lo && p1 < a.cand_hi) lcand[nt][j] += x[j + 2];
-              }
-            }
-            // P -> bf16 hi + lo, then transpose to the B operand of PV.
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const float p0 = x[2 * j], p1 = x[2 * j + 1];
-              const uint32_t hi = pack_bf16x2(p0, p1);
-              const float2 hf = unpack_bf16x2(hi);
-              const uint32_t lo = pack_bf16x2(p0 - hf.x, p1 - hf.y);
-              pb_hi[nt][j] = movmatrix_trans(hi);
-              pb_lo[nt][j] = movmatrix_trans(lo);
-            }
-          }
-
-          // O^T += V^T . P^T
-#pragma unroll
-          for (int mt = 0; mt < kMT; ++mt) {
-            uint32_t vf[4];
-            ldmatrix_x4_trans(vf, swz(vb, rowV, mt * 2 + chV));
+          for (int ks = 0; ks < kMT; ks += 2) {
+            uint32_t af[4], ag[4];
+            ldmatrix_x4(af, swz(kb_[tt], rowA, ks * 2 + chA));
+            ldmatrix_x4(ag, swz(kb_[tt], rowA, (ks + 1) * 2 + chA));
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              mma_bf16_16816(o[nt][mt], vf, pb_hi[nt][0], pb_hi[nt][1]);
-              mma_bf16_16816(o[nt][mt], vf, pb_lo[nt][0], pb_lo[nt][1]);
+              mma_bf16_16816(s[tt][nt], af, qb[nt][ks][0], qb[nt][ks][1]);
+              mma_bf16_16816(s2[nt], ag, qb[nt][ks + 1][0], qb[nt][ks + 1][1]);
             }
           }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) s[tt][nt][i] += s2[nt][i];
       }
-      __syncwarp();
-      if (lane == 0 && !dead) mbar_arrive(&empty[slot]);
-      if (++slot == kStages) {
-        slot = 0;
-        phase ^= 1;
+
+      // mask, scale, online softmax over the warp's TT tiles at once
+      uint32_t pb_hi[TT][NT][2], pb_lo[TT][NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float x[TT][4];
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int hh = nt * 8 + cq + (i & 1);
+            const bool v = (rmask[tt][i >> 1] >> hh) & 1u;
+            x[tt][i] = (v && hh < a.G) ? s[tt][nt][i] * a.scale_log2 : NEG_INF;
+          }
+        if (MODE == kDenseExtras && a.logits) {
+#pragma unroll
+          for (int tt = 0; tt < TT; ++tt) {
+            if (!act[tt] || kind_[tt] != 0) continue;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int hh = nt * 8 + cq + (i & 1);
+              const int pos = pos0_[tt] + r0 + 8 * (i >> 1);
+              if (hh < a.G && pos < a.L)
+                a.logits[((size_t)cur_b * a.Hq + cur_g * a.G + hh) * a.ld + pos] = s[tt][nt][i] * a.scale;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float tm = NEG_INF;
+#pragma unroll
+          for (int tt = 0; tt < TT; ++tt) tm = fmaxf(tm, fmaxf(x[tt][j], x[tt][j + 2]));
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+          tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+          const float mnew = fmaxf(mrun[nt][j], tm);
+          const float mref = (mnew == NEG_INF) ? 0.f : mnew;
+          const float alpha = fast_exp2(mrun[nt][j] - mref);
+          mrun[nt][j] = mnew;
+          lrun[nt][j] *= alpha;
+          if (MODE == kDenseExtras) lcand[nt][j] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt) {
+            o[nt][mt][j] *= alpha;
+            o[nt][mt][j + 2] *= alpha;
+          }
+#pragma unroll
+          for (int tt = 0; tt < TT; ++tt) {
+            x[tt][j] = fast_exp2(x[tt][j] - mref);
+            x[tt][j + 2] = fast_exp2(x[tt][j + 2] - mref);
+            lrun[nt][j] += x[tt][j] + x[tt][j + 2];
+            if (MODE == kDenseExtras && kind_[tt] == 0) {
+              const int p0 = pos0_[tt] + r0, p1 = p0 + 8;
+              if (p0 >= a.cand_lo && p0 < a.cand_hi) lcand[nt][j] += x[tt][j];
+              if (p1 >= a.cand_lo && p1 < a.cand_hi) lcand[nt][j] += x[tt][j + 2];
+            }
+          }
+        }
+        // P -> bf16 hi + lo, then transpose to the B operand of PV.
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float p0 = x[tt][2 * j], p1 = x[tt][2 * j + 1];
+            const uint32_t hi = pack_bf16x2(p0, p1);
+            const float2 hf = unpack_bf16x2(hi);
+            const uint32_t lo = pack_bf16x2(p0 - hf.x, p1 - hf.y);
+            pb_hi[tt][nt][j] = movmatrix_trans(hi);
+            pb_lo[tt][nt][j] = movmatrix_trans(lo);
+          }
+      }
+
+      // O^T += V^T . P^T
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) {
+        if (!act[tt]) continue;
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+          uint32_t vf[4];
+          ldmatrix_x4_trans(vf, swz(vb_[tt], rowV, mt * 2 + chV));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_bf16_16816(o[nt][mt], vf, pb_hi[tt][nt][0], pb_hi[tt][nt][1]);
+            mma_bf16_16816(o[nt][mt], vf, pb_lo[tt][nt][0], pb_lo[tt][nt][1]);
+          }
+        }
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (++slot == kStages) {
+      slot = 0;
+      phase ^= 1;
+    }
+    if (!(flags & 2)) continue;
 
-    // ---- merge the four warps' partial softmax states of this item
+    // ---- last stage of the item: this warp's partial softmax state goes to
+    // global memory as it is (m, l, l_cand and the unnormalised O of each
+    // query head); the combine kernel merges all partials.
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -450,102 +591,129 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           lrun[nt][j] += __shfl_xor_sync(0xffffffffu, lrun[nt][j], sh);
           if (MODE == kDenseExtras) lcand[nt][j] += __shfl_xor_sync(0xffffffffu, lcand[nt][j], sh);
         }
-    constexpr int H8 = S::kHeads;
-    if (lane < 4) {
+    float* part = a.part + ((size_t)item * kConsumerWarps + warp) * a.G * (D + 4);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int hh = nt * 8 + cq + j;
-          float* st = sstat + (warp * H8 + hh) * 3;
-          st[0] = mrun[nt][j];
-          st[1] = lrun[nt][j];
-          st[2] = lcand[nt][j];
-        }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int hh = nt * 8 + cq + (i & 1);
           const int d = mt * 16 + r0 + (i >> 1) * 8;
-          so[(warp * H8 + hh) * D + d] = o[nt][mt][i];
+          if (hh < a.G) part[hh * (D + 4) + d] = o[nt][mt][i];
         }
-    named_barrier(1, kConsumerWarps * 32);
-    float* part = a.part + (size_t)item * a.G * (D + 4);
-    for (int idx = ctid; idx < a.G * D; idx += kConsumerWarps * 32) {
-      const int hh = idx / D, d = idx - hh * D;
-      float M = NEG_INF;
+      if (lane < 4) {
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sstat[(w * H8 + hh) * 3]);
-      const float mref = (M == NEG_INF) ? 0.f : M;
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w)
-        acc += exp2f(sstat[(w * H8 + hh) * 3] - mref) * so[(w * H8 + hh) * D + d];
-      part[hh * (D + 4) + d] = acc;
-      if (d == 0) {
-        float l = 0.f, lc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float wt = exp2f(sstat[(w * H8 + hh) * 3] - mref);
-          l += wt * sstat[(w * H8 + hh) * 3 + 1];
-          lc += wt * sstat[(w * H8 + hh) * 3 + 2];
+        for (int j = 0; j < 2; ++j) {
+          const int hh = nt * 8 + cq + j;
+          if (hh < a.G) {
+            part[hh * (D + 4) + D] = mrun[nt][j];
+            part[hh * (D + 4) + D + 1] = lrun[nt][j];
+            part[hh * (D + 4) + D + 2] = lcand[nt][j];
+          }
         }
-        part[hh * (D + 4) + D] = M;
-        part[hh * (D + 4) + D + 1] = l;
-        part[hh * (D + 4) + D + 2] = lc;
       }
     }
-    named_barrier(1, kConsumerWarps * 32);
   }
 }
 
-// Merge the per-chunk partials of every (b, query head): one warp each.
+// Merge the partials of every (b, query head): one CTA of kCombWarps warps
+// each.  Pass 1: the largest m.  Pass 2: warp w folds partials w, w + 8, ...
+// with four partials' loads in flight per step; the warps' sums meet in
+// shared memory.
+constexpr int kCombWarps = 8;
+
 template <int D>
-__global__ void attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq,
-                                    int Hkv, int G, float* __restrict__ out, float* __restrict__ lse,
-                                    float* __restrict__ lse_cand, const int32_t* n_rows, int p_max,
-                                    int* err) {
+__global__ void __launch_bounds__(kCombWarps * 32)
+    attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
+                        float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
+                        const int32_t* n_rows, int p_max, int* err, int* ctr) {
   constexpr int kPer = D / 32;
-  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wid >= B * Hq) return;
-  const int b = wid / Hq, hq = wid - b * Hq;
+  __shared__ float red[kCombWarps][D + 4];
+  __shared__ float mx[kCombWarps];
+  if (blockIdx.x == 0 && threadIdx.x == 0) ctr[0] = 0;   // the attention kernel is done with it
+  const int row = blockIdx.x;   // b * Hq + hq
+  const int b = row / Hq, hq = row - b * Hq;
   const int g = hq / G, hh = hq - g * G;
   const int bg = b * Hkv + g;
-  if (n_rows && lane == 0 && hh == 0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (n_rows && threadIdx.x == 0 && hh == 0) {
     const int nr = n_rows[bg];
     if (nr < 0 || nr > p_max) latch_error(err, SFI_ERR_DEVICE_CHECK, kSiteAttnRows);
   }
   const size_t stride = (size_t)G * (D + 4);
-  const float* base = part + (size_t)bg * n_chunks * stride + (size_t)hh * (D + 4);
+  const int n = n_chunks * kConsumerWarps;   // one partial per consumer warp and work item
+  const float* base = part + (size_t)bg * n * stride + (size_t)hh * (D + 4);
   float M = -INFINITY;
-  for (int c = lane; c < n_chunks; c += 32) M = fmaxf(M, base[c * stride + D]);
+  for (int c = threadIdx.x; c < n; c += blockDim.x) M = fmaxf(M, __ldg(base + c * stride + D));
 #pragma unroll
   for (int sh = 16; sh >= 1; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+  if (lane == 0) mx[warp] = M;
+  __syncthreads();
+  M = mx[0];
+#pragma unroll
+  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, mx[w]);
   const float mref = (M == -INFINITY) ? 0.f : M;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   float l = 0.f, lc = 0.f;
-  for (int c = 0; c < n_chunks; ++c) {
-    const float* pc = base + c * stride;
-    const float w = exp2f(pc[D] - mref);
-    l += w * pc[D + 1];
-    lc += w * pc[D + 2];
+  for (int c0 = warp; c0 < n; c0 += 4 * kCombWarps) {
+    float st[4][3];
+    float ov[4][kPer];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) acc[k] += w * pc[lane * kPer + k];
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * kCombWarps;
+      if (c < n) {
+        const float* pc = base + c * stride;
+        st[u][0] = __ldg(pc + D);
+        st[u][1] = __ldg(pc + D + 1);
+        st[u][2] = __ldg(pc + D + 2);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) ov[u][k] = __ldg(pc + lane * kPer + k);
+      } else {
+        st[u][0] = -INFINITY;
+        st[u][1] = st[u][2] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) ov[u][k] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = exp2f(st[u][0] - mref);
+      l += w * st[u][1];
+      lc += w * st[u][2];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] += w * ov[u][k];
+    }
   }
-  const float inv = 1.f / l;
-  float* orow = out + ((size_t)b * Hq + hq) * D + lane * kPer;
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) orow[k] = acc[k] * inv;
+  for (int k = 0; k < kPer; ++k) red[warp][lane * kPer + k] = acc[k];
   if (lane == 0) {
-    if (lse) lse[(size_t)b * Hq + hq] = (M + log2f(l)) * kLn2;
-    if (lse_cand) lse_cand[(size_t)b * Hq + hq] = lc > 0.f ? (M + log2f(lc)) * kLn2 : -INFINITY;
+    red[warp][D] = l;
+    red[warp][D + 1] = lc;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float lt = 0.f, lct = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      lt += red[w][D];
+      lct += red[w][D + 1];
+    }
+    const float inv = 1.f / lt;
+    float* orow = out + (size_t)row * D + lane * kPer;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCombWarps; ++w) t += red[w][lane * kPer + k];
+      orow[k] = t * inv;
+    }
+    if (lane == 0) {
+      if (lse) lse[row] = (M + log2f(lt)) * kLn2;
+      if (lse_cand) lse_cand[row] = lct > 0.f ? (M + log2f(lct)) * kLn2 : -INFINITY;
+    }
   }
 }
 
@@ -575,15 +743,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// rows x D bf16 matrix, box of 16 rows x 64 columns, 128-byte swizzle.
+// rows x D bf16 matrix viewed as [D/64 column blocks][rows][64 columns]: one
+// box is a whole 16-row tile, landing as [block][16 rows][128 B] with the
+// 128-byte swizzle (4 KB per load at D = 128).
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 16};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(D / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128};
+  cuuint32_t box[3] = {64, 16, (cuuint32_t)(D / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -617,45 +787,57 @@ sfi_status launch_attn(int D, int G, const CUtensorMap& tk, const CUtensorMap& t
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int* err,
-                          cudaStream_t st) {
+                          int* ctr, cudaStream_t st) {
   const int G = s.Hq / s.Hkv;
-  const int warps = s.B * s.Hq;
-  const int grid = (warps + 3) / 4;
+  const int grid = s.B * s.Hq;
   if (D == 128)
-    attn_combine_kernel<128><<<grid, 128, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
-                                                   lse_cand, n_rows, p_max, err);
+    attn_combine_kernel<128><<<grid, kCombWarps * 32, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
+                                                   lse_cand, n_rows, p_max, err, ctr);
   else
-    attn_combine_kernel<64><<<grid, 128, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
-                                                  lse_cand, n_rows, p_max, err);
+    attn_combine_kernel<64><<<grid, kCombWarps * 32, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
+                                                  lse_cand, n_rows, p_max, err, ctr);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 }  // namespace
 
 // Tiles of 16 rows per chunk for the dense step: about 8 work items per SM,
-// at least 8 tiles, a multiple of the 4-tile stage.
+// at least 8 tiles and at most kMaxChunkTiles, a multiple of the 4-tile stage.
 int dense_chunk_tiles(const sfi_shape& s, int L) {
   const long T = (L + kPage - 1) / kPage;
   const long bh = (long)s.B * s.Hkv;
   long ct = (T * bh + 8L * num_sms() - 1) / (8L * num_sms());
   ct = std::max(ct, 8L);
-  ct = (ct + kTilesPerStage - 1) / kTilesPerStage * kTilesPerStage;
-  return (int)ct;
+  ct = (ct + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
+  return (int)std::min<long>(ct, kMaxChunkTiles);
 }
 
-int fast_chunks(const sfi_shape& s, int p_max, int n_recent) {
+int dense_chunks_bound(const sfi_shape& s) {
+  const long T = (long)s.max_pages;
   const long bh = (long)s.B * s.Hkv;
-  const long tiles_max = (p_max + kPage - 1) / kPage + n_recent / kPage + 2;
-  long nc = (8L * num_sms() + bh - 1) / bh;
-  nc = std::min(nc, std::max(1L, tiles_max / 8));
+  const long a = (8L * num_sms() + bh - 1) / bh + 1;
+  const long b = (T + kMaxChunkTiles - 1) / kMaxChunkTiles;
+  return (int)std::min<long>((T + 7) / 8, std::max(a, b));
+}
+
+// Chunks per (b, kv head) for the fast step: items of about 32 tiles for the
+// expected packed size (n_sink + K rows), never more than kMaxChunkTiles tiles
+// even when the packed buffer is full.
+int fast_chunks(const sfi_shape& s, int p_max, int n_recent, int k_est) {
+  const long t_rec = n_recent / kPage + 2;
+  const long t_max = (p_max + kPage - 1) / kPage + t_rec;
+  const long t_est = std::min<long>((k_est + kPage - 1) / kPage + 1, (p_max + kPage - 1) / kPage) + t_rec;
+  long nc = std::max<long>((t_est + 31) / 32, (t_max + kMaxChunkTiles - 1) / kMaxChunkTiles);
   return (int)std::max(nc, 1L);
 }
 
-size_t attn_part_bytes(int n_items, int G, int D) { return (size_t)n_items * G * (D + 4) * sizeof(float); }
+size_t attn_part_bytes(int n_items, int G, int D) {
+  return (size_t)n_items * kConsumerWarps * G * (D + 4) * sizeof(float);
+}
 
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
-                          float* out, const sfi_dense_extras* ex, float* part, size_t part_bytes,
-                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+                          float* out, const sfi_dense_extras* ex, int* ctr, float* part,
+                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
   const int G = s.Hq / s.Hkv;
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
@@ -665,6 +847,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   a.num_pages = s.num_pages; a.max_pages = s.max_pages;
   a.page_table = kv.page_table;
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.ctr = ctr;
   a.chunk_tiles = dense_chunk_tiles(s, L);
   const int T = (L + kPage - 1) / kPage;
   a.n_chunks = (T + a.chunk_tiles - 1) / a.chunk_tiles;
@@ -691,7 +874,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
   r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0,
-                     kv.err, st);
+                     kv.err, ctr, st);
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
     dim3 grid((L + 1023) / 1024 < 64 ? (L + 1023) / 1024 : 64, s.B * s.Hq);
@@ -702,10 +885,11 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
 }
 
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
-                         const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse,
+                         const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
                          cudaEvent_t ev_end) {
   const int G = s.Hq / s.Hkv;
+  if ((long)s.B * s.Hkv > kMaxBH) return SFI_ERR_UNSUPPORTED;
   CUtensorMap tk, tv, tpk, tpv;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
   const uint64_t prows = (uint64_t)s.B * s.Hkv * pk.p_max;
@@ -717,7 +901,8 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   a.num_pages = s.num_pages; a.max_pages = s.max_pages;
   a.page_table = kv.page_table;
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
-  a.n_chunks = fast_chunks(s, pk.p_max, p.n_recent);
+  a.ctr = ctr;
+  a.n_chunks = fast_chunks(s, pk.p_max, p.n_recent, std::max(budget_k(p, L), 0) * 1 + p.n_sink);
   a.n_items = s.B * s.Hkv * a.n_chunks;
   if (attn_part_bytes(a.n_items, G, s.D) > part_bytes) return SFI_ERR_WORKSPACE;
   a.part = part;
@@ -732,7 +917,8 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   sfi_status r = launch_attn<kFast>(s.D, G, tk, tv, tpk, tpv, a, st);
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
-  return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, kv.err, st);
+  return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, kv.err, ctr,
+                        st);
 }
 
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,

@@ -9,14 +9,15 @@
 // up to the next multiple of 16.  The candidate range is cut into tiles of
 // kCTile positions.  compact_count: per tile, rebuild the union bitmask in
 // shared memory from the sorted selections (binary search per head) and count
-// the rows.  compact_gather: the same bitmask, an ordered block scan, then one
-// warp per row copies the K and V rows (128-bit loads/stores) from the pages.
+// the rows.  compact_gather: the same bitmask, an ordered block scan, the page
+// of every row in one round of independent loads, then the K and V rows are
+// copied in 16-byte units with eight loads in flight per lane.
 #include "common.cuh"
 #include "internal.h"
 
 namespace sfi {
 
-constexpr int kCTile = 4096;
+constexpr int kCTile = 2048;
 constexpr int kCThreads = 256;
 
 struct CompactArgs {
@@ -94,34 +95,17 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactA
   }
 }
 
-__device__ __forceinline__ void copy_row(const CompactArgs& a, int b, int g, int p, int r, int lane) {
-  const int page = a.pt[(size_t)b * a.max_pages + p / kPage];
-  const int chunks = a.D / 8;   // 16-byte chunks per row
-  const size_t dst = ((size_t)(b * a.Hkv + g) * a.p_max + r) * chunks;
-  if ((unsigned)page >= (unsigned)a.num_pages) {
-    if (lane == 0) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
-    for (int i = lane; i < 2 * chunks; i += 32) {
-      uint4* d = (i < chunks) ? a.pk : a.pv;
-      d[dst + (i % chunks)] = make_uint4(0, 0, 0, 0);
-    }
-    return;
-  }
-  const size_t src = ((size_t)(page * a.Hkv + g) * kPage + p % kPage) * chunks;
-  for (int i = lane; i < 2 * chunks; i += 32) {
-    if (i < chunks) a.pk[dst + i] = __ldg(a.kpool + src + i);
-    else a.pv[dst + i - chunks] = __ldg(a.vpool + src + i - chunks);
-  }
-}
-
 __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const CompactArgs a) {
   __shared__ uint32_t mask[kCTile];
   __shared__ int32_t rows[kCTile];
+  __shared__ int32_t pgs[kCTile];
   __shared__ int ranges[64];
   __shared__ int wtot[64];
   __shared__ int base_s, total_s;
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kCThreads / 32;
   const int t_lo = a.lo + blockIdx.x * kCTile;
   const int t_n = min(kCTile, a.lo + a.nC - t_lo);
   build_tile_mask(a, b, g, t_lo, t_n, mask, ranges);
@@ -149,7 +133,7 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   __syncthreads();
   if (threadIdx.x == 0) {
     int s = 0;
-    for (int w = 0; w < kCThreads / 32; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       const int t = wtot[w];
       wtot[32 + w] = s;
       s += t;
@@ -162,48 +146,90 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   for (int u = 0; u < kPer; ++u)
     if (j0 + u < t_n && mask[j0 + u] != 0u) rows[off++] = j0 + u;
   __syncthreads();
-  const int base = base_s, total = total_s;
+  const int base = base_s;
+  const int total = min(total_s, max(a.p_max - base, 0));
+  if (total < total_s && threadIdx.x == 0) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
+  // page of every row (independent loads), positions and head masks
   int32_t* pos = a.pos + (size_t)bg * a.p_max;
   uint32_t* hm = a.headmask + (size_t)bg * a.p_max;
-  for (int i = warp; i < total; i += kCThreads / 32) {
-    const int r = base + i;
-    if (r >= a.p_max) {
-      if (lane == 0) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
-      break;
+  for (int i = threadIdx.x; i < total; i += kCThreads) {
+    const int p = t_lo + rows[i];
+    int page = a.pt[(size_t)b * a.max_pages + p / kPage];
+    if ((unsigned)page >= (unsigned)a.num_pages) {
+      latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
+      page = -1;
     }
-    const int j = rows[i];
-    if (lane == 0) {
-      pos[r] = t_lo + j;
-      hm[r] = mask[j];
-    }
-    copy_row(a, b, g, t_lo + j, r, lane);
+    pgs[i] = page;
+    pos[base + i] = p;
+    hm[base + i] = mask[rows[i]];
   }
-  // sinks (first tile) and the tail (last tile)
+  __syncthreads();
+  // copy K and V rows: 16-byte units, eight in flight per lane
+  const int chunks = a.D / 8;
+  const int upr = 2 * chunks;
+  const int nunits = total * upr;
+  const size_t dst0 = ((size_t)bg * a.p_max + base) * chunks;
+  for (int u0 = warp * 256; u0 < nunits; u0 += kWarps * 256) {
+    uint4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int u = u0 + k * 32 + lane;
+      v[k] = make_uint4(0, 0, 0, 0);
+      if (u < nunits) {
+        const int i = u / upr, c = u - i * upr;
+        const int page = pgs[i];
+        if (page >= 0) {
+          const int p = t_lo + rows[i];
+          const size_t src = ((size_t)(page * a.Hkv + g) * kPage + p % kPage) * chunks;
+          v[k] = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int u = u0 + k * 32 + lane;
+      if (u < nunits) {
+        const int i = u / upr, c = u - i * upr;
+        if (c < chunks) a.pk[dst0 + (size_t)i * chunks + c] = v[k];
+        else a.pv[dst0 + (size_t)i * chunks + c - chunks] = v[k];
+      }
+    }
+  }
+  // sinks (first tile) and the zero tail (last tile)
   const uint32_t all = a.G >= 32 ? 0xffffffffu : ((1u << a.G) - 1u);
   if (blockIdx.x == 0) {
-    for (int i = warp; i < a.n_sink; i += kCThreads / 32) {
-      if (i >= a.p_max) break;
-      if (lane == 0) {
+    const int ns = min(a.n_sink, a.p_max);
+    for (int u = threadIdx.x; u < ns * upr; u += kCThreads) {
+      const int i = u / upr, c = u - i * upr;
+      const int page = a.pt[(size_t)b * a.max_pages + i / kPage];
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if ((unsigned)page < (unsigned)a.num_pages) {
+        const size_t src = ((size_t)(page * a.Hkv + g) * kPage + i % kPage) * chunks;
+        v = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
+      } else if (c == 0) {
+        latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
+      }
+      const size_t dst = ((size_t)bg * a.p_max + i) * chunks;
+      if (c < chunks) a.pk[dst + c] = v;
+      else a.pv[dst + c - chunks] = v;
+      if (c == 0) {
         pos[i] = i;
         hm[i] = all;
       }
-      copy_row(a, b, g, i, i, lane);
     }
   }
   if (blockIdx.x == gridDim.x - 1) {
-    const int n = min(base + total, a.p_max);
+    const int n = min(base + total_s, a.p_max);
     if (threadIdx.x == 0) a.n_rows[bg] = n;
     const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
-    const int chunks = a.D / 8;
-    for (int r = n + warp; r < pad_end; r += kCThreads / 32) {
-      if (lane == 0) {
+    for (int u = threadIdx.x; u < (pad_end - n) * upr; u += kCThreads) {
+      const int r = n + u / upr, c = u % upr;
+      const size_t dst = ((size_t)bg * a.p_max + r) * chunks;
+      if (c < chunks) a.pk[dst + c] = make_uint4(0, 0, 0, 0);
+      else a.pv[dst + c - chunks] = make_uint4(0, 0, 0, 0);
+      if (c == 0) {
         pos[r] = -1;
         hm[r] = 0u;
-      }
-      const size_t dst = ((size_t)bg * a.p_max + r) * chunks;
-      for (int i = lane; i < 2 * chunks; i += 32) {
-        uint4* d = (i < chunks) ? a.pk : a.pv;
-        d[dst + (i % chunks)] = make_uint4(0, 0, 0, 0);
       }
     }
   }

@@ -171,6 +171,8 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   const CtxLayout l = ctx_layout(c->s, c->p);
   if (bytes < l.total) return SFI_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
+  // the first 256 bytes hold the attention kernels' work counter: zero it once
+  if (cudaMemset(w, 0, 256) != cudaSuccess) return SFI_ERR_CUDA;
   c->ws = w;
   c->ws_bytes = bytes;
   c->part = reinterpret_cast<float*>(w + l.part_off);
@@ -223,7 +225,8 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   if (!c->cur_slow) {
     cudaEvent_t b, e;
     timing_events(c, 0, &b, &e);
-    return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, c->part, c->part_bytes, main, b, e);
+    return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, reinterpret_cast<int*>(c->ws), c->part,
+                         c->part_bytes, main, b, e);
   }
 
   const int buf = layer & 1;
@@ -237,7 +240,8 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   {
     cudaEvent_t b, e;
     timing_events(c, 1, &b, &e);
-    SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, c->part, c->part_bytes, main, b, e));
+    SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
+                           main, b, e));
   }
   SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
   cudaStream_t side = c->side;
@@ -245,10 +249,11 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   const int nC = L - p.n_recent - p.n_sink;
   const int K = budget_k(p, L);
   if (K < 1) return SFI_ERR_SHAPE;
-  SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, nC,
+  const int ld_s = (nC + 3) / 4 * 4;
+  SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
                             c->stats, side));
   SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, nC, K, p.n_sink, c->sel_idx, c->sel_ld, side));
+  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, c->sel_idx, c->sel_ld, side));
   SFI_TRY(run_compact(s, p, *kv, c->sel_idx, c->sel_ld, K, *packed, c->tile_counts, c->tc_bytes, L,
                       side));
   SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));

@@ -44,16 +44,17 @@ struct WsLayout {
 WsLayout ws_layout(const sfi_shape& s, const sfi_params& p);
 
 int dense_chunk_tiles(const sfi_shape& s, int L);
-int fast_chunks(const sfi_shape& s, int p_max, int n_recent);
+int dense_chunks_bound(const sfi_shape& s);
+int fast_chunks(const sfi_shape& s, int p_max, int n_recent, int k_est);
 size_t attn_part_bytes(int n_items, int G, int D);
 int packed_rows_capacity(const sfi_shape& s, const sfi_params& p);
 int budget_k(const sfi_params& p, int L);   // -1 if |C| < 1
 
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
-                          float* out, const sfi_dense_extras* ex, float* part, size_t part_bytes,
-                          cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
+                          float* out, const sfi_dense_extras* ex, int* ctr, float* part,
+                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
-                         const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse,
+                         const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
                          cudaEvent_t ev_end);
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld,
@@ -74,5 +75,6 @@ sfi_status run_compact(const sfi_shape& s, const sfi_params& p, const sfi_paged_
                        int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st);
 int compact_tiles(int nC);
 int score_tile(int G);
+int stat_chunks(int nC);
 
 }  // namespace sfi

@@ -12,8 +12,9 @@
 //   exclusivity l'' = l' - alpha_cross * [h != argmax_h' l'_{h',j}]
 //   top-K      K largest l'' per query head, ties to the lower position.
 //
-// Kernels: select_stats (per (b, kv head): nbar and 1 / sum kappa pi, fp64
-// sums), select_scores (one CTA per (b, kv group, candidate tile) holding all
+// Kernels: stats_norm / stats_prior (per (b, kv head) and chunk of C: fp64
+// partial sums of the norms and of kappa pi; every consumer reduces the
+// partials in the same fixed order), select_scores (one CTA per (b, kv group, candidate tile) holding all
 // G heads plus a halo of w on each side in shared memory, so soft-NMS and the
 // cross-head owner need no second pass over memory), topk_kernel (one CTA
 // per row: 3-pass MSB radix select on order-preserving uint32 keys, then one
@@ -25,7 +26,8 @@
 
 namespace sfi {
 
-constexpr int kStatThreads = 1024;
+constexpr int kStatThreads = 256;
+constexpr int kStatChunk = 4096;
 
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
 #pragma unroll
@@ -45,28 +47,61 @@ __device__ __forceinline__ double block_sum_d(double v, double* red) {
   return red[0];
 }
 
+// Sum of the per-chunk partials part[k * 2 + which], k < nch, by warp 0 in a
+// fixed order (every CTA that needs it gets the bit-identical value).
+__device__ __forceinline__ double reduce_parts(const double* part, int nch, int which, double* bcast) {
+  if (threadIdx.x < 32) {
+    double t = 0.0;
+    for (int k = threadIdx.x; k < nch; k += 32) t += part[k * 2 + which];
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) t += __shfl_xor_sync(0xffffffffu, t, sh);
+    if (threadIdx.x == 0) *bcast = t;
+  }
+  __syncthreads();
+  const double r = *bcast;
+  __syncthreads();
+  return r;
+}
+
 __device__ __forceinline__ float kappa_of(float nbar, float n) {
   return n > 0.f ? fminf(1.f, nbar / n) : 1.f;
 }
 
 __device__ __forceinline__ float pi_of(int L, int j) { return logf((float)(1 + L - j)); }
 
-// stats[bg] = {nbar, 1 / sum_C kappa pi}
-__global__ void __launch_bounds__(kStatThreads) select_stats_kernel(int L, int lo, int hi,
-                                                                    const float* __restrict__ norms,
-                                                                    int64_t norm_ld, float2* stats) {
+__device__ __forceinline__ float nbar_of(double sum_norms, int nC) { return (float)(sum_norms / (double)nC); }
+
+// part[bg][chunk][0] = sum of key norms over the chunk of C
+__global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC, const float* __restrict__ norms,
+                                                                  int64_t norm_ld, double* part, int nch) {
   __shared__ double red[32];
-  const int bg = blockIdx.x;
+  const int bg = blockIdx.y;
+  const float* n = norms + (size_t)bg * norm_ld + lo;
+  const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
+  double sacc = 0.0;
+  for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) sacc += (double)n[c];
+  const double t = block_sum_d(sacc, red);
+  if (threadIdx.x == 0) part[((size_t)bg * nch + blockIdx.x) * 2] = t;
+}
+
+// part[bg][chunk][1] = sum of kappa * pi over the chunk of C
+__global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
+                                                                   const float* __restrict__ norms,
+                                                                   int64_t norm_ld, double* part, int nch) {
+  __shared__ double red[32];
+  __shared__ double bc;
+  const int bg = blockIdx.y;
+  double* pbg = part + (size_t)bg * nch * 2;
+  const float nbar = nbar_of(reduce_parts(pbg, nch, 0, &bc), nC);
   const float* n = norms + (size_t)bg * norm_ld;
-  double s = 0.0;
-  for (int j = lo + threadIdx.x; j < hi; j += blockDim.x) s += (double)n[j];
-  const double tot = block_sum_d(s, red);
-  const float nbar = (float)(tot / (double)(hi - lo));
+  const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double z = 0.0;
-  for (int j = lo + threadIdx.x; j < hi; j += blockDim.x)
+  for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
+    const int j = lo + c;
     z += (double)(kappa_of(nbar, n[j]) * pi_of(L, j));
-  const double ztot = block_sum_d(z, red);
-  if (threadIdx.x == 0) stats[bg] = make_float2(nbar, (float)(1.0 / ztot));
+  }
+  const double t = block_sum_d(z, red);
+  if (threadIdx.x == 0) pbg[blockIdx.x * 2 + 1] = t;
 }
 
 struct ScoreArgs {
@@ -77,7 +112,8 @@ struct ScoreArgs {
   const float* lse_cand;
   const float* norms;
   int64_t norm_ld;
-  const float2* stats;
+  const double* stat_part;   // [B*Hkv][nch][2]
+  int nch;
   float* scores;
   int64_t ld_s;
 };
@@ -92,7 +128,10 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
   const int c0 = blockIdx.x * a.tile;
   const int tile_n = min(a.tile, a.nC - c0);
-  const float2 st = a.stats[bg];
+  __shared__ double bc;
+  const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
+  const float nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
+  const float inv_z = (float)(1.0 / reduce_parts(pbg, a.nch, 1, &bc));
   const float* nrm = a.norms + (size_t)bg * a.norm_ld;
 
   // prior over the haloed tile
@@ -101,7 +140,7 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
     float r = 0.f;
     if (c >= 0 && c < a.nC) {
       const int j = a.lo + c;
-      r = kappa_of(st.x, nrm[j]) * pi_of(a.L, j) * st.y;
+      r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * inv_z;
     }
     rr[k] = r;
   }
@@ -219,6 +258,50 @@ __device__ __forceinline__ int block_prefix_excl(int v, int* wtot, int* total) {
   return r;
 }
 
+// Keys of one block-wide slab of kSlab = 16 * kTopkThreads scores starting at
+// `base`: coalesced loads (float4 when the row allows it); element u of a
+// thread sits at index slab_index(base, u).  Padding keys are 0, below the
+// image of every float but a negative NaN, and are never counted.
+constexpr int kPerThread = 16;
+constexpr int kSlab = kPerThread * kTopkThreads;
+
+template <bool VEC>
+__device__ __forceinline__ int slab_index(int base, int u) {
+  return VEC ? base + (u >> 2) * (4 * kTopkThreads) + threadIdx.x * 4 + (u & 3)
+             : base + u * kTopkThreads + threadIdx.x;
+}
+
+template <bool VEC>
+__device__ __forceinline__ void load_slab(const float* row, int n, int base, uint32_t (&k)[kPerThread]) {
+  if (VEC) {
+#pragma unroll
+    for (int v = 0; v < kPerThread / 4; ++v) {
+      const int j = base + v * (4 * kTopkThreads) + threadIdx.x * 4;
+      if (j + 4 <= n) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(row + j));
+        k[4 * v + 0] = float_key(f.x);
+        k[4 * v + 1] = float_key(f.y);
+        k[4 * v + 2] = float_key(f.z);
+        k[4 * v + 3] = float_key(f.w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) k[4 * v + e] = (j + e < n) ? float_key(__ldg(row + j + e)) : 0u;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int j = base + u * kTopkThreads + threadIdx.x;
+      k[u] = (j < n) ? float_key(__ldg(row + j)) : 0u;
+    }
+  }
+}
+
+// One CTA per row.  Keys are order-preserving uint32 images of the scores.
+// Three MSB radix passes (11, 11, 10 bits) find the key T of the K-th largest
+// and how many keys equal to T to keep (the lowest positions first); one
+// ordered pass writes the positions ascending.
+template <bool VEC>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(int n, const float* __restrict__ scores,
                                                             int64_t ld_s, int K, int offset,
                                                             int32_t* __restrict__ idx, int64_t ld_i) {
@@ -238,19 +321,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(int n, const float* 
     const uint32_t dmask = (1u << widths[pass]) - 1u;
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < n; base += blockDim.x) {
-      const int j = base + threadIdx.x;
-      bool in = false;
-      uint32_t bin = 0;
-      if (j < n) {
-        const uint32_t key = float_key(row[j]);
-        in = (key & pmask) == prefix;
-        bin = (key >> sh) & dmask;
-      }
-      const unsigned act = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const unsigned peers = __match_any_sync(act, bin);
-        if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+    for (int base = 0; base < n; base += kSlab) {
+      uint32_t k[kPerThread];
+      load_slab<VEC>(row, n, base, k);
+#pragma unroll
+      for (int u = 0; u < kPerThread; ++u) {
+        const bool in = slab_index<VEC>(base, u) < n && (k[u] & pmask) == prefix;
+        const uint32_t bin = (k[u] >> sh) & dmask;
+        const unsigned act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const unsigned peers = __match_any_sync(act, bin);
+          if ((int)(__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+        }
       }
     }
     __syncthreads();
@@ -272,42 +354,43 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(int n, const float* 
     k_rem -= sel_above;
     __syncthreads();
   }
-  const uint32_t T = prefix;   // key of the K-th largest; take k_rem of the ties
-  // ordered output pass
+  const uint32_t T = prefix;   // key of the K-th largest; keep k_rem of the ties
+  // ordered pass: 4 consecutive elements per thread per round, rounds in order
   int gt_run = 0, eq_run = 0;
-  constexpr int kPerThread = 4;
-  for (int base = 0; base < n; base += blockDim.x * kPerThread) {
-    const int j0 = base + threadIdx.x * kPerThread;
-    int ngt = 0, neq = 0;
-    uint32_t kinds = 0;   // 2 bits per element: 1 = gt, 2 = eq
+  for (int base = 0; base < n; base += 4 * kTopkThreads) {
+    const int j0 = base + threadIdx.x * 4;
+    uint32_t k[4];
+    if (VEC && j0 + 4 <= n) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(row + j0));
+      k[0] = float_key(f.x);
+      k[1] = float_key(f.y);
+      k[2] = float_key(f.z);
+      k[3] = float_key(f.w);
+    } else {
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-      const int j = j0 + u;
-      if (j < n) {
-        const uint32_t key = float_key(row[j]);
-        if (key > T) {
-          ++ngt;
-          kinds |= 1u << (2 * u);
-        } else if (key == T) {
-          ++neq;
-          kinds |= 2u << (2 * u);
-        }
+      for (int e = 0; e < 4; ++e) k[e] = (j0 + e < n) ? float_key(__ldg(row + j0 + e)) : 0u;
+    }
+    int ngt = 0, neq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j0 + e < n) {
+        ngt += k[e] > T;
+        neq += k[e] == T;
       }
     }
-    const int packed = (neq << 16) | ngt;
-    const int ex = block_prefix_excl(packed, wtot, &total);
+    const int ex = block_prefix_excl((neq << 16) | ngt, wtot, &total);
     int gt_before = gt_run + (ex & 0xffff);
     int eq_before = eq_run + (ex >> 16);
 #pragma unroll
-    for (int u = 0; u < kPerThread; ++u) {
-      const uint32_t kd = (kinds >> (2 * u)) & 3u;
-      if (kd == 1u) {
+    for (int e = 0; e < 4; ++e) {
+      if (j0 + e >= n) break;
+      if (k[e] > T) {
         const int at = gt_before + min(eq_before, k_rem);
-        if (at < K) out[at] = offset + j0 + u;
+        if (at < K) out[at] = offset + j0 + e;
         ++gt_before;
-      } else if (kd == 2u) {
+      } else if (k[e] == T) {
         const int at = gt_before + eq_before;
-        if (eq_before < k_rem && at < K) out[at] = offset + j0 + u;
+        if (eq_before < k_rem && at < K) out[at] = offset + j0 + e;
         ++eq_before;
       }
     }
@@ -324,15 +407,20 @@ size_t score_smem(int G, int tile, int w) {
   return ((size_t)G * (tile + 2 * w) + (size_t)G * tile + (tile + 2 * w)) * sizeof(float);
 }
 
+int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }
+
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws, cudaStream_t st) {
   const int G = s.Hq / s.Hkv;
   const int lo = p.n_sink, hi = L - p.n_recent;
   const int nC = hi - lo;
-  float2* stats = reinterpret_cast<float2*>(stat_ws);
+  double* part = reinterpret_cast<double*>(stat_ws);
+  const int nch = stat_chunks(nC);
   const int64_t norm_ld = (int64_t)s.max_pages * kPage;
-  select_stats_kernel<<<s.B * s.Hkv, kStatThreads, 0, st>>>(L, lo, hi, kv.key_norms, norm_ld, stats);
+  dim3 sgrid(nch, s.B * s.Hkv);
+  stats_norm_kernel<<<sgrid, kStatThreads, 0, st>>>(lo, nC, kv.key_norms, norm_ld, part, nch);
+  stats_prior_kernel<<<sgrid, kStatThreads, 0, st>>>(L, lo, nC, kv.key_norms, norm_ld, part, nch);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
@@ -343,7 +431,8 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;
-  a.norms = kv.key_norms; a.norm_ld = norm_ld; a.stats = stats;
+  a.norms = kv.key_norms; a.norm_ld = norm_ld;
+  a.stat_part = part; a.nch = nch;
   a.scores = scores; a.ld_s = ld_s;
   const size_t smem = score_smem(G, a.tile, a.w);
   static DeviceOnce attr;
@@ -359,7 +448,9 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset,
                     int32_t* idx, int64_t ld_i, cudaStream_t st) {
   if (rows <= 0) return SFI_OK;
-  topk_kernel<<<rows, kTopkThreads, 0, st>>>(n, scores, ld_s, K, offset, idx, ld_i);
+  const bool vec = (ld_s % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
+  if (vec) topk_kernel<true><<<rows, kTopkThreads, 0, st>>>(n, scores, ld_s, K, offset, idx, ld_i);
+  else topk_kernel<false><<<rows, kTopkThreads, 0, st>>>(n, scores, ld_s, K, offset, idx, ld_i);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

@@ -27,7 +27,7 @@ def _cfg(B, Hq, Hkv, D, L, **kw):
 def _setup(cfg):
     li = W.make_layer(cfg, 0, "cpu")
     layer = alloc_layer(cfg, li, DEV)
-    ws = torch.empty(S.sfi_workspace_size(shape_of(cfg), params_of(cfg)), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(S.sfi_workspace_size(shape_of(cfg), params_of(cfg)), dtype=torch.uint8, device=DEV)
     return li, layer, ws
 
 
