@@ -66,6 +66,13 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   w.cmp_off = off;
   w.cmp_bytes = align_up((size_t)bh * compact_tiles((int)nC) * sizeof(int32_t), 256);
   off += w.cmp_bytes;
+  w.bits_ld = (nC + 31) / 32;
+  w.bits_off = off;
+  w.bits_bytes = align_up((size_t)s.B * s.Hq * w.bits_ld * sizeof(uint32_t), 256);
+  off += w.bits_bytes;
+  w.mm_off = off;
+  w.mm_bytes = align_up((size_t)s.B * s.Hq * 2 * sizeof(uint32_t), 256);
+  off += w.mm_bytes;
   w.total = off;
   return w;
 }
@@ -256,17 +263,20 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
   if (!kv || !kv->key_norms || !logits || !lse_cand || !scores) return SFI_ERR_INVALID_ARG;
   if (ld < L) return SFI_ERR_SHAPE;
   const WsLayout w = ws_layout(*shape, *params);
-  if (!ws || ws_bytes < w.stat_off + w.stat_bytes) return SFI_ERR_WORKSPACE;
+  if (!ws || ws_bytes < w.total) return SFI_ERR_WORKSPACE;
   const int nC = L - params->n_recent - params->n_sink;
   return run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, nC,
-                           static_cast<char*>(ws) + w.stat_off, (cudaStream_t)stream);
+                           static_cast<char*>(ws) + w.stat_off,
+                           reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.mm_off),
+                           (cudaStream_t)stream);
 }
 
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
                     int32_t offset, int32_t* idx, int64_t ld_i, sfi_stream stream) {
   if (!scores || !idx) return SFI_ERR_INVALID_ARG;
   if (rows < 0 || n < 1 || K < 1 || K > n || ld_s < n || ld_i < K) return SFI_ERR_SHAPE;
-  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, (cudaStream_t)stream);
+  if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
+  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, nullptr, 0, nullptr, (cudaStream_t)stream);
 }
 
 sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
@@ -287,9 +297,12 @@ sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sf
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + w.sel_off);
   const int ld_s = (nC + 3) / 4 * 4;
   cudaStream_t st = (cudaStream_t)stream;
+  uint32_t* mm = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.mm_off);
+  if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
   SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s,
-                            static_cast<char*>(ws) + w.stat_off, st));
-  SFI_TRY(run_topk(shape->B * shape->Hq, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, st));
+                            static_cast<char*>(ws) + w.stat_off, mm, st));
+  SFI_TRY(run_topk(shape->B * shape->Hq, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0,
+                   mm, st));
   if (K_out) *K_out = K;
   return SFI_OK;
 }
@@ -306,10 +319,12 @@ sfi_status sfi_compact(const sfi_shape* shape, const sfi_params* params, const s
   const int nC = L - params->n_recent - params->n_sink;
   if (K < 1 || K > nC || sel_ld < K) return SFI_ERR_SHAPE;
   const WsLayout w = ws_layout(*shape, *params);
-  if (!ws || ws_bytes < w.cmp_off + w.cmp_bytes) return SFI_ERR_WORKSPACE;
-  return run_compact(*shape, *params, *kv, sel_idx, sel_ld, K, *packed,
-                     reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.cmp_off), w.cmp_bytes, L,
-                     (cudaStream_t)stream);
+  if (!ws || ws_bytes < w.total) return SFI_ERR_WORKSPACE;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.bits_off);
+  cudaStream_t st = (cudaStream_t)stream;
+  SFI_TRY(run_idx_to_bits(*shape, *params, *kv, L, sel_idx, sel_ld, K, bits, w.bits_ld, st));
+  return run_compact_bits(*shape, *params, *kv, bits, w.bits_ld, *packed,
+                          reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.cmp_off), w.cmp_bytes, L, st);
 }
 
 sfi_status sfi_poll_error(const sfi_paged_kv* kv, int32_t* code) {

@@ -155,11 +155,17 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile_base, int row, int ci) {
   return tile_base + (ci >> 3) * kBoxBytes + row * 128 + ((((ci & 7) ^ (row & 7))) << 4);
 }
 
+// Tensor maps of one launch.  k, v: the page pools, one box = one 16-row
+// tile of one (page, KV head).  pk, pv: the packed buffers, one box = one
+// tile; pk8, pv8: the packed buffers viewed as [tiles][column block][16
+// rows][64 columns], one box = a whole stage of consecutive tiles.
+struct Maps {
+  CUtensorMap k, v, pk, pv, pk8, pv8;
+};
+
 template <int D, int NT, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                const __grid_constant__ CUtensorMap tpk, const __grid_constant__ CUtensorMap tpv,
-                const AttnArgs a) {
+    attn_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   using S = Smem<D, NT>;
   using P = Plan<D, NT>;
   constexpr int kStages = S::kStages;
@@ -194,11 +200,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // ------------------------------------------------------------ producer warp
   if (warp == kConsumerWarps) {
     if (lane == 0) {
-      prefetch_tensormap(&tk);
-      prefetch_tensormap(&tv);
+      prefetch_tensormap(&maps.k);
+      prefetch_tensormap(&maps.v);
       if (MODE == kFast) {
-        prefetch_tensormap(&tpk);
-        prefetch_tensormap(&tpv);
+        prefetch_tensormap(&maps.pk);
+        prefetch_tensormap(&maps.pv);
+        prefetch_tensormap(&maps.pk8);
+        prefetch_tensormap(&maps.pv8);
       }
     }
     const int BH = a.B * a.Hkv;
@@ -282,6 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               uint8_t* sv = sk + P::kKBytes;
               if (st == 0) bytes += G * D * 2;
               int ys[kTPS];
+              int n_pk = 0;   // packed tiles lead the stage
               for (int i = 0; i < nt; ++i) {
                 const int t = t0 + i;
                 int kind, y, pos0;
@@ -290,6 +299,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   pos0 = t * kPage;
                   y = it.bg * a.p_max + pos0;
                   bytes += 2 * P::kTileBytes + 64;
+                  ++n_pk;
                 } else {
                   const int pg = item_page(it, t);
                   const int page = ptbuf[pg - p_lo];
@@ -313,16 +323,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               if (st == 0)
                 bulk_load(sq + slot * P::kQBytes, a.q + ((size_t)it.b * a.Hq + it.g * G) * D, G * D * 2,
                           &full[slot]);
-              for (int i = 0; i < nt; ++i) {
+              int i0 = 0;
+              if (MODE == kFast && n_pk > 0) {
+                // head masks of the stage's packed tiles: one copy
+                bulk_load(smask + slot * kTPS * 16, a.headmask + (size_t)it.bg * a.p_max + m.pos0[0],
+                          n_pk * 64, &full[slot]);
+                if (n_pk == kTPS) {
+                  // a whole stage of consecutive packed tiles: one box each for K and V
+                  const int tile0 = ys[0] / kPage;
+                  tma_load_4d(sk, &maps.pk8, 0, 0, 0, tile0, &full[slot], policy);
+                  tma_load_4d(sv, &maps.pv8, 0, 0, 0, tile0, &full[slot], policy);
+                  i0 = nt;
+                }
+              }
+              for (int i = i0; i < nt; ++i) {
                 const int kind = (kinds >> (2 * i)) & 3;
                 if (kind == 2) continue;
-                const CUtensorMap* mk = kind == 1 ? &tpk : &tk;
-                const CUtensorMap* mv = kind == 1 ? &tpv : &tv;
+                const CUtensorMap* mk = kind == 1 ? &maps.pk : &maps.k;
+                const CUtensorMap* mv = kind == 1 ? &maps.pv : &maps.v;
                 tma_load_3d(sk + i * P::kTileBytes, mk, 0, ys[i], 0, &full[slot], policy);
                 tma_load_3d(sv + i * P::kTileBytes, mv, 0, ys[i], 0, &full[slot], policy);
-                if (kind == 1)
-                  bulk_load(smask + (slot * kTPS + i) * 16,
-                            a.headmask + (size_t)it.bg * a.p_max + m.pos0[i], 64, &full[slot]);
               }
             }
           } else {
@@ -618,10 +638,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // Merge the partials of every (b, query head): one CTA of kCombWarps warps
-// each.  Pass 1: the largest m.  Pass 2: warp w folds partials w, w + 8, ...
-// with four partials' loads in flight per step; the warps' sums meet in
-// shared memory.
-constexpr int kCombWarps = 8;
+// each.  Pass 1: the largest m.  Pass 2: warp w folds partials w,
+// w + kCombWarps, ... with eight partials' loads in flight per step; the
+// warps' sums meet in shared memory.
+constexpr int kCombWarps = 16;
 
 template <int D>
 __global__ void __launch_bounds__(kCombWarps * 32)
@@ -658,11 +678,12 @@ __global__ void __launch_bounds__(kCombWarps * 32)
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   float l = 0.f, lc = 0.f;
-  for (int c0 = warp; c0 < n; c0 += 4 * kCombWarps) {
-    float st[4][3];
-    float ov[4][kPer];
+  constexpr int kIn = 8;   // partials in flight per warp
+  for (int c0 = warp; c0 < n; c0 += kIn * kCombWarps) {
+    float st[kIn][3];
+    float ov[kIn][kPer];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kIn; ++u) {
       const int c = c0 + u * kCombWarps;
       if (c < n) {
         const float* pc = base + c * stride;
@@ -679,7 +700,7 @@ __global__ void __launch_bounds__(kCombWarps * 32)
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kIn; ++u) {
       const float w = exp2f(st[u][0] - mref);
       l += w * st[u][1];
       lc += w * st[u][2];
@@ -759,9 +780,24 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int D) {
   return r == CUDA_SUCCESS;
 }
 
+// rows (a multiple of 16) x D bf16 matrix viewed as [tiles][D/64][16][64]:
+// one box = `nt` consecutive 16-row tiles, landing exactly as `nt`
+// single-tile boxes would, one after another.
+bool make_map_tiles(CUtensorMap* m, const void* base, uint64_t rows, int D, int nt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, 16, (cuuint64_t)(D / 64), (cuuint64_t)(rows / 16)};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, 128, (cuuint64_t)16 * D * 2};
+  cuuint32_t box[4] = {64, 16, (cuuint32_t)(D / 64), (cuuint32_t)nt};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int NT, int MODE>
-sfi_status launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tpk,
-                         const CUtensorMap& tpv, const AttnArgs& a, cudaStream_t st) {
+sfi_status launch_attn_t(const Maps& maps, const AttnArgs& a, cudaStream_t st) {
   using S = Smem<D, NT>;
   auto kern = attn_kernel<D, NT, MODE>;
   static DeviceOnce attr;   // per instantiation and device
@@ -769,21 +805,21 @@ sfi_status launch_attn_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUt
       !attr.mark(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal)))
     return SFI_ERR_CUDA;
   const int grid = std::min(a.n_items, num_sms());
-  kern<<<grid, kAttnThreads, S::kTotal, st>>>(tk, tv, tpk, tpv, a);
+  kern<<<grid, kAttnThreads, S::kTotal, st>>>(maps, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 template <int MODE>
-sfi_status launch_attn(int D, int G, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tpk, const CUtensorMap& tpv, const AttnArgs& a,
-                       cudaStream_t st) {
+sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaStream_t st) {
   if (D == 128) {
-    if (G <= 8) return launch_attn_t<128, 1, MODE>(tk, tv, tpk, tpv, a, st);
-    return launch_attn_t<128, 2, MODE>(tk, tv, tpk, tpv, a, st);
+    if (G <= 8) return launch_attn_t<128, 1, MODE>(maps, a, st);
+    return launch_attn_t<128, 2, MODE>(maps, a, st);
   }
-  if (G <= 8) return launch_attn_t<64, 1, MODE>(tk, tv, tpk, tpv, a, st);
-  return launch_attn_t<64, 2, MODE>(tk, tv, tpk, tpv, a, st);
+  if (G <= 8) return launch_attn_t<64, 1, MODE>(maps, a, st);
+  return launch_attn_t<64, 2, MODE>(maps, a, st);
 }
+
+int stage_tiles(int D, int G) { return (G <= 8) ? 8 : 4; }
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int* err,
@@ -839,9 +875,11 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
   const int G = s.Hq / s.Hkv;
-  CUtensorMap tk, tv;
+  Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
-  if (!make_map(&tk, kv.k_pool, rows, s.D) || !make_map(&tv, kv.v_pool, rows, s.D)) return SFI_ERR_CUDA;
+  if (!make_map(&maps.k, kv.k_pool, rows, s.D) || !make_map(&maps.v, kv.v_pool, rows, s.D)) return SFI_ERR_CUDA;
+  maps.pk = maps.pk8 = maps.k;
+  maps.pv = maps.pv8 = maps.v;
   AttnArgs a{};
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G; a.L = L;
   a.num_pages = s.num_pages; a.max_pages = s.max_pages;
@@ -868,8 +906,8 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   }
   if (ev_begin) cudaEventRecord(ev_begin, st);
   sfi_status r;
-  if (extras) r = launch_attn<kDenseExtras>(s.D, G, tk, tv, tk, tv, a, st);
-  else r = launch_attn<kDense>(s.D, G, tk, tv, tk, tv, a, st);
+  if (extras) r = launch_attn<kDenseExtras>(s.D, G, maps, a, st);
+  else r = launch_attn<kDense>(s.D, G, maps, a, st);
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
@@ -890,11 +928,13 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
                          cudaEvent_t ev_end) {
   const int G = s.Hq / s.Hkv;
   if ((long)s.B * s.Hkv > kMaxBH) return SFI_ERR_UNSUPPORTED;
-  CUtensorMap tk, tv, tpk, tpv;
+  Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
   const uint64_t prows = (uint64_t)s.B * s.Hkv * pk.p_max;
-  if (!make_map(&tk, kv.k_pool, rows, s.D) || !make_map(&tv, kv.v_pool, rows, s.D) ||
-      !make_map(&tpk, pk.k, prows, s.D) || !make_map(&tpv, pk.v, prows, s.D))
+  const int nts = stage_tiles(s.D, G);
+  if (!make_map(&maps.k, kv.k_pool, rows, s.D) || !make_map(&maps.v, kv.v_pool, rows, s.D) ||
+      !make_map(&maps.pk, pk.k, prows, s.D) || !make_map(&maps.pv, pk.v, prows, s.D) ||
+      !make_map_tiles(&maps.pk8, pk.k, prows, s.D, nts) || !make_map_tiles(&maps.pv8, pk.v, prows, s.D, nts))
     return SFI_ERR_CUDA;
   AttnArgs a{};
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G; a.L = L;
@@ -914,7 +954,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   a.rec_lo = std::max(L - p.n_recent, 0);
   a.err = kv.err;
   if (ev_begin) cudaEventRecord(ev_begin, st);
-  sfi_status r = launch_attn<kFast>(s.D, G, tk, tv, tpk, tpv, a, st);
+  sfi_status r = launch_attn<kFast>(s.D, G, maps, a, st);
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
   return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, kv.err, ctr,

@@ -6,24 +6,27 @@
 // Per (sequence, KV head): rows = sink tokens [0, n_sink), then the union of
 // the group's per-head selections in ascending position order, each with a
 // bitmask of the query heads that chose it (sinks: all heads), then zero rows
-// up to the next multiple of 16.  The candidate range is cut into tiles of
-// kCTile positions.  compact_count: per tile, rebuild the union bitmask in
-// shared memory from the sorted selections (binary search per head) and count
-// the rows.  compact_gather: the same bitmask, an ordered block scan, the page
-// of every row in one round of independent loads, then the K and V rows are
-// copied in 16-byte units with eight loads in flight per lane.
+// up to the next multiple of 16.  Selections arrive as one bitmap per query
+// head over the candidate range (bit c = position n_sink + c), as the top-K
+// kernel writes them.  A tile is 256 bitmap words (8192 positions); each
+// thread owns one word: the OR of the group's words is the union, its
+// popcount the row count.  compact_count writes the per-tile counts;
+// compact_gather scans them, writes positions and head masks, looks up every
+// row's page in one round of independent loads, then copies the K and V rows
+// in 16-byte units with eight loads in flight per lane.
 #include "common.cuh"
 #include "internal.h"
 
 namespace sfi {
 
-constexpr int kCTile = 2048;
+constexpr int kCWords = 256;
 constexpr int kCThreads = 256;
 
 struct CompactArgs {
-  int Hkv, G, Hq, D, n_sink, lo, nC, K, sel_ld, n_tiles;
+  int Hkv, G, Hq, D, n_sink, lo, nC, nw, n_tiles;
   int max_pages, num_pages, p_max;
-  const int32_t* sel;
+  const uint32_t* bits;   // [B*Hq][ld_b]
+  int64_t ld_b;
   const int32_t* pt;
   const uint4* kpool;
   const uint4* vpool;
@@ -32,58 +35,29 @@ struct CompactArgs {
   int32_t* pos;
   uint32_t* headmask;
   int32_t* n_rows;
-  int32_t* tile_counts;   // [B*Hkv, n_tiles]
+  int32_t* tile_counts;   // [B*Hkv][n_tiles]
   int* err;
 };
 
-__device__ int lower_bound_i(const int32_t* a, int n, int v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] < v) lo = mid + 1;
-    else hi = mid;
+template <int GM>
+__device__ __forceinline__ uint32_t union_word(const CompactArgs& a, int b, int g, int w, uint32_t (&hw)[GM]) {
+  uint32_t u = 0u;
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    hw[h] = (h < a.G && w < a.nw) ? __ldg(a.bits + ((size_t)b * a.Hq + g * a.G + h) * a.ld_b + w) : 0u;
+    u |= hw[h];
   }
-  return lo;
+  return u;
 }
 
-// Bitmask of the tile's candidate positions in shared memory.
-__device__ void build_tile_mask(const CompactArgs& a, int b, int g, int t_lo, int t_n,
-                                uint32_t* mask, int* ranges) {
-  for (int i = threadIdx.x; i < kCTile; i += blockDim.x) mask[i] = 0u;
-  if (threadIdx.x < a.G) {
-    const int32_t* sh = a.sel + ((size_t)b * a.Hq + g * a.G + threadIdx.x) * a.sel_ld;
-    ranges[2 * threadIdx.x] = lower_bound_i(sh, a.K, t_lo);
-    ranges[2 * threadIdx.x + 1] = lower_bound_i(sh, a.K, t_lo + t_n);
-  }
-  __syncthreads();
-  for (int h = 0; h < a.G; ++h) {
-    const int32_t* sh = a.sel + ((size_t)b * a.Hq + g * a.G + h) * a.sel_ld;
-    const int r0 = ranges[2 * h], r1 = ranges[2 * h + 1];
-    for (int i = r0 + threadIdx.x; i < r1; i += blockDim.x) {
-      const int p = sh[i] - t_lo;
-      if ((unsigned)p < (unsigned)t_n) atomicOr(&mask[p], 1u << h);
-    }
-  }
-  __syncthreads();
-}
-
+template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactArgs a) {
-  __shared__ uint32_t mask[kCTile];
-  __shared__ int ranges[64];
   __shared__ int wsum[kCThreads / 32];
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
-  const int t_lo = a.lo + blockIdx.x * kCTile;
-  const int t_n = min(kCTile, a.lo + a.nC - t_lo);
-  // selections must lie in the candidate range: count the ones that do not
-  if (blockIdx.x == 0 && threadIdx.x < a.G) {
-    const int32_t* sh = a.sel + ((size_t)b * a.Hq + g * a.G + threadIdx.x) * a.sel_ld;
-    if (a.K > 0 && (sh[0] < a.lo || sh[a.K - 1] >= a.lo + a.nC))
-      latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactIdx);
-  }
-  build_tile_mask(a, b, g, t_lo, t_n, mask, ranges);
-  int c = 0;
-  for (int i = threadIdx.x; i < t_n; i += blockDim.x) c += mask[i] != 0u;
+  uint32_t hw[GM];
+  const uint32_t u = union_word<GM>(a, b, g, blockIdx.x * kCWords + threadIdx.x, hw);
+  int c = __popc(u);
 #pragma unroll
   for (int sh = 16; sh >= 1; sh >>= 1) c += __shfl_xor_sync(0xffffffffu, c, sh);
   if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = c;
@@ -95,20 +69,20 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactA
   }
 }
 
+template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const CompactArgs a) {
-  __shared__ uint32_t mask[kCTile];
-  __shared__ int32_t rows[kCTile];
-  __shared__ int32_t pgs[kCTile];
-  __shared__ int ranges[64];
-  __shared__ int wtot[64];
+  extern __shared__ int32_t csm[];
+  int32_t* rp = csm;                       // position of each row of the tile
+  int32_t* rg = csm + kCWords * 32;        // its page (-1: bad page-table entry)
+  __shared__ int wtot[kCThreads / 32 + 1];
   __shared__ int base_s, total_s;
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kWarps = kCThreads / 32;
-  const int t_lo = a.lo + blockIdx.x * kCTile;
-  const int t_n = min(kCTile, a.lo + a.nC - t_lo);
-  build_tile_mask(a, b, g, t_lo, t_n, mask, ranges);
+  const int w = blockIdx.x * kCWords + threadIdx.x;
+  uint32_t hw[GM];
+  const uint32_t u = union_word<GM>(a, b, g, w, hw);
   // rows before this tile
   if (warp == 0) {
     int s = 0;
@@ -117,12 +91,8 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
     for (int sh = 16; sh >= 1; sh >>= 1) s += __shfl_xor_sync(0xffffffffu, s, sh);
     if (lane == 0) base_s = a.n_sink + s;
   }
-  // ordered compaction of the tile: each thread owns kCTile / kCThreads consecutive slots
-  constexpr int kPer = kCTile / kCThreads;
-  const int j0 = threadIdx.x * kPer;
-  int cnt = 0;
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) cnt += (j0 + u < t_n) && mask[j0 + u] != 0u;
+  // rank of this word's rows inside the tile
+  const int cnt = __popc(u);
   int x = cnt;
 #pragma unroll
   for (int sh = 1; sh < 32; sh <<= 1) {
@@ -133,35 +103,44 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   __syncthreads();
   if (threadIdx.x == 0) {
     int s = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const int t = wtot[w];
-      wtot[32 + w] = s;
+    for (int i = 0; i < kWarps; ++i) {
+      const int t = wtot[i];
+      wtot[i] = s;
       s += t;
     }
     total_s = s;
   }
   __syncthreads();
-  int off = x - cnt + wtot[32 + warp];
-#pragma unroll
-  for (int u = 0; u < kPer; ++u)
-    if (j0 + u < t_n && mask[j0 + u] != 0u) rows[off++] = j0 + u;
-  __syncthreads();
   const int base = base_s;
   const int total = min(total_s, max(a.p_max - base, 0));
   if (total < total_s && threadIdx.x == 0) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
-  // page of every row (independent loads), positions and head masks
   int32_t* pos = a.pos + (size_t)bg * a.p_max;
   uint32_t* hm = a.headmask + (size_t)bg * a.p_max;
+  int r = x - cnt + wtot[warp];
+  uint32_t t = u;
+  while (t) {
+    const int bit = __ffs(t) - 1;
+    t &= t - 1u;
+    if (r < total) {
+      const int p = a.lo + w * 32 + bit;
+      uint32_t m = 0u;
+#pragma unroll
+      for (int h = 0; h < GM; ++h) m |= ((hw[h] >> bit) & 1u) << h;
+      pos[base + r] = p;
+      hm[base + r] = m;
+      rp[r] = p;
+    }
+    ++r;
+  }
+  __syncthreads();
   for (int i = threadIdx.x; i < total; i += kCThreads) {
-    const int p = t_lo + rows[i];
-    int page = a.pt[(size_t)b * a.max_pages + p / kPage];
+    const int p = rp[i];
+    int page = __ldg(a.pt + (size_t)b * a.max_pages + p / kPage);
     if ((unsigned)page >= (unsigned)a.num_pages) {
       latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
       page = -1;
     }
-    pgs[i] = page;
-    pos[base + i] = p;
-    hm[base + i] = mask[rows[i]];
+    rg[i] = page;
   }
   __syncthreads();
   // copy K and V rows: 16-byte units, eight in flight per lane
@@ -173,13 +152,13 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
     uint4 v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int u = u0 + k * 32 + lane;
+      const int un = u0 + k * 32 + lane;
       v[k] = make_uint4(0, 0, 0, 0);
-      if (u < nunits) {
-        const int i = u / upr, c = u - i * upr;
-        const int page = pgs[i];
+      if (un < nunits) {
+        const int i = un / upr, c = un - i * upr;
+        const int page = rg[i];
         if (page >= 0) {
-          const int p = t_lo + rows[i];
+          const int p = rp[i];
           const size_t src = ((size_t)(page * a.Hkv + g) * kPage + p % kPage) * chunks;
           v[k] = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
         }
@@ -187,9 +166,9 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int u = u0 + k * 32 + lane;
-      if (u < nunits) {
-        const int i = u / upr, c = u - i * upr;
+      const int un = u0 + k * 32 + lane;
+      if (un < nunits) {
+        const int i = un / upr, c = un - i * upr;
         if (c < chunks) a.pk[dst0 + (size_t)i * chunks + c] = v[k];
         else a.pv[dst0 + (size_t)i * chunks + c - chunks] = v[k];
       }
@@ -199,8 +178,8 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   const uint32_t all = a.G >= 32 ? 0xffffffffu : ((1u << a.G) - 1u);
   if (blockIdx.x == 0) {
     const int ns = min(a.n_sink, a.p_max);
-    for (int u = threadIdx.x; u < ns * upr; u += kCThreads) {
-      const int i = u / upr, c = u - i * upr;
+    for (int un = threadIdx.x; un < ns * upr; un += kCThreads) {
+      const int i = un / upr, c = un - i * upr;
       const int page = a.pt[(size_t)b * a.max_pages + i / kPage];
       uint4 v = make_uint4(0, 0, 0, 0);
       if ((unsigned)page < (unsigned)a.num_pages) {
@@ -222,44 +201,85 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
     const int n = min(base + total_s, a.p_max);
     if (threadIdx.x == 0) a.n_rows[bg] = n;
     const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
-    for (int u = threadIdx.x; u < (pad_end - n) * upr; u += kCThreads) {
-      const int r = n + u / upr, c = u % upr;
-      const size_t dst = ((size_t)bg * a.p_max + r) * chunks;
+    for (int un = threadIdx.x; un < (pad_end - n) * upr; un += kCThreads) {
+      const int rr = n + un / upr, c = un % upr;
+      const size_t dst = ((size_t)bg * a.p_max + rr) * chunks;
       if (c < chunks) a.pk[dst + c] = make_uint4(0, 0, 0, 0);
       else a.pv[dst + c - chunks] = make_uint4(0, 0, 0, 0);
       if (c == 0) {
-        pos[r] = -1;
-        hm[r] = 0u;
+        pos[rr] = -1;
+        hm[rr] = 0u;
       }
     }
   }
 }
 
-int compact_tiles(int nC) { return (nC + kCTile - 1) / kCTile; }
+// Selections as ascending positions -> one bitmap per query head.
+__global__ void __launch_bounds__(256) idx_to_bits_kernel(const int32_t* __restrict__ sel, int sel_ld, int K,
+                                                          int lo, int nC, uint32_t* bits, int64_t ld_b,
+                                                          int* err) {
+  const int row = blockIdx.x;
+  const int nw = (nC + 31) / 32;
+  uint32_t* brow = bits + (size_t)row * ld_b;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) brow[i] = 0u;
+  __syncthreads();
+  const int32_t* s = sel + (size_t)row * sel_ld;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    const int c = s[i] - lo;
+    if ((unsigned)c < (unsigned)nC) atomicOr(&brow[c >> 5], 1u << (c & 31));
+    else latch_error(err, SFI_ERR_DEVICE_CHECK, kSiteCompactIdx);
+  }
+}
 
-sfi_status run_compact(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
-                       const int32_t* sel_idx, int sel_ld, int K, const sfi_packed& pk,
-                       int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st) {
+int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
+
+template <int GM>
+sfi_status launch_compact(const CompactArgs& a, int BH, cudaStream_t st) {
+  const size_t smem = 2 * kCWords * 32 * sizeof(int32_t);
+  static DeviceOnce attr;
+  if (!attr.done() &&
+      !attr.mark(cudaFuncSetAttribute(compact_gather_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)))
+    return SFI_ERR_CUDA;
+  dim3 grid(a.n_tiles, BH);
+  compact_count_kernel<GM><<<grid, kCThreads, 0, st>>>(a);
+  compact_gather_kernel<GM><<<grid, kCThreads, smem, st>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+}
+
+sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
+                            const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,
+                            int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st) {
   CompactArgs a{};
   a.Hkv = s.Hkv; a.G = s.Hq / s.Hkv; a.Hq = s.Hq; a.D = s.D;
   a.n_sink = p.n_sink;
   a.lo = p.n_sink;
   a.nC = L_slow - p.n_recent - p.n_sink;
-  a.K = K; a.sel_ld = sel_ld;
+  a.nw = (a.nC + 31) / 32;
   a.n_tiles = compact_tiles(a.nC);
   if ((size_t)s.B * s.Hkv * a.n_tiles * sizeof(int32_t) > tc_bytes) return SFI_ERR_WORKSPACE;
   a.max_pages = s.max_pages; a.num_pages = s.num_pages; a.p_max = pk.p_max;
-  a.sel = sel_idx; a.pt = kv.page_table;
+  a.bits = bits; a.ld_b = ld_b;
+  a.pt = kv.page_table;
   a.kpool = reinterpret_cast<const uint4*>(kv.k_pool);
   a.vpool = reinterpret_cast<const uint4*>(kv.v_pool);
   a.pk = reinterpret_cast<uint4*>(pk.k);
   a.pv = reinterpret_cast<uint4*>(pk.v);
   a.pos = pk.pos; a.headmask = pk.headmask; a.n_rows = pk.n_rows;
   a.tile_counts = tile_counts; a.err = kv.err;
-  dim3 grid(a.n_tiles, s.B * s.Hkv);
-  compact_count_kernel<<<grid, kCThreads, 0, st>>>(a);
-  if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
-  compact_gather_kernel<<<grid, kCThreads, 0, st>>>(a);
+  const int BH = s.B * s.Hkv;
+  if (a.G <= 1) return launch_compact<1>(a, BH, st);
+  if (a.G <= 2) return launch_compact<2>(a, BH, st);
+  if (a.G <= 4) return launch_compact<4>(a, BH, st);
+  if (a.G <= 8) return launch_compact<8>(a, BH, st);
+  return launch_compact<16>(a, BH, st);
+}
+
+sfi_status run_idx_to_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L_slow,
+                           const int32_t* sel_idx, int sel_ld, int K, uint32_t* bits, int64_t ld_b,
+                           cudaStream_t st) {
+  const int nC = L_slow - p.n_recent - p.n_sink;
+  idx_to_bits_kernel<<<s.B * s.Hq, 256, 0, st>>>(sel_idx, sel_ld, K, p.n_sink, nC, bits, ld_b, kv.err);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

@@ -37,8 +37,9 @@ struct sfi_ctx {
   int64_t ld = 0;
   void* stats = nullptr;
   float* scores = nullptr;
-  int32_t* sel_idx = nullptr;
-  int sel_ld = 0;
+  uint32_t* bits = nullptr;
+  int64_t bits_ld = 0;
+  uint32_t* rowmm = nullptr;
   int32_t* tile_counts = nullptr;
   size_t tc_bytes = 0;
   // timing of the attention kernels (kind 0 fast, 1 dense)
@@ -52,7 +53,8 @@ namespace {
 
 struct CtxLayout {
   size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, stat_off, stat_bytes, score_off,
-      score_bytes, sel_off, sel_bytes, tc_off, tc_bytes, total;
+      score_bytes, bits_off, bits_bytes, mm_off, mm_bytes, tc_off, tc_bytes, total;
+  int64_t bits_ld;
 };
 
 CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
@@ -74,10 +76,13 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
   c.score_off = off;
   c.score_bytes = w.sel_bytes;
   off += c.score_bytes;
-  const long kmax = std::max(budget_k(p, Lmax), 1);
-  c.sel_off = off;
-  c.sel_bytes = align_up((size_t)s.B * s.Hq * kmax * sizeof(int32_t), 256);
-  off += c.sel_bytes;
+  c.bits_off = off;
+  c.bits_bytes = w.bits_bytes;
+  c.bits_ld = w.bits_ld;
+  off += c.bits_bytes;
+  c.mm_off = off;
+  c.mm_bytes = w.mm_bytes;
+  off += c.mm_bytes;
   c.tc_off = off;
   c.tc_bytes = w.cmp_bytes;
   off += c.tc_bytes;
@@ -185,8 +190,9 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   }
   c->stats = w + l.stat_off;
   c->scores = reinterpret_cast<float*>(w + l.score_off);
-  c->sel_ld = std::max(budget_k(c->p, c->s.max_pages * kPage), 1);
-  c->sel_idx = reinterpret_cast<int32_t*>(w + l.sel_off);
+  c->bits = reinterpret_cast<uint32_t*>(w + l.bits_off);
+  c->bits_ld = l.bits_ld;
+  c->rowmm = reinterpret_cast<uint32_t*>(w + l.mm_off);
   c->tile_counts = reinterpret_cast<int32_t*>(w + l.tc_off);
   c->tc_bytes = l.tc_bytes;
   return SFI_OK;
@@ -250,12 +256,13 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   const int K = budget_k(p, L);
   if (K < 1) return SFI_ERR_SHAPE;
   const int ld_s = (nC + 3) / 4 * 4;
+  if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
   SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                            c->stats, side));
+                            c->stats, c->rowmm, side));
   SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, c->sel_idx, c->sel_ld, side));
-  SFI_TRY(run_compact(s, p, *kv, c->sel_idx, c->sel_ld, K, *packed, c->tile_counts, c->tc_bytes, L,
-                      side));
+  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, c->rowmm,
+                   side));
+  SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->tile_counts, c->tc_bytes, L, side));
   SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
   if (c->overlap) {
     c->pending[layer] = 1;

@@ -39,6 +39,9 @@ struct WsLayout {
   size_t sel_off, sel_bytes;        // Selector: per-(b,kv) stats + scores
   size_t stat_off, stat_bytes;
   size_t cmp_off, cmp_bytes;        // compaction tile counts
+  size_t bits_off, bits_bytes;      // selection bitmaps [B*Hq][bits_ld]
+  size_t mm_off, mm_bytes;          // per-row min / max keys of the scores
+  int64_t bits_ld;
   size_t total;
 };
 WsLayout ws_layout(const sfi_shape& s, const sfi_params& p);
@@ -67,12 +70,18 @@ sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int
 
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
-                             float* scores, int64_t ld_s, void* stat_ws, cudaStream_t st);
+                             float* scores, int64_t ld_s, void* stat_ws, uint32_t* rowmm,
+                             cudaStream_t st);
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset,
-                    int32_t* idx, int64_t ld_i, cudaStream_t st);
-sfi_status run_compact(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
-                       const int32_t* sel_idx, int sel_ld, int K, const sfi_packed& pk,
-                       int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st);
+                    int32_t* idx, int64_t ld_i, uint32_t* bits, int64_t ld_b, const uint32_t* rowmm,
+                    cudaStream_t st);
+int topk_max_n();
+sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
+                            const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,
+                            int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st);
+sfi_status run_idx_to_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L_slow,
+                           const int32_t* sel_idx, int sel_ld, int K, uint32_t* bits, int64_t ld_b,
+                           cudaStream_t st);
 int compact_tiles(int nC);
 int score_tile(int G);
 int stat_chunks(int nC);

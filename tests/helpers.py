@@ -56,21 +56,27 @@ def assert_attn_close(o, ref, what=""):
 
 def ambiguous_positions(ell: np.ndarray, ell1: np.ndarray, window: int, G: int) -> np.ndarray:
     """bool [G, nC]: elements whose soft-NMS or cross-head decision rests on a
-    near-tie (relative gap < NEAR_TIE) in the oracle's float64 scores."""
+    near-tie (relative gap < NEAR_TIE) in the oracle's float64 scores.
+
+    A head's l'' at position j depends on its own soft-NMS penalty and on the
+    owner of j, and the owner depends on every head's l' at j.  So a near-tie
+    in any head's dominance test at j (which can move that head's l' by up to
+    alpha_soft) or between the top two heads makes all heads at j ambiguous."""
     w = window // 2
     Gh, n = ell.shape
-    amb = np.zeros((Gh, n), bool)
+    nms = np.zeros((Gh, n), bool)
     scale = np.maximum(np.abs(ell), 1e-30)
     for d in range(1, w + 1):
         diff = np.abs(ell[:, d:] - ell[:, :-d])
         near = diff < NEAR_TIE * np.maximum(scale[:, d:], scale[:, :-d])
-        amb[:, d:] |= near
-        amb[:, :-d] |= near
+        nms[:, d:] |= near
+        nms[:, :-d] |= near
+    amb = nms.copy()
     if G > 1:
         s = np.sort(ell1, axis=0)
         top, second = s[-1], s[-2]
         near_owner = np.abs(top - second) < NEAR_TIE * np.maximum(np.abs(top), 1e-30)
-        amb |= near_owner[None, :]
+        amb |= (near_owner | nms.any(axis=0))[None, :]
     return amb
 
 
