@@ -173,6 +173,24 @@ sfi_status sfi_dense_attn(const sfi_shape* shape, const sfi_paged_kv* kv, int32_
                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
                           void* ws, size_t ws_bytes, sfi_stream stream);
 
+/* sfi_dense_attn without a workspace argument, for callers that cannot
+ * allocate device memory where they call it: serving runtimes whose pool
+ * hands the library only input and output tensors, plugin or embedded hosts
+ * without access to the CUDA allocator, code that must not allocate during
+ * CUDA graph capture.  The paper has no counterpart to this entry point.
+ * Arguments and results are those of sfi_dense_attn.  The scratch (a work
+ * counter and the split-K partials) is a static 16 MiB device array that
+ * every GPU loading the library holds until the process exits; a call whose
+ * partials would not fit returns SFI_ERR_WORKSPACE and launches nothing.
+ * Nothing is allocated.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress), so make it before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (the counter is cleared at the start of every call): calls that
+ * overlap on the GPU race, so order them (one stream, or events). */
+sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                                  const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
+                                  sfi_stream stream);
+
 /* f = exp(logits - lse) over j < L for every (b, hq) row. */
 sfi_status sfi_attn_probs(const sfi_shape* shape, int32_t L, const float* logits, int64_t ld,
                           const float* lse, float* probs, sfi_stream stream);

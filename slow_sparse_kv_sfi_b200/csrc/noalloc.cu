@@ -1,0 +1,91 @@
+// Dense attention whose scratch lives in a static device array, for callers
+// that cannot allocate device memory at the point of the call.
+//
+// sfi_dense_attn needs scratch (a work counter and the split-K partials) and
+// takes it as a caller-allocated workspace.  Some callers have no way to
+// provide one: serving runtimes whose memory pool hands the library only the
+// input and output tensors, plugin or embedded hosts that have no access to
+// the CUDA allocator, and code that must not allocate while a CUDA graph is
+// being captured.  This entry point runs the same kernels with the scratch
+// taken from g_noalloc_scratch, a file-scope device array of
+// kNoAllocScratchBytes that every GPU which loads the library holds until the
+// process exits.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sfi {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
+constexpr size_t kCounterBytes = 256;                         // work counter, then partials
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_mu;
+void* g_addr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device.  The first call
+// on a device looks it up (host code only holds a stand-in for the symbol).
+sfi_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SFI_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SFI_ERR_CUDA;
+    g_addr[dev] = p;
+  }
+  *out = g_addr[dev];
+  return SFI_OK;
+}
+
+__global__ void zero_counter_kernel(int* ctr) { ctr[0] = 0; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace sfi
+
+using namespace sfi;
+
+extern "C" sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                                             const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
+                                             sfi_stream stream) {
+  if (!shape || !kv || !q || !out) return SFI_ERR_INVALID_ARG;
+  const sfi_shape& s = *shape;
+  if (s.B < 1 || s.Hq < 1 || s.Hkv < 1 || s.Hq % s.Hkv != 0) return SFI_ERR_SHAPE;
+  const int G = s.Hq / s.Hkv;
+  if (G > 16) return SFI_ERR_UNSUPPORTED;
+  if (s.D != 64 && s.D != 128) return SFI_ERR_UNSUPPORTED;
+  if (s.page_size != kPage) return SFI_ERR_UNSUPPORTED;
+  if (s.max_pages < 1 || s.num_pages < 1) return SFI_ERR_SHAPE;
+  if ((long long)s.num_pages * s.Hkv * kPage >= (1LL << 31)) return SFI_ERR_SHAPE;
+  if (L < 1 || L > s.max_pages * kPage) return SFI_ERR_SHAPE;
+  if (!kv->k_pool || !kv->v_pool || !kv->page_table) return SFI_ERR_INVALID_ARG;
+  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool) || !aligned16(q)) return SFI_ERR_INVALID_ARG;
+  if (extras) {
+    if ((extras->logits || extras->probs) && extras->ld < L) return SFI_ERR_SHAPE;
+    if (extras->probs && !extras->lse) return SFI_ERR_INVALID_ARG;
+    if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
+      return SFI_ERR_SHAPE;
+  }
+  // partials this call needs, against the static capacity
+  const int T = (L + kPage - 1) / kPage;
+  const int ct = dense_chunk_tiles(s, L);
+  const int n_items = s.B * s.Hkv * ((T + ct - 1) / ct);
+  const size_t part_cap = kNoAllocScratchBytes - kCounterBytes;
+  if (attn_part_bytes(n_items, G, s.D) > part_cap) return SFI_ERR_WORKSPACE;
+  void* base = nullptr;
+  const sfi_status r = scratch_address(&base);
+  if (r != SFI_OK) return r;
+  char* b = static_cast<char*>(base);
+  int* ctr = reinterpret_cast<int*>(b);
+  cudaStream_t st = (cudaStream_t)stream;
+  // the area keeps whatever the last call left: the work counter must start at zero
+  zero_counter_kernel<<<1, 1, 0, st>>>(ctr);
+  if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
+  return run_dense_attn(s, *kv, L, q, out, extras, ctr, reinterpret_cast<float*>(b + kCounterBytes), part_cap, st,
+                        nullptr, nullptr);
+}

@@ -75,6 +75,7 @@ def _declare(L):
         "sfi_append_kv": (C.c_int, [P, P, I32, P, P, P]),
         "sfi_key_norms": (C.c_int, [P, P, I32, I32, P]),
         "sfi_dense_attn": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
+        "sfi_dense_attn_noalloc": (C.c_int, [P, P, I32, P, P, P, P]),
         "sfi_attn_probs": (C.c_int, [P, I32, P, I64, P, P, P]),
         "sfi_fast_attn": (C.c_int, [P, P, P, I32, P, P, P, P, P, SZ, P]),
         "sfi_select_scores": (C.c_int, [P, P, P, I32, P, I64, P, P, P, SZ, P]),
@@ -98,7 +99,8 @@ def _declare(L):
 
 
 EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_rows", "sfi_budget",
-            "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_attn_probs", "sfi_fast_attn",
+            "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_noalloc",
+            "sfi_attn_probs", "sfi_fast_attn",
             "sfi_select_scores", "sfi_topk", "sfi_select", "sfi_compact", "sfi_poll_error",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
             "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_timing"]
@@ -182,6 +184,13 @@ def sfi_dense_attn(shape, kv, L, q, out, ws, extras: Optional[DenseExtras] = Non
     _check(lib().sfi_dense_attn(C.byref(shape), C.byref(kv), L, _p(q), _p(out), _ref(extras),
                                 _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "sfi_dense_attn")
+
+
+def sfi_dense_attn_noalloc(shape, kv, L, q, out, extras: Optional[DenseExtras] = None, stream=None):
+    """sfi_dense_attn with its scratch in the library's static device array
+    (no workspace, nothing allocated)."""
+    _check(lib().sfi_dense_attn_noalloc(C.byref(shape), C.byref(kv), L, _p(q), _p(out), _ref(extras),
+                                        _stream(stream)), "sfi_dense_attn_noalloc")
 
 
 def sfi_attn_probs(shape, L, logits, ld, lse, probs, stream=None):
