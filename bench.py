@@ -391,7 +391,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
                 "launches": dense_n, "avg_launch_us": 1000 * dense_ms / max(dense_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
     value = world * tokens / t_sfi * args.steps
-    launches_per_run = NL * (n_slow * 8 + (T - n_slow) * 3)
+    launches_per_run = NL * (n_slow * 9 + (T - n_slow) * 3)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000 * t_sfi / args.steps, "higher_is_better": True,
@@ -432,6 +432,28 @@ def run_sfi(args, cfg, rank, world, dist_on):
     bench.ctx.close()
 
 
+def run_layer_probe(args, cfg):
+    """A few launches of every hot-path kernel on one layer of the workload
+    (for profiler captures): per repetition one slow layer-step (dense
+    attention with logits, Selector, compaction) and one fast layer-step."""
+    cfg1 = cfg.replace(n_layers=1)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    li = W.make_layer(cfg1, 0, dev)
+    layer = alloc_layer(cfg1, li, dev)
+    ctx = S.Context(shape_of(cfg1), params_of(cfg1), 1, overlap=False, device=dev)
+    out = torch.empty(cfg1.B, cfg1.Hq, cfg1.D, device=dev)
+    torch.cuda.synchronize()
+    for r in range(args.layer_probe):
+        for t in range(2):   # step 0 is slow, step 1 fast
+            ctx.decode_step(0, t, 0, cfg1.seq_len(t), layer.kv, layer.packed, li.q[t], li.k_new[t],
+                            li.v_new[t], out)
+        ctx.join()
+    torch.cuda.synchronize()
+    assert S.sfi_poll_error(layer.kv) == 0
+    ctx.close()
+    print(json.dumps({"layer_probe": cfg1.name, "repetitions": args.layer_probe}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,6 +463,8 @@ def main():
     ap.add_argument("--impl", default="sfi", choices=["sfi", "reference"])
     ap.add_argument("--decode-steps", type=int, default=0, help="override the workload's decode steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layer-probe", type=int, default=0,
+                    help="only run this many slow+fast layer-steps of one layer (profiler captures)")
     args = ap.parse_args()
     cfg = W.CONFIG_BY_NAME[args.config]
     if args.decode_steps:
@@ -453,7 +477,9 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-    if args.impl == "reference":
+    if args.layer_probe:
+        run_layer_probe(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg, rank, world)
     else:
         if not torch.cuda.is_available():
