@@ -11,9 +11,10 @@
 // kernel writes them.  A tile is 256 bitmap words (8192 positions); each
 // thread owns one word: the OR of the group's words is the union, its
 // popcount the row count.  compact_count writes the per-tile counts;
-// compact_gather scans them, writes positions and head masks, looks up every
-// row's page in one round of independent loads, then copies the K and V rows
-// in 16-byte units with eight loads in flight per lane.
+// compact_gather scans them and writes positions, head masks and n_rows;
+// compact_copy then copies the K and V rows in 16-byte units, eight loads in
+// flight per thread, over fixed 128-row blocks (the selection is far from
+// uniform over positions, so per-tile copying would be imbalanced).
 #include "common.cuh"
 #include "internal.h"
 
@@ -71,9 +72,6 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactA
 
 template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const CompactArgs a) {
-  extern __shared__ int32_t csm[];
-  int32_t* rp = csm;                       // position of each row of the tile
-  int32_t* rg = csm + kCWords * 32;        // its page (-1: bad page-table entry)
   __shared__ int wtot[kCThreads / 32 + 1];
   __shared__ int base_s, total_s;
   const int bg = blockIdx.y;
@@ -128,87 +126,87 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
       for (int h = 0; h < GM; ++h) m |= ((hw[h] >> bit) & 1u) << h;
       pos[base + r] = p;
       hm[base + r] = m;
-      rp[r] = p;
     }
     ++r;
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < total; i += kCThreads) {
-    const int p = rp[i];
-    int page = __ldg(a.pt + (size_t)b * a.max_pages + p / kPage);
-    if ((unsigned)page >= (unsigned)a.num_pages) {
-      latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
-      page = -1;
-    }
-    rg[i] = page;
-  }
-  __syncthreads();
-  // copy K and V rows: 16-byte units, eight in flight per lane
-  const int chunks = a.D / 8;
-  const int upr = 2 * chunks;
-  const int nunits = total * upr;
-  const size_t dst0 = ((size_t)bg * a.p_max + base) * chunks;
-  for (int u0 = warp * 256; u0 < nunits; u0 += kWarps * 256) {
-    uint4 v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int un = u0 + k * 32 + lane;
-      v[k] = make_uint4(0, 0, 0, 0);
-      if (un < nunits) {
-        const int i = un / upr, c = un - i * upr;
-        const int page = rg[i];
-        if (page >= 0) {
-          const int p = rp[i];
-          const size_t src = ((size_t)(page * a.Hkv + g) * kPage + p % kPage) * chunks;
-          v[k] = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
-        }
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int un = u0 + k * 32 + lane;
-      if (un < nunits) {
-        const int i = un / upr, c = un - i * upr;
-        if (c < chunks) a.pk[dst0 + (size_t)i * chunks + c] = v[k];
-        else a.pv[dst0 + (size_t)i * chunks + c - chunks] = v[k];
-      }
-    }
-  }
-  // sinks (first tile) and the zero tail (last tile)
+  // sinks (first tile) and the tail (last tile); rows are copied by compact_copy
   const uint32_t all = a.G >= 32 ? 0xffffffffu : ((1u << a.G) - 1u);
   if (blockIdx.x == 0) {
-    const int ns = min(a.n_sink, a.p_max);
-    for (int un = threadIdx.x; un < ns * upr; un += kCThreads) {
-      const int i = un / upr, c = un - i * upr;
-      const int page = a.pt[(size_t)b * a.max_pages + i / kPage];
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if ((unsigned)page < (unsigned)a.num_pages) {
-        const size_t src = ((size_t)(page * a.Hkv + g) * kPage + i % kPage) * chunks;
-        v = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
-      } else if (c == 0) {
-        latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
-      }
-      const size_t dst = ((size_t)bg * a.p_max + i) * chunks;
-      if (c < chunks) a.pk[dst + c] = v;
-      else a.pv[dst + c - chunks] = v;
-      if (c == 0) {
-        pos[i] = i;
-        hm[i] = all;
-      }
+    for (int i = threadIdx.x; i < min(a.n_sink, a.p_max); i += kCThreads) {
+      pos[i] = i;
+      hm[i] = all;
     }
   }
   if (blockIdx.x == gridDim.x - 1) {
     const int n = min(base + total_s, a.p_max);
     if (threadIdx.x == 0) a.n_rows[bg] = n;
     const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
-    for (int un = threadIdx.x; un < (pad_end - n) * upr; un += kCThreads) {
-      const int rr = n + un / upr, c = un % upr;
-      const size_t dst = ((size_t)bg * a.p_max + rr) * chunks;
-      if (c < chunks) a.pk[dst + c] = make_uint4(0, 0, 0, 0);
-      else a.pv[dst + c - chunks] = make_uint4(0, 0, 0, 0);
-      if (c == 0) {
-        pos[rr] = -1;
-        hm[rr] = 0u;
+    for (int rr = n + threadIdx.x; rr < pad_end; rr += kCThreads) {
+      pos[rr] = -1;
+      hm[rr] = 0u;
+    }
+  }
+}
+
+// Copy the K and V rows of the packed buffer from the pages (rows past
+// n_rows up to the next multiple of 16: zeros).  Grid: 128-row blocks of
+// every (b, KV head); blocks past the rows in use return at once, so the
+// copy work is spread evenly whatever the selection looks like.
+constexpr int kCopyRows = 128;
+
+__global__ void __launch_bounds__(256) compact_copy_kernel(const CompactArgs a) {
+  __shared__ int32_t pg[kCopyRows];
+  __shared__ int32_t pp[kCopyRows];
+  const int bg = blockIdx.y;
+  const int b = bg / a.Hkv, g = bg - b * a.Hkv;
+  const int n = min(max(a.n_rows[bg], 0), a.p_max);
+  const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
+  const int r0 = blockIdx.x * kCopyRows;
+  if (r0 >= pad_end) return;
+  const int nr = min(kCopyRows, pad_end - r0);
+  const int32_t* pos = a.pos + (size_t)bg * a.p_max;
+  if (threadIdx.x < nr) {
+    const int r = r0 + threadIdx.x;
+    int page = -1, p = 0;
+    if (r < n) {
+      p = pos[r];
+      const int pi = p / kPage;
+      if (p >= 0 && pi < a.max_pages) page = __ldg(a.pt + (size_t)b * a.max_pages + pi);
+      if ((unsigned)page >= (unsigned)a.num_pages) {
+        latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
+        page = -1;
+      }
+    }
+    pg[threadIdx.x] = page;
+    pp[threadIdx.x] = p;
+  }
+  __syncthreads();
+  const int chunks = a.D / 8;
+  const int upr = 2 * chunks;
+  const int nunits = nr * upr;
+  const size_t dst0 = ((size_t)bg * a.p_max + r0) * chunks;
+  for (int u0 = threadIdx.x; u0 < nunits; u0 += 8 * 256) {
+    uint4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int un = u0 + k * 256;
+      v[k] = make_uint4(0, 0, 0, 0);
+      if (un < nunits) {
+        const int i = un / upr, c = un - i * upr;
+        const int page = pg[i];
+        if (page >= 0) {
+          const size_t src = ((size_t)(page * a.Hkv + g) * kPage + pp[i] % kPage) * chunks;
+          v[k] = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int un = u0 + k * 256;
+      if (un < nunits) {
+        const int i = un / upr, c = un - i * upr;
+        if (c < chunks) a.pk[dst0 + (size_t)i * chunks + c] = v[k];
+        else a.pv[dst0 + (size_t)i * chunks + c - chunks] = v[k];
       }
     }
   }
@@ -235,15 +233,11 @@ int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
 
 template <int GM>
 sfi_status launch_compact(const CompactArgs& a, int BH, cudaStream_t st) {
-  const size_t smem = 2 * kCWords * 32 * sizeof(int32_t);
-  static DeviceOnce attr;
-  if (!attr.done() &&
-      !attr.mark(cudaFuncSetAttribute(compact_gather_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem)))
-    return SFI_ERR_CUDA;
   dim3 grid(a.n_tiles, BH);
   compact_count_kernel<GM><<<grid, kCThreads, 0, st>>>(a);
-  compact_gather_kernel<GM><<<grid, kCThreads, smem, st>>>(a);
+  compact_gather_kernel<GM><<<grid, kCThreads, 0, st>>>(a);
+  dim3 cgrid((a.p_max + kCopyRows - 1) / kCopyRows, BH);
+  compact_copy_kernel<<<cgrid, 256, 0, st>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
