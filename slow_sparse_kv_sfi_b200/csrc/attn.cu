@@ -37,7 +37,8 @@ namespace sfi {
 constexpr int kConsumerWarps = 4;
 constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = 16 * 128;   // 16 rows x 128 bytes: one column block of a tile
-constexpr int kChunkAlign = 8;        // chunk lengths are multiples of the largest stage
+constexpr long kDenseItemsPerSm = 8;  // dense step: work items per SM
+constexpr long kFastItemTiles = 64;   // fast step: target tiles per work item
 
 enum AttnMode : int { kDense = 0, kDenseExtras = 1, kFast = 2 };
 
@@ -49,7 +50,7 @@ struct AttnArgs {
   float* part;          // [n_items][G][D + 4]
   int* ctr;             // work counter (zero on entry; the combine kernel re-zeroes it)
   int n_chunks;         // chunks per (b, kv head)
-  int chunk_tiles;      // dense: tiles per chunk (multiple of kChunkAlign, <= kMaxChunkTiles)
+  int chunk_tiles;      // dense: tiles per chunk (a multiple of the stage, <= kMaxChunkTiles)
   int n_items;
   float scale_log2;     // log2(e) / sqrt(D)
   float scale;          // 1 / sqrt(D)
@@ -71,15 +72,17 @@ constexpr int kMaxBH = 512;
 // Shared-memory plan.  A tile is 16 rows of K (or V): one TMA box of
 // [D/64 column blocks][16 rows][128 B], 128B-swizzled.  Each consumer warp
 // takes TT tiles of every stage, so a stage holds 4 * TT tiles of K and V.
+// kCps CTAs share an SM; together they keep about 192 KB of copies in flight.
 template <int D, int NT>
 struct Plan {
-  static constexpr int TT = (NT == 1) ? 2 : 1;
+  static constexpr int kCps = (NT == 1) ? 2 : 1;
+  static constexpr int TT = (NT == 1 && kCps == 1) ? 2 : 1;
   static constexpr int kTPS = 4 * TT;
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kHalves * kBoxBytes;
   static constexpr int kKBytes = kTPS * kTileBytes;
   static constexpr int kStageBytes = 2 * kKBytes;
-  static constexpr int kStages = (D == 128) ? (NT == 1 ? 3 : 6) : (NT == 1 ? 6 : 12);
+  static constexpr int kStages = (192 * 1024 / kCps) / kStageBytes;
   static constexpr int kHeads = NT * 8;
   static constexpr int kQBytes = kHeads * D * 2;
 };
@@ -107,7 +110,7 @@ struct Smem {
   static constexpr int kNrOff = kPtOff + kMaxChunkTiles * 4;
   static constexpr int kBarOff = kNrOff + kMaxBH * 4;
   static constexpr int kTotal = kBarOff + 2 * kStages * 8 + 64 + 1024;   // + alignment slack
-  static_assert(kTotal <= 227 * 1024, "shared memory budget");
+  static_assert(kTotal * P::kCps + 1024 * P::kCps <= 228 * 1024, "shared memory budget");
 };
 
 // Tile range and page range of one work item.
@@ -118,7 +121,7 @@ struct Item {
   int first_page;         // page number of tile n_packed_tiles (fast) or tile 0 (dense)
 };
 
-template <int MODE>
+template <int MODE, int TPS>
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const int* nrows_s) {
   Item it;
   it.bg = item / a.n_chunks;
@@ -138,7 +141,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const i
     it.first_page = a.rec_lo / kPage;
     const int T = it.n_packed_tiles + ((a.L - 1) / kPage - it.first_page + 1);
     int ct = (T + a.n_chunks - 1) / a.n_chunks;
-    ct = (ct + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
+    ct = (ct + TPS - 1) / TPS * TPS;
     it.t_begin = min(T, c * ct);
     it.t_end = min(T, it.t_begin + ct);
   }
@@ -164,7 +167,7 @@ struct Maps {
 };
 
 template <int D, int NT, int MODE>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     attn_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   using S = Smem<D, NT>;
   using P = Plan<D, NT>;
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int j = 0; j < kMaxChunkTiles / 32; ++j) regs[j] = 0;
       if (item >= a.n_items) return;
-      const Item it = decode_item<MODE>(a, item, nrows_s);
+      const Item it = decode_item<MODE, kTPS>(a, item, nrows_s);
       const int p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
       const int p_hi = item_page(it, max(it.t_end, it.n_packed_tiles));
       const int32_t* row = a.page_table + (size_t)it.b * a.max_pages;
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int nst = 1;
       int p_lo = 0;
       if (item < a.n_items) {
-        it = decode_item<MODE>(a, item, nrows_s);
+        it = decode_item<MODE, kTPS>(a, item, nrows_s);
         nst = max(1, (it.t_end - it.t_begin + kTPS - 1) / kTPS);
         p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
       }
@@ -377,7 +380,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 
   // ------------------------------------------------------------ consumers
-  const int ctid = threadIdx.x;          // 0..127
   const int r0 = lane >> 2;              // accumulator rows r0, r0 + 8
   const int cq = (lane & 3) * 2;         // accumulator columns cq, cq + 1
   const int rowA = (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -385,7 +387,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int rowV = (lane & 7) + ((lane >> 4) & 1) * 8;
   const int chV = (lane >> 3) & 1;
   const float NEG_INF = -INFINITY;
-  constexpr int H8 = P::kHeads;
 
   int slot = 0;
   uint32_t phase = 0;
@@ -801,10 +802,13 @@ sfi_status launch_attn_t(const Maps& maps, const AttnArgs& a, cudaStream_t st) {
   using S = Smem<D, NT>;
   auto kern = attn_kernel<D, NT, MODE>;
   static DeviceOnce attr;   // per instantiation and device
-  if (!attr.done() &&
-      !attr.mark(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal)))
-    return SFI_ERR_CUDA;
-  const int grid = std::min(a.n_items, num_sms());
+  if (!attr.done()) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (!attr.mark(e)) return SFI_ERR_CUDA;
+  }
+  const int grid = std::min(a.n_items, num_sms() * Plan<D, NT>::kCps);
   kern<<<grid, kAttnThreads, S::kTotal, st>>>(maps, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
@@ -818,8 +822,6 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
   if (G <= 8) return launch_attn_t<64, 1, MODE>(maps, a, st);
   return launch_attn_t<64, 2, MODE>(maps, a, st);
 }
-
-int stage_tiles(int D, int G) { return (G <= 8) ? 8 : 4; }
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int* err,
@@ -837,33 +839,62 @@ sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shap
 
 }  // namespace
 
-// Tiles of 16 rows per chunk for the dense step: about 8 work items per SM,
-// at least 8 tiles and at most kMaxChunkTiles, a multiple of the 4-tile stage.
+namespace {
+
+// CTAs of one attention launch that run at once, and the tiles of one stage.
+struct AttnGrid {
+  long ctas;
+  int tps;
+};
+
+template <int D, int NT>
+AttnGrid grid_of() {
+  return AttnGrid{(long)num_sms() * Plan<D, NT>::kCps, Plan<D, NT>::kTPS};
+}
+
+AttnGrid attn_grid(int D, int G) {
+  if (D == 128) return G <= 8 ? grid_of<128, 1>() : grid_of<128, 2>();
+  return G <= 8 ? grid_of<64, 1>() : grid_of<64, 2>();
+}
+
+}  // namespace
+
+// Tiles of 16 rows per chunk for the dense step: about kDenseItemsPerSm items
+// per SM, at least 8 tiles and at most kMaxChunkTiles, a multiple of the stage.
 int dense_chunk_tiles(const sfi_shape& s, int L) {
+  const AttnGrid g = attn_grid(s.D, s.Hq / s.Hkv);
   const long T = (L + kPage - 1) / kPage;
   const long bh = (long)s.B * s.Hkv;
-  long ct = (T * bh + 8L * num_sms() - 1) / (8L * num_sms());
+  const long n = kDenseItemsPerSm * num_sms();
+  long ct = (T * bh + n - 1) / n;
   ct = std::max(ct, 8L);
-  ct = (ct + kChunkAlign - 1) / kChunkAlign * kChunkAlign;
+  ct = (ct + g.tps - 1) / g.tps * g.tps;
   return (int)std::min<long>(ct, kMaxChunkTiles);
 }
 
+// Upper bound of the dense chunks per (b, kv head) at any L <= max_pages * 16.
 int dense_chunks_bound(const sfi_shape& s) {
   const long T = (long)s.max_pages;
   const long bh = (long)s.B * s.Hkv;
-  const long a = (8L * num_sms() + bh - 1) / bh + 1;
+  const long a = (kDenseItemsPerSm * num_sms() + bh - 1) / bh + 1;
   const long b = (T + kMaxChunkTiles - 1) / kMaxChunkTiles;
   return (int)std::min<long>((T + 7) / 8, std::max(a, b));
 }
 
-// Chunks per (b, kv head) for the fast step: items of about 32 tiles for the
-// expected packed size (n_sink + K rows), never more than kMaxChunkTiles tiles
-// even when the packed buffer is full.
+// Chunks per (b, kv head) for the fast step.  The expected tiles (n_sink + K
+// packed rows plus the recent window) are cut so that every CTA of the launch
+// gets the same whole number of items of at most about kFastItemTiles tiles;
+// an item never exceeds kMaxChunkTiles tiles, even with a full packed buffer.
+// The result never decreases as k_est grows.
 int fast_chunks(const sfi_shape& s, int p_max, int n_recent, int k_est) {
+  const AttnGrid g = attn_grid(s.D, s.Hq / s.Hkv);
+  const long bh = (long)s.B * s.Hkv;
   const long t_rec = n_recent / kPage + 2;
   const long t_max = (p_max + kPage - 1) / kPage + t_rec;
   const long t_est = std::min<long>((k_est + kPage - 1) / kPage + 1, (p_max + kPage - 1) / kPage) + t_rec;
-  long nc = std::max<long>((t_est + 31) / 32, (t_max + kMaxChunkTiles - 1) / kMaxChunkTiles);
+  const long per_cta = std::max<long>(1, (bh * t_est + g.ctas * kFastItemTiles - 1) / (g.ctas * kFastItemTiles));
+  long nc = std::min<long>((per_cta * g.ctas + bh - 1) / bh, t_est);
+  nc = std::max<long>(nc, (t_max + kMaxChunkTiles - 1) / kMaxChunkTiles);
   return (int)std::max(nc, 1L);
 }
 
@@ -931,7 +962,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
   const uint64_t prows = (uint64_t)s.B * s.Hkv * pk.p_max;
-  const int nts = stage_tiles(s.D, G);
+  const int nts = attn_grid(s.D, G).tps;
   if (!make_map(&maps.k, kv.k_pool, rows, s.D) || !make_map(&maps.v, kv.v_pool, rows, s.D) ||
       !make_map(&maps.pk, pk.k, prows, s.D) || !make_map(&maps.pv, pk.v, prows, s.D) ||
       !make_map_tiles(&maps.pk8, pk.k, prows, s.D, nts) || !make_map_tiles(&maps.pv8, pk.v, prows, s.D, nts))
