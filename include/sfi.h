@@ -155,7 +155,8 @@ sfi_status sfi_packed_rows(const sfi_shape* shape, const sfi_params* params, int
 sfi_status sfi_budget(const sfi_params* params, int32_t L, int32_t* K);
 
 /* Append one token per (sequence, KV head) at position L-1 and record its key
- * norm.  k_new, v_new: bf16 [B, Hkv, D]. */
+ * norm (fp64 sum of squares of the stored bf16 key, rounded once to fp32) when
+ * kv->key_norms is non-NULL.  k_new, v_new: bf16 [B, Hkv, D], 16-byte aligned. */
 sfi_status sfi_append_kv(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
                          const sfi_bf16* k_new, const sfi_bf16* v_new, sfi_stream stream);
 
@@ -172,6 +173,20 @@ sfi_status sfi_key_norms(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t
 sfi_status sfi_dense_attn(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
                           void* ws, size_t ws_bytes, sfi_stream stream);
+
+/* sfi_append_kv and sfi_dense_attn in one launch: the work item of each
+ * (b, kv head) that holds position L - 1 first writes k_new / v_new (bf16
+ * [B, Hkv, D], 16-byte aligned) into that row of the pages and its key norm
+ * into kv->key_norms (when non-NULL), then attends over [0, L) as
+ * sfi_dense_attn does.  Results are those of the two calls in a row, bit for
+ * bit; a page-table entry outside the pool is latched in kv->err
+ * (SFI_ERR_DEVICE_CHECK) and that row is neither written nor attended.  The
+ * pages fold the append into the decode step ([ES] §2; [ZH] §2.1) and do not
+ * say how it is launched. */
+sfi_status sfi_dense_attn_append(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                                 const sfi_bf16* k_new, const sfi_bf16* v_new, const sfi_bf16* q,
+                                 float* out, const sfi_dense_extras* extras, void* ws, size_t ws_bytes,
+                                 sfi_stream stream);
 
 /* sfi_dense_attn without a workspace argument, for callers that cannot
  * allocate device memory where they call it: serving runtimes whose pool
@@ -203,6 +218,14 @@ sfi_status sfi_fast_attn(const sfi_shape* shape, const sfi_params* params,
                          const sfi_paged_kv* kv, int32_t L, const sfi_bf16* q,
                          const sfi_packed* packed, float* out, float* lse, void* ws,
                          size_t ws_bytes, sfi_stream stream);
+
+/* sfi_append_kv and sfi_fast_attn in one launch (the step's token lies in the
+ * recent window); append semantics, alignment and errors as for
+ * sfi_dense_attn_append. */
+sfi_status sfi_fast_attn_append(const sfi_shape* shape, const sfi_params* params,
+                                const sfi_paged_kv* kv, int32_t L, const sfi_bf16* k_new,
+                                const sfi_bf16* v_new, const sfi_bf16* q, const sfi_packed* packed,
+                                float* out, float* lse, void* ws, size_t ws_bytes, sfi_stream stream);
 
 /* Selector scores ([FR] "B. Le Sélecteur"; [NL] "De Selector"; [ZH] §2.2):
  * for the candidates C = [n_sink, L - n_recent) of a slow step at context L,
@@ -279,10 +302,13 @@ sfi_status sfi_ctx_join(sfi_ctx* ctx, sfi_stream stream);
 
 /* Per-kernel CUDA-event timing of the attention kernels launched by
  * sfi_decode_step (kind 0 = fast-attention main kernel, 1 = dense main
- * kernel).  Enabled with sfi_ctx_set_timing; sfi_ctx_timing synchronises on
- * the recorded events and returns total milliseconds and launch count since
- * the last reset. */
-sfi_status sfi_ctx_set_timing(sfi_ctx* ctx, int32_t enable);
+ * kernel).  sfi_ctx_set_timing(ctx, n): n = 0 off; n > 0 brackets the
+ * attention launches of layers 0, n, 2n, ... with an event pair (an event
+ * between two launches keeps the second from starting early, so sparse
+ * sampling leaves the other layers' launches overlapped).  sfi_ctx_timing
+ * synchronises on the recorded events and returns total milliseconds and
+ * launch count since the last reset. */
+sfi_status sfi_ctx_set_timing(sfi_ctx* ctx, int32_t layer_stride);
 sfi_status sfi_ctx_timing(sfi_ctx* ctx, int32_t kind, double* total_ms, int64_t* launches,
                           int32_t reset);
 

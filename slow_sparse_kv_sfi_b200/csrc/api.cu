@@ -139,6 +139,46 @@ sfi_status check_packed(const sfi_shape* s, const sfi_params* p, const sfi_packe
     if (_r != SFI_OK) return _r;       \
   } while (0)
 
+// Shared bodies of the attention entry points with and without the fused
+// append of the step's token (tok == nullptr: none).
+sfi_status dense_attn_impl(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L, const StepToken* tok,
+                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras, void* ws,
+                           size_t ws_bytes, sfi_stream stream) {
+  SFI_TRY(check_shape(shape));
+  SFI_TRY(check_kv(kv));
+  SFI_TRY(check_L(shape, L));
+  if (!q || !out) return SFI_ERR_INVALID_ARG;
+  if (extras) {
+    if ((extras->logits || extras->probs) && extras->ld < L) return SFI_ERR_SHAPE;
+    if (extras->probs && !extras->lse) return SFI_ERR_INVALID_ARG;
+    if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
+      return SFI_ERR_SHAPE;
+  }
+  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
+  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
+  const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
+  return run_dense_attn(*shape, *kv, L, q, out, extras, static_cast<int*>(ws),
+                        reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
+                        (cudaStream_t)stream, nullptr, nullptr, tok);
+}
+
+sfi_status fast_attn_impl(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv, int32_t L,
+                          const StepToken* tok, const sfi_bf16* q, const sfi_packed* packed, float* out,
+                          float* lse, void* ws, size_t ws_bytes, sfi_stream stream) {
+  SFI_TRY(check_shape(shape));
+  SFI_TRY(check_params(params));
+  SFI_TRY(check_kv(kv));
+  SFI_TRY(check_sparse_L(shape, params, L));
+  SFI_TRY(check_packed(shape, params, packed));
+  if (!q || !out) return SFI_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
+  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
+  const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
+  return run_fast_attn(*shape, *params, *kv, L, q, *packed, out, lse, static_cast<int*>(ws),
+                       reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
+                       (cudaStream_t)stream, nullptr, nullptr, tok);
+}
+
 }  // namespace
 }  // namespace sfi
 
@@ -192,7 +232,7 @@ sfi_status sfi_append_kv(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t
   SFI_TRY(check_shape(shape));
   SFI_TRY(check_kv(kv));
   SFI_TRY(check_L(shape, L));
-  if (!k_new || !v_new) return SFI_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SFI_ERR_INVALID_ARG;
   return run_append(*shape, *kv, L, k_new, v_new, (cudaStream_t)stream);
 }
 
@@ -208,22 +248,16 @@ sfi_status sfi_key_norms(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t
 sfi_status sfi_dense_attn(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
                           void* ws, size_t ws_bytes, sfi_stream stream) {
-  SFI_TRY(check_shape(shape));
-  SFI_TRY(check_kv(kv));
-  SFI_TRY(check_L(shape, L));
-  if (!q || !out) return SFI_ERR_INVALID_ARG;
-  if (extras) {
-    if ((extras->logits || extras->probs) && extras->ld < L) return SFI_ERR_SHAPE;
-    if (extras->probs && !extras->lse) return SFI_ERR_INVALID_ARG;
-    if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
-      return SFI_ERR_SHAPE;
-  }
-  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
-  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
-  const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
-  return run_dense_attn(*shape, *kv, L, q, out, extras, static_cast<int*>(ws),
-                        reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
-                        (cudaStream_t)stream, nullptr, nullptr);
+  return dense_attn_impl(shape, kv, L, nullptr, q, out, extras, ws, ws_bytes, stream);
+}
+
+sfi_status sfi_dense_attn_append(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
+                                 const sfi_bf16* k_new, const sfi_bf16* v_new, const sfi_bf16* q,
+                                 float* out, const sfi_dense_extras* extras, void* ws, size_t ws_bytes,
+                                 sfi_stream stream) {
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SFI_ERR_INVALID_ARG;
+  const StepToken tok{k_new, v_new};
+  return dense_attn_impl(shape, kv, L, &tok, q, out, extras, ws, ws_bytes, stream);
 }
 
 sfi_status sfi_attn_probs(const sfi_shape* shape, int32_t L, const float* logits, int64_t ld,
@@ -239,18 +273,16 @@ sfi_status sfi_fast_attn(const sfi_shape* shape, const sfi_params* params,
                          const sfi_paged_kv* kv, int32_t L, const sfi_bf16* q,
                          const sfi_packed* packed, float* out, float* lse, void* ws,
                          size_t ws_bytes, sfi_stream stream) {
-  SFI_TRY(check_shape(shape));
-  SFI_TRY(check_params(params));
-  SFI_TRY(check_kv(kv));
-  SFI_TRY(check_sparse_L(shape, params, L));
-  SFI_TRY(check_packed(shape, params, packed));
-  if (!q || !out) return SFI_ERR_INVALID_ARG;
-  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
-  if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
-  const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
-  return run_fast_attn(*shape, *params, *kv, L, q, *packed, out, lse, static_cast<int*>(ws),
-                       reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
-                       (cudaStream_t)stream, nullptr, nullptr);
+  return fast_attn_impl(shape, params, kv, L, nullptr, q, packed, out, lse, ws, ws_bytes, stream);
+}
+
+sfi_status sfi_fast_attn_append(const sfi_shape* shape, const sfi_params* params,
+                                const sfi_paged_kv* kv, int32_t L, const sfi_bf16* k_new,
+                                const sfi_bf16* v_new, const sfi_bf16* q, const sfi_packed* packed,
+                                float* out, float* lse, void* ws, size_t ws_bytes, sfi_stream stream) {
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SFI_ERR_INVALID_ARG;
+  const StepToken tok{k_new, v_new};
+  return fast_attn_impl(shape, params, kv, L, &tok, q, packed, out, lse, ws, ws_bytes, stream);
 }
 
 sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,

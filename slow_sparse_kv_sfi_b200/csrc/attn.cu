@@ -64,6 +64,14 @@ struct AttnArgs {
   int p_max;
   int rec_lo;           // L - n_recent
   int* err;
+  // the step's token, appended at L - 1 by the item holding the last tile
+  // (k_new == nullptr: already in the cache)
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pool;
+  __nv_bfloat16* v_pool;
+  float* norms;
+  int64_t norm_ld;
 };
 
 constexpr int kMaxChunkTiles = 256;
@@ -117,6 +125,7 @@ struct Smem {
 struct Item {
   int bg, b, g;
   int t_begin, t_end;     // tiles of the item
+  int t_total;            // tiles of the whole (b, kv head); the last one holds position L - 1
   int n_packed_tiles;     // tiles before this index are packed-buffer tiles
   int first_page;         // page number of tile n_packed_tiles (fast) or tile 0 (dense)
 };
@@ -130,6 +139,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const i
   it.g = it.bg - it.b * a.Hkv;
   if (MODE != kFast) {
     const int T = (a.L + kPage - 1) / kPage;
+    it.t_total = T;
     it.t_begin = min(T, c * a.chunk_tiles);
     it.t_end = min(T, it.t_begin + a.chunk_tiles);
     it.n_packed_tiles = 0;
@@ -140,6 +150,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const i
     it.n_packed_tiles = (nr + kPage - 1) / kPage;
     it.first_page = a.rec_lo / kPage;
     const int T = it.n_packed_tiles + ((a.L - 1) / kPage - it.first_page + 1);
+    it.t_total = T;
     int ct = (T + a.n_chunks - 1) / a.n_chunks;
     ct = (ct + TPS - 1) / TPS * TPS;
     it.t_begin = min(T, c * ct);
@@ -199,6 +210,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dep_enter();
 
   // ------------------------------------------------------------ producer warp
   if (warp == kConsumerWarps) {
@@ -268,6 +280,14 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
         it = decode_item<MODE, kTPS>(a, item, nrows_s);
         nst = max(1, (it.t_end - it.t_begin + kTPS - 1) / kTPS);
         p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
+        // the item holding position L - 1 first appends the step's token
+        // there (the whole warp), before any copy of that tile is issued
+        if (a.k_new && it.t_begin < it.t_end && it.t_end == it.t_total) {
+          const int pos = a.L - 1;
+          append_row_warp<D>(lane, it.bg, it.g, pos, ptbuf[pos / kPage - p_lo], a.Hkv, a.num_pages, a.k_pool,
+                             a.v_pool, a.k_new, a.v_new, a.norms, a.norm_ld, a.err);
+          __syncwarp();
+        }
       }
       for (int st = 0; st < nst; ++st) {
         bool good = true;
@@ -649,6 +669,7 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
                         float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
                         const int32_t* n_rows, int p_max, int* err, int* ctr) {
+  grid_dep_enter();
   constexpr int kPer = D / 32;
   __shared__ float red[kCombWarps][D + 4];
   __shared__ float mx[kCombWarps];
@@ -741,6 +762,7 @@ __global__ void __launch_bounds__(kCombWarps * 32)
 
 __global__ void probs_kernel(int L, int Hq, const float* __restrict__ logits, int64_t ld,
                              const float* __restrict__ lse, float* __restrict__ probs) {
+  grid_dep_enter();
   const int row = blockIdx.y;
   const float m = lse[row];
   const float* z = logits + (size_t)row * ld;
@@ -809,7 +831,7 @@ sfi_status launch_attn_t(const Maps& maps, const AttnArgs& a, cudaStream_t st) {
     if (!attr.mark(e)) return SFI_ERR_CUDA;
   }
   const int grid = std::min(a.n_items, num_sms() * Plan<D, NT>::kCps);
-  kern<<<grid, kAttnThreads, S::kTotal, st>>>(maps, a);
+  launch_k(kern, dim3(grid), dim3(kAttnThreads), S::kTotal, st, maps, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -829,11 +851,11 @@ sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shap
   const int G = s.Hq / s.Hkv;
   const int grid = s.B * s.Hq;
   if (D == 128)
-    attn_combine_kernel<128><<<grid, kCombWarps * 32, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
-                                                   lse_cand, n_rows, p_max, err, ctr);
+    launch_k(attn_combine_kernel<128>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
+             out, lse, lse_cand, n_rows, p_max, err, ctr);
   else
-    attn_combine_kernel<64><<<grid, kCombWarps * 32, 0, st>>>(part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse,
-                                                  lse_cand, n_rows, p_max, err, ctr);
+    launch_k(attn_combine_kernel<64>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
+             out, lse, lse_cand, n_rows, p_max, err, ctr);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -902,9 +924,24 @@ size_t attn_part_bytes(int n_items, int G, int D) {
   return (size_t)n_items * kConsumerWarps * G * (D + 4) * sizeof(float);
 }
 
+namespace {
+
+void set_token(AttnArgs& a, const sfi_shape& s, const sfi_paged_kv& kv, const StepToken* tok) {
+  if (!tok) return;
+  a.k_new = reinterpret_cast<const __nv_bfloat16*>(tok->k_new);
+  a.v_new = reinterpret_cast<const __nv_bfloat16*>(tok->v_new);
+  a.k_pool = reinterpret_cast<__nv_bfloat16*>(kv.k_pool);
+  a.v_pool = reinterpret_cast<__nv_bfloat16*>(kv.v_pool);
+  a.norms = kv.key_norms;
+  a.norm_ld = (int64_t)s.max_pages * kPage;
+}
+
+}  // namespace
+
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
-                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
+                          const StepToken* tok) {
   const int G = s.Hq / s.Hkv;
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
@@ -926,6 +963,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   a.scale = 1.0f / sqrtf((float)s.D);
   a.scale_log2 = kLog2e * a.scale;
   a.err = kv.err;
+  set_token(a, s, kv, tok);
   const bool extras = ex && (ex->logits || ex->probs || ex->lse_cand);
   float* zbuf = nullptr;
   if (extras) {
@@ -947,7 +985,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
     dim3 grid((L + 1023) / 1024 < 64 ? (L + 1023) / 1024 : 64, s.B * s.Hq);
-    probs_kernel<<<grid, 256, 0, st>>>(L, s.Hq, zbuf, ex->ld, lse_tmp, ex->probs);
+    launch_k(probs_kernel, dim3(grid), dim3(256), 0, st, L, s.Hq, zbuf, ex->ld, lse_tmp, ex->probs);
     if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   }
   return SFI_OK;
@@ -956,7 +994,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end) {
+                         cudaEvent_t ev_end, const StepToken* tok) {
   const int G = s.Hq / s.Hkv;
   if ((long)s.B * s.Hkv > kMaxBH) return SFI_ERR_UNSUPPORTED;
   Maps maps;
@@ -984,6 +1022,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   a.p_max = pk.p_max;
   a.rec_lo = std::max(L - p.n_recent, 0);
   a.err = kv.err;
+  set_token(a, s, kv, tok);
   if (ev_begin) cudaEventRecord(ev_begin, st);
   sfi_status r = launch_attn<kFast>(s.D, G, maps, a, st);
   if (ev_end) cudaEventRecord(ev_end, st);
@@ -995,7 +1034,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,
                           float* probs, cudaStream_t st) {
   dim3 grid((L + 1023) / 1024 < 64 ? (L + 1023) / 1024 : 64, s.B * s.Hq);
-  probs_kernel<<<grid, 256, 0, st>>>(L, s.Hq, logits, ld, lse, probs);
+  launch_k(probs_kernel, dim3(grid), dim3(256), 0, st, L, s.Hq, logits, ld, lse, probs);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

@@ -16,6 +16,21 @@
 
 namespace sfi {
 
+// Programmatic dependent launch.  The library launches its kernels with
+// programmatic stream serialization, so a kernel may be scheduled while the
+// previous kernel on its stream is still running.  Every kernel therefore
+// calls grid_dep_wait() before its first global-memory access (read or
+// write); it returns once the previous kernel has finished and its writes are
+// visible.  grid_dep_launch() lets the next kernel get scheduled early.  Both
+// are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_enter() {
+  grid_dep_wait();
+  grid_dep_launch();
+}
+
+
 constexpr int kPage = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -53,6 +68,12 @@ __device__ __forceinline__ void fence_barrier_init() {
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders this thread's earlier generic-proxy global writes before later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -200,6 +221,54 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Append of one decode token by one warp: row `pos` of (b, kv head h) in the
+// paged cache receives k_new / v_new (bf16 [B, Hkv, D] at row bg = b * Hkv + h),
+// and norms[bg * norm_ld + pos] (when non-null) the fp32 rounding of the
+// fp64-accumulated Euclidean norm of the stored key.  Lane l moves elements
+// [l * D / 32, (l + 1) * D / 32).  A page-table entry outside the pool is
+// latched as SFI_ERR_DEVICE_CHECK and nothing is written; returns whether the
+// row was written.  The writes are fenced for later TMA reads of the row.
+template <int D>
+__device__ __forceinline__ bool append_row_warp(int lane, int bg, int h, int pos, int page, int Hkv, int num_pages,
+                                                __nv_bfloat16* kpool, __nv_bfloat16* vpool,
+                                                const __nv_bfloat16* knew, const __nv_bfloat16* vnew,
+                                                float* norms, int64_t norm_ld, int* err) {
+  static_assert(D == 64 || D == 128, "head dim");
+  if ((unsigned)page >= (unsigned)num_pages) {
+    if (lane == 0) latch_error(err, SFI_ERR_DEVICE_CHECK, kSiteAppend);
+    return false;
+  }
+  constexpr int E = D / 32;
+  const size_t src = (size_t)bg * D + lane * E;
+  const size_t dst = ((size_t)(page * Hkv + h) * kPage + pos % kPage) * D + lane * E;
+  uint32_t kx[E / 2], vx[E / 2];
+  if constexpr (E == 4) {
+    const uint2 k2 = *reinterpret_cast<const uint2*>(knew + src);
+    const uint2 v2 = *reinterpret_cast<const uint2*>(vnew + src);
+    *reinterpret_cast<uint2*>(kpool + dst) = k2;
+    *reinterpret_cast<uint2*>(vpool + dst) = v2;
+    kx[0] = k2.x;
+    kx[1] = k2.y;
+  } else {
+    kx[0] = *reinterpret_cast<const uint32_t*>(knew + src);
+    vx[0] = *reinterpret_cast<const uint32_t*>(vnew + src);
+    *reinterpret_cast<uint32_t*>(kpool + dst) = kx[0];
+    *reinterpret_cast<uint32_t*>(vpool + dst) = vx[0];
+  }
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const float2 f = unpack_bf16x2(kx[i]);
+    ss += (double)f.x * f.x + (double)f.y * f.y;
+  }
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+  if (lane == 0 && norms) norms[(size_t)bg * norm_ld + pos] = (float)sqrt(ss);
+  fence_proxy_async_global();
+  (void)vx;
+  return true;
 }
 
 }  // namespace sfi

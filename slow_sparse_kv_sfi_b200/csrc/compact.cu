@@ -53,6 +53,7 @@ __device__ __forceinline__ uint32_t union_word(const CompactArgs& a, int b, int 
 
 template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactArgs a) {
+  grid_dep_enter();
   __shared__ int wsum[kCThreads / 32];
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactA
 
 template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const CompactArgs a) {
+  grid_dep_enter();
   __shared__ int wtot[kCThreads / 32 + 1];
   __shared__ int base_s, total_s;
   const int bg = blockIdx.y;
@@ -155,6 +157,7 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
 constexpr int kCopyRows = 128;
 
 __global__ void __launch_bounds__(256) compact_copy_kernel(const CompactArgs a) {
+  grid_dep_enter();
   __shared__ int32_t pg[kCopyRows];
   __shared__ int32_t pp[kCopyRows];
   const int bg = blockIdx.y;
@@ -216,6 +219,7 @@ __global__ void __launch_bounds__(256) compact_copy_kernel(const CompactArgs a) 
 __global__ void __launch_bounds__(256) idx_to_bits_kernel(const int32_t* __restrict__ sel, int sel_ld, int K,
                                                           int lo, int nC, uint32_t* bits, int64_t ld_b,
                                                           int* err) {
+  grid_dep_enter();
   const int row = blockIdx.x;
   const int nw = (nC + 31) / 32;
   uint32_t* brow = bits + (size_t)row * ld_b;
@@ -234,10 +238,10 @@ int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
 template <int GM>
 sfi_status launch_compact(const CompactArgs& a, int BH, cudaStream_t st) {
   dim3 grid(a.n_tiles, BH);
-  compact_count_kernel<GM><<<grid, kCThreads, 0, st>>>(a);
-  compact_gather_kernel<GM><<<grid, kCThreads, 0, st>>>(a);
+  launch_k(compact_count_kernel<GM>, dim3(grid), dim3(kCThreads), 0, st, a);
+  launch_k(compact_gather_kernel<GM>, dim3(grid), dim3(kCThreads), 0, st, a);
   dim3 cgrid((a.p_max + kCopyRows - 1) / kCopyRows, BH);
-  compact_copy_kernel<<<cgrid, 256, 0, st>>>(a);
+  launch_k(compact_copy_kernel, dim3(cgrid), dim3(256), 0, st, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -273,7 +277,8 @@ sfi_status run_idx_to_bits(const sfi_shape& s, const sfi_params& p, const sfi_pa
                            const int32_t* sel_idx, int sel_ld, int K, uint32_t* bits, int64_t ld_b,
                            cudaStream_t st) {
   const int nC = L_slow - p.n_recent - p.n_sink;
-  idx_to_bits_kernel<<<s.B * s.Hq, 256, 0, st>>>(sel_idx, sel_ld, K, p.n_sink, nC, bits, ld_b, kv.err);
+  launch_k(idx_to_bits_kernel, dim3(s.B * s.Hq), dim3(256), 0, st, sel_idx, sel_ld, K, p.n_sink, nC, bits, ld_b,
+           kv.err);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

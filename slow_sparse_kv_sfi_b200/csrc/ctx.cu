@@ -42,8 +42,9 @@ struct sfi_ctx {
   uint32_t* rowmm = nullptr;
   int32_t* tile_counts = nullptr;
   size_t tc_bytes = 0;
-  // timing of the attention kernels (kind 0 fast, 1 dense)
-  bool timing = false;
+  // timing of the attention kernels (kind 0 fast, 1 dense) of every
+  // timing-th layer (0: off)
+  int timing = 0;
   std::vector<cudaEvent_t> tev[2];
   size_t tused[2] = {0, 0};
 };
@@ -99,9 +100,9 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
 sfi_status cu(cudaError_t e) { return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA; }
 
 // Event pair for one timed launch, or nulls when timing is off.
-void timing_events(sfi_ctx* c, int kind, cudaEvent_t* b, cudaEvent_t* e) {
+void timing_events(sfi_ctx* c, int kind, int layer, cudaEvent_t* b, cudaEvent_t* e) {
   *b = *e = nullptr;
-  if (!c->timing) return;
+  if (c->timing <= 0 || layer % c->timing != 0) return;
   auto& v = c->tev[kind];
   if (c->tused[kind] + 2 > v.size()) {
     for (int i = 0; i < 256; ++i) {
@@ -205,6 +206,8 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   if (!c || !c->ws) return SFI_ERR_WORKSPACE;
   if (layer < 0 || layer >= c->n_layers || step < 0) return SFI_ERR_INVALID_ARG;
   if (!kv || !packed || !q || !k_new || !v_new || !out || !kv->key_norms) return SFI_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u) != 0)
+    return SFI_ERR_INVALID_ARG;
   if (L < c->p.n_sink + c->p.n_recent + 1 || L > c->s.max_pages * kPage) return SFI_ERR_SHAPE;
   if (packed->p_max < packed_rows_capacity(c->s, c->p)) return SFI_ERR_SHAPE;
   const sfi_shape& s = c->s;
@@ -226,13 +229,13 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
     SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
     c->pending[layer] = 0;
   }
-  SFI_TRY(run_append(s, *kv, L, k_new, v_new, main));
-
+  // the attention launch appends the step's token itself
+  const StepToken tok{k_new, v_new};
   if (!c->cur_slow) {
     cudaEvent_t b, e;
-    timing_events(c, 0, &b, &e);
+    timing_events(c, 0, layer, &b, &e);
     return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, reinterpret_cast<int*>(c->ws), c->part,
-                         c->part_bytes, main, b, e);
+                         c->part_bytes, main, b, e, &tok);
   }
 
   const int buf = layer & 1;
@@ -245,9 +248,9 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   ex.cand_hi = L - p.n_recent;
   {
     cudaEvent_t b, e;
-    timing_events(c, 1, &b, &e);
+    timing_events(c, 1, layer, &b, &e);
     SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
-                           main, b, e));
+                           main, b, e, &tok));
   }
   SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
   cudaStream_t side = c->side;
@@ -283,9 +286,9 @@ sfi_status sfi_ctx_join(sfi_ctx* c, sfi_stream stream) {
   return SFI_OK;
 }
 
-sfi_status sfi_ctx_set_timing(sfi_ctx* c, int32_t enable) {
-  if (!c) return SFI_ERR_INVALID_ARG;
-  c->timing = enable != 0;
+sfi_status sfi_ctx_set_timing(sfi_ctx* c, int32_t layer_stride) {
+  if (!c || layer_stride < 0) return SFI_ERR_INVALID_ARG;
+  c->timing = layer_stride;
   return SFI_OK;
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <utility>
 #include <cstddef>
 #include <cstdint>
 
@@ -33,6 +34,26 @@ struct DeviceOnce {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launches a kernel of the library with programmatic stream serialization:
+// its launch and prologue overlap the tail of the previous kernel on `st`.
+// Every kernel of the library waits for that kernel (grid_dep_wait) before
+// touching global memory, so stream order is kept.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Workspace carving: the per-op calls take one caller-provided buffer.
 struct WsLayout {
   size_t part_off, part_bytes;      // attention split-K partials
@@ -53,13 +74,21 @@ size_t attn_part_bytes(int n_items, int G, int D);
 int packed_rows_capacity(const sfi_shape& s, const sfi_params& p);
 int budget_k(const sfi_params& p, int L);   // -1 if |C| < 1
 
+// The decode step's new token (bf16 [B, Hkv, D] each), appended at L - 1 by
+// the attention launch itself.
+struct StepToken {
+  const sfi_bf16* k_new;
+  const sfi_bf16* v_new;
+};
+
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
-                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end);
+                          size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
+                          const StepToken* tok = nullptr);
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end);
+                         cudaEvent_t ev_end, const StepToken* tok = nullptr);
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld,
                           const float* lse, float* probs, cudaStream_t st);
 

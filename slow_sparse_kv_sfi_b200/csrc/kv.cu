@@ -8,37 +8,21 @@
 
 namespace sfi {
 
-// One CTA per (b, kv head), one thread per element of the row.
-__global__ void append_kernel(int Hkv, int D, int L, int max_pages, int num_pages,
-                              const int32_t* __restrict__ pt, __nv_bfloat16* kpool,
-                              __nv_bfloat16* vpool, const __nv_bfloat16* __restrict__ knew,
-                              const __nv_bfloat16* __restrict__ vnew, float* norms, int64_t norm_ld,
-                              int* err) {
-  __shared__ double wsum[4];
-  const int bg = blockIdx.x;
+// One warp per (b, kv head).
+template <int D>
+__global__ void __launch_bounds__(128) append_kernel(int BH, int Hkv, int L, int max_pages, int num_pages,
+                                                     const int32_t* __restrict__ pt, __nv_bfloat16* kpool,
+                                                     __nv_bfloat16* vpool, const __nv_bfloat16* __restrict__ knew,
+                                                     const __nv_bfloat16* __restrict__ vnew, float* norms,
+                                                     int64_t norm_ld, int* err) {
+  grid_dep_enter();
+  const int bg = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (bg >= BH) return;
   const int b = bg / Hkv, h = bg - b * Hkv;
   const int pos = L - 1;
   const int page = pt[(size_t)b * max_pages + pos / kPage];
-  if ((unsigned)page >= (unsigned)num_pages) {
-    if (threadIdx.x == 0) latch_error(err, SFI_ERR_DEVICE_CHECK, kSiteAppend);
-    return;
-  }
-  const size_t row = ((size_t)(page * Hkv + h) * kPage + pos % kPage) * D;
-  const int t = threadIdx.x;
-  const __nv_bfloat16 k = knew[(size_t)bg * D + t];
-  kpool[row + t] = k;
-  vpool[row + t] = vnew[(size_t)bg * D + t];
-  const double x = (double)__bfloat162float(k);
-  double s = x * x;
-#pragma unroll
-  for (int sh = 16; sh >= 1; sh >>= 1) s += __shfl_xor_sync(0xffffffffu, s, sh);
-  if ((t & 31) == 0) wsum[t >> 5] = s;
-  __syncthreads();
-  if (t == 0) {
-    double tot = 0.0;
-    for (int w = 0; w < D / 32; ++w) tot += wsum[w];
-    if (norms) norms[(size_t)bg * norm_ld + pos] = (float)sqrt(tot);
-  }
+  append_row_warp<D>(threadIdx.x & 31, bg, h, pos, page, Hkv, num_pages, kpool, vpool, knew, vnew, norms, norm_ld,
+                     err);
 }
 
 // One warp per (b, kv head, position) in [lo, hi).
@@ -47,6 +31,7 @@ __global__ void key_norms_kernel(int Hkv, int lo, int hi, int max_pages, int num
                                  const int32_t* __restrict__ pt,
                                  const __nv_bfloat16* __restrict__ kpool, float* norms,
                                  int64_t norm_ld, int* err) {
+  grid_dep_enter();
   const int bg = blockIdx.y;
   const int b = bg / Hkv, h = bg - b * Hkv;
   const int lane = threadIdx.x & 31;
@@ -71,11 +56,19 @@ __global__ void key_norms_kernel(int Hkv, int lo, int hi, int max_pages, int num
 
 sfi_status run_append(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* k_new,
                       const sfi_bf16* v_new, cudaStream_t st) {
-  append_kernel<<<s.B * s.Hkv, s.D, 0, st>>>(
-      s.Hkv, s.D, L, s.max_pages, s.num_pages, kv.page_table,
-      reinterpret_cast<__nv_bfloat16*>(kv.k_pool), reinterpret_cast<__nv_bfloat16*>(kv.v_pool),
-      reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
-      kv.key_norms, (int64_t)s.max_pages * kPage, kv.err);
+  const int BH = s.B * s.Hkv;
+  auto* kp = reinterpret_cast<__nv_bfloat16*>(kv.k_pool);
+  auto* vp = reinterpret_cast<__nv_bfloat16*>(kv.v_pool);
+  const auto* kn = reinterpret_cast<const __nv_bfloat16*>(k_new);
+  const auto* vn = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  const int64_t ld = (int64_t)s.max_pages * kPage;
+  const dim3 grid((BH + 3) / 4);
+  if (s.D == 128)
+    launch_k(append_kernel<128>, grid, dim3(128), 0, st, BH, s.Hkv, L, s.max_pages, s.num_pages, kv.page_table, kp, vp,
+             kn, vn, kv.key_norms, ld, kv.err);
+  else
+    launch_k(append_kernel<64>, grid, dim3(128), 0, st, BH, s.Hkv, L, s.max_pages, s.num_pages, kv.page_table, kp, vp,
+             kn, vn, kv.key_norms, ld, kv.err);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -86,11 +79,11 @@ sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int
   const auto* kp = reinterpret_cast<const __nv_bfloat16*>(kv.k_pool);
   const int64_t ld = (int64_t)s.max_pages * kPage;
   if (s.D == 128)
-    key_norms_kernel<128><<<grid, 256, 0, st>>>(s.Hkv, lo, hi, s.max_pages, s.num_pages,
-                                                kv.page_table, kp, kv.key_norms, ld, kv.err);
+    launch_k(key_norms_kernel<128>, dim3(grid), dim3(256), 0, st, s.Hkv, lo, hi, s.max_pages, s.num_pages,
+             kv.page_table, kp, kv.key_norms, ld, kv.err);
   else
-    key_norms_kernel<64><<<grid, 256, 0, st>>>(s.Hkv, lo, hi, s.max_pages, s.num_pages,
-                                               kv.page_table, kp, kv.key_norms, ld, kv.err);
+    launch_k(key_norms_kernel<64>, dim3(grid), dim3(256), 0, st, s.Hkv, lo, hi, s.max_pages, s.num_pages,
+             kv.page_table, kp, kv.key_norms, ld, kv.err);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

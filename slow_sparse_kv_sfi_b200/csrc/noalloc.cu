@@ -41,7 +41,10 @@ sfi_status scratch_address(void** out) {
   return SFI_OK;
 }
 
-__global__ void zero_counter_kernel(int* ctr) { ctr[0] = 0; }
+__global__ void zero_counter_kernel(int* ctr) {
+  grid_dep_enter();
+  ctr[0] = 0;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -84,7 +87,7 @@ extern "C" sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_p
   int* ctr = reinterpret_cast<int*>(b);
   cudaStream_t st = (cudaStream_t)stream;
   // the area keeps whatever the last call left: the work counter must start at zero
-  zero_counter_kernel<<<1, 1, 0, st>>>(ctr);
+  launch_k(zero_counter_kernel, dim3(1), dim3(1), 0, st, ctr);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   return run_dense_attn(s, *kv, L, q, out, extras, ctr, reinterpret_cast<float*>(b + kCounterBytes), part_cap, st,
                         nullptr, nullptr);

@@ -77,6 +77,7 @@ __device__ __forceinline__ float nbar_of(double sum_norms, int nC) { return (flo
 __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC, const float* __restrict__ norms,
                                                                   int64_t norm_ld, double* part, int nch,
                                                                   uint32_t* rowmm, int G) {
+  grid_dep_enter();
   __shared__ double red[32];
   const int bg = blockIdx.y;
   if (rowmm && blockIdx.x == 0 && threadIdx.x < G) {   // the score kernel folds into these
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC
 __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
                                                                    const float* __restrict__ norms,
                                                                    int64_t norm_ld, double* part, int nch) {
+  grid_dep_enter();
   __shared__ double red[32];
   __shared__ double bc;
   const int bg = blockIdx.y;
@@ -133,6 +135,7 @@ struct ScoreArgs {
 // and writes l''; it also folds the order keys into per-row min / max.
 template <int GM>
 __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
+  grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
   float* ell = sm;                    // [G][W]
@@ -341,6 +344,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(int n, const float* 
                                                             int32_t* __restrict__ idx, int64_t ld_i,
                                                             uint32_t* __restrict__ bits, int64_t ld_b,
                                                             const uint32_t* __restrict__ rowmm) {
+  grid_dep_enter();
   extern __shared__ uint32_t tsm[];
   const int nw = (n + 31) / 32;
   uint32_t* sel = tsm;                           // [nw]
@@ -535,7 +539,7 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
       !attr.mark(cudaFuncSetAttribute(select_scores_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       200 * 1024)))
     return SFI_ERR_CUDA;
-  select_scores_kernel<GM><<<grid, 256, smem, st>>>(a);
+  launch_k(select_scores_kernel<GM>, dim3(grid), dim3(256), smem, st, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -550,8 +554,9 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   const int nch = stat_chunks(nC);
   const int64_t norm_ld = (int64_t)s.max_pages * kPage;
   dim3 sgrid(nch, s.B * s.Hkv);
-  stats_norm_kernel<<<sgrid, kStatThreads, 0, st>>>(lo, nC, kv.key_norms, norm_ld, part, nch, rowmm, G);
-  stats_prior_kernel<<<sgrid, kStatThreads, 0, st>>>(L, lo, nC, kv.key_norms, norm_ld, part, nch);
+  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch, rowmm,
+           G);
+  launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
@@ -586,7 +591,8 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
       !attr.mark(cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)topk_smem(topk_max_n()))))
     return SFI_ERR_CUDA;
-  topk_kernel<false><<<rows, kTopkThreads, smem, st>>>(n, scores, ld_s, K, offset, idx, ld_i, bits, ld_b, rowmm);
+  launch_k(topk_kernel<false>, dim3(rows), dim3(kTopkThreads), smem, st, n, scores, ld_s, K, offset, idx, ld_i, bits,
+           ld_b, rowmm);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

@@ -75,9 +75,11 @@ def _declare(L):
         "sfi_append_kv": (C.c_int, [P, P, I32, P, P, P]),
         "sfi_key_norms": (C.c_int, [P, P, I32, I32, P]),
         "sfi_dense_attn": (C.c_int, [P, P, I32, P, P, P, P, SZ, P]),
+        "sfi_dense_attn_append": (C.c_int, [P, P, I32, P, P, P, P, P, P, SZ, P]),
         "sfi_dense_attn_noalloc": (C.c_int, [P, P, I32, P, P, P, P]),
         "sfi_attn_probs": (C.c_int, [P, I32, P, I64, P, P, P]),
         "sfi_fast_attn": (C.c_int, [P, P, P, I32, P, P, P, P, P, SZ, P]),
+        "sfi_fast_attn_append": (C.c_int, [P, P, P, I32, P, P, P, P, P, P, P, SZ, P]),
         "sfi_select_scores": (C.c_int, [P, P, P, I32, P, I64, P, P, P, SZ, P]),
         "sfi_topk": (C.c_int, [I32, I32, P, I64, I32, I32, P, I64, P]),
         "sfi_select": (C.c_int, [P, P, P, I32, P, I64, P, P, I32, C.POINTER(I32), P, SZ, P]),
@@ -99,8 +101,8 @@ def _declare(L):
 
 
 EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_rows", "sfi_budget",
-            "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_noalloc",
-            "sfi_attn_probs", "sfi_fast_attn",
+            "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_append",
+            "sfi_dense_attn_noalloc", "sfi_attn_probs", "sfi_fast_attn", "sfi_fast_attn_append",
             "sfi_select_scores", "sfi_topk", "sfi_select", "sfi_compact", "sfi_poll_error",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
             "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_timing"]
@@ -186,6 +188,14 @@ def sfi_dense_attn(shape, kv, L, q, out, ws, extras: Optional[DenseExtras] = Non
            "sfi_dense_attn")
 
 
+def sfi_dense_attn_append(shape, kv, L, k_new, v_new, q, out, ws, extras: Optional[DenseExtras] = None,
+                          stream=None):
+    """sfi_append_kv + sfi_dense_attn in one launch."""
+    _check(lib().sfi_dense_attn_append(C.byref(shape), C.byref(kv), L, _p(k_new), _p(v_new), _p(q), _p(out),
+                                       _ref(extras), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "sfi_dense_attn_append")
+
+
 def sfi_dense_attn_noalloc(shape, kv, L, q, out, extras: Optional[DenseExtras] = None, stream=None):
     """sfi_dense_attn with its scratch in the library's static device array
     (no workspace, nothing allocated)."""
@@ -202,6 +212,13 @@ def sfi_fast_attn(shape, params, kv, L, q, packed, out, ws, lse=None, stream=Non
     _check(lib().sfi_fast_attn(C.byref(shape), C.byref(params), C.byref(kv), L, _p(q), C.byref(packed),
                                _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(),
                                _stream(stream)), "sfi_fast_attn")
+
+
+def sfi_fast_attn_append(shape, params, kv, L, k_new, v_new, q, packed, out, ws, lse=None, stream=None):
+    """sfi_append_kv + sfi_fast_attn in one launch."""
+    _check(lib().sfi_fast_attn_append(C.byref(shape), C.byref(params), C.byref(kv), L, _p(k_new), _p(v_new),
+                                      _p(q), C.byref(packed), _p(out), _p(lse), _p(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)), "sfi_fast_attn_append")
 
 
 def sfi_select_scores(shape, params, kv, L, logits, ld, lse_cand, scores, ws, stream=None):
@@ -261,8 +278,9 @@ class Context:
     def join(self, stream=None):
         _check(lib().sfi_ctx_join(self.h, _stream(stream)), "sfi_ctx_join")
 
-    def set_timing(self, enable: bool):
-        _check(lib().sfi_ctx_set_timing(self.h, int(enable)), "sfi_ctx_set_timing")
+    def set_timing(self, layer_stride: int):
+        """Time the attention launches of layers 0, n, 2n, ... (n = layer_stride; 0 = off)."""
+        _check(lib().sfi_ctx_set_timing(self.h, int(layer_stride)), "sfi_ctx_set_timing")
 
     def timing(self, kind: int, reset: bool = True):
         ms = C.c_double(0)
