@@ -139,10 +139,11 @@ const char* sfi_version(void);
 
 /* Bytes of scratch the per-op calls below need for contexts up to
  * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes
- * (16-byte aligned).  Ownership stays with the caller.  The first 256 bytes
- * hold a work counter of the attention kernels: they must be zero before the
- * first call, and every call leaves them zero.  Calls that share one ws must
- * not run concurrently. */
+ * (16-byte aligned).  Ownership stays with the caller.  The scratch must be
+ * zero-filled before its first use (the first 256 bytes hold a work counter
+ * of the attention kernels, other parts the top-K histograms); every
+ * successful call leaves it ready for the next one (after an error, zero it
+ * again).  Calls that share one ws must not run concurrently. */
 sfi_status sfi_workspace_size(const sfi_shape* shape, const sfi_params* params, size_t* bytes);
 
 /* Packed-buffer row capacity p_max needed for contexts up to max_pages*16:
@@ -238,11 +239,19 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
                              const float* lse_cand, float* scores, void* ws, size_t ws_bytes,
                              sfi_stream stream);
 
-/* Per-row top-K: the K largest of scores[r, 0:n] (ties -> lower index),
- * written ascending as idx[r, 0:K] = offset + column.  rows = number of rows;
- * scores row stride ld_s, idx row stride ld_i (elements). */
+/* Per-row top-K: the K largest of scores[r, 0:n] (finite values; ties ->
+ * lower index), written ascending as idx[r, 0:K] = offset + column.  rows =
+ * number of rows; scores row stride ld_s, idx row stride ld_i (elements);
+ * n <= 262144.  ws: device scratch of sfi_topk_workspace_size bytes, 16-byte
+ * aligned, zero-filled before its first use; every successful call leaves it
+ * ready for the next one (after an error, zero it again).  Every row is cut
+ * into slices with one CTA each: a histogram of linear bins over the row's
+ * [min, max], the boundary bin of the K-th score, an exact radix select of
+ * the threshold among the boundary candidates, ties in position order. */
+sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes);
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
-                    int32_t offset, int32_t* idx, int64_t ld_i, sfi_stream stream);
+                    int32_t offset, int32_t* idx, int64_t ld_i, void* ws, size_t ws_bytes,
+                    sfi_stream stream);
 
 /* Full Selector = sfi_select_scores + sfi_topk.  sel_idx int32 [B, Hq, sel_ld]
  * receives K ascending absolute positions per query head; *K_out = K. */

@@ -50,6 +50,8 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   const int Lmax = s.max_pages * kPage;
   const long dense_chunks = dense_chunks_bound(s);
   const int kmax = std::max(budget_k(p, Lmax), 0);
+  // the fast step's chunk count grows with the expected selection size, which
+  // is largest at L_max
   const long fast_items = bh * fast_chunks(s, packed_rows_capacity(s, p), p.n_recent, kmax + p.n_sink);
   const long items = std::max(bh * dense_chunks, fast_items);
   size_t off = 256;   // first 256 bytes reserved
@@ -70,9 +72,9 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   w.bits_off = off;
   w.bits_bytes = align_up((size_t)s.B * s.Hq * w.bits_ld * sizeof(uint32_t), 256);
   off += w.bits_bytes;
-  w.mm_off = off;
-  w.mm_bytes = align_up((size_t)s.B * s.Hq * 2 * sizeof(uint32_t), 256);
-  off += w.mm_bytes;
+  w.tk_off = off;
+  w.tk_bytes = align_up(topk_scratch_bytes(s.B * s.Hq, (int)std::min<long>(nC, topk_max_n())), 256);
+  off += w.tk_bytes;
   w.total = off;
   return w;
 }
@@ -298,17 +300,27 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
   if (!ws || ws_bytes < w.total) return SFI_ERR_WORKSPACE;
   const int nC = L - params->n_recent - params->n_sink;
   return run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, nC,
-                           static_cast<char*>(ws) + w.stat_off,
-                           reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.mm_off),
-                           (cudaStream_t)stream);
+                           static_cast<char*>(ws) + w.stat_off, (cudaStream_t)stream);
+}
+
+sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes) {
+  if (!bytes) return SFI_ERR_INVALID_ARG;
+  if (rows < 0 || n < 1) return SFI_ERR_SHAPE;
+  if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
+  *bytes = topk_scratch_bytes(rows, n);
+  return SFI_OK;
 }
 
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
-                    int32_t offset, int32_t* idx, int64_t ld_i, sfi_stream stream) {
+                    int32_t offset, int32_t* idx, int64_t ld_i, void* ws, size_t ws_bytes,
+                    sfi_stream stream) {
   if (!scores || !idx) return SFI_ERR_INVALID_ARG;
   if (rows < 0 || n < 1 || K < 1 || K > n || ld_s < n || ld_i < K) return SFI_ERR_SHAPE;
   if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, nullptr, 0, nullptr, (cudaStream_t)stream);
+  if (!ws || !aligned16(ws) || ws_bytes < topk_scratch_bytes(rows, n))
+    return SFI_ERR_WORKSPACE;
+  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, nullptr, 0, topk_scratch(ws, rows, n),
+                  (cudaStream_t)stream);
 }
 
 sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
@@ -329,12 +341,12 @@ sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sf
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + w.sel_off);
   const int ld_s = (nC + 3) / 4 * 4;
   cudaStream_t st = (cudaStream_t)stream;
-  uint32_t* mm = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.mm_off);
   if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
   SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s,
-                            static_cast<char*>(ws) + w.stat_off, mm, st));
-  SFI_TRY(run_topk(shape->B * shape->Hq, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0,
-                   mm, st));
+                            static_cast<char*>(ws) + w.stat_off, st));
+  const int rows = shape->B * shape->Hq;
+  SFI_TRY(run_topk(rows, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0,
+                   topk_scratch(static_cast<char*>(ws) + w.tk_off, rows, nC), st));
   if (K_out) *K_out = K;
   return SFI_OK;
 }

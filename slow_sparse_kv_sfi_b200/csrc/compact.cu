@@ -12,8 +12,8 @@
 // thread owns one word: the OR of the group's words is the union, its
 // popcount the row count.  compact_count writes the per-tile counts;
 // compact_gather scans them and writes positions, head masks and n_rows;
-// compact_copy then copies the K and V rows in 16-byte units, eight loads in
-// flight per thread, over fixed 128-row blocks (the selection is far from
+// compact_copy then copies the K and V rows, one warp per row, eight rows in
+// flight per warp, over fixed 128-row blocks (the selection is far from
 // uniform over positions, so per-tile copying would be imbalanced).
 #include "common.cuh"
 #include "internal.h"
@@ -153,13 +153,23 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
 // Copy the K and V rows of the packed buffer from the pages (rows past
 // n_rows up to the next multiple of 16: zeros).  Grid: 128-row blocks of
 // every (b, KV head); blocks past the rows in use return at once, so the
-// copy work is spread evenly whatever the selection looks like.
+// copy work is spread evenly whatever the selection looks like.  A warp moves
+// whole rows: for D = 128 lanes 0-15 carry the K row and lanes 16-31 the V
+// row (16 bytes each), for D = 64 one warp pass moves two rows; eight passes
+// are in flight per warp.
 constexpr int kCopyRows = 128;
+constexpr int kCopyWarps = 8;
 
-__global__ void __launch_bounds__(256) compact_copy_kernel(const CompactArgs a) {
+template <int D>
+__global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const CompactArgs a) {
   grid_dep_enter();
-  __shared__ int32_t pg[kCopyRows];
-  __shared__ int32_t pp[kCopyRows];
+  constexpr int kUnits = D / 8;                 // 16-byte units of one K (or V) row
+  constexpr int kRowUnits = 2 * kUnits;         // K then V
+  constexpr int kRowsPerPass = 32 / kRowUnits;  // rows one warp moves per pass
+  constexpr int kRowsPerWarp = kCopyRows / kCopyWarps;
+  constexpr int kIn = 8;                        // passes in flight
+  static_assert(kRowsPerWarp % (kIn * kRowsPerPass) == 0 || kRowsPerWarp == kIn * kRowsPerPass, "copy plan");
+  __shared__ long long src[kCopyRows];          // unit offset of the row in the pools, -1: zero row
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
   const int n = min(max(a.n_rows[bg], 0), a.p_max);
@@ -168,54 +178,45 @@ __global__ void __launch_bounds__(256) compact_copy_kernel(const CompactArgs a) 
   if (r0 >= pad_end) return;
   const int nr = min(kCopyRows, pad_end - r0);
   const int32_t* pos = a.pos + (size_t)bg * a.p_max;
-  if (threadIdx.x < nr) {
+  if (threadIdx.x < kCopyRows) {
     const int r = r0 + threadIdx.x;
-    int page = -1, p = 0;
-    if (r < n) {
-      p = pos[r];
+    long long off = -1;
+    if (threadIdx.x < nr && r < n) {
+      const int p = pos[r];
       const int pi = p / kPage;
+      int page = -1;
       if (p >= 0 && pi < a.max_pages) page = __ldg(a.pt + (size_t)b * a.max_pages + pi);
-      if ((unsigned)page >= (unsigned)a.num_pages) {
-        latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
-        page = -1;
-      }
+      if ((unsigned)page >= (unsigned)a.num_pages) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
+      else off = ((long long)(page * a.Hkv + g) * kPage + p % kPage) * kUnits;
     }
-    pg[threadIdx.x] = page;
-    pp[threadIdx.x] = p;
+    src[threadIdx.x] = off;
   }
   __syncthreads();
-  const int chunks = a.D / 8;
-  const int upr = 2 * chunks;
-  const int nunits = nr * upr;
-  const size_t dst0 = ((size_t)bg * a.p_max + r0) * chunks;
-  for (int u0 = threadIdx.x; u0 < nunits; u0 += 8 * 256) {
-    uint4 v[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / kRowUnits;             // row of the pass
+  const int u = lane % kRowUnits;
+  const bool isv = u >= kUnits;
+  const int cu = isv ? u - kUnits : u;
+  const uint4* from = isv ? a.vpool : a.kpool;
+  uint4* to = isv ? a.pv : a.pk;
+  const size_t dst0 = ((size_t)bg * a.p_max + r0) * kUnits + cu;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int un = u0 + k * 256;
-      v[k] = make_uint4(0, 0, 0, 0);
-      if (un < nunits) {
-        const int i = un / upr, c = un - i * upr;
-        const int page = pg[i];
-        if (page >= 0) {
-          const size_t src = ((size_t)(page * a.Hkv + g) * kPage + pp[i] % kPage) * chunks;
-          v[k] = (c < chunks) ? __ldg(a.kpool + src + c) : __ldg(a.vpool + src + c - chunks);
-        }
-      }
+  for (int i0 = 0; i0 < kRowsPerWarp; i0 += kIn * kRowsPerPass) {
+    uint4 v[kIn];
+#pragma unroll
+    for (int k = 0; k < kIn; ++k) {
+      const int r = warp * kRowsPerWarp + i0 + k * kRowsPerPass + sub;
+      const long long off = (r < nr) ? src[r] : -1;
+      v[k] = off >= 0 ? __ldg(from + off + cu) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int un = u0 + k * 256;
-      if (un < nunits) {
-        const int i = un / upr, c = un - i * upr;
-        if (c < chunks) a.pk[dst0 + (size_t)i * chunks + c] = v[k];
-        else a.pv[dst0 + (size_t)i * chunks + c - chunks] = v[k];
-      }
+    for (int k = 0; k < kIn; ++k) {
+      const int r = warp * kRowsPerWarp + i0 + k * kRowsPerPass + sub;
+      if (r < nr) to[dst0 + (size_t)r * kUnits] = v[k];
     }
   }
 }
 
-// Selections as ascending positions -> one bitmap per query head.
 __global__ void __launch_bounds__(256) idx_to_bits_kernel(const int32_t* __restrict__ sel, int sel_ld, int K,
                                                           int lo, int nC, uint32_t* bits, int64_t ld_b,
                                                           int* err) {
@@ -241,7 +242,8 @@ sfi_status launch_compact(const CompactArgs& a, int BH, cudaStream_t st) {
   launch_k(compact_count_kernel<GM>, dim3(grid), dim3(kCThreads), 0, st, a);
   launch_k(compact_gather_kernel<GM>, dim3(grid), dim3(kCThreads), 0, st, a);
   dim3 cgrid((a.p_max + kCopyRows - 1) / kCopyRows, BH);
-  launch_k(compact_copy_kernel, dim3(cgrid), dim3(256), 0, st, a);
+  if (a.D == 128) launch_k(compact_copy_kernel<128>, cgrid, dim3(kCopyWarps * 32), 0, st, a);
+  else launch_k(compact_copy_kernel<64>, cgrid, dim3(kCopyWarps * 32), 0, st, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 

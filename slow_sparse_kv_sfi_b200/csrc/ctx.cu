@@ -39,7 +39,7 @@ struct sfi_ctx {
   float* scores = nullptr;
   uint32_t* bits = nullptr;
   int64_t bits_ld = 0;
-  uint32_t* rowmm = nullptr;
+  char* topk_ws = nullptr;
   int32_t* tile_counts = nullptr;
   size_t tc_bytes = 0;
   // timing of the attention kernels (kind 0 fast, 1 dense) of every
@@ -54,7 +54,7 @@ namespace {
 
 struct CtxLayout {
   size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, stat_off, stat_bytes, score_off,
-      score_bytes, bits_off, bits_bytes, mm_off, mm_bytes, tc_off, tc_bytes, total;
+      score_bytes, bits_off, bits_bytes, tc_off, tc_bytes, tk_off, tk_bytes, total;
   int64_t bits_ld;
 };
 
@@ -81,12 +81,12 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
   c.bits_bytes = w.bits_bytes;
   c.bits_ld = w.bits_ld;
   off += c.bits_bytes;
-  c.mm_off = off;
-  c.mm_bytes = w.mm_bytes;
-  off += c.mm_bytes;
   c.tc_off = off;
   c.tc_bytes = w.cmp_bytes;
   off += c.tc_bytes;
+  c.tk_off = off;
+  c.tk_bytes = w.tk_bytes;
+  off += c.tk_bytes;
   c.total = off;
   return c;
 }
@@ -177,8 +177,10 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   const CtxLayout l = ctx_layout(c->s, c->p);
   if (bytes < l.total) return SFI_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
-  // the first 256 bytes hold the attention kernels' work counter: zero it once
+  // the attention kernels' work counter (first 256 bytes) and the top-K
+  // state start at zero; every step leaves them so
   if (cudaMemset(w, 0, 256) != cudaSuccess) return SFI_ERR_CUDA;
+  if (cudaMemset(w + l.tk_off, 0, l.tk_bytes) != cudaSuccess) return SFI_ERR_CUDA;
   c->ws = w;
   c->ws_bytes = bytes;
   c->part = reinterpret_cast<float*>(w + l.part_off);
@@ -193,8 +195,8 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   c->scores = reinterpret_cast<float*>(w + l.score_off);
   c->bits = reinterpret_cast<uint32_t*>(w + l.bits_off);
   c->bits_ld = l.bits_ld;
-  c->rowmm = reinterpret_cast<uint32_t*>(w + l.mm_off);
   c->tile_counts = reinterpret_cast<int32_t*>(w + l.tc_off);
+  c->topk_ws = w + l.tk_off;
   c->tc_bytes = l.tc_bytes;
   return SFI_OK;
 }
@@ -261,10 +263,10 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   const int ld_s = (nC + 3) / 4 * 4;
   if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
   SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                            c->stats, c->rowmm, side));
+                            c->stats, side));
   SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, c->rowmm,
-                   side));
+  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld,
+                   topk_scratch(c->topk_ws, s.B * s.Hq, nC), side));
   SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->tile_counts, c->tc_bytes, L, side));
   SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
   if (c->overlap) {

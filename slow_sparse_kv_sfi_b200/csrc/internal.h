@@ -61,7 +61,7 @@ struct WsLayout {
   size_t stat_off, stat_bytes;
   size_t cmp_off, cmp_bytes;        // compaction tile counts
   size_t bits_off, bits_bytes;      // selection bitmaps [B*Hq][bits_ld]
-  size_t mm_off, mm_bytes;          // per-row min / max keys of the scores
+  size_t tk_off, tk_bytes;          // top-K scratch (zero before the first call)
   int64_t bits_ld;
   size_t total;
 };
@@ -99,11 +99,24 @@ sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int
 
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
-                             float* scores, int64_t ld_s, void* stat_ws, uint32_t* rowmm,
+                             float* scores, int64_t ld_s, void* stat_ws,
                              cudaStream_t st);
-sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset,
-                    int32_t* idx, int64_t ld_i, uint32_t* bits, int64_t ld_b, const uint32_t* rowmm,
-                    cudaStream_t st);
+// Scratch of the top-K kernels for `rows` rows of n scores (topk.cu).  ghist
+// and done must be zero before the first call; every call leaves them zero.
+struct TopkScratch {
+  int* ghist;         // [rows][4096] digit histogram
+  int* done;          // [rows] arrival counter of the digit kernels
+  int* info;          // [rows][4] threshold prefix, scores to take, digit mask
+  uint32_t* ties;     // [rows][words_ld] scores equal to the threshold
+  uint32_t* bits;     // [rows][words_ld] bitmap when the caller wants positions only
+  int64_t words_ld;
+};
+size_t topk_scratch_bytes(int rows, int n);
+TopkScratch topk_scratch(void* base, int rows, int n);
+// K largest of every row (ties to the lower index): bitmap bits[rows][ld_b]
+// and / or ascending positions idx[rows][ld_i] (+ offset).
+sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
+                    int64_t ld_i, uint32_t* bits, int64_t ld_b, const TopkScratch& w, cudaStream_t st);
 int topk_max_n();
 sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                             const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,

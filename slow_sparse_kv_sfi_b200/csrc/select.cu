@@ -17,10 +17,7 @@
 // partials in the same fixed order), select_scores (one CTA per (b, kv group,
 // candidate tile) holding all G heads plus a halo of w on each side in shared
 // memory, so soft-NMS and the cross-head owner need no second pass over
-// memory; it also records each row's min and max), topk_kernel (one CTA per
-// row: linear bins over [min, max], boundary-bin candidates resolved exactly
-// by MSB radix select on order-preserving uint32 keys, ties by position; a
-// selection bitmap and / or ascending positions out).
+// memory); the top-K follows in topk.cu.
 #include <algorithm>
 
 #include "common.cuh"
@@ -75,15 +72,10 @@ __device__ __forceinline__ float nbar_of(double sum_norms, int nC) { return (flo
 
 // part[bg][chunk][0] = sum of key norms over the chunk of C
 __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC, const float* __restrict__ norms,
-                                                                  int64_t norm_ld, double* part, int nch,
-                                                                  uint32_t* rowmm, int G) {
+                                                                  int64_t norm_ld, double* part, int nch) {
   grid_dep_enter();
   __shared__ double red[32];
   const int bg = blockIdx.y;
-  if (rowmm && blockIdx.x == 0 && threadIdx.x < G) {   // the score kernel folds into these
-    rowmm[((size_t)bg * G + threadIdx.x) * 2] = 0xffffffffu;
-    rowmm[((size_t)bg * G + threadIdx.x) * 2 + 1] = 0u;
-  }
   const float* n = norms + (size_t)bg * norm_ld + lo;
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double sacc = 0.0;
@@ -125,14 +117,13 @@ struct ScoreArgs {
   int nch;
   float* scores;
   int64_t ld_s;
-  uint32_t* rowmm;           // [B*Hq][2]: min / max order key of each score row
 };
 
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes the log-score
 // of every head of the group over the tile plus a halo of w on each side to
 // shared memory (NaN outside C: a NaN never dominates).  Phase 2: the thread
 // of a position applies soft-NMS to every head in registers, picks the owner
-// and writes l''; it also folds the order keys into per-row min / max.
+// and writes l''.
 template <int GM>
 __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   grid_dep_enter();
@@ -153,36 +144,47 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   const size_t row0 = (size_t)b * a.Hq + (size_t)g * G;
   const float* z0 = a.logits + row0 * a.ld + a.lo;
   const float nan = __int_as_float(0x7fc00000);
-  for (int k = threadIdx.x; k < W; k += blockDim.x) {
-    const int c = c0 - a.w + k;
-    if (c >= 0 && c < a.nC) {
-      const int j = a.lo + c;
-      const float r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * inv_z;
-      float zv[GM];
+  float lsec[GM];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) zv[h] = (h < G) ? z0[(size_t)h * a.ld + c] : 0.f;
+  for (int h = 0; h < GM; ++h) lsec[h] = (h < G) ? a.lse_cand[row0 + h] : 0.f;
+  // kU positions per thread and round: all their loads are issued first
+  constexpr int kU = GM >= 8 ? 2 : 4;
+  for (int k0 = threadIdx.x; k0 < W; k0 += kU * blockDim.x) {
+    float nv[kU], zv[kU][GM];
+    bool in[kU];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-          const float ft = expf(zv[h] - a.lse_cand[row0 + h]);
-          const float s = (1.f - lam) * ft + lam * r;
-          ell[h * W + k] = logf(s + 1e-30f);
+    for (int u = 0; u < kU; ++u) {
+      const int c = c0 - a.w + k0 + u * blockDim.x;
+      in[u] = k0 + u * blockDim.x < W && c >= 0 && c < a.nC;
+      const int cc = in[u] ? c : 0;
+      nv[u] = in[u] ? nrm[a.lo + cc] : 1.f;
+#pragma unroll
+      for (int h = 0; h < GM; ++h) zv[u][h] = (in[u] && h < G) ? z0[(size_t)h * a.ld + cc] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int k = k0 + u * blockDim.x;
+      if (k >= W) continue;
+      if (in[u]) {
+        const int j = a.lo + c0 - a.w + k;
+        const float r = kappa_of(nbar, nv[u]) * pi_of(a.L, j) * inv_z;
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          if (h < G) {
+            const float ft = expf(zv[u][h] - lsec[h]);
+            const float sv = (1.f - lam) * ft + lam * r;
+            ell[h * W + k] = logf(sv + 1e-30f);
+          }
         }
-      }
-    } else {
+      } else {
 #pragma unroll
-      for (int h = 0; h < GM; ++h)
-        if (h < G) ell[h * W + k] = nan;
+        for (int h = 0; h < GM; ++h)
+          if (h < G) ell[h * W + k] = nan;
+      }
     }
   }
   __syncthreads();
   const float inv_w = 1.f / (float)a.w;
-  uint32_t kmin[GM], kmax[GM];
-#pragma unroll
-  for (int h = 0; h < GM; ++h) {
-    kmin[h] = 0xffffffffu;
-    kmax[h] = 0u;
-  }
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
     float l1[GM];
 #pragma unroll
@@ -214,323 +216,17 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
       if (h < G) {
         const float v = l1[h] - (h != owner ? a.alpha_cross : 0.f);
         a.scores[(row0 + h) * a.ld_s + c0 + k] = v;
-        const uint32_t key = float_key(v);
-        kmin[h] = min(kmin[h], key);
-        kmax[h] = max(kmax[h], key);
-      }
-    }
-  }
-  if (a.rowmm) {
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      if (h >= G) continue;
-      uint32_t mn = kmin[h], mx = kmax[h];
-#pragma unroll
-      for (int sh = 16; sh >= 1; sh >>= 1) {
-        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, sh));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
-      }
-      if ((threadIdx.x & 31) == 0) {
-        atomicMin(&a.rowmm[(row0 + h) * 2], mn);
-        atomicMax(&a.rowmm[(row0 + h) * 2 + 1], mx);
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- top-K
-constexpr int kTopkThreads = 1024;
-constexpr int kBins = 4096;       // first digit: linear bins over [min, max] of the row
-constexpr int kRBins = 2048;      // exact radix digits (11 bits)
-constexpr int kCap = 4096;        // boundary-bin candidates resolved in shared memory
-constexpr int kTopkMaxWords = 8192;
-
-// Reverse (suffix) inclusive scan of one value per thread across the block.
-__device__ __forceinline__ int block_suffix_incl(int v, int* wtot) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int sh = 1; sh < 32; sh <<= 1) {
-    const int y = __shfl_down_sync(0xffffffffu, x, sh);
-    if (lane + sh < 32) x += y;
-  }
-  if (lane == 0) wtot[w] = x;   // total of this warp
-  __syncthreads();
-  if (w == 0) {
-    const int nwarps = blockDim.x >> 5;
-    int t = lane < nwarps ? wtot[lane] : 0;
-    int s = t;
-#pragma unroll
-    for (int sh = 1; sh < 32; sh <<= 1) {
-      const int y = __shfl_down_sync(0xffffffffu, s, sh);
-      if (lane + sh < 32) s += y;
-    }
-    wtot[32 + lane] = s - t;      // sum of warps after this one
-  }
-  __syncthreads();
-  const int r = x + wtot[32 + w];
-  __syncthreads();
-  return r;
-}
-
-// Exclusive prefix scan of one value per thread across the block.
-__device__ __forceinline__ int block_prefix_excl(int v, int* wtot, int* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int sh = 1; sh < 32; sh <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, sh);
-    if (lane >= sh) x += y;
-  }
-  if (lane == 31) wtot[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    const int nwarps = blockDim.x >> 5;
-    const int t = lane < nwarps ? wtot[lane] : 0;
-    int s = t;
-#pragma unroll
-    for (int sh = 1; sh < 32; sh <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, sh);
-      if (lane >= sh) s += y;
-    }
-    wtot[32 + lane] = s - t;
-    if (lane == 31) *total = s;
-  }
-  __syncthreads();
-  const int r = x - v + wtot[32 + w];
-  __syncthreads();
-  return r;
-}
-
-__device__ __forceinline__ float key_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Bin b of `hist` (nb bins, held 1024 / nb... by the block) containing the
-// k-th largest element counted from the top: sets *bin and *above (elements
-// in higher bins).  Each thread owns nb / blockDim consecutive bins.
-__device__ __forceinline__ void find_bin(const int* hist, int nb, int k, int* wtot, int* s_bin,
-                                         int* s_above) {
-  const int per = nb / blockDim.x;
-  const int b0 = threadIdx.x * per;
-  int mine = 0;
-  for (int i = 0; i < per; ++i) mine += hist[b0 + i];
-  const int incl = block_suffix_incl(mine, wtot);
-  int above = incl - mine;   // bins after this thread's
-  for (int i = per - 1; i >= 0; --i) {
-    const int h = hist[b0 + i];
-    if (above < k && above + h >= k) {
-      *s_bin = b0 + i;
-      *s_above = above;
-    }
-    above += h;
-  }
-  __syncthreads();
-}
-
-// One CTA per row: the K largest scores (ties to the lower index) as a
-// selection bitmap and / or K ascending positions.
-//  1. linear bins over [min, max] of the row (from the score kernel, or one
-//     extra pass): histogram, the boundary bin and how many to take from it;
-//  2. one pass: elements above the boundary bin are selected (warp ballots
-//     become bitmap words), boundary-bin elements are candidates;
-//  3. exact MSB radix select of the boundary among the candidates in shared
-//     memory (or, if they do not fit, over the row restricted to the bin);
-//  4. ties at the threshold key: the lowest positions first;
-//  5. bitmap and/or ordered positions out.
-template <bool VEC>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(int n, const float* __restrict__ scores,
-                                                            int64_t ld_s, int K, int offset,
-                                                            int32_t* __restrict__ idx, int64_t ld_i,
-                                                            uint32_t* __restrict__ bits, int64_t ld_b,
-                                                            const uint32_t* __restrict__ rowmm) {
-  grid_dep_enter();
-  extern __shared__ uint32_t tsm[];
-  const int nw = (n + 31) / 32;
-  uint32_t* sel = tsm;                           // [nw]
-  uint32_t* tie = sel + nw;                      // [nw]
-  int* hist = reinterpret_cast<int*>(tie + nw);  // [kBins]
-  uint32_t* ckey = reinterpret_cast<uint32_t*>(hist + kBins);   // [kCap]
-  int* cidx = reinterpret_cast<int*>(ckey + kCap);               // [kCap]
-  __shared__ int wtot[64];
-  __shared__ int s_bin, s_above, s_total, s_nc;
-  __shared__ uint32_t s_mn, s_mx;
-  const int row_id = blockIdx.x;
-  const float* row = scores + (size_t)row_id * ld_s;
-  const int tid = threadIdx.x, lane = tid & 31;
-
-  for (int i = tid; i < nw; i += blockDim.x) sel[i] = tie[i] = 0u;
-  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
-  if (tid == 0) {
-    s_nc = 0;
-    s_mn = 0xffffffffu;
-    s_mx = 0u;
-  }
-  __syncthreads();
-  // -- 0. key range
-  uint32_t mn, mx;
-  if (rowmm) {
-    mn = rowmm[2 * row_id];
-    mx = rowmm[2 * row_id + 1];
-  } else {
-    uint32_t a = 0xffffffffu, c = 0u;
-    for (int j = tid; j < n; j += blockDim.x) {
-      const uint32_t k = float_key(__ldg(row + j));
-      a = min(a, k);
-      c = max(c, k);
-    }
-    atomicMin(&s_mn, a);
-    atomicMax(&s_mx, c);
-    __syncthreads();
-    mn = s_mn;
-    mx = s_mx;
-  }
-  const float vmin = key_float(mn), vmax = key_float(mx);
-  const float scale = (vmax > vmin) ? (float)(kBins - 1) / (vmax - vmin) : 0.f;
-  auto bin_of = [&](float v) -> int {
-    const int bb = (int)((v - vmin) * scale);
-    return min(max(bb, 0), kBins - 1);
-  };
-  // -- 1. histogram of linear bins
-  for (int j = tid; j < n; j += blockDim.x) atomicAdd(&hist[bin_of(__ldg(row + j))], 1);
-  __syncthreads();
-  find_bin(hist, kBins, K, wtot, &s_bin, &s_above);
-  const int b1 = s_bin;
-  int k_rem = K - s_above;   // to take from bin b1 (>= 1)
-  // -- 2. above the bin: selected; in the bin: candidates
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int j = base + tid;
-    int bb = -1;
-    uint32_t key = 0u;
-    if (j < n) {
-      const float v = __ldg(row + j);
-      bb = bin_of(v);
-      key = float_key(v);
-    }
-    const unsigned up = __ballot_sync(0xffffffffu, bb > b1);
-    if (lane == 0 && j < n) sel[j >> 5] = up;
-    const unsigned cand = __ballot_sync(0xffffffffu, bb == b1);
-    if (cand) {
-      int slot0 = 0;
-      if (lane == 0) slot0 = atomicAdd(&s_nc, __popc(cand));
-      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-      if (bb == b1) {
-        const int at = slot0 + __popc(cand & ((1u << lane) - 1u));
-        if (at < kCap) {
-          ckey[at] = key;
-          cidx[at] = j;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  const int nc = s_nc;
-  const bool fits = nc <= kCap;
-  // -- 3. exact threshold key T among the bin's elements: MSB radix, 11/11/10 bits
-  uint32_t prefix = 0, pmask = 0;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sh = shifts[pass];
-    const uint32_t dmask = (1u << widths[pass]) - 1u;
-    for (int i = tid; i < kRBins; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    if (fits) {
-      for (int c = tid; c < nc; c += blockDim.x) {
-        const uint32_t k = ckey[c];
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> sh) & dmask], 1);
-      }
-    } else {
-      for (int j = tid; j < n; j += blockDim.x) {
-        const float v = __ldg(row + j);
-        const uint32_t k = float_key(v);
-        if (bin_of(v) == b1 && (k & pmask) == prefix) atomicAdd(&hist[(k >> sh) & dmask], 1);
-      }
-    }
-    __syncthreads();
-    find_bin(hist, kRBins, k_rem, wtot, &s_bin, &s_above);
-    prefix |= (uint32_t)s_bin << sh;
-    pmask |= dmask << sh;
-    k_rem -= s_above;
-  }
-  const uint32_t T = prefix;   // take k_rem of the keys equal to T, lowest positions first
-  // -- 4. mark the bin's elements above T, and the ties
-  if (fits) {
-    for (int c = tid; c < nc; c += blockDim.x) {
-      const uint32_t k = ckey[c];
-      const int j = cidx[c];
-      if (k > T) atomicOr(&sel[j >> 5], 1u << (j & 31));
-      else if (k == T) atomicOr(&tie[j >> 5], 1u << (j & 31));
-    }
-  } else {
-    for (int j = tid; j < n; j += blockDim.x) {
-      const float v = __ldg(row + j);
-      const uint32_t k = float_key(v);
-      if (bin_of(v) != b1) continue;
-      if (k > T) atomicOr(&sel[j >> 5], 1u << (j & 31));
-      else if (k == T) atomicOr(&tie[j >> 5], 1u << (j & 31));
-    }
-  }
-  __syncthreads();
-  // -- 5. the first k_rem ties in position order join the selection
-  const int per = (nw + blockDim.x - 1) / blockDim.x;
-  const int w0 = tid * per;
-  {
-    int mine = 0;
-    for (int i = 0; i < per; ++i)
-      if (w0 + i < nw) mine += __popc(tie[w0 + i]);
-    int before = block_prefix_excl(mine, wtot, &s_total);
-    for (int i = 0; i < per && before < k_rem; ++i) {
-      if (w0 + i >= nw) break;
-      uint32_t t = tie[w0 + i];
-      uint32_t take = 0u;
-      while (t && before < k_rem) {
-        const uint32_t lowbit = t & (~t + 1u);
-        take |= lowbit;
-        t ^= lowbit;
-        ++before;
-      }
-      sel[w0 + i] |= take;
-    }
-  }
-  __syncthreads();
-  // -- 6. outputs
-  if (bits) {
-    uint32_t* brow = bits + (size_t)row_id * ld_b;
-    for (int i = tid; i < nw; i += blockDim.x) brow[i] = sel[i];
-  }
-  if (idx) {
-    int32_t* out = idx + (size_t)row_id * ld_i;
-    int mine = 0;
-    for (int i = 0; i < per; ++i)
-      if (w0 + i < nw) mine += __popc(sel[w0 + i]);
-    int at = block_prefix_excl(mine, wtot, &s_total);
-    for (int i = 0; i < per; ++i) {
-      if (w0 + i >= nw) break;
-      uint32_t t = sel[w0 + i];
-      while (t) {
-        const int bpos = __ffs(t) - 1;
-        t &= t - 1u;
-        if (at < K) out[at] = offset + (w0 + i) * 32 + bpos;
-        ++at;
       }
     }
   }
 }
 
 // ---------------------------------------------------------------- host
-int score_tile(int G) { return std::max(256, 8192 / G); }
+int score_tile(int G) { return std::max(256, 4096 / G); }
 
 size_t score_smem(int G, int tile, int w) { return (size_t)G * (tile + 2 * w) * sizeof(float); }
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }
-
-int topk_max_n() { return kTopkMaxWords * 32; }
-
-size_t topk_smem(int n) {
-  const size_t nw = (size_t)(n + 31) / 32;
-  return (2 * nw + kBins + 2 * kCap) * sizeof(uint32_t);
-}
 
 template <int GM>
 sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
@@ -545,7 +241,7 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
 
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
-                             float* scores, int64_t ld_s, void* stat_ws, uint32_t* rowmm,
+                             float* scores, int64_t ld_s, void* stat_ws,
                              cudaStream_t st) {
   const int G = s.Hq / s.Hkv;
   const int lo = p.n_sink, hi = L - p.n_recent;
@@ -554,8 +250,7 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   const int nch = stat_chunks(nC);
   const int64_t norm_ld = (int64_t)s.max_pages * kPage;
   dim3 sgrid(nch, s.B * s.Hkv);
-  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch, rowmm,
-           G);
+  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch);
   launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
@@ -570,7 +265,6 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.norms = kv.key_norms; a.norm_ld = norm_ld;
   a.stat_part = part; a.nch = nch;
   a.scores = scores; a.ld_s = ld_s;
-  a.rowmm = rowmm;
   const size_t smem = score_smem(G, a.tile, a.w);
   dim3 grid((nC + a.tile - 1) / a.tile, s.B * s.Hkv);
   if (G <= 1) return launch_scores<1>(a, grid, smem, st);
@@ -578,22 +272,6 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   if (G <= 4) return launch_scores<4>(a, grid, smem, st);
   if (G <= 8) return launch_scores<8>(a, grid, smem, st);
   return launch_scores<16>(a, grid, smem, st);
-}
-
-sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset,
-                    int32_t* idx, int64_t ld_i, uint32_t* bits, int64_t ld_b, const uint32_t* rowmm,
-                    cudaStream_t st) {
-  if (rows <= 0) return SFI_OK;
-  if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  const size_t smem = topk_smem(n);
-  static DeviceOnce attr;
-  if (!attr.done() &&
-      !attr.mark(cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)topk_smem(topk_max_n()))))
-    return SFI_ERR_CUDA;
-  launch_k(topk_kernel<false>, dim3(rows), dim3(kTopkThreads), smem, st, n, scores, ld_s, K, offset, idx, ld_i, bits,
-           ld_b, rowmm);
-  return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 }  // namespace sfi

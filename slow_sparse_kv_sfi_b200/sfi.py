@@ -81,7 +81,8 @@ def _declare(L):
         "sfi_fast_attn": (C.c_int, [P, P, P, I32, P, P, P, P, P, SZ, P]),
         "sfi_fast_attn_append": (C.c_int, [P, P, P, I32, P, P, P, P, P, P, P, SZ, P]),
         "sfi_select_scores": (C.c_int, [P, P, P, I32, P, I64, P, P, P, SZ, P]),
-        "sfi_topk": (C.c_int, [I32, I32, P, I64, I32, I32, P, I64, P]),
+        "sfi_topk_workspace_size": (C.c_int, [I32, I32, C.POINTER(SZ)]),
+        "sfi_topk": (C.c_int, [I32, I32, P, I64, I32, I32, P, I64, P, SZ, P]),
         "sfi_select": (C.c_int, [P, P, P, I32, P, I64, P, P, I32, C.POINTER(I32), P, SZ, P]),
         "sfi_compact": (C.c_int, [P, P, P, I32, P, I32, I32, P, P, SZ, P]),
         "sfi_poll_error": (C.c_int, [P, C.POINTER(I32)]),
@@ -103,7 +104,7 @@ def _declare(L):
 EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_rows", "sfi_budget",
             "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_append",
             "sfi_dense_attn_noalloc", "sfi_attn_probs", "sfi_fast_attn", "sfi_fast_attn_append",
-            "sfi_select_scores", "sfi_topk", "sfi_select", "sfi_compact", "sfi_poll_error",
+            "sfi_select_scores", "sfi_topk_workspace_size", "sfi_topk", "sfi_select", "sfi_compact", "sfi_poll_error",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
             "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_timing"]
 
@@ -227,9 +228,16 @@ def sfi_select_scores(shape, params, kv, L, logits, ld, lse_cand, scores, ws, st
                                    _stream(stream)), "sfi_select_scores")
 
 
-def sfi_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, stream=None):
-    _check(lib().sfi_topk(rows, n, _p(scores), ld_s, K, offset, _p(idx), ld_i, _stream(stream)),
-           "sfi_topk")
+def sfi_topk_workspace_size(rows, n) -> int:
+    v = C.c_size_t(0)
+    _check(lib().sfi_topk_workspace_size(rows, n, C.byref(v)), "sfi_topk_workspace_size")
+    return v.value
+
+
+def sfi_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, ws, stream=None):
+    """ws: zero-filled scratch of sfi_topk_workspace_size(rows, n) bytes (left zero-filled)."""
+    _check(lib().sfi_topk(rows, n, _p(scores), ld_s, K, offset, _p(idx), ld_i, _p(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "sfi_topk")
 
 
 def sfi_select(shape, params, kv, L, logits, ld, lse_cand, sel_idx, sel_ld, ws, stream=None) -> int:

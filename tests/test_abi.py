@@ -81,14 +81,19 @@ def test_null_pointers_rejected_before_any_launch(S):
     lib = S.lib()
     assert lib.sfi_dense_attn(C.byref(sh), C.byref(kv), 100, None, None, None, None, 0, None) == 1
     assert lib.sfi_append_kv(C.byref(sh), C.byref(kv), 100, None, None, None) == 1
-    assert lib.sfi_topk(4, 10, None, 10, 3, 0, None, 3, None) == 1
+    assert lib.sfi_topk(4, 10, None, 10, 3, 0, None, 3, None, 0, None) == 1
     # misaligned pool pointer
     kv = S.PagedKV(8, 16, 16, 16, None)
     assert lib.sfi_key_norms(C.byref(sh), C.byref(kv), 0, 10, None) == 1
     # context longer than the cache
     kv = S.PagedKV(16, 16, 16, 16, None)
     assert lib.sfi_append_kv(C.byref(sh), C.byref(kv), 161, 16, 16, None) == 2
-    assert lib.sfi_topk(4, 10, 16, 10, 11, 0, 16, 11, None) == 2   # K > n
+    assert lib.sfi_topk(4, 10, 16, 10, 11, 0, 16, 11, 16, 1 << 20, None) == 2   # K > n
+    # a workspace smaller than sfi_topk_workspace_size is refused before any launch
+    need = C.c_size_t(0)
+    assert lib.sfi_topk_workspace_size(4, 10, C.byref(need)) == 0 and need.value > 0
+    assert lib.sfi_topk(4, 10, 16, 10, 3, 0, 16, 3, 16, need.value - 1, None) == 7
+    assert lib.sfi_topk(4, 10, 16, 10, 3, 0, 16, 3, None, need.value, None) == 7
     assert lib.sfi_ctx_set_workspace(None, None, 0) == 1
 
 

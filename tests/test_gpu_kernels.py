@@ -181,7 +181,8 @@ def test_selector_scores_topk_and_compaction(B, Hq, Hkv, D, L, kw):
     S.sfi_select_scores(shape, params, layer.kv, L, logits, L, lse_c, scores, ws)
     K = S.sfi_budget(params, L)
     sel = torch.empty(B, Hq, K + 3, dtype=torch.int32, device=DEV)
-    S.sfi_topk(B * Hq, nC, scores, nC, K, lo, sel, K + 3)
+    tws = torch.zeros(S.sfi_topk_workspace_size(B * Hq, nC), dtype=torch.uint8, device=DEV)
+    S.sfi_topk(B * Hq, nC, scores, nC, K, lo, sel, K + 3, tws)
     sel2 = torch.empty_like(sel)
     assert S.sfi_select(shape, params, layer.kv, L, logits, L, lse_c, sel2, K + 3, ws) == K
     S.sfi_compact(shape, params, layer.kv, L, sel2, K + 3, K, layer.packed, ws)
