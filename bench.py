@@ -198,20 +198,31 @@ class Bench:
 
 
 def _sync_barrier(dist_on):
-    torch.cuda.synchronize()
+    """Device idle on every rank, then all ranks meet."""
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     if dist_on:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def _max_over_ranks(x, dist_on):
+    """The largest x over all ranks (the slowest rank's time)."""
     if not dist_on:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(world, units_per_rank_run, runs, seconds):
+    """Whole-job throughput: every rank (replica) processed units_per_rank_run
+    per run, `runs` runs took `seconds` on the slowest rank."""
+    return world * units_per_rank_run * runs / seconds
 
 
 def _timed(fn, K, dist_on):
@@ -397,7 +408,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
                 "algorithmic_bytes_per_launch": dense_bytes_slow / max(dense_n / k, 1),
                 "launches": dense_n, "avg_launch_us": 1000 * dense_ms / max(dense_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
-    value = world * tokens / t_sfi * args.steps
+    value = aggregate_rate(world, tokens, args.steps, t_sfi)
     # fast layer-step: attention (with the append) + combine; slow: the same
     # two, then 2 statistics + scores + top-K + 3 compaction kernels (side stream)
     launches_per_run = NL * (n_slow * 9 + (T - n_slow) * 2)
@@ -412,12 +423,12 @@ def run_sfi(args, cfg, rank, world, dist_on):
                    "l2": "inputs larger than L2 (KV cache %.1f GB)" %
                          (NL * 2 * cfg.num_pages * cfg.Hkv * 16 * D * 2 / 1e9)},
         "roofline": roof,
-        "e2e": {"value": world * tokens / t_e2e * args.steps, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": aggregate_rate(world, tokens, args.steps, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_run * args.steps,
         "clocks": clk,
         "breakdown": {
-            "dense_full_kv_tok_s": world * tokens / t_dense * args.steps,
+            "dense_full_kv_tok_s": aggregate_rate(world, tokens, args.steps, t_dense),
             "speedup_vs_dense": t_dense / t_sfi,
             "fast_step_tok_s": B * NL / (statistics.mean(st_fast) / 1e3) if st_fast else None,
             "slow_step_tok_s": B * NL / (statistics.mean(st_slow) / 1e3) if st_slow else None,
@@ -481,6 +492,11 @@ def main():
         cfg = cfg.replace(steps=args.decode_steps)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 alone; the other ranks exit at once
+        if rank == 0:
+            run_reference(args, cfg, rank, world)
+        return
     dist_on = world > 1
     if dist_on:
         import datetime
@@ -489,8 +505,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     if args.layer_probe:
         run_layer_probe(args, cfg)
-    elif args.impl == "reference":
-        run_reference(args, cfg, rank, world)
     else:
         if not torch.cuda.is_available():
             raise SystemExit("bench.py --impl sfi needs a CUDA device")
