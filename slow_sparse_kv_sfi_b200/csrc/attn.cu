@@ -659,10 +659,11 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
 }
 
 // Merge the partials of every (b, query head): one CTA of kCombWarps warps
-// each.  Pass 1: the largest m.  Pass 2: warp w folds partials w,
-// w + kCombWarps, ... with eight partials' loads in flight per step; the
-// warps' sums meet in shared memory.
-constexpr int kCombWarps = 16;
+// each, one pass.  Warp w folds partials w, w + kCombWarps, ... (eight loads
+// in flight per lane, each partial's m, l, l_C and a 4-column slice of O per
+// lane) into a running (m, l, l_C, O) with online rescaling; the warps' states
+// meet in shared memory, where thread d merges column d.
+constexpr int kCombWarps = 24;
 
 template <int D>
 __global__ void __launch_bounds__(kCombWarps * 32)
@@ -670,9 +671,9 @@ __global__ void __launch_bounds__(kCombWarps * 32)
                         float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
                         const int32_t* n_rows, int p_max, int* err, int* ctr) {
   grid_dep_enter();
-  constexpr int kPer = D / 32;
+  constexpr int kPer = D / 32;     // columns of O per lane
+  static_assert(kPer == 4 || kPer == 2, "head dim");
   __shared__ float red[kCombWarps][D + 4];
-  __shared__ float mx[kCombWarps];
   if (blockIdx.x == 0 && threadIdx.x == 0) ctr[0] = 0;   // the attention kernel is done with it
   const int row = blockIdx.x;   // b * Hq + hq
   const int b = row / Hq, hq = row - b * Hq;
@@ -686,20 +687,10 @@ __global__ void __launch_bounds__(kCombWarps * 32)
   const size_t stride = (size_t)G * (D + 4);
   const int n = n_chunks * kConsumerWarps;   // one partial per consumer warp and work item
   const float* base = part + (size_t)bg * n * stride + (size_t)hh * (D + 4);
-  float M = -INFINITY;
-  for (int c = threadIdx.x; c < n; c += blockDim.x) M = fmaxf(M, __ldg(base + c * stride + D));
-#pragma unroll
-  for (int sh = 16; sh >= 1; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
-  if (lane == 0) mx[warp] = M;
-  __syncthreads();
-  M = mx[0];
-#pragma unroll
-  for (int w = 1; w < kCombWarps; ++w) M = fmaxf(M, mx[w]);
-  const float mref = (M == -INFINITY) ? 0.f : M;
+  float m = -INFINITY, l = 0.f, lc = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  float l = 0.f, lc = 0.f;
   constexpr int kIn = 8;   // partials in flight per warp
   for (int c0 = warp; c0 < n; c0 += kIn * kCombWarps) {
     float st[kIn][3];
@@ -712,8 +703,17 @@ __global__ void __launch_bounds__(kCombWarps * 32)
         st[u][0] = __ldg(pc + D);
         st[u][1] = __ldg(pc + D + 1);
         st[u][2] = __ldg(pc + D + 2);
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) ov[u][k] = __ldg(pc + lane * kPer + k);
+        if constexpr (kPer == 4) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(pc + lane * 4));
+          ov[u][0] = v.x;
+          ov[u][1] = v.y;
+          ov[u][2] = v.z;
+          ov[u][3] = v.w;
+        } else {
+          const float2 v = __ldg(reinterpret_cast<const float2*>(pc + lane * 2));
+          ov[u][0] = v.x;
+          ov[u][1] = v.y;
+        }
       } else {
         st[u][0] = -INFINITY;
         st[u][1] = st[u][2] = 0.f;
@@ -721,39 +721,48 @@ __global__ void __launch_bounds__(kCombWarps * 32)
         for (int k = 0; k < kPer; ++k) ov[u][k] = 0.f;
       }
     }
+    float mb = m;
+#pragma unroll
+    for (int u = 0; u < kIn; ++u) mb = fmaxf(mb, st[u][0]);
+    const float mref = (mb == -INFINITY) ? 0.f : mb;
+    const float a = fast_exp2(m - mref);
+    l *= a;
+    lc *= a;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) acc[k] *= a;
 #pragma unroll
     for (int u = 0; u < kIn; ++u) {
-      const float w = exp2f(st[u][0] - mref);
+      const float w = fast_exp2(st[u][0] - mref);
       l += w * st[u][1];
       lc += w * st[u][2];
 #pragma unroll
       for (int k = 0; k < kPer; ++k) acc[k] += w * ov[u][k];
     }
+    m = mb;
   }
 #pragma unroll
   for (int k = 0; k < kPer; ++k) red[warp][lane * kPer + k] = acc[k];
   if (lane == 0) {
-    red[warp][D] = l;
-    red[warp][D + 1] = lc;
+    red[warp][D] = m;
+    red[warp][D + 1] = l;
+    red[warp][D + 2] = lc;
   }
   __syncthreads();
-  if (warp == 0) {
-    float lt = 0.f, lct = 0.f;
-#pragma unroll
+  if (threadIdx.x < D) {
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int w = 0; w < kCombWarps; ++w) M = fmaxf(M, red[w][D]);
+    const float mref = (M == -INFINITY) ? 0.f : M;
+    float lt = 0.f, lct = 0.f, o = 0.f;
+#pragma unroll 8
     for (int w = 0; w < kCombWarps; ++w) {
-      lt += red[w][D];
-      lct += red[w][D + 1];
+      const float wt = fast_exp2(red[w][D] - mref);
+      lt += wt * red[w][D + 1];
+      lct += wt * red[w][D + 2];
+      o += wt * red[w][threadIdx.x];
     }
-    const float inv = 1.f / lt;
-    float* orow = out + (size_t)row * D + lane * kPer;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < kCombWarps; ++w) t += red[w][lane * kPer + k];
-      orow[k] = t * inv;
-    }
-    if (lane == 0) {
+    out[(size_t)row * D + threadIdx.x] = o / lt;
+    if (threadIdx.x == 0) {
       if (lse) lse[row] = (M + log2f(lt)) * kLn2;
       if (lse_cand) lse_cand[row] = lct > 0.f ? (M + log2f(lct)) * kLn2 : -INFINITY;
     }
