@@ -177,10 +177,9 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   const CtxLayout l = ctx_layout(c->s, c->p);
   if (bytes < l.total) return SFI_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
-  // the attention kernels' work counter (first 256 bytes) and the top-K
-  // state start at zero; every step leaves them so
-  if (cudaMemset(w, 0, 256) != cudaSuccess) return SFI_ERR_CUDA;
-  if (cudaMemset(w + l.tk_off, 0, l.tk_bytes) != cudaSuccess) return SFI_ERR_CUDA;
+  // the counters in the workspace (attention work counter, combine and top-K
+  // arrival counters, histograms) start at zero; every step leaves them so
+  if (cudaMemset(w, 0, l.total) != cudaSuccess) return SFI_ERR_CUDA;
   c->ws = w;
   c->ws_bytes = bytes;
   c->part = reinterpret_cast<float*>(w + l.part_off);

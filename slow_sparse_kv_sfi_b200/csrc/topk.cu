@@ -44,19 +44,21 @@ __host__ __device__ constexpr Digit digit_of(int pass) {
 }
 
 // The 32 scores of this thread in slice [s0, s0 + kSlice) of a row, as keys:
-// element e of load u is score s0 + (u * kTkThreads + tid) * 4 + e.
-// Scores past n are flagged absent.
+// element e of load u is score s0 + (u * kTkThreads + tid) * 4 + e, so every
+// warp-wide load reads 512 consecutive bytes.  All eight loads are issued
+// before any is used.  Scores past n read as key 0 and are flagged by the
+// callers.
 struct SliceKeys {
   uint32_t k[8][4];
 };
 
+__device__ __forceinline__ int pos_of(int s0, int u, int e) { return s0 + (u * kTkThreads + threadIdx.x) * 4 + e; }
+
 __device__ __forceinline__ void load_keys(const float* row, int n, int s0, bool vec, SliceKeys& x) {
-  const int tid = threadIdx.x;
   if (vec && s0 + kSlice <= n) {
-    // a whole slice: all eight loads are issued before any is used
     float4 f[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(row + s0 + (u * kTkThreads + tid) * 4));
+    for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(row + pos_of(s0, u, 0)));
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       x.k[u][0] = float_key(f[u].x);
@@ -70,7 +72,7 @@ __device__ __forceinline__ void load_keys(const float* row, int n, int s0, bool 
     for (int u = 0; u < 8; ++u)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int j = s0 + (u * kTkThreads + tid) * 4 + e;
+        const int j = pos_of(s0, u, e);
         f[u][e] = j < n ? __ldg(row + j) : 0.f;
       }
 #pragma unroll
@@ -79,8 +81,6 @@ __device__ __forceinline__ void load_keys(const float* row, int n, int s0, bool 
       for (int e = 0; e < 4; ++e) x.k[u][e] = float_key(f[u][e]);
   }
 }
-
-__device__ __forceinline__ int pos_of(int s0, int u, int e) { return s0 + (u * kTkThreads + threadIdx.x) * 4 + e; }
 
 // Reverse (suffix) inclusive scan of one value per thread across the block;
 // wtot holds 64 ints.
@@ -184,7 +184,6 @@ __global__ void __launch_bounds__(kTkThreads) topk_digit_kernel(const TopkArgs a
   __shared__ int wtot[64];
   __shared__ int s_last, s_bin, s_above;
   const int row = blockIdx.y, s0 = blockIdx.x * kSlice;
-  const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kNb; i += kTkThreads) hist[i] = 0;
   SliceKeys x;
   load_keys(a.scores + (size_t)row * a.ld_s, a.n, s0, a.vec, x);
@@ -193,24 +192,36 @@ __global__ void __launch_bounds__(kTkThreads) topk_digit_kernel(const TopkArgs a
   const uint32_t pmask = PASS == 0 ? 0u : (uint32_t)info[2];
   const int k = PASS == 0 ? a.K : info[1];
   __syncthreads();
+  // Neighbouring scores share digits, and the bins of a row's bulk are few:
+  // a lane whose 4 scores share one digit counts them as one, and a run of
+  // such lanes with one digit adds once (from its first lane); lanes with
+  // mixed digits add their scores one by one.
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
+  for (int u = 0; u < 8; ++u) {
+    int d[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const uint32_t key = x.k[u][e];
-      const bool p = pos_of(s0, u, e) < a.n && (key & pmask) == prefix;
-      const int d = p ? (int)((key >> dg.shift) & kDm) : -1;
-      // Neighbouring scores share digits: across the warp (positions 4 apart)
-      // a run of lanes with one digit adds its length once, from its first lane.
-      const int dprev = __shfl_up_sync(0xffffffffu, d, 1);
-      const bool head = lane == 0 || dprev != d;
-      const unsigned heads = __ballot_sync(0xffffffffu, head);
-      if (head && p) {
+      d[e] = (pos_of(s0, u, e) < a.n && (key & pmask) == prefix) ? (int)((key >> dg.shift) & kDm) : -1;
+    }
+    const bool uni = d[0] == d[1] && d[0] == d[2] && d[0] == d[3];
+    const int dl = uni ? d[0] : -2;
+    const int dprev = __shfl_up_sync(0xffffffffu, dl, 1);
+    const bool head = lane == 0 || dprev != dl;
+    const unsigned heads = __ballot_sync(0xffffffffu, head);
+    if (uni) {
+      if (head && dl >= 0) {
         const unsigned later = heads & ~((2u << lane) - 1u);   // run heads after this lane
         const int next = later ? __ffs(later) - 1 : 32;
-        atomicAdd(&hist[d], next - lane);
+        atomicAdd(&hist[dl], 4 * (next - lane));
       }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (d[e] >= 0) atomicAdd(&hist[d[e]], 1);
     }
+  }
   __syncthreads();
   int* gh = a.w.ghist + (size_t)row * kDigitBins;
   for (int i = threadIdx.x; i < kNb; i += kTkThreads)
