@@ -24,6 +24,7 @@ independent replica; the decode path has no cross-GPU exchange.
 from __future__ import annotations
 
 import argparse
+import ctypes as C
 import hashlib
 import json
 import os
@@ -157,13 +158,23 @@ class Bench:
         vn = self.vn if vn is None else vn
         out = self.out if out is None else out
         slows = []
+        # raw addresses of every (step, layer) slice: [T, layers, ...] contiguous
+        NL = len(self.layers)
+        qb, qs = q.data_ptr(), q[0, 0].numel() * q.element_size()
+        kb, ks = kn.data_ptr(), kn[0, 0].numel() * kn.element_size()
+        vb, vs = vn.data_ptr(), vn[0, 0].numel() * vn.element_size()
+        ob, os_ = out.data_ptr(), out[0].numel() * out.element_size()
+        refs = [(C.byref(layer.kv), C.byref(layer.packed)) for layer in self.layers]
+        stream = torch.cuda.current_stream().cuda_stream
+        step_fn = self.ctx.decode_step_ptr
         for t in range(cfg.steps):
             L = cfg.seq_len(t)
             bprev = int(self.boundary[t - 1]) if t > 0 else 0
             slow = False
-            for l, layer in enumerate(self.layers):
-                slow = self.ctx.decode_step(l, t, bprev, L, layer.kv, layer.packed, q[t, l], kn[t, l],
-                                            vn[t, l], out[l])
+            for l in range(NL):
+                i = t * NL + l
+                slow = step_fn(l, t, bprev, L, refs[l][0], refs[l][1], qb + i * qs, kb + i * ks, vb + i * vs,
+                               ob + l * os_, stream)
             slows.append(slow)
             if step_events is not None:
                 step_events[t].record()
@@ -185,14 +196,22 @@ class Bench:
         """Every decode step copies that step's inputs (all layers) from pinned
         host memory and reads all layers' outputs back."""
         cfg = self.cfg
+        NL = len(self.layers)
+        qs, ks, vs = (dq[0].numel() * dq.element_size(), dk[0].numel() * dk.element_size(),
+                      dv[0].numel() * dv.element_size())
+        os_ = self.out[0].numel() * self.out.element_size()
+        refs = [(C.byref(layer.kv), C.byref(layer.packed)) for layer in self.layers]
+        stream = torch.cuda.current_stream().cuda_stream
+        step_fn = self.ctx.decode_step_ptr
         for t in range(cfg.steps):
             dq.copy_(host_q[t], non_blocking=True)
             dk.copy_(host_k[t], non_blocking=True)
             dv.copy_(host_v[t], non_blocking=True)
             L = cfg.seq_len(t)
             bprev = int(self.boundary[t - 1]) if t > 0 else 0
-            for l, layer in enumerate(self.layers):
-                self.ctx.decode_step(l, t, bprev, L, layer.kv, layer.packed, dq[l], dk[l], dv[l], self.out[l])
+            for l in range(NL):
+                step_fn(l, t, bprev, L, refs[l][0], refs[l][1], dq.data_ptr() + l * qs, dk.data_ptr() + l * ks,
+                        dv.data_ptr() + l * vs, self.out.data_ptr() + l * os_, stream)
             host_out[t].copy_(self.out, non_blocking=True)
         self.ctx.join()
 

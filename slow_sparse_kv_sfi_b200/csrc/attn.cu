@@ -257,22 +257,30 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     uint32_t phase = 0;
     int inflight = 0;
     bool ok = true;
-    int nxt2 = 0;
-    if (lane == 0) nxt2 = atomicAdd(a.ctr, 1);
+    // The next item is drawn late in the current one (two stages before its
+    // end, leaving time to fetch its page-table entries): a CTA holds no work
+    // it cannot start soon, so CTAs that finish early take what remains.
+    bool drawn = false;
+    auto draw_next = [&]() {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(a.ctr, 1);
+      nxt = __shfl_sync(0xffffffffu, v, 0);
+      prefetch(nxt, pf);
+      drawn = true;
+    };
     while (ok) {
       const int item = nxt;
-      // publish this item's page entries, then start fetching the next item's
+      // publish this item's page entries
       __syncwarp();
 #pragma unroll
       for (int j = 0; j < kMaxChunkTiles / 32; ++j) ptbuf[j * 32 + lane] = pf[j];
       __syncwarp();
-      nxt = __shfl_sync(0xffffffffu, nxt2, 0);
-      if (item < a.n_items) {
-        prefetch(nxt, pf);
-        if (lane == 0) nxt2 = (nxt < a.n_items) ? atomicAdd(a.ctr, 1) : a.n_items;
-      }
-      // one stage per kTPS tiles; an item without tiles still sends one
-      // (empty) stage so the consumers write its partial; item == n_items: stop.
+      drawn = item >= a.n_items;
+      // one stage per kTPS tiles; item == n_items: stop.  A dense item without
+      // tiles still sends one (empty) stage so the consumers write its
+      // partial; a fast-step chunk past its (b, kv head)'s tiles is skipped
+      // (the combine kernel reads only the chunks holding tiles), so its CTA
+      // does not take one real item more than the others at the end.
       Item it{};
       int nst = 1;
       int p_lo = 0;
@@ -288,8 +296,13 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
                              a.v_pool, a.k_new, a.v_new, a.norms, a.norm_ld, a.err);
           __syncwarp();
         }
+        if (MODE == kFast && it.t_begin >= it.t_end) {
+          draw_next();
+          continue;
+        }
       }
       for (int st = 0; st < nst; ++st) {
+        if (!drawn && st >= nst - 2) draw_next();
         bool good = true;
         if (lane == 0) {
           good = !*abort_flag && mbar_wait(&empty[slot], phase ^ 1, a.err, kSiteAttnProducer);
@@ -669,7 +682,7 @@ template <int D>
 __global__ void __launch_bounds__(kCombWarps * 32)
     attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
                         float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
-                        const int32_t* n_rows, int p_max, int* err, int* ctr) {
+                        const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr) {
   grid_dep_enter();
   constexpr int kPer = D / 32;     // columns of O per lane
   static_assert(kPer == 4 || kPer == 2, "head dim");
@@ -685,8 +698,19 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     if (nr < 0 || nr > p_max) latch_error(err, SFI_ERR_DEVICE_CHECK, kSiteAttnRows);
   }
   const size_t stride = (size_t)G * (D + 4);
-  const int n = n_chunks * kConsumerWarps;   // one partial per consumer warp and work item
-  const float* base = part + (size_t)bg * n * stride + (size_t)hh * (D + 4);
+  // one partial per consumer warp and work item; the fast step's chunks past
+  // the (b, kv head)'s tiles were skipped
+  int chunks = n_chunks;
+  if (n_rows) {
+    int nr = n_rows[bg];
+    if (nr < 0 || nr > p_max) nr = nr < 0 ? 0 : p_max;
+    const int T = (nr + kPage - 1) / kPage + rec_tiles;
+    int ct = (T + n_chunks - 1) / n_chunks;
+    ct = (ct + tps - 1) / tps * tps;
+    chunks = (T + ct - 1) / ct;
+  }
+  const int n = chunks * kConsumerWarps;
+  const float* base = part + (size_t)bg * n_chunks * kConsumerWarps * stride + (size_t)hh * (D + 4);
   float m = -INFINITY, l = 0.f, lc = 0.f;
   float acc[kPer];
 #pragma unroll
@@ -828,6 +852,58 @@ bool make_map_tiles(CUtensorMap* m, const void* base, uint64_t rows, int D, int 
   return r == CUDA_SUCCESS;
 }
 
+static_assert(sizeof(Maps) == sizeof(AttnMapCache::maps), "tensor-map cache size");
+
+// The launch's tensor maps: from the cache when it was built from the same
+// pointers and sizes, else encoded (and kept in the cache, if there is one).
+bool paged_maps(Maps* m, const sfi_paged_kv& kv, uint64_t rows, int D, AttnMapCache* c) {
+  if (c && c->paged && c->k_pool == kv.k_pool && c->v_pool == kv.v_pool && c->rows == rows && c->D == D) {
+    const Maps* cm = reinterpret_cast<const Maps*>(c->maps);
+    m->k = cm->k;
+    m->v = cm->v;
+    return true;
+  }
+  if (!make_map(&m->k, kv.k_pool, rows, D) || !make_map(&m->v, kv.v_pool, rows, D)) return false;
+  if (c) {
+    Maps* cm = reinterpret_cast<Maps*>(c->maps);
+    cm->k = m->k;
+    cm->v = m->v;
+    c->k_pool = kv.k_pool;
+    c->v_pool = kv.v_pool;
+    c->rows = rows;
+    c->D = D;
+    c->paged = true;
+    c->packed = false;   // the packed maps are checked against the same D
+  }
+  return true;
+}
+
+bool packed_maps(Maps* m, const sfi_packed& pk, uint64_t prows, int D, int nts, AttnMapCache* c) {
+  if (c && c->packed && c->pk == pk.k && c->pv == pk.v && c->prows == prows && c->D == D) {
+    const Maps* cm = reinterpret_cast<const Maps*>(c->maps);
+    m->pk = cm->pk;
+    m->pv = cm->pv;
+    m->pk8 = cm->pk8;
+    m->pv8 = cm->pv8;
+    return true;
+  }
+  if (!make_map(&m->pk, pk.k, prows, D) || !make_map(&m->pv, pk.v, prows, D) ||
+      !make_map_tiles(&m->pk8, pk.k, prows, D, nts) || !make_map_tiles(&m->pv8, pk.v, prows, D, nts))
+    return false;
+  if (c && c->paged && c->D == D) {
+    Maps* cm = reinterpret_cast<Maps*>(c->maps);
+    cm->pk = m->pk;
+    cm->pv = m->pv;
+    cm->pk8 = m->pk8;
+    cm->pv8 = m->pv8;
+    c->pk = pk.k;
+    c->pv = pk.v;
+    c->prows = prows;
+    c->packed = true;
+  }
+  return true;
+}
+
 template <int D, int NT, int MODE>
 sfi_status launch_attn_t(const Maps& maps, const AttnArgs& a, cudaStream_t st) {
   using S = Smem<D, NT>;
@@ -855,16 +931,16 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
 }
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
-                          float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int* err,
-                          int* ctr, cudaStream_t st) {
+                          float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int rec_tiles, int tps,
+                          int* err, int* ctr, cudaStream_t st) {
   const int G = s.Hq / s.Hkv;
   const int grid = s.B * s.Hq;
   if (D == 128)
     launch_k(attn_combine_kernel<128>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, err, ctr);
+             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr);
   else
     launch_k(attn_combine_kernel<64>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, err, ctr);
+             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -950,11 +1026,11 @@ void set_token(AttnArgs& a, const sfi_shape& s, const sfi_paged_kv& kv, const St
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
-                          const StepToken* tok) {
+                          const StepToken* tok, AttnMapCache* cache) {
   const int G = s.Hq / s.Hkv;
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
-  if (!make_map(&maps.k, kv.k_pool, rows, s.D) || !make_map(&maps.v, kv.v_pool, rows, s.D)) return SFI_ERR_CUDA;
+  if (!paged_maps(&maps, kv, rows, s.D, cache)) return SFI_ERR_CUDA;
   maps.pk = maps.pk8 = maps.k;
   maps.pv = maps.pv8 = maps.v;
   AttnArgs a{};
@@ -989,7 +1065,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
-  r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0,
+  r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0, 0, 1,
                      kv.err, ctr, st);
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
@@ -1003,16 +1079,14 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end, const StepToken* tok) {
+                         cudaEvent_t ev_end, const StepToken* tok, AttnMapCache* cache) {
   const int G = s.Hq / s.Hkv;
   if ((long)s.B * s.Hkv > kMaxBH) return SFI_ERR_UNSUPPORTED;
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
   const uint64_t prows = (uint64_t)s.B * s.Hkv * pk.p_max;
   const int nts = attn_grid(s.D, G).tps;
-  if (!make_map(&maps.k, kv.k_pool, rows, s.D) || !make_map(&maps.v, kv.v_pool, rows, s.D) ||
-      !make_map(&maps.pk, pk.k, prows, s.D) || !make_map(&maps.pv, pk.v, prows, s.D) ||
-      !make_map_tiles(&maps.pk8, pk.k, prows, s.D, nts) || !make_map_tiles(&maps.pv8, pk.v, prows, s.D, nts))
+  if (!paged_maps(&maps, kv, rows, s.D, cache) || !packed_maps(&maps, pk, prows, s.D, nts, cache))
     return SFI_ERR_CUDA;
   AttnArgs a{};
   a.B = s.B; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G; a.L = L;
@@ -1036,8 +1110,9 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   sfi_status r = launch_attn<kFast>(s.D, G, maps, a, st);
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
-  return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, kv.err, ctr,
-                        st);
+  const int rec_tiles = (L - 1) / kPage - a.rec_lo / kPage + 1;
+  return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, rec_tiles, nts, kv.err,
+                        ctr, st);
 }
 
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,

@@ -42,6 +42,7 @@ struct sfi_ctx {
   char* topk_ws = nullptr;
   int32_t* tile_counts = nullptr;
   size_t tc_bytes = 0;
+  std::vector<sfi::AttnMapCache> maps;   // per layer
   // timing of the attention kernels (kind 0 fast, 1 dense) of every
   // timing-th layer (0: off)
   int timing = 0;
@@ -140,6 +141,7 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->ev_dense.resize(n_layers, nullptr);
   c->ev_sel.resize(n_layers, nullptr);
   c->pending.assign(n_layers, 0);
+  c->maps.resize(n_layers);
   for (int i = 0; i < n_layers && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
@@ -236,7 +238,7 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
     cudaEvent_t b, e;
     timing_events(c, 0, layer, &b, &e);
     return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, reinterpret_cast<int*>(c->ws), c->part,
-                         c->part_bytes, main, b, e, &tok);
+                         c->part_bytes, main, b, e, &tok, &c->maps[layer]);
   }
 
   const int buf = layer & 1;
@@ -251,7 +253,7 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
     cudaEvent_t b, e;
     timing_events(c, 1, layer, &b, &e);
     SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
-                           main, b, e, &tok));
+                           main, b, e, &tok, &c->maps[layer]));
   }
   SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
   cudaStream_t side = c->side;

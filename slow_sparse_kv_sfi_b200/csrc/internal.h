@@ -74,6 +74,21 @@ size_t attn_part_bytes(int n_items, int G, int D);
 int packed_rows_capacity(const sfi_shape& s, const sfi_params& p);
 int budget_k(const sfi_params& p, int L);   // -1 if |C| < 1
 
+// Tensor maps of one layer's paged cache and packed buffer, kept by the
+// decode-step driver so that a launch does not encode them again (a host
+// cost paid on every call otherwise).  Valid while the pointers and sizes
+// they were built from are unchanged; the attention calls check that.
+struct AttnMapCache {
+  const void* k_pool = nullptr;
+  const void* v_pool = nullptr;
+  const void* pk = nullptr;
+  const void* pv = nullptr;
+  uint64_t rows = 0, prows = 0;
+  int D = 0;
+  bool paged = false, packed = false;
+  alignas(128) unsigned char maps[6 * 128];   // the kernel's tensor maps (k, v, pk, pv, pk8, pv8)
+};
+
 // The decode step's new token (bf16 [B, Hkv, D] each), appended at L - 1 by
 // the attention launch itself.
 struct StepToken {
@@ -84,11 +99,11 @@ struct StepToken {
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
-                          const StepToken* tok = nullptr);
+                          const StepToken* tok = nullptr, AttnMapCache* maps = nullptr);
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end, const StepToken* tok = nullptr);
+                         cudaEvent_t ev_end, const StepToken* tok = nullptr, AttnMapCache* maps = nullptr);
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld,
                           const float* lse, float* probs, cudaStream_t st);
 

@@ -274,6 +274,7 @@ class Context:
         _check(lib().sfi_ctx_workspace_size(h, C.byref(n)), "sfi_ctx_workspace_size")
         self.ws = torch.empty(n.value, dtype=torch.uint8, device=device or "cuda")
         _check(lib().sfi_ctx_set_workspace(h, _p(self.ws), n.value), "sfi_ctx_set_workspace")
+        self._slow = C.c_int32(0)
 
     def decode_step(self, layer, step, boundary_prev, L, kv, packed, q, k_new, v_new, out,
                     stream=None) -> bool:
@@ -282,6 +283,17 @@ class Context:
                                      C.byref(packed), _p(q), _p(k_new), _p(v_new), _p(out),
                                      _stream(stream), C.byref(slow)), "sfi_decode_step")
         return bool(slow.value)
+
+    def decode_step_ptr(self, layer, step, boundary_prev, L, kv_ref, packed_ref, q, k_new, v_new, out,
+                        stream) -> bool:
+        """decode_step with raw device addresses (ints), C.byref(...) of the
+        cache and packed structs and a raw stream handle: no tensor
+        marshalling, for drivers that issue many layer-steps."""
+        st = lib().sfi_decode_step(self.h, layer, step, boundary_prev, L, kv_ref, packed_ref, q, k_new, v_new, out,
+                                   stream, C.byref(self._slow))
+        if st != 0:
+            raise SFIError(st, "sfi_decode_step")
+        return bool(self._slow.value)
 
     def join(self, stream=None):
         _check(lib().sfi_ctx_join(self.h, _stream(stream)), "sfi_ctx_join")
