@@ -163,6 +163,12 @@ SEL_SHAPES = [
     (2, 8, 2, 128, 6000, dict(budget_frac=0.15)),
     (1, 32, 2, 128, 3000, dict(budget_frac=0.2, outlier_frac=0.005, query_mode="clusters")),
     (2, 4, 4, 64, 2500, dict(budget_frac=0.2)),     # G = 1
+    # Selector settings of the ablation sweep
+    (1, 16, 4, 128, 4000, dict(budget_frac=0.2, lam=0.0)),                       # evidence only
+    (1, 16, 4, 128, 4000, dict(budget_frac=0.2, lam=1.0, lam_clip=1.0)),         # prior only
+    (1, 16, 4, 128, 4000, dict(budget_frac=0.2, lam=0.8, lam_clip=0.5)),         # clip active
+    (1, 16, 4, 128, 4000, dict(budget_frac=0.2, alpha_soft=0.0, alpha_cross=0.0)),
+    (1, 16, 4, 128, 4000, dict(budget_frac=0.2, nms_window=8, alpha_soft=1.0, alpha_cross=0.25)),
 ]
 
 
