@@ -171,7 +171,11 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
           if (h < G) {
-            const float ft = expf(zv[u][h] - lsec[h]);
+            // exp through the hardware's base-2 approximation (relative
+            // error ~1e-7); the log stays the accurate one, since the
+            // selection compares scores that can sit an ulp apart and an
+            // approximate log does not keep their order
+            const float ft = fast_exp2((zv[u][h] - lsec[h]) * kLog2e);
             const float sv = (1.f - lam) * ft + lam * r;
             ell[h * W + k] = logf(sv + 1e-30f);
           }
