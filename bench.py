@@ -474,8 +474,11 @@ def run_sfi(args, cfg, rank, world, dist_on):
 
 def run_layer_probe(args, cfg):
     """A few launches of every hot-path kernel on one layer of the workload
-    (for profiler captures): per repetition one slow layer-step (dense
-    attention with logits, Selector, compaction) and one fast layer-step."""
+    (for profiler captures): per repetition a slow layer-step that builds the
+    packed buffer (dense attention with logits, Selector, full compaction), a
+    fast layer-step, and after 15 more fast steps a slow layer-step that
+    refreshes the buffer incrementally, as the decode loop's later slow steps
+    do."""
     cfg1 = cfg.replace(n_layers=1)
     dev = torch.device("cuda", torch.cuda.current_device())
     li = W.make_layer(cfg1, 0, dev)
@@ -484,8 +487,8 @@ def run_layer_probe(args, cfg):
     out = torch.empty(cfg1.B, cfg1.Hq, cfg1.D, device=dev)
     torch.cuda.synchronize()
     for r in range(args.layer_probe):
-        for t in range(2):   # step 0 is slow, step 1 fast
-            ctx.decode_step(0, t, 0, cfg1.seq_len(t), layer.kv, layer.packed, li.q[t], li.k_new[t],
+        for t in range(18):   # steps 0 and 16 slow (a boundary at step 15), the rest fast
+            ctx.decode_step(0, t, int(t == 16), cfg1.seq_len(t), layer.kv, layer.packed, li.q[t], li.k_new[t],
                             li.v_new[t], out)
         ctx.join()
     torch.cuda.synchronize()

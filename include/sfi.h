@@ -98,8 +98,9 @@ typedef struct {
 
 /* Contiguous packed buffer of one layer ([ES] §3 item 2, [NL] Memory-Coalesced
  * Kernel, [ZH] §2.3): per (sequence, KV head) the sink rows, then the union of
- * the group's selected positions in ascending order, then zero rows up to a
- * multiple of 16.
+ * the group's selected positions (ascending after sfi_compact; after
+ * sfi_compact_incremental, rows that stayed selected keep their slots), then
+ * zero rows up to a multiple of 16.  Readers treat the rows as a set.
  *  k, v      bf16  [B, Hkv, p_max, D]
  *  pos       int32 [B, Hkv, p_max]   cache position of each row
  *  headmask  uint32[B, Hkv, p_max]   bit h set: query head h of the group
@@ -270,6 +271,25 @@ sfi_status sfi_compact(const sfi_shape* shape, const sfi_params* params, const s
                        int32_t L, const int32_t* sel_idx, int32_t sel_ld, int32_t K,
                        sfi_packed* packed, void* ws, size_t ws_bytes, sfi_stream stream);
 
+/* Incremental compaction (the support of consecutive slow steps overlaps
+ * strongly, "Slow-Fast Inference", within-sentence support stability): same
+ * arguments and result set as sfi_compact, but `packed` must hold the previous
+ * compaction of the same sequences and KV heads (by sfi_compact or this call,
+ * same params, cache rows unchanged since), unless fresh != 0 or its n_rows is
+ * 0.  Rows whose position stays selected keep their slot (head mask
+ * rewritten); with U the new union and n_new = n_sink + |U|, the slots in
+ * [n_sink, n_new) that are not kept receive, in slot order, the positions of
+ * U not in the previous buffer (ascending) and then the kept rows at slots >=
+ * n_new (in slot order), copied from the pages.  Rows [n_new, next multiple
+ * of 16): zero, pos -1, mask 0.  A fresh buffer gets the layout of
+ * sfi_compact.  packed->p_max must be at least the packed row capacity
+ * (SFI_ERR_SHAPE otherwise).  ws as for sfi_select: zero-filled before its
+ * first use, left so by every call. */
+sfi_status sfi_compact_incremental(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
+                                   int32_t L, const int32_t* sel_idx, int32_t sel_ld, int32_t K,
+                                   sfi_packed* packed, int32_t fresh, void* ws, size_t ws_bytes,
+                                   sfi_stream stream);
+
 /* Read the latched device error word of kv (synchronous), then clear it. */
 sfi_status sfi_poll_error(const sfi_paged_kv* kv, int32_t* code);
 
@@ -305,6 +325,13 @@ sfi_status sfi_decode_step(sfi_ctx* ctx, int32_t layer, int32_t step, int32_t bo
                            int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
                            const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
                            float* out, sfi_stream stream, int32_t* was_slow);
+
+/* Compaction used by slow steps: incremental != 0 (the default) refreshes a
+ * layer's packed buffer with sfi_compact_incremental's layout once that buffer
+ * holds this context's previous refresh of the layer (the first slow step of
+ * a layer, step 0, a new workspace or another packed buffer rebuild it
+ * fully); 0: sfi_compact's full rebuild at every slow step. */
+sfi_status sfi_ctx_set_compaction(sfi_ctx* ctx, int32_t incremental);
 
 /* Make `stream` wait for every outstanding side-stream refresh of ctx. */
 sfi_status sfi_ctx_join(sfi_ctx* ctx, sfi_stream stream);

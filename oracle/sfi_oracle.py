@@ -322,6 +322,48 @@ def compact(selected: np.ndarray, n_sink: int):
     return np.asarray(pos, np.int64), np.asarray(hm, np.uint32)
 
 
+def compact_incremental(prev_pos, n_prev: int, selected: np.ndarray, n_sink: int):
+    """Packed rows of one (sequence, KV head) refreshed from the previous
+    buffer's rows prev_pos[:n_prev] (n_prev = 0: none) rather than rebuilt.
+
+    READING (the pages name the coalesced buffer and the stability of the
+    support across consecutive slow steps — "Slow-Fast Inference",
+    within-sentence support stability — but no refresh rule): with U the new
+    union (as `compact` forms it) and n_new = n_sink + |U|,
+      * a previous row whose position is in U keeps its slot;
+      * holes: slots in [n_sink, n_new) holding no kept row, ascending;
+      * movers: positions of U not among the previous rows, ascending, then
+        the positions of kept rows at slots >= n_new, by slot;
+      * the i-th mover goes to the i-th hole.
+    Head masks are those of U.  Returns (pos int64 [n_new], headmask uint32
+    [n_new], moved: the number of rows written from the cache).
+    """
+    pos_full, hm_full = compact(selected, n_sink)
+    mask_of = dict(zip(pos_full.tolist(), hm_full.tolist()))
+    union = [p for p in pos_full.tolist()[n_sink:]]
+    n_new = n_sink + len(union)
+    if n_prev == 0:
+        return pos_full, hm_full, n_new
+    prev = [int(p) for p in prev_pos[:n_prev]]
+    in_union = set(union)
+    layout = {}
+    for s_ in range(n_sink):
+        layout[s_] = s_
+    kept_slots = [s_ for s_ in range(n_sink, n_prev) if prev[s_] in in_union]
+    for s_ in kept_slots:
+        if s_ < n_new:
+            layout[s_] = prev[s_]
+    prev_set = set(prev[n_sink:])
+    holes = [s_ for s_ in range(n_sink, n_new) if s_ not in layout]
+    movers = [p for p in union if p not in prev_set] + [prev[s_] for s_ in kept_slots if s_ >= n_new]
+    assert len(movers) == len(holes)
+    for s_, p in zip(holes, movers):
+        layout[s_] = p
+    pos = np.asarray([layout[s_] for s_ in range(n_new)], np.int64)
+    hm = np.asarray([mask_of[p] for p in pos.tolist()], np.uint32)
+    return pos, hm, len(movers)
+
+
 # ----------------------------------------------------------------------------
 # Trigger
 # ----------------------------------------------------------------------------

@@ -66,7 +66,7 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   w.sel_bytes = align_up((size_t)s.B * s.Hq * ((nC + 3) / 4 * 4) * sizeof(float), 256);
   off += w.sel_bytes;
   w.cmp_off = off;
-  w.cmp_bytes = align_up((size_t)bh * compact_tiles((int)nC) * sizeof(int32_t), 256);
+  w.cmp_bytes = align_up(compact_scratch_bytes(s, p), 256);
   off += w.cmp_bytes;
   w.bits_ld = (nC + 31) / 32;
   w.bits_off = off;
@@ -368,7 +368,29 @@ sfi_status sfi_compact(const sfi_shape* shape, const sfi_params* params, const s
   cudaStream_t st = (cudaStream_t)stream;
   SFI_TRY(run_idx_to_bits(*shape, *params, *kv, L, sel_idx, sel_ld, K, bits, w.bits_ld, st));
   return run_compact_bits(*shape, *params, *kv, bits, w.bits_ld, *packed,
-                          reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.cmp_off), w.cmp_bytes, L, st);
+                          compact_scratch(static_cast<char*>(ws) + w.cmp_off, *shape, *params), L, st);
+}
+
+sfi_status sfi_compact_incremental(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
+                                   int32_t L, const int32_t* sel_idx, int32_t sel_ld, int32_t K,
+                                   sfi_packed* packed, int32_t fresh, void* ws, size_t ws_bytes,
+                                   sfi_stream stream) {
+  SFI_TRY(check_shape(shape));
+  SFI_TRY(check_params(params));
+  SFI_TRY(check_kv(kv));
+  SFI_TRY(check_sparse_L(shape, params, L));
+  SFI_TRY(check_packed(shape, params, packed));
+  if (!sel_idx) return SFI_ERR_INVALID_ARG;
+  const int nC = L - params->n_recent - params->n_sink;
+  if (K < 1 || K > nC || sel_ld < K) return SFI_ERR_SHAPE;
+  if (packed->p_max < packed_rows_capacity(*shape, *params)) return SFI_ERR_SHAPE;
+  const WsLayout w = ws_layout(*shape, *params);
+  if (!ws || ws_bytes < w.total) return SFI_ERR_WORKSPACE;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + w.bits_off);
+  cudaStream_t st = (cudaStream_t)stream;
+  SFI_TRY(run_idx_to_bits(*shape, *params, *kv, L, sel_idx, sel_ld, K, bits, w.bits_ld, st));
+  return run_compact_inc(*shape, *params, *kv, bits, w.bits_ld, *packed,
+                         compact_scratch(static_cast<char*>(ws) + w.cmp_off, *shape, *params), L, fresh != 0, st);
 }
 
 sfi_status sfi_poll_error(const sfi_paged_kv* kv, int32_t* code) {

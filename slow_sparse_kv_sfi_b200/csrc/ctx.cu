@@ -10,6 +10,7 @@
 // layer i waits for that refresh before it touches the layer's cache or
 // packed buffer.  A logits buffer is rewritten only after the side stream has
 // finished reading it.
+#include <algorithm>
 #include <vector>
 
 #include "common.cuh"
@@ -40,8 +41,11 @@ struct sfi_ctx {
   uint32_t* bits = nullptr;
   int64_t bits_ld = 0;
   char* topk_ws = nullptr;
-  int32_t* tile_counts = nullptr;
-  size_t tc_bytes = 0;
+  sfi::CompactScratch cmp;
+  // compaction: incremental (rows that stay selected keep their slots) once
+  // a layer's packed buffer holds this context's previous result
+  int incremental = 1;
+  std::vector<const void*> packed_seen;   // per layer: pos pointer of the last refresh
   std::vector<sfi::AttnMapCache> maps;   // per layer
   // timing of the attention kernels (kind 0 fast, 1 dense) of every
   // timing-th layer (0: off)
@@ -142,6 +146,7 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->ev_sel.resize(n_layers, nullptr);
   c->pending.assign(n_layers, 0);
   c->maps.resize(n_layers);
+  c->packed_seen.assign(n_layers, nullptr);
   for (int i = 0; i < n_layers && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
@@ -196,9 +201,10 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   c->scores = reinterpret_cast<float*>(w + l.score_off);
   c->bits = reinterpret_cast<uint32_t*>(w + l.bits_off);
   c->bits_ld = l.bits_ld;
-  c->tile_counts = reinterpret_cast<int32_t*>(w + l.tc_off);
+  c->cmp = compact_scratch(w + l.tc_off, c->s, c->p);
   c->topk_ws = w + l.tk_off;
-  c->tc_bytes = l.tc_bytes;
+  // a new workspace holds no previous-selection state
+  std::fill(c->packed_seen.begin(), c->packed_seen.end(), nullptr);
   return SFI_OK;
 }
 
@@ -268,13 +274,28 @@ sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boun
   SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
   SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld,
                    topk_scratch(c->topk_ws, s.B * s.Hq, nC), side));
-  SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->tile_counts, c->tc_bytes, L, side));
+  if (c->incremental && packed->p_max >= c->cmp.cap) {
+    // step 0 starts a new decode: cache rows copied before may have changed
+    const bool fresh = step == 0 || c->packed_seen[layer] != packed->pos;
+    SFI_TRY(run_compact_inc(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, fresh, side));
+    c->packed_seen[layer] = packed->pos;
+  } else {
+    SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, side));
+    c->packed_seen[layer] = nullptr;
+  }
   SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
   if (c->overlap) {
     c->pending[layer] = 1;
   } else {
     SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
   }
+  return SFI_OK;
+}
+
+sfi_status sfi_ctx_set_compaction(sfi_ctx* c, int32_t incremental) {
+  if (!c) return SFI_ERR_INVALID_ARG;
+  c->incremental = incremental ? 1 : 0;
+  std::fill(c->packed_seen.begin(), c->packed_seen.end(), nullptr);
   return SFI_OK;
 }
 

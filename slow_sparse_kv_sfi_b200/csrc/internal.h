@@ -133,9 +133,28 @@ TopkScratch topk_scratch(void* base, int rows, int n);
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
                     int64_t ld_i, uint32_t* bits, int64_t ld_b, const TopkScratch& w, cudaStream_t st);
 int topk_max_n();
+// Compaction scratch (inside the workspace): per-tile counts of the full
+// compaction, and the incremental compaction's counts, previous-position
+// bitmap (zero between calls), mover and hole lists.
+struct CompactScratch {
+  int32_t* wcounts = nullptr;   // [BH][n_tiles][2]
+  size_t wcount_bytes = 0;
+  int32_t* scounts = nullptr;   // [BH][slot tiles][2]
+  uint32_t* oldbits = nullptr;  // [BH][nw]
+  int32_t* mover_pos = nullptr; // [BH][cap]
+  int32_t* hole_slot = nullptr; // [BH][cap]
+  int32_t* info = nullptr;      // [BH][4]
+  int cap = 0;                  // packed_rows_capacity
+};
+size_t compact_scratch_bytes(const sfi_shape& s, const sfi_params& p);
+CompactScratch compact_scratch(void* base, const sfi_shape& s, const sfi_params& p);
 sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                             const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,
-                            int32_t* tile_counts, size_t tc_bytes, int L_slow, cudaStream_t st);
+                            const CompactScratch& cs, int L_slow, cudaStream_t st);
+// fresh: build from scratch (sinks + union ascending) whatever the buffer holds
+sfi_status run_compact_inc(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
+                           const uint32_t* bits, int64_t ld_b, const sfi_packed& pk, const CompactScratch& cs,
+                           int L_slow, bool fresh, cudaStream_t st);
 sfi_status run_idx_to_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L_slow,
                            const int32_t* sel_idx, int sel_ld, int K, uint32_t* bits, int64_t ld_b,
                            cudaStream_t st);

@@ -121,9 +121,9 @@ struct ScoreArgs {
 
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes the log-score
 // of every head of the group over the tile plus a halo of w on each side to
-// shared memory (NaN outside C: a NaN never dominates).  Phase 2: the thread
-// of a position applies soft-NMS to every head in registers, picks the owner
-// and writes l''.
+// shared memory (NaN outside C: a NaN never dominates).  Phase 2 finds every
+// head's nearest dominator (two passes, below), then the thread of a position
+// applies soft-NMS to every head, picks the owner and writes l''.
 template <int GM>
 __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   grid_dep_enter();
@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   const int tile_n = min(a.tile, a.nC - c0);
   const int G = a.G;
   __shared__ double bc;
+  __shared__ int qn;
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
   const float nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
   const float inv_z = (float)(1.0 / reduce_parts(pbg, a.nch, 1, &bc));
@@ -187,6 +188,65 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
       }
     }
   }
+  if (threadIdx.x == 0) qn = 0;
+  __syncthreads();
+  // Phase 2a: distances 1..kNear of every head for every position (no early
+  // exit, so a warp does not wait for its local maxima); positions with a head
+  // still undecided go to a queue.  2b: the queue, scanned to w with all lanes
+  // busy.  dom = distance of the nearest dominator, 0: none within w.
+  constexpr int kNear = 4;
+  uint16_t* dom = reinterpret_cast<uint16_t*>(ell + G * W);            // [G][tile]
+  uint32_t* queue = reinterpret_cast<uint32_t*>(dom + G * a.tile);     // [tile]
+  const int lane = threadIdx.x & 31;
+  for (int k0 = 0; k0 < tile_n; k0 += blockDim.x) {
+    const int k = k0 + threadIdx.x;
+    uint32_t open = 0u;
+    if (k < tile_n) {
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          const float* row = ell + h * W + a.w + k;
+          const float e = row[0];
+          int d_hit = 0;
+#pragma unroll
+          for (int d = kNear; d >= 1; --d) {   // descending: the nearest hit stays
+            const int dd = min(d, a.w);
+            if (d <= a.w && (row[-dd] >= e || row[dd] > e)) d_hit = d;   // NaN compares false
+          }
+          dom[h * a.tile + k] = (uint16_t)d_hit;
+          if (d_hit == 0 && a.w > kNear) open |= 1u << h;
+        }
+      }
+    }
+    const unsigned ball = __ballot_sync(0xffffffffu, open != 0u);
+    if (ball) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&qn, __popc(ball));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (open) queue[base + __popc(ball & ((1u << lane) - 1u))] = (uint32_t)k | (open << 16);
+    }
+  }
+  __syncthreads();
+  const int nq = qn;
+  for (int qi = threadIdx.x; qi < nq; qi += blockDim.x) {
+    const uint32_t ent = queue[qi];
+    const int k = (int)(ent & 0xffffu);
+    uint32_t open = ent >> 16;
+    while (open) {
+      const int h = __ffs(open) - 1;
+      open &= open - 1u;
+      const float* row = ell + h * W + a.w + k;
+      const float e = row[0];
+      int d_hit = 0;
+      for (int d = kNear + 1; d <= a.w; ++d) {
+        if (row[-d] >= e || row[d] > e) {
+          d_hit = d;
+          break;
+        }
+      }
+      dom[h * a.tile + k] = (uint16_t)d_hit;
+    }
+  }
   __syncthreads();
   const float inv_w = 1.f / (float)a.w;
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
@@ -195,16 +255,9 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
     for (int h = 0; h < GM; ++h) {
       l1[h] = -INFINITY;
       if (h < G) {
-        const float* row = ell + h * W + a.w + k;
-        const float e = row[0];
-        float pen = 0.f;
-        for (int d = 1; d <= a.w; ++d) {
-          if (row[-d] >= e || row[d] > e) {   // NaN (outside C) compares false
-            pen = 1.f - (float)(d - 1) * inv_w;
-            break;
-          }
-        }
-        l1[h] = e - a.alpha_soft * pen;
+        const int d = dom[h * a.tile + k];
+        const float pen = d > 0 ? 1.f - (float)(d - 1) * inv_w : 0.f;
+        l1[h] = ell[h * W + a.w + k] - a.alpha_soft * pen;
       }
     }
     int owner = 0;
@@ -228,7 +281,11 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
 // ---------------------------------------------------------------- host
 int score_tile(int G) { return std::max(256, 4096 / G); }
 
-size_t score_smem(int G, int tile, int w) { return (size_t)G * (tile + 2 * w) * sizeof(float); }
+// log-scores with halo, nearest-dominator distances, queue of undecided positions
+size_t score_smem(int G, int tile, int w) {
+  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(uint16_t) +
+         (size_t)tile * sizeof(uint32_t);
+}
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }
 

@@ -85,6 +85,7 @@ def _declare(L):
         "sfi_topk": (C.c_int, [I32, I32, P, I64, I32, I32, P, I64, P, SZ, P]),
         "sfi_select": (C.c_int, [P, P, P, I32, P, I64, P, P, I32, C.POINTER(I32), P, SZ, P]),
         "sfi_compact": (C.c_int, [P, P, P, I32, P, I32, I32, P, P, SZ, P]),
+        "sfi_compact_incremental": (C.c_int, [P, P, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "sfi_poll_error": (C.c_int, [P, C.POINTER(I32)]),
         "sfi_ctx_create": (C.c_int, [P, P, I32, I32, C.POINTER(P)]),
         "sfi_ctx_destroy": (C.c_int, [P]),
@@ -93,6 +94,7 @@ def _declare(L):
         "sfi_decode_step": (C.c_int, [P, I32, I32, I32, I32, P, P, P, P, P, P, P, C.POINTER(I32)]),
         "sfi_ctx_join": (C.c_int, [P, P]),
         "sfi_ctx_set_timing": (C.c_int, [P, I32]),
+        "sfi_ctx_set_compaction": (C.c_int, [P, I32]),
         "sfi_ctx_timing": (C.c_int, [P, I32, C.POINTER(C.c_double), C.POINTER(I64), I32]),
     }
     for name, (res, args) in sig.items():
@@ -104,9 +106,11 @@ def _declare(L):
 EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_rows", "sfi_budget",
             "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_append",
             "sfi_dense_attn_noalloc", "sfi_attn_probs", "sfi_fast_attn", "sfi_fast_attn_append",
-            "sfi_select_scores", "sfi_topk_workspace_size", "sfi_topk", "sfi_select", "sfi_compact", "sfi_poll_error",
+            "sfi_select_scores", "sfi_topk_workspace_size", "sfi_topk", "sfi_select", "sfi_compact",
+            "sfi_compact_incremental", "sfi_poll_error",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
-            "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_timing"]
+            "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_compaction",
+            "sfi_ctx_timing"]
 
 
 def _check(st: int, where: str):
@@ -254,6 +258,12 @@ def sfi_compact(shape, params, kv, L, sel_idx, sel_ld, K, packed, ws, stream=Non
            "sfi_compact")
 
 
+def sfi_compact_incremental(shape, params, kv, L, sel_idx, sel_ld, K, packed, fresh, ws, stream=None):
+    _check(lib().sfi_compact_incremental(C.byref(shape), C.byref(params), C.byref(kv), L, _p(sel_idx), sel_ld, K,
+                                         C.byref(packed), int(fresh), _p(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "sfi_compact_incremental")
+
+
 def sfi_poll_error(kv) -> int:
     code = C.c_int32(0)
     _check(lib().sfi_poll_error(C.byref(kv), C.byref(code)), "sfi_poll_error")
@@ -264,7 +274,7 @@ class Context:
     """Owns an sfi_ctx (side stream, per-layer events) and its workspace tensor."""
 
     def __init__(self, shape: Shape, params: Params, n_layers: int, overlap: bool = True,
-                 device=None):
+                 device=None, incremental: bool = True):
         self.shape, self.params = shape, params
         h = C.c_void_p()
         _check(lib().sfi_ctx_create(C.byref(shape), C.byref(params), n_layers, int(overlap),
@@ -274,6 +284,7 @@ class Context:
         _check(lib().sfi_ctx_workspace_size(h, C.byref(n)), "sfi_ctx_workspace_size")
         self.ws = torch.empty(n.value, dtype=torch.uint8, device=device or "cuda")
         _check(lib().sfi_ctx_set_workspace(h, _p(self.ws), n.value), "sfi_ctx_set_workspace")
+        _check(lib().sfi_ctx_set_compaction(h, int(incremental)), "sfi_ctx_set_compaction")
         self._slow = C.c_int32(0)
 
     def decode_step(self, layer, step, boundary_prev, L, kv, packed, q, k_new, v_new, out,

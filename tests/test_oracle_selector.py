@@ -229,6 +229,66 @@ def test_compact_hand_worked():
     np.testing.assert_array_equal(hm, g["headmask"])
 
 
+def test_compact_incremental_hand_worked():
+    g = _golden("compact_incremental_example.json")
+    for case in g["cases"]:
+        prev = np.array(case["prev_pos"])
+        pos, hm, moved = O.compact_incremental(prev, len(prev), np.array(case["selected"]), g["n_sink"])
+        np.testing.assert_array_equal(pos, case["pos"])
+        np.testing.assert_array_equal(hm, case["headmask"])
+        assert moved == case["moved"]
+
+
+def _random_selection(rng, lo, hi, G, K, prev=None, keep=0.9):
+    out = []
+    for h in range(G):
+        base = rng.choice(np.arange(lo, hi), size=K, replace=False) if prev is None else prev[h].copy()
+        if prev is not None:
+            swap = rng.random(K) > keep
+            fresh = rng.choice(np.setdiff1d(np.arange(lo, hi), base), size=int(swap.sum()), replace=False)
+            base[swap] = fresh
+        out.append(np.sort(base))
+    return np.stack(out)
+
+
+def test_compact_incremental_fresh_equals_full_compaction():
+    rng = np.random.default_rng(3)
+    sel = _random_selection(rng, 4, 300, 4, 40)
+    pos, hm, moved = O.compact_incremental(np.zeros(0), 0, sel, 4)
+    ref_pos, ref_hm = O.compact(sel, 4)
+    np.testing.assert_array_equal(pos, ref_pos)
+    np.testing.assert_array_equal(hm, ref_hm)
+    assert moved == len(pos)
+
+
+@pytest.mark.parametrize("keep", [1.0, 0.95, 0.5, 0.0])
+def test_compact_incremental_is_the_union_with_stable_slots(keep):
+    """Against the full compaction (pinned above): the same (position, mask)
+    rows as a set; every previous row that stays selected and fits below n_new
+    keeps its slot; exactly the entering and displaced rows are written."""
+    rng = np.random.default_rng(int(keep * 100))
+    n_sink, G = 4, 4
+    prev_sel = _random_selection(rng, n_sink, 400, G, 30)
+    prev_pos, _, _ = O.compact_incremental(np.zeros(0), 0, prev_sel, n_sink)
+    for _ in range(6):
+        sel = _random_selection(rng, n_sink, 400, G, 30, prev_sel, keep)
+        pos, hm, moved = O.compact_incremental(prev_pos, len(prev_pos), sel, n_sink)
+        ref_pos, ref_hm = O.compact(sel, n_sink)
+        assert sorted(zip(pos.tolist(), hm.tolist())) == sorted(zip(ref_pos.tolist(), ref_hm.tolist()))
+        assert len(set(pos.tolist())) == len(pos)
+        new = set(ref_pos.tolist())
+        same = [s for s in range(min(len(pos), len(prev_pos))) if prev_pos[s] in new and pos[s] == prev_pos[s]]
+        should = [s for s in range(min(len(pos), len(prev_pos))) if prev_pos[s] in new]
+        assert same == should
+        entering = len(new - set(prev_pos.tolist()))
+        displaced = sum(1 for s in range(len(pos), len(prev_pos)) if prev_pos[s] in new)
+        assert moved == entering + displaced
+        assert moved == sum(1 for s in range(n_sink, len(pos)) if s >= len(prev_pos) or pos[s] != prev_pos[s])
+        if keep == 1.0:
+            assert moved == 0
+        prev_pos, prev_sel = pos, sel
+
+
 def test_trigger_hand_worked():
     for case in _golden("trigger_example.json")["cases"]:
         got = O.trigger(np.array(case["boundary"], np.int8), case["M"])
