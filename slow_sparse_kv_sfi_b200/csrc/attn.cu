@@ -231,12 +231,12 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     }
     const uint64_t policy = l2_policy_evict_first();
     const int G = a.G;
-    // Work items come from a global counter; the next item's index and page
-    // table entries are fetched one item ahead so their latency overlaps the
-    // current item's copies.
-    int nxt = 0;
-    if (lane == 0) nxt = atomicAdd(a.ctr, 1);
-    nxt = __shfl_sync(0xffffffffu, nxt, 0);
+    // CTA i starts on item i without a round trip to memory (the grid is no
+    // larger than the CTAs that fit at once); the later items come from a
+    // global counter, offset by the grid.  The next
+    // item's index and page table entries are fetched ahead so their latency
+    // overlaps the current item's copies.
+    int nxt = blockIdx.x;
     int pf[kMaxChunkTiles / 32];
     auto prefetch = [&](int item, int* regs) {
 #pragma unroll
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     bool drawn = false;
     auto draw_next = [&]() {
       int v = 0;
-      if (lane == 0) v = atomicAdd(a.ctr, 1);
+      if (lane == 0) v = atomicAdd(a.ctr, 1) + (int)gridDim.x;
       nxt = __shfl_sync(0xffffffffu, v, 0);
       prefetch(nxt, pf);
       drawn = true;
