@@ -243,9 +243,10 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
 /* Per-row top-K: the K largest of scores[r, 0:n] (finite values; ties ->
  * lower index), written ascending as idx[r, 0:K] = offset + column.  rows =
  * number of rows; scores row stride ld_s, idx row stride ld_i (elements);
- * n <= 262144.  ws: device scratch of sfi_topk_workspace_size bytes, 16-byte
- * aligned, zero-filled before its first use; every successful call leaves it
- * ready for the next one (after an error, zero it again).  Every row is cut
+ * n <= 262144.  ws: device scratch of sfi_topk_workspace_size(rows, n) bytes,
+ * 16-byte aligned, zero-filled before its first use; every successful call
+ * leaves it ready for the next one with the same rows (zero it again after an
+ * error or before a call with another row count).  Every row is cut
  * into slices with one CTA each: a histogram of linear bins over the row's
  * [min, max], the boundary bin of the K-th score, an exact radix select of
  * the threshold among the boundary candidates, ties in position order. */
@@ -320,7 +321,8 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* ctx, void* ws, size_t bytes);
  *     fast step: wait for this layer's pending refresh, then sparse attention
  *     over packed + recent -> out.
  *  q bf16 [B,Hq,D]; k_new, v_new bf16 [B,Hkv,D]; out fp32 [B,Hq,D].
- *  *was_slow (may be NULL) receives the step's decision. */
+ *  *was_slow (may be NULL) receives the step's decision (1 when any sequence
+ *  is slow, after sfi_decode_step_rows on the same context). */
 sfi_status sfi_decode_step(sfi_ctx* ctx, int32_t layer, int32_t step, int32_t boundary_prev,
                            int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
                            const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
@@ -332,6 +334,23 @@ sfi_status sfi_decode_step(sfi_ctx* ctx, int32_t layer, int32_t step, int32_t bo
  * a layer, step 0, a new workspace or another packed buffer rebuild it
  * fully); 0: sfi_compact's full rebuild at every slow step. */
 sfi_status sfi_ctx_set_compaction(sfi_ctx* ctx, int32_t incremental);
+
+/* Per-sequence triggers ([ES] §2 Pasos Lentos: the boundary that makes a
+ * step slow is a token of one sequence): sfi_decode_step with one trigger
+ * per sequence.  boundary_prev: host int32 [B], sequence b emitted a boundary
+ * token at the previous step (NULL: none).  At layer 0 every sequence b is
+ * decided: slow when step == 0, boundary_prev[b] != 0, or step minus its last
+ * slow step >= refresh_budget.  A step whose sequences are all slow (all
+ * fast) runs as in sfi_decode_step; a mixed step runs, per layer, the dense
+ * attention on the slow sequences (and, on the side stream, the Selector and
+ * compaction of their packed buffers) and the fast attention on the others.
+ * slow_rows: host int32 [B] receiving the decisions (may be NULL).  B <= 256
+ * (SFI_ERR_UNSUPPORTED otherwise).  sfi_decode_step on the same context
+ * applies its boundary flag to every sequence. */
+sfi_status sfi_decode_step_rows(sfi_ctx* ctx, int32_t layer, int32_t step, const int32_t* boundary_prev,
+                                int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
+                                const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
+                                float* out, sfi_stream stream, int32_t* slow_rows);
 
 /* Make `stream` wait for every outstanding side-stream refresh of ctx. */
 sfi_status sfi_ctx_join(sfi_ctx* ctx, sfi_stream stream);

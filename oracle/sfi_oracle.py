@@ -384,6 +384,16 @@ def trigger(boundary: np.ndarray, refresh_budget: int) -> np.ndarray:
     return slow
 
 
+def trigger_rows(boundary: np.ndarray, refresh_budget: int) -> np.ndarray:
+    """Slow-step schedules of a batch whose sequences trigger independently:
+    `trigger` applied to every sequence's own boundary stream (boundary
+    [B, T] -> bool [B, T]).
+    READING: the boundary that makes a step slow is a token of one sequence
+    ([ES] "2. Metodología", Pasos Lentos), so in a batch each sequence has its
+    own schedule and its own refresh budget."""
+    return np.stack([trigger(np.asarray(row), refresh_budget) for row in boundary])
+
+
 # ----------------------------------------------------------------------------
 # A whole decode run (one layer), for end-to-end checks on small workloads
 # ----------------------------------------------------------------------------

@@ -72,6 +72,7 @@ struct AttnArgs {
   __nv_bfloat16* v_pool;
   float* norms;
   int64_t norm_ld;
+  RowMap rows;          // the sequences of this launch
 };
 
 constexpr int kMaxChunkTiles = 256;
@@ -133,10 +134,12 @@ struct Item {
 template <int MODE, int TPS>
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int item, const int* nrows_s) {
   Item it;
-  it.bg = item / a.n_chunks;
-  const int c = item - it.bg * a.n_chunks;
-  it.b = it.bg / a.Hkv;
-  it.g = it.bg - it.b * a.Hkv;
+  const int bgl = item / a.n_chunks;   // logical (row of the launch, kv head)
+  const int c = item - bgl * a.n_chunks;
+  const int bl = bgl / a.Hkv;
+  it.g = bgl - bl * a.Hkv;
+  it.b = a.rows.phys(bl);
+  it.bg = it.b * a.Hkv + it.g;
   if (MODE != kFast) {
     const int T = (a.L + kPage - 1) / kPage;
     it.t_total = T;
@@ -179,7 +182,7 @@ struct Maps {
 
 template <int D, int NT, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
-    attn_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
+    attn_kernel(const __grid_constant__ Maps maps, const __grid_constant__ AttnArgs a) {
   using S = Smem<D, NT>;
   using P = Plan<D, NT>;
   constexpr int kStages = S::kStages;
@@ -682,16 +685,19 @@ template <int D>
 __global__ void __launch_bounds__(kCombWarps * 32)
     attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
                         float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
-                        const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr) {
+                        const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
+                        const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   constexpr int kPer = D / 32;     // columns of O per lane
   static_assert(kPer == 4 || kPer == 2, "head dim");
   __shared__ float red[kCombWarps][D + 4];
   if (blockIdx.x == 0 && threadIdx.x == 0) ctr[0] = 0;   // the attention kernel is done with it
-  const int row = blockIdx.x;   // b * Hq + hq
-  const int b = row / Hq, hq = row - b * Hq;
+  const int bl = blockIdx.x / Hq, hq = blockIdx.x - bl * Hq;   // logical row of the launch, query head
+  const int b = rows.phys(bl);
+  const int row = b * Hq + hq;
   const int g = hq / G, hh = hq - g * G;
-  const int bg = b * Hkv + g;
+  const int bg = b * Hkv + g;            // the sequence's (b, kv head)
+  const int bgl = bl * Hkv + g;          // its partials
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (n_rows && threadIdx.x == 0 && hh == 0) {
     const int nr = n_rows[bg];
@@ -710,7 +716,7 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     chunks = (T + ct - 1) / ct;
   }
   const int n = chunks * kConsumerWarps;
-  const float* base = part + (size_t)bg * n_chunks * kConsumerWarps * stride + (size_t)hh * (D + 4);
+  const float* base = part + (size_t)bgl * n_chunks * kConsumerWarps * stride + (size_t)hh * (D + 4);
   float m = -INFINITY, l = 0.f, lc = 0.f;
   float acc[kPer];
 #pragma unroll
@@ -932,15 +938,15 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int rec_tiles, int tps,
-                          int* err, int* ctr, cudaStream_t st) {
+                          int* err, int* ctr, cudaStream_t st, const RowMap& rows) {
   const int G = s.Hq / s.Hkv;
-  const int grid = s.B * s.Hq;
+  const int grid = rows.count(s.B) * s.Hq;
   if (D == 128)
     launch_k(attn_combine_kernel<128>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr);
+             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr, rows);
   else
     launch_k(attn_combine_kernel<64>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr);
+             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr, rows);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -1026,8 +1032,9 @@ void set_token(AttnArgs& a, const sfi_shape& s, const sfi_paged_kv& kv, const St
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
-                          const StepToken* tok, AttnMapCache* cache) {
+                          const StepToken* tok, AttnMapCache* cache, const RowMap& rmap) {
   const int G = s.Hq / s.Hkv;
+  if (rmap.count(s.B) < 1 || rmap.count(s.B) > s.B) return SFI_ERR_SHAPE;
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
   if (!paged_maps(&maps, kv, rows, s.D, cache)) return SFI_ERR_CUDA;
@@ -1042,7 +1049,9 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   a.chunk_tiles = dense_chunk_tiles(s, L);
   const int T = (L + kPage - 1) / kPage;
   a.n_chunks = (T + a.chunk_tiles - 1) / a.chunk_tiles;
-  a.n_items = s.B * s.Hkv * a.n_chunks;
+  // chunking of the whole batch also for a subset: the partials fit the workspace
+  a.rows = rmap;
+  a.n_items = rmap.count(s.B) * s.Hkv * a.n_chunks;
   if (attn_part_bytes(a.n_items, G, s.D) > part_bytes) return SFI_ERR_WORKSPACE;
   a.part = part;
   a.scale = 1.0f / sqrtf((float)s.D);
@@ -1066,9 +1075,10 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
   r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0, 0, 1,
-                     kv.err, ctr, st);
+                     kv.err, ctr, st, rmap);
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
+    if (rmap.n) return SFI_ERR_UNSUPPORTED;   // probabilities of the whole batch only
     dim3 grid((L + 1023) / 1024 < 64 ? (L + 1023) / 1024 : 64, s.B * s.Hq);
     launch_k(probs_kernel, dim3(grid), dim3(256), 0, st, L, s.Hq, zbuf, ex->ld, lse_tmp, ex->probs);
     if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
@@ -1079,8 +1089,9 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end, const StepToken* tok, AttnMapCache* cache) {
+                         cudaEvent_t ev_end, const StepToken* tok, AttnMapCache* cache, const RowMap& rmap) {
   const int G = s.Hq / s.Hkv;
+  if (rmap.count(s.B) < 1 || rmap.count(s.B) > s.B) return SFI_ERR_SHAPE;
   if ((long)s.B * s.Hkv > kMaxBH) return SFI_ERR_UNSUPPORTED;
   Maps maps;
   const uint64_t rows = (uint64_t)s.num_pages * s.Hkv * kPage;
@@ -1095,7 +1106,8 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
   a.ctr = ctr;
   a.n_chunks = fast_chunks(s, pk.p_max, p.n_recent, std::max(budget_k(p, L), 0) * 1 + p.n_sink);
-  a.n_items = s.B * s.Hkv * a.n_chunks;
+  a.rows = rmap;
+  a.n_items = rmap.count(s.B) * s.Hkv * a.n_chunks;
   if (attn_part_bytes(a.n_items, G, s.D) > part_bytes) return SFI_ERR_WORKSPACE;
   a.part = part;
   a.scale = 1.0f / sqrtf((float)s.D);
@@ -1112,7 +1124,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   if (r != SFI_OK) return r;
   const int rec_tiles = (L - 1) / kPage - a.rec_lo / kPage + 1;
   return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, rec_tiles, nts, kv.err,
-                        ctr, st);
+                        ctr, st, rmap);
 }
 
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,

@@ -38,6 +38,7 @@ struct CompactArgs {
   int32_t* n_rows;
   int32_t* tile_counts;   // [B*Hkv][n_tiles]
   int* err;
+  RowMap rows;            // bits and scratch: logical rows; everything else: the sequences
 };
 
 template <int GM>
@@ -52,7 +53,7 @@ __device__ __forceinline__ uint32_t union_word(const CompactArgs& a, int b, int 
 }
 
 template <int GM>
-__global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactArgs a) {
+__global__ void __launch_bounds__(kCThreads) compact_count_kernel(const __grid_constant__ CompactArgs a) {
   grid_dep_enter();
   __shared__ int wsum[kCThreads / 32];
   const int bg = blockIdx.y;
@@ -72,12 +73,14 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const CompactA
 }
 
 template <int GM>
-__global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const CompactArgs a) {
+__global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const __grid_constant__ CompactArgs a) {
   grid_dep_enter();
   __shared__ int wtot[kCThreads / 32 + 1];
   __shared__ int base_s, total_s;
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
+  const int bp = a.rows.phys(b);                  // the sequence
+  const int bgp = bp * a.Hkv + g;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kWarps = kCThreads / 32;
   const int w = blockIdx.x * kCWords + threadIdx.x;
@@ -114,8 +117,8 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   const int base = base_s;
   const int total = min(total_s, max(a.p_max - base, 0));
   if (total < total_s && threadIdx.x == 0) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
-  int32_t* pos = a.pos + (size_t)bg * a.p_max;
-  uint32_t* hm = a.headmask + (size_t)bg * a.p_max;
+  int32_t* pos = a.pos + (size_t)bgp * a.p_max;
+  uint32_t* hm = a.headmask + (size_t)bgp * a.p_max;
   int r = x - cnt + wtot[warp];
   uint32_t t = u;
   while (t) {
@@ -141,7 +144,7 @@ __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const Compact
   }
   if (blockIdx.x == gridDim.x - 1) {
     const int n = min(base + total_s, a.p_max);
-    if (threadIdx.x == 0) a.n_rows[bg] = n;
+    if (threadIdx.x == 0) a.n_rows[bgp] = n;
     const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
     for (int rr = n + threadIdx.x; rr < pad_end; rr += kCThreads) {
       pos[rr] = -1;
@@ -161,7 +164,7 @@ constexpr int kCopyRows = 128;
 constexpr int kCopyWarps = 8;
 
 template <int D>
-__global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const CompactArgs a) {
+__global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const __grid_constant__ CompactArgs a) {
   grid_dep_enter();
   constexpr int kUnits = D / 8;                 // 16-byte units of one K (or V) row
   constexpr int kRowUnits = 2 * kUnits;         // K then V
@@ -170,14 +173,16 @@ __global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const Com
   constexpr int kIn = 8;                        // passes in flight
   static_assert(kRowsPerWarp % (kIn * kRowsPerPass) == 0 || kRowsPerWarp == kIn * kRowsPerPass, "copy plan");
   __shared__ long long src[kCopyRows];          // unit offset of the row in the pools, -1: zero row
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
-  const int n = min(max(a.n_rows[bg], 0), a.p_max);
+  const int bp = a.rows.phys(b);                  // the sequence
+  const int bgp = bp * a.Hkv + g;
+  const int n = min(max(a.n_rows[bgp], 0), a.p_max);
   const int pad_end = min((n + kPage - 1) / kPage * kPage, a.p_max);
   const int r0 = blockIdx.x * kCopyRows;
   if (r0 >= pad_end) return;
   const int nr = min(kCopyRows, pad_end - r0);
-  const int32_t* pos = a.pos + (size_t)bg * a.p_max;
+  const int32_t* pos = a.pos + (size_t)bgp * a.p_max;
   if (threadIdx.x < kCopyRows) {
     const int r = r0 + threadIdx.x;
     long long off = -1;
@@ -185,7 +190,7 @@ __global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const Com
       const int p = pos[r];
       const int pi = p / kPage;
       int page = -1;
-      if (p >= 0 && pi < a.max_pages) page = __ldg(a.pt + (size_t)b * a.max_pages + pi);
+      if (p >= 0 && pi < a.max_pages) page = __ldg(a.pt + (size_t)bp * a.max_pages + pi);
       if ((unsigned)page >= (unsigned)a.num_pages) latch_error(a.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
       else off = ((long long)(page * a.Hkv + g) * kPage + p % kPage) * kUnits;
     }
@@ -199,7 +204,7 @@ __global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const Com
   const int cu = isv ? u - kUnits : u;
   const uint4* from = isv ? a.vpool : a.kpool;
   uint4* to = isv ? a.pv : a.pk;
-  const size_t dst0 = ((size_t)bg * a.p_max + r0) * kUnits + cu;
+  const size_t dst0 = ((size_t)bgp * a.p_max + r0) * kUnits + cu;
 #pragma unroll
   for (int i0 = 0; i0 < kRowsPerWarp; i0 += kIn * kRowsPerPass) {
     uint4 v[kIn];
@@ -307,21 +312,23 @@ __device__ __forceinline__ int block_scan2(int x, int* sh, int* total) {
   return before + v - x;
 }
 
-__device__ __forceinline__ int n_old_of(const IncArgs& a, int bg) {
+__device__ __forceinline__ int n_old_of(const IncArgs& a, int bgp) {
   if (a.fresh) return 0;
-  const int n = a.c.n_rows[bg];
+  const int n = a.c.n_rows[bgp];
   return (n < a.c.n_sink || n > a.cap) ? 0 : n;
 }
 
 template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_old_kernel(const IncArgs a) {
+__global__ void __launch_bounds__(kCThreads) inc_old_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
   const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
-  const int n_old = n_old_of(a, bg);
+  const int bp = a.c.rows.phys(b);                // the sequence
+  const int bgp = bp * a.c.Hkv + g;
+  const int n_old = n_old_of(a, bgp);
   if (blockIdx.x == 0 && threadIdx.x == 0) a.info[bg * 4] = n_old;
-  const int32_t* pos = a.c.pos + (size_t)bg * a.c.p_max;
-  uint32_t* hm = a.c.headmask + (size_t)bg * a.c.p_max;
+  const int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
+  uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
   uint32_t* ob = a.oldbits + (size_t)bg * a.c.nw;
   constexpr int kPer = kSTile / kCThreads;
   int c[kPer];
@@ -344,7 +351,7 @@ __global__ void __launch_bounds__(kCThreads) inc_old_kernel(const IncArgs a) {
 }
 
 template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_count_kernel(const IncArgs a) {
+__global__ void __launch_bounds__(kCThreads) inc_count_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
   __shared__ int sh[kCThreads / 32];
   const int bg = blockIdx.y;
@@ -386,13 +393,14 @@ __device__ __forceinline__ int n_new_of(const IncArgs& a, int bg) {
   return a.c.n_sink + all;
 }
 
-__global__ void __launch_bounds__(kCThreads) inc_slots_kernel(const IncArgs a) {
+__global__ void __launch_bounds__(kCThreads) inc_slots_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
   __shared__ int sh[kCThreads / 32];
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
+  const int bgp = a.c.rows.phys(bg / a.c.Hkv) * a.c.Hkv + bg % a.c.Hkv;
   const int n_old = a.info[bg * 4];
   const int n_new = min(n_new_of(a, bg), a.cap);
-  const uint32_t* hm = a.c.headmask + (size_t)bg * a.c.p_max;
+  const uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
   int x = 0;
 #pragma unroll
   for (int i = 0; i < kSTile / kCThreads; ++i) {
@@ -411,11 +419,13 @@ __global__ void __launch_bounds__(kCThreads) inc_slots_kernel(const IncArgs a) {
 }
 
 template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_list_kernel(const IncArgs a) {
+__global__ void __launch_bounds__(kCThreads) inc_list_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
   __shared__ int sh[kCThreads / 32];
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
   const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
+  const int bp = a.c.rows.phys(b);                // the sequence
+  const int bgp = bp * a.c.Hkv + g;
   int32_t* mv = a.mover_pos + (size_t)bg * a.cap;
   const int32_t* wc = a.wcounts + (size_t)bg * a.c.n_tiles * 2;
   if ((int)blockIdx.x < a.c.n_tiles) {
@@ -454,8 +464,8 @@ __global__ void __launch_bounds__(kCThreads) inc_list_kernel(const IncArgs a) {
     a.info[bg * 4 + 2] = h_all;
     a.info[bg * 4 + 3] = e_all + m_all;
   }
-  const int32_t* pos = a.c.pos + (size_t)bg * a.c.p_max;
-  const uint32_t* hm = a.c.headmask + (size_t)bg * a.c.p_max;
+  const int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
+  const uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
   int32_t* hs = a.hole_slot + (size_t)bg * a.cap;
   int hr = h_before, mr = e_all + m_before;
 #pragma unroll 1
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(kCThreads) inc_list_kernel(const IncArgs a) {
 }
 
 template <int D, int GM>
-__global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const IncArgs a) {
+__global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
   constexpr int kUnits = D / 8;
   constexpr int kRowUnits = 2 * kUnits;
@@ -483,8 +493,10 @@ __global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const IncArgs
   constexpr int kIn = 8;
   __shared__ long long src[kCopyRows];
   __shared__ int dst[kCopyRows];
-  const int bg = blockIdx.y;
+  const int bg = blockIdx.y;                    // logical (row, kv head)
   const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
+  const int bp = a.c.rows.phys(b);                // the sequence
+  const int bgp = bp * a.c.Hkv + g;
   const int4 inf = *reinterpret_cast<const int4*>(a.info + bg * 4);
   const int n_want = inf.y;
   const int n_new = min(n_want, a.cap);
@@ -495,11 +507,11 @@ __global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const IncArgs
   const int n_sf = fresh ? a.c.n_sink : 0;
   const int items = n_holes + n_pad + n_sf;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
-    a.c.n_rows[bg] = n_new;
+    a.c.n_rows[bgp] = n_new;
     if (n_want > a.cap || n_mov < n_holes) latch_error(a.c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
   }
-  int32_t* pos = a.c.pos + (size_t)bg * a.c.p_max;
-  uint32_t* hm = a.c.headmask + (size_t)bg * a.c.p_max;
+  int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
+  uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
   // 128-item chunks, strided over the blocks of this (b, KV head)
   for (int i0 = blockIdx.x * kCopyRows; i0 < items; i0 += gridDim.x * kCopyRows) {
     const int nr = min(kCopyRows, items - i0);
@@ -529,7 +541,7 @@ __global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const IncArgs
         if (p >= 0) {
           const int pi = p / kPage;
           int page = -1;
-          if (pi < a.c.max_pages) page = __ldg(a.c.pt + (size_t)b * a.c.max_pages + pi);
+          if (pi < a.c.max_pages) page = __ldg(a.c.pt + (size_t)bp * a.c.max_pages + pi);
           if ((unsigned)page >= (unsigned)a.c.num_pages) latch_error(a.c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
           else off = ((long long)(page * a.c.Hkv + g) * kPage + p % kPage) * kUnits;
         }
@@ -545,7 +557,7 @@ __global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const IncArgs
     const int cu = isv ? u - kUnits : u;
     const uint4* from = isv ? a.c.vpool : a.c.kpool;
     uint4* to = isv ? a.c.pv : a.c.pk;
-    const size_t base = (size_t)bg * a.c.p_max * kUnits + cu;
+    const size_t base = (size_t)bgp * a.c.p_max * kUnits + cu;
 #pragma unroll
     for (int i0r = 0; i0r < kRowsPerWarp; i0r += kIn * kRowsPerPass) {
       uint4 v[kIn];
@@ -656,11 +668,14 @@ CompactArgs compact_args(const sfi_shape& s, const sfi_params& p, const sfi_page
 
 sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                             const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,
-                            const CompactScratch& cs, int L_slow, cudaStream_t st) {
+                            const CompactScratch& cs, int L_slow, cudaStream_t st, const RowMap& rows) {
+  const int nb = rows.count(s.B);
+  if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
   CompactArgs a = compact_args(s, p, kv, bits, ld_b, pk, L_slow);
-  if ((size_t)s.B * s.Hkv * a.n_tiles * sizeof(int32_t) > cs.wcount_bytes) return SFI_ERR_WORKSPACE;
+  a.rows = rows;
+  if ((size_t)nb * s.Hkv * a.n_tiles * sizeof(int32_t) > cs.wcount_bytes) return SFI_ERR_WORKSPACE;
   a.tile_counts = cs.wcounts;
-  const int BH = s.B * s.Hkv;
+  const int BH = nb * s.Hkv;
   if (a.G <= 1) return launch_compact<1>(a, BH, st);
   if (a.G <= 2) return launch_compact<2>(a, BH, st);
   if (a.G <= 4) return launch_compact<4>(a, BH, st);
@@ -670,18 +685,21 @@ sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_p
 
 sfi_status run_compact_inc(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                            const uint32_t* bits, int64_t ld_b, const sfi_packed& pk, const CompactScratch& cs,
-                           int L_slow, bool fresh, cudaStream_t st) {
+                           int L_slow, bool fresh, cudaStream_t st, const RowMap& rows) {
+  const int nb = rows.count(s.B);
+  if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
   IncArgs a{};
   a.c = compact_args(s, p, kv, bits, ld_b, pk, L_slow);
+  a.c.rows = rows;
   a.cap = cs.cap;
   if (a.cap % kPage != 0 || pk.p_max < a.cap) return SFI_ERR_SHAPE;
   a.n_stiles = inc_slot_tiles(a.cap);
   if (fresh)   // same layout as the full compaction, which copies faster
-    return run_compact_bits(s, p, kv, bits, ld_b, pk, cs, L_slow, st);
+    return run_compact_bits(s, p, kv, bits, ld_b, pk, cs, L_slow, st, rows);
   a.fresh = 0;
   a.wcounts = cs.wcounts; a.scounts = cs.scounts; a.oldbits = cs.oldbits;
   a.mover_pos = cs.mover_pos; a.hole_slot = cs.hole_slot; a.info = cs.info;
-  const int BH = s.B * s.Hkv;
+  const int BH = nb * s.Hkv;
   if (a.c.G <= 1) return launch_inc<1>(a, BH, st);
   if (a.c.G <= 2) return launch_inc<2>(a, BH, st);
   if (a.c.G <= 4) return launch_inc<4>(a, BH, st);

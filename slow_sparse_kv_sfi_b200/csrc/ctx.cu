@@ -27,7 +27,13 @@ struct sfi_ctx {
   std::vector<cudaEvent_t> ev_dense, ev_sel;
   std::vector<uint8_t> pending;
   cudaEvent_t ev_buf_free[2] = {nullptr, nullptr};
-  int cur_step = -1, cur_slow = 0, last_slow = 0;
+  int cur_step = -1;
+  // per-sequence trigger state: the last slow step of every sequence and the
+  // decision of the current step (layer 0 decides, the other layers reuse it)
+  std::vector<int> last_slow;
+  std::vector<uint8_t> row_slow;
+  int n_slow = 0;
+  sfi::RowMap slow_rows, fast_rows;   // lists of a mixed step
   // workspace carving
   char* ws = nullptr;
   size_t ws_bytes = 0;
@@ -124,6 +130,126 @@ void timing_events(sfi_ctx* c, int kind, int layer, cudaEvent_t* b, cudaEvent_t*
 }  // namespace
 }  // namespace sfi
 
+namespace sfi {
+namespace {
+
+sfi_status check_step(const sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv* kv,
+                      const sfi_packed* packed, const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
+                      const float* out) {
+  if (!c || !c->ws) return SFI_ERR_WORKSPACE;
+  if (layer < 0 || layer >= c->n_layers || step < 0) return SFI_ERR_INVALID_ARG;
+  if (!kv || !packed || !q || !k_new || !v_new || !out || !kv->key_norms) return SFI_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u) != 0)
+    return SFI_ERR_INVALID_ARG;
+  if (L < c->p.n_sink + c->p.n_recent + 1 || L > c->s.max_pages * kPage) return SFI_ERR_SHAPE;
+  if (packed->p_max < packed_rows_capacity(c->s, c->p)) return SFI_ERR_SHAPE;
+  return SFI_OK;
+}
+
+// Trigger of every sequence for the step (layer 0): slow at step 0, after a
+// boundary token of that sequence, or when its refresh budget runs out.
+// boundary(b) gives the sequence's previous-step boundary flag.
+template <class F>
+sfi_status decide(sfi_ctx* c, int step, F boundary) {
+  const int B = c->s.B;
+  int n = 0;
+  for (int b = 0; b < B; ++b) {
+    const bool slow = step == 0 || boundary(b) || (step - c->last_slow[b]) >= c->p.refresh_budget;
+    if (slow) c->last_slow[b] = step;
+    c->row_slow[b] = slow ? 1 : 0;
+    n += slow ? 1 : 0;
+  }
+  c->cur_step = step;
+  c->n_slow = n;
+  if (n > 0 && n < B) {   // a mixed step: the two lists
+    if (B > kMaxRowMap) return SFI_ERR_UNSUPPORTED;
+    c->slow_rows.n = c->fast_rows.n = 0;
+    for (int b = 0; b < B; ++b) {
+      RowMap& m = c->row_slow[b] ? c->slow_rows : c->fast_rows;
+      m.b[m.n++] = (int16_t)b;
+    }
+  }
+  return SFI_OK;
+}
+
+// One layer of the current step: the slow path (dense attention, then the
+// Selector and compaction on the side stream) on the slow sequences, the
+// fast path on the others.
+sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv* kv, sfi_packed* packed,
+                     const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new, float* out,
+                     cudaStream_t main) {
+  const sfi_shape& s = c->s;
+  const sfi_params& p = c->p;
+  const int B = s.B;
+  const RowMap all{};
+  const RowMap& slow_map = c->n_slow == B ? all : c->slow_rows;
+  const RowMap& fast_map = c->n_slow == 0 ? all : c->fast_rows;
+
+  // this layer's previous refresh must land before its cache or packed buffer is touched
+  if (c->pending[layer]) {
+    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
+    c->pending[layer] = 0;
+  }
+  // the attention launches append the step's token themselves
+  const StepToken tok{k_new, v_new};
+  if (c->n_slow > 0) {
+    const int buf = layer & 1;
+    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
+    sfi_dense_extras ex{};
+    ex.logits = c->logits[buf];
+    ex.ld = c->ld;
+    ex.lse_cand = c->lse_cand[buf];
+    ex.cand_lo = p.n_sink;
+    ex.cand_hi = L - p.n_recent;
+    {
+      cudaEvent_t b, e;
+      timing_events(c, 1, layer, &b, &e);
+      SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
+                             main, b, e, &tok, &c->maps[layer], slow_map));
+    }
+    SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
+    cudaStream_t side = c->side;
+    SFI_TRY(cu(cudaStreamWaitEvent(side, c->ev_dense[layer], 0)));
+    const int nC = L - p.n_recent - p.n_sink;
+    const int K = budget_k(p, L);
+    if (K < 1) return SFI_ERR_SHAPE;
+    const int ld_s = (nC + 3) / 4 * 4;
+    if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
+    const int rows = slow_map.count(B) * s.Hq;   // logical rows of the Selector
+    SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
+                              c->stats, side, slow_map));
+    SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
+    // the scratch is laid out for the whole batch whatever the rows of this
+    // step, so its zero-state histograms stay where the last call cleared them
+    SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld,
+                     topk_scratch(c->topk_ws, B * s.Hq, nC), side));
+    if (c->incremental && packed->p_max >= c->cmp.cap) {
+      // step 0 starts a new decode: cache rows copied before may have changed
+      const bool fresh = step == 0 || c->packed_seen[layer] != packed->pos;
+      SFI_TRY(run_compact_inc(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, fresh, side, slow_map));
+      c->packed_seen[layer] = packed->pos;
+    } else {
+      SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, side, slow_map));
+      c->packed_seen[layer] = nullptr;
+    }
+    SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
+  }
+  if (c->n_slow < B) {
+    cudaEvent_t b, e;
+    timing_events(c, 0, layer, &b, &e);
+    SFI_TRY(run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, reinterpret_cast<int*>(c->ws), c->part,
+                          c->part_bytes, main, b, e, &tok, &c->maps[layer], fast_map));
+  }
+  if (c->n_slow > 0) {
+    if (c->overlap) c->pending[layer] = 1;
+    else SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
+  }
+  return SFI_OK;
+}
+
+}  // namespace
+}  // namespace sfi
+
 using namespace sfi;
 
 extern "C" {
@@ -147,6 +273,8 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->pending.assign(n_layers, 0);
   c->maps.resize(n_layers);
   c->packed_seen.assign(n_layers, nullptr);
+  c->last_slow.assign(shape->B, 0);
+  c->row_slow.assign(shape->B, 0);
   for (int i = 0; i < n_layers && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
@@ -208,88 +336,29 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   return SFI_OK;
 }
 
+
 sfi_status sfi_decode_step(sfi_ctx* c, int32_t layer, int32_t step, int32_t boundary_prev,
                            int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
                            const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
                            float* out, sfi_stream stream, int32_t* was_slow) {
-  if (!c || !c->ws) return SFI_ERR_WORKSPACE;
-  if (layer < 0 || layer >= c->n_layers || step < 0) return SFI_ERR_INVALID_ARG;
-  if (!kv || !packed || !q || !k_new || !v_new || !out || !kv->key_norms) return SFI_ERR_INVALID_ARG;
-  if (((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15u) != 0)
-    return SFI_ERR_INVALID_ARG;
-  if (L < c->p.n_sink + c->p.n_recent + 1 || L > c->s.max_pages * kPage) return SFI_ERR_SHAPE;
-  if (packed->p_max < packed_rows_capacity(c->s, c->p)) return SFI_ERR_SHAPE;
-  const sfi_shape& s = c->s;
-  const sfi_params& p = c->p;
-  cudaStream_t main = (cudaStream_t)stream;
+  SFI_TRY(check_step(c, layer, step, L, kv, packed, q, k_new, v_new, out));
+  if (layer == 0) SFI_TRY(decide(c, step, [&](int) { return boundary_prev != 0; }));
+  else if (step != c->cur_step) return SFI_ERR_INVALID_ARG;   // layer 0 decides the step
+  if (was_slow) *was_slow = c->n_slow > 0 ? 1 : 0;
+  return run_layer(c, layer, step, L, kv, packed, q, k_new, v_new, out, (cudaStream_t)stream);
+}
 
-  if (layer == 0) {
-    const bool slow = step == 0 || boundary_prev != 0 || (step - c->last_slow) >= p.refresh_budget;
-    if (slow) c->last_slow = step;
-    c->cur_step = step;
-    c->cur_slow = slow ? 1 : 0;
-  } else if (step != c->cur_step) {
-    return SFI_ERR_INVALID_ARG;   // layer 0 decides the step
-  }
-  if (was_slow) *was_slow = c->cur_slow;
-
-  // this layer's previous refresh must land before its cache or packed buffer is touched
-  if (c->pending[layer]) {
-    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
-    c->pending[layer] = 0;
-  }
-  // the attention launch appends the step's token itself
-  const StepToken tok{k_new, v_new};
-  if (!c->cur_slow) {
-    cudaEvent_t b, e;
-    timing_events(c, 0, layer, &b, &e);
-    return run_fast_attn(s, p, *kv, L, q, *packed, out, nullptr, reinterpret_cast<int*>(c->ws), c->part,
-                         c->part_bytes, main, b, e, &tok, &c->maps[layer]);
-  }
-
-  const int buf = layer & 1;
-  SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
-  sfi_dense_extras ex{};
-  ex.logits = c->logits[buf];
-  ex.ld = c->ld;
-  ex.lse_cand = c->lse_cand[buf];
-  ex.cand_lo = p.n_sink;
-  ex.cand_hi = L - p.n_recent;
-  {
-    cudaEvent_t b, e;
-    timing_events(c, 1, layer, &b, &e);
-    SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
-                           main, b, e, &tok, &c->maps[layer]));
-  }
-  SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
-  cudaStream_t side = c->side;
-  SFI_TRY(cu(cudaStreamWaitEvent(side, c->ev_dense[layer], 0)));
-  const int nC = L - p.n_recent - p.n_sink;
-  const int K = budget_k(p, L);
-  if (K < 1) return SFI_ERR_SHAPE;
-  const int ld_s = (nC + 3) / 4 * 4;
-  if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                            c->stats, side));
-  SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-  SFI_TRY(run_topk(s.B * s.Hq, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld,
-                   topk_scratch(c->topk_ws, s.B * s.Hq, nC), side));
-  if (c->incremental && packed->p_max >= c->cmp.cap) {
-    // step 0 starts a new decode: cache rows copied before may have changed
-    const bool fresh = step == 0 || c->packed_seen[layer] != packed->pos;
-    SFI_TRY(run_compact_inc(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, fresh, side));
-    c->packed_seen[layer] = packed->pos;
-  } else {
-    SFI_TRY(run_compact_bits(s, p, *kv, c->bits, c->bits_ld, *packed, c->cmp, L, side));
-    c->packed_seen[layer] = nullptr;
-  }
-  SFI_TRY(cu(cudaEventRecord(c->ev_sel[layer], side)));
-  if (c->overlap) {
-    c->pending[layer] = 1;
-  } else {
-    SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_sel[layer], 0)));
-  }
-  return SFI_OK;
+sfi_status sfi_decode_step_rows(sfi_ctx* c, int32_t layer, int32_t step, const int32_t* boundary_prev,
+                                int32_t L, const sfi_paged_kv* kv, sfi_packed* packed,
+                                const sfi_bf16* q, const sfi_bf16* k_new, const sfi_bf16* v_new,
+                                float* out, sfi_stream stream, int32_t* slow_rows) {
+  SFI_TRY(check_step(c, layer, step, L, kv, packed, q, k_new, v_new, out));
+  if (c->s.B > kMaxRowMap) return SFI_ERR_UNSUPPORTED;
+  if (layer == 0) SFI_TRY(decide(c, step, [&](int b) { return boundary_prev && boundary_prev[b] != 0; }));
+  else if (step != c->cur_step) return SFI_ERR_INVALID_ARG;
+  if (slow_rows)
+    for (int b = 0; b < c->s.B; ++b) slow_rows[b] = c->row_slow[b];
+  return run_layer(c, layer, step, L, kv, packed, q, k_new, v_new, out, (cudaStream_t)stream);
 }
 
 sfi_status sfi_ctx_set_compaction(sfi_ctx* c, int32_t incremental) {

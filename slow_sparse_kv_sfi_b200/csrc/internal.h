@@ -89,6 +89,22 @@ struct AttnMapCache {
   alignas(128) unsigned char maps[6 * 128];   // the kernel's tensor maps (k, v, pk, pv, pk8, pv8)
 };
 
+// Sequences of one launch (per-sequence triggers: a step whose sequences are
+// partly slow and partly fast runs the slow path on some, the fast path on
+// the others).  Logical row i indexes what the launch owns — work items,
+// split-K partials, Selector statistics, scores, top-K rows, selection
+// bitmaps, compaction scratch — and stands for sequence b[i], which indexes
+// what persists — cache pages, key norms, logits, packed buffers, outputs.
+// n == 0: every sequence, in order.  Passed by value into the kernels, so a
+// launch queued on the side stream never sees a later step's rows.
+constexpr int kMaxRowMap = 256;
+struct RowMap {
+  int32_t n = 0;
+  int16_t b[kMaxRowMap];
+  __host__ __device__ __forceinline__ int count(int B) const { return n ? n : B; }
+  __host__ __device__ __forceinline__ int phys(int i) const { return n ? (int)b[i] : i; }
+};
+
 // The decode step's new token (bf16 [B, Hkv, D] each), appended at L - 1 by
 // the attention launch itself.
 struct StepToken {
@@ -99,11 +115,13 @@ struct StepToken {
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
-                          const StepToken* tok = nullptr, AttnMapCache* maps = nullptr);
+                          const StepToken* tok = nullptr, AttnMapCache* maps = nullptr,
+                          const RowMap& rows = RowMap());
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
-                         cudaEvent_t ev_end, const StepToken* tok = nullptr, AttnMapCache* maps = nullptr);
+                         cudaEvent_t ev_end, const StepToken* tok = nullptr, AttnMapCache* maps = nullptr,
+                         const RowMap& rows = RowMap());
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld,
                           const float* lse, float* probs, cudaStream_t st);
 
@@ -115,7 +133,7 @@ sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st);
+                             cudaStream_t st, const RowMap& rows = RowMap());
 // Scratch of the top-K kernels for `rows` rows of n scores (topk.cu).  ghist
 // and done must be zero before the first call; every call leaves them zero.
 struct TopkScratch {
@@ -150,11 +168,12 @@ size_t compact_scratch_bytes(const sfi_shape& s, const sfi_params& p);
 CompactScratch compact_scratch(void* base, const sfi_shape& s, const sfi_params& p);
 sfi_status run_compact_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                             const uint32_t* bits, int64_t ld_b, const sfi_packed& pk,
-                            const CompactScratch& cs, int L_slow, cudaStream_t st);
+                            const CompactScratch& cs, int L_slow, cudaStream_t st,
+                            const RowMap& rows = RowMap());
 // fresh: build from scratch (sinks + union ascending) whatever the buffer holds
 sfi_status run_compact_inc(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                            const uint32_t* bits, int64_t ld_b, const sfi_packed& pk, const CompactScratch& cs,
-                           int L_slow, bool fresh, cudaStream_t st);
+                           int L_slow, bool fresh, cudaStream_t st, const RowMap& rows = RowMap());
 sfi_status run_idx_to_bits(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L_slow,
                            const int32_t* sel_idx, int sel_ld, int K, uint32_t* bits, int64_t ld_b,
                            cudaStream_t st);

@@ -70,13 +70,22 @@ __device__ __forceinline__ float pi_of(int L, int j) { return logf((float)(1 + L
 
 __device__ __forceinline__ float nbar_of(double sum_norms, int nC) { return (float)(sum_norms / (double)nC); }
 
-// part[bg][chunk][0] = sum of key norms over the chunk of C
+// Key-norm row of the launch's logical (row, kv head) bgl.
+__device__ __forceinline__ const float* norm_row(const float* norms, int64_t norm_ld, const RowMap& rows, int Hkv,
+                                                 int bgl) {
+  const int bl = bgl / Hkv;
+  return norms + ((size_t)rows.phys(bl) * Hkv + (bgl - bl * Hkv)) * norm_ld;
+}
+
+// part[bgl][chunk][0] = sum of key norms over the chunk of C (bgl: logical
+// (row, kv head) of the launch)
 __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC, const float* __restrict__ norms,
-                                                                  int64_t norm_ld, double* part, int nch) {
+                                                                  int64_t norm_ld, double* part, int nch, int Hkv,
+                                                                  const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   __shared__ double red[32];
   const int bg = blockIdx.y;
-  const float* n = norms + (size_t)bg * norm_ld + lo;
+  const float* n = norm_row(norms, norm_ld, rows, Hkv, bg) + lo;
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double sacc = 0.0;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) sacc += (double)n[c];
@@ -84,17 +93,18 @@ __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC
   if (threadIdx.x == 0) part[((size_t)bg * nch + blockIdx.x) * 2] = t;
 }
 
-// part[bg][chunk][1] = sum of kappa * pi over the chunk of C
+// part[bgl][chunk][1] = sum of kappa * pi over the chunk of C
 __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
                                                                    const float* __restrict__ norms,
-                                                                   int64_t norm_ld, double* part, int nch) {
+                                                                   int64_t norm_ld, double* part, int nch, int Hkv,
+                                                                   const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   __shared__ double red[32];
   __shared__ double bc;
   const int bg = blockIdx.y;
   double* pbg = part + (size_t)bg * nch * 2;
   const float nbar = nbar_of(reduce_parts(pbg, nch, 0, &bc), nC);
-  const float* n = norms + (size_t)bg * norm_ld;
+  const float* n = norm_row(norms, norm_ld, rows, Hkv, bg);
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double z = 0.0;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
@@ -115,8 +125,9 @@ struct ScoreArgs {
   int64_t norm_ld;
   const double* stat_part;   // [B*Hkv][nch][2]
   int nch;
-  float* scores;
+  float* scores;         // logical rows of the launch
   int64_t ld_s;
+  RowMap rows;
 };
 
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes the log-score
@@ -125,13 +136,14 @@ struct ScoreArgs {
 // head's nearest dominator (two passes, below), then the thread of a position
 // applies soft-NMS to every head, picks the owner and writes l''.
 template <int GM>
-__global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
   grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
   float* ell = sm;                    // [G][W]
-  const int bg = blockIdx.y;
-  const int b = bg / a.Hkv, g = bg - b * a.Hkv;
+  const int bg = blockIdx.y;                        // logical (row, kv head)
+  const int bl = bg / a.Hkv, g = bg - bl * a.Hkv;
+  const int b = a.rows.phys(bl);                    // the sequence
   const int c0 = blockIdx.x * a.tile;
   const int tile_n = min(a.tile, a.nC - c0);
   const int G = a.G;
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
   const float nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
   const float inv_z = (float)(1.0 / reduce_parts(pbg, a.nch, 1, &bc));
-  const float* nrm = a.norms + (size_t)bg * a.norm_ld;
+  const float* nrm = a.norms + ((size_t)b * a.Hkv + g) * a.norm_ld;
   const float lam = a.lam;
   const size_t row0 = (size_t)b * a.Hq + (size_t)g * G;
   const float* z0 = a.logits + row0 * a.ld + a.lo;
@@ -272,7 +284,7 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const ScoreArgs a) {
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
         const float v = l1[h] - (h != owner ? a.alpha_cross : 0.f);
-        a.scores[(row0 + h) * a.ld_s + c0 + k] = v;
+        a.scores[((size_t)bl * a.Hq + (size_t)g * G + h) * a.ld_s + c0 + k] = v;
       }
     }
   }
@@ -303,16 +315,20 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st) {
+                             cudaStream_t st, const RowMap& rows) {
   const int G = s.Hq / s.Hkv;
+  const int nb = rows.count(s.B);
+  if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
   const int lo = p.n_sink, hi = L - p.n_recent;
   const int nC = hi - lo;
   double* part = reinterpret_cast<double*>(stat_ws);
   const int nch = stat_chunks(nC);
   const int64_t norm_ld = (int64_t)s.max_pages * kPage;
-  dim3 sgrid(nch, s.B * s.Hkv);
-  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch);
-  launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch);
+  dim3 sgrid(nch, nb * s.Hkv);
+  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch,
+           s.Hkv, rows);
+  launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
+           s.Hkv, rows);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
@@ -326,8 +342,9 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.norms = kv.key_norms; a.norm_ld = norm_ld;
   a.stat_part = part; a.nch = nch;
   a.scores = scores; a.ld_s = ld_s;
+  a.rows = rows;
   const size_t smem = score_smem(G, a.tile, a.w);
-  dim3 grid((nC + a.tile - 1) / a.tile, s.B * s.Hkv);
+  dim3 grid((nC + a.tile - 1) / a.tile, nb * s.Hkv);
   if (G <= 1) return launch_scores<1>(a, grid, smem, st);
   if (G <= 2) return launch_scores<2>(a, grid, smem, st);
   if (G <= 4) return launch_scores<4>(a, grid, smem, st);

@@ -92,6 +92,7 @@ def _declare(L):
         "sfi_ctx_workspace_size": (C.c_int, [P, C.POINTER(SZ)]),
         "sfi_ctx_set_workspace": (C.c_int, [P, P, SZ]),
         "sfi_decode_step": (C.c_int, [P, I32, I32, I32, I32, P, P, P, P, P, P, P, C.POINTER(I32)]),
+        "sfi_decode_step_rows": (C.c_int, [P, I32, I32, P, I32, P, P, P, P, P, P, P, P]),
         "sfi_ctx_join": (C.c_int, [P, P]),
         "sfi_ctx_set_timing": (C.c_int, [P, I32]),
         "sfi_ctx_set_compaction": (C.c_int, [P, I32]),
@@ -109,7 +110,7 @@ EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_r
             "sfi_select_scores", "sfi_topk_workspace_size", "sfi_topk", "sfi_select", "sfi_compact",
             "sfi_compact_incremental", "sfi_poll_error",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
-            "sfi_decode_step", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_compaction",
+            "sfi_decode_step", "sfi_decode_step_rows", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_compaction",
             "sfi_ctx_timing"]
 
 
@@ -294,6 +295,20 @@ class Context:
                                      C.byref(packed), _p(q), _p(k_new), _p(v_new), _p(out),
                                      _stream(stream), C.byref(slow)), "sfi_decode_step")
         return bool(slow.value)
+
+    def decode_step_rows(self, layer, step, boundary_prev, L, kv, packed, q, k_new, v_new, out,
+                         stream=None):
+        """One layer-step with a trigger per sequence; boundary_prev: B flags
+        (or None).  Returns the per-sequence slow decisions."""
+        B = self.shape.B
+        bnd = None
+        if boundary_prev is not None:
+            bnd = (C.c_int32 * B)(*[int(x) for x in boundary_prev])
+        slow = (C.c_int32 * B)()
+        _check(lib().sfi_decode_step_rows(self.h, layer, step, bnd, L, C.byref(kv), C.byref(packed), _p(q),
+                                          _p(k_new), _p(v_new), _p(out), _stream(stream), slow),
+               "sfi_decode_step_rows")
+        return [bool(x) for x in slow]
 
     def decode_step_ptr(self, layer, step, boundary_prev, L, kv_ref, packed_ref, q, k_new, v_new, out,
                         stream) -> bool:

@@ -122,7 +122,7 @@ CONFIG_BY_NAME = {c.name: c for c in CONFIGS}
 
 _TAGS = {"page_table": 1, "k": 2, "v": 3, "kscale": 4, "outlier": 5, "planted": 6,
          "qnoise": 7, "knew": 8, "vnew": 9, "boundary": 10, "clusters": 11,
-         "switch": 12}
+         "switch": 12, "boundary_rows": 13}
 
 
 def _seed(cfg: SFIConfig, layer: int, what: str, extra: int = 0) -> int:
@@ -151,6 +151,17 @@ def boundary_stream(cfg: SFIConfig) -> np.ndarray:
         return b
     rng = _np_rng(cfg, 0, "boundary")
     return (rng.random(T) < cfg.boundary_p).astype(np.int8)
+
+
+def boundary_rows(cfg: SFIConfig) -> np.ndarray:
+    """int8[B, T]: boundary tokens of every sequence of the batch, drawn
+    independently (Bernoulli(boundary_p) per sequence and step), for decoding
+    with a trigger per sequence."""
+    T, B = cfg.steps, cfg.B
+    if cfg.boundary_mode != "bernoulli":
+        return np.broadcast_to(boundary_stream(cfg), (B, T)).copy()
+    rng = _np_rng(cfg, 0, "boundary_rows")
+    return (rng.random((B, T)) < cfg.boundary_p).astype(np.int8)
 
 
 def page_table(cfg: SFIConfig, layer: int) -> np.ndarray:

@@ -289,6 +289,12 @@ def test_compact_incremental_is_the_union_with_stable_slots(keep):
         prev_pos, prev_sel = pos, sel
 
 
+def test_trigger_rows_hand_worked():
+    g = _golden("trigger_rows_example.json")
+    got = O.trigger_rows(np.array(g["boundary"], np.int8), g["M"])
+    np.testing.assert_array_equal(got.astype(int), g["slow"])
+
+
 def test_trigger_hand_worked():
     for case in _golden("trigger_example.json")["cases"]:
         got = O.trigger(np.array(case["boundary"], np.int8), case["M"])
