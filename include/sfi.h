@@ -246,10 +246,11 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
  * n <= 262144.  ws: device scratch of sfi_topk_workspace_size(rows, n) bytes,
  * 16-byte aligned, zero-filled before its first use; every successful call
  * leaves it ready for the next one with the same rows (zero it again after an
- * error or before a call with another row count).  Every row is cut
- * into slices with one CTA each: a histogram of linear bins over the row's
- * [min, max], the boundary bin of the K-th score, an exact radix select of
- * the threshold among the boundary candidates, ties in position order. */
+ * error or before a call with another row count).  Exact radix select over
+ * order-preserving 32-bit keys of the scores: three digit passes (12, 12 and
+ * 8 bits; every row cut into slices of 8192 with one CTA each, the last CTA
+ * of a row narrowing the threshold prefix), then a pass marking the scores
+ * above the threshold and one taking the ties in position order. */
 sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes);
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
                     int32_t offset, int32_t* idx, int64_t ld_i, void* ws, size_t ws_bytes,
