@@ -88,6 +88,7 @@ class Clocks:
         self.index = index
         self.proc = None
         self.path = None
+        self.fh = None
 
     def start(self):
         try:
@@ -98,6 +99,10 @@ class Clocks:
                  "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            if self.fh is not None:
+                self.fh.close()
+            if self.path:
+                os.unlink(self.path)
 
     def stop(self):
         if self.proc is None:
