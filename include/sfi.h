@@ -72,12 +72,17 @@ typedef struct {
  *                         ([NL] "De Selector", [ZH] §2.2, §4 ablations)
  *  alpha_soft, nms_window  soft-NMS strength and full window width (w = window/2)
  *  alpha_cross             cross-head exclusivity penalty      ([FR] §2.B)
- *  refresh_budget          M: a slow step at least every M steps ([ES] §2) */
+ *  refresh_budget          M: a slow step at least every M steps ([ES] §2)
+ *  evidence_window         W: the Selector's evidence averages the attention
+ *                          distributions of the last W queries ([ES] §2, [ZH]
+ *                          §2.2 "window"); 0 or 1: the slow step's query only.
+ *                          W <= n_recent, W <= 32 and W * G <= 16. */
 typedef struct {
   int32_t n_sink, n_recent, k_fixed;
   double budget_frac;   /* K = floor(budget_frac * L) in double precision */
   float lambda, lambda_clip, alpha_soft, alpha_cross;
   int32_t nms_window, refresh_budget;
+  int32_t evidence_window;
 } sfi_params;
 
 /* The paged KV cache of one layer ([NL] "Systeemontwerp": the recent window is
@@ -234,7 +239,12 @@ sfi_status sfi_fast_attn_append(const sfi_shape* shape, const sfi_params* params
  * evidence f~ = exp(z - lse_cand), prior r from key norms and positions,
  * s = (1-l) f~ + l r, log-score, soft-NMS, cross-head exclusivity.
  *  logits    fp32 [B, Hq, ld] from sfi_dense_attn;  lse_cand fp32 [B, Hq]
- *  scores    fp32 [B, Hq, |C|] refined log-scores l''. */
+ *  scores    fp32 [B, Hq, |C|] refined log-scores l''.
+ * With W = params->evidence_window > 1 the evidence is the mean over W
+ * queries of exp(z_i - lse_cand_i), and logits / lse_cand hold B x Hkv x W x G
+ * rows: row ((b * Hkv + g) * W + i) * G + h is query i of head h of group g
+ * (the layout sfi_dense_attn writes for a query tensor of Hkv * W * G heads
+ * ordered that way). */
 sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
                              const sfi_paged_kv* kv, int32_t L, const float* logits, int64_t ld,
                              const float* lse_cand, float* scores, void* ws, size_t ws_bytes,

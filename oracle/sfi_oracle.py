@@ -162,6 +162,18 @@ def evidence(f: np.ndarray, lo: int, hi: int) -> np.ndarray:
     return fc / fc.sum(axis=1, keepdims=True)
 
 
+def evidence_window(fs: Sequence[np.ndarray], lo: int, hi: int) -> np.ndarray:
+    """Evidence over a window of queries: the mean of the restricted,
+    renormalised distributions of the last W queries, f~_{h,j} =
+    (1/W) sum_i f_{i,h,j} / sum_{c in C} f_{i,h,c}  ([ES] "2. Metodología", the
+    slow step's window; [ZH] "2.2", 证据分布).
+    READING: equal weights; fs[i] is the attention distribution of the query
+    i steps back over the current cache.  Its positions in C all precede that
+    query's own context end (W <= n_recent), so the restriction to C is the
+    same either way.  W = 1 is `evidence`."""
+    return np.mean([evidence(f, lo, hi) for f in fs], axis=0)
+
+
 def prior(norms: np.ndarray, L: int, lo: int, hi: int) -> np.ndarray:
     """Prior r from cache statistics, shared by the query heads of one KV head
     ([ZH] "2.2", 先验分布: a key-norm factor that suppresses spuriously high

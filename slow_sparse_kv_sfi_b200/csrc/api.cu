@@ -105,6 +105,8 @@ sfi_status check_params(const sfi_params* p) {
       !(p->alpha_cross >= 0.f) || !std::isfinite(p->alpha_soft) || !std::isfinite(p->alpha_cross))
     return SFI_ERR_INVALID_ARG;
   if (p->refresh_budget < 1) return SFI_ERR_INVALID_ARG;
+  if (p->evidence_window < 0 || p->evidence_window > 32 || p->evidence_window > p->n_recent)
+    return SFI_ERR_INVALID_ARG;
   return SFI_OK;
 }
 

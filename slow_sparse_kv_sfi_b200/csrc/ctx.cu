@@ -34,6 +34,13 @@ struct sfi_ctx {
   std::vector<uint8_t> row_slow;
   int n_slow = 0;
   sfi::RowMap slow_rows, fast_rows;   // lists of a mixed step
+  // evidence window of W queries: per layer a ring of the last W steps'
+  // queries (slot = step mod W) and the step each slot holds (-1: none)
+  int win = 1;
+  char* ring = nullptr;
+  size_t ring_layer_bytes = 0;
+  float* wout = nullptr;
+  std::vector<int> slot_step;   // [n_layers][win]
   // workspace carving
   char* ws = nullptr;
   size_t ws_bytes = 0;
@@ -64,24 +71,36 @@ namespace sfi {
 namespace {
 
 struct CtxLayout {
-  size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, stat_off, stat_bytes, score_off,
-      score_bytes, bits_off, bits_bytes, tc_off, tc_bytes, tk_off, tk_bytes, total;
+  size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, lsec_bytes, stat_off, stat_bytes, score_off,
+      score_bytes, bits_off, bits_bytes, tc_off, tc_bytes, tk_off, tk_bytes, ring_off, ring_layer_bytes,
+      wout_off, total;
   int64_t bits_ld;
 };
 
-CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
+// The slow step's dense-attention shape: with an evidence window of W
+// queries, the group's last W queries are Hkv * W * G heads of one launch.
+sfi_shape window_shape(const sfi_shape& s, const sfi_params& p) {
+  sfi_shape w = s;
+  w.Hq = s.Hkv * evidence_window(p) * (s.Hq / s.Hkv);
+  return w;
+}
+
+CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p, int n_layers) {
   const WsLayout w = ws_layout(s, p);
+  const sfi_shape sw = window_shape(s, p);
+  const int W = evidence_window(p);
   CtxLayout c{};
   const int Lmax = s.max_pages * kPage;
   size_t off = 256;
   c.part_off = off;
-  c.part_bytes = w.part_bytes;
+  c.part_bytes = W > 1 ? std::max(w.part_bytes, ws_layout(sw, p).part_bytes) : w.part_bytes;
   off += c.part_bytes;
   c.logit_off = off;
-  c.logit_bytes = align_up((size_t)s.B * s.Hq * Lmax * sizeof(float), 256);
+  c.logit_bytes = align_up((size_t)s.B * sw.Hq * Lmax * sizeof(float), 256);
   off += 2 * c.logit_bytes;
   c.lsec_off = off;
-  off += 2 * align_up((size_t)s.B * s.Hq * sizeof(float), 256);
+  c.lsec_bytes = align_up((size_t)s.B * sw.Hq * sizeof(float), 256);
+  off += 2 * c.lsec_bytes;
   c.stat_off = off;
   c.stat_bytes = w.stat_bytes;
   off += c.stat_bytes;
@@ -98,6 +117,13 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p) {
   c.tk_off = off;
   c.tk_bytes = w.tk_bytes;
   off += c.tk_bytes;
+  // evidence window: every layer's last W queries, [B][Hkv][W][G][D] bf16,
+  // and the window launch's outputs [B][Hkv * W * G][D] fp32
+  c.ring_off = off;
+  c.ring_layer_bytes = W > 1 ? align_up((size_t)s.B * sw.Hq * s.D * 2, 256) : 0;
+  off += (size_t)n_layers * c.ring_layer_bytes;
+  c.wout_off = off;
+  off += W > 1 ? align_up((size_t)s.B * sw.Hq * s.D * sizeof(float), 256) : 0;
   c.total = off;
   return c;
 }
@@ -192,6 +218,23 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
   }
   // the attention launches append the step's token themselves
   const StepToken tok{k_new, v_new};
+  const int W = c->win, G = s.Hq / s.Hkv;
+  char* ring = c->ring + (size_t)layer * c->ring_layer_bytes;
+  uint32_t wmask = 1u;
+  if (W > 1) {
+    // the step's queries into the layer's ring (after the wait above: the
+    // last refresh of this layer has read the slot this overwrites)
+    int* ss = &c->slot_step[(size_t)layer * W];
+    if (step == 0) std::fill(ss, ss + W, -1);
+    const int slot = step % W;
+    const size_t row = (size_t)G * s.D * sizeof(sfi_bf16);
+    SFI_TRY(cu(cudaMemcpy2DAsync(ring + slot * row, W * row, q, row, row, (size_t)s.B * s.Hkv,
+                                 cudaMemcpyDeviceToDevice, main)));
+    ss[slot] = step;
+    wmask = 0u;
+    for (int i = 0; i < W; ++i)
+      if (ss[i] >= 0 && ss[i] > step - W) wmask |= 1u << i;
+  }
   if (c->n_slow > 0) {
     const int buf = layer & 1;
     SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
@@ -204,8 +247,20 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
     {
       cudaEvent_t b, e;
       timing_events(c, 1, layer, &b, &e);
-      SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
-                             main, b, e, &tok, &c->maps[layer], slow_map));
+      if (W == 1) {
+        SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
+                               main, b, e, &tok, &c->maps[layer], slow_map));
+      } else {
+        // one pass over the cache for the group's last W queries (Hkv * W * G
+        // heads); the outputs of the step's own queries are copied out
+        const sfi_shape sw = window_shape(s, p);
+        SFI_TRY(run_dense_attn(sw, *kv, L, reinterpret_cast<const sfi_bf16*>(ring), c->wout, &ex,
+                               reinterpret_cast<int*>(c->ws), c->part, c->part_bytes, main, b, e, &tok,
+                               &c->maps[layer], slow_map));
+        const size_t orow = (size_t)G * s.D * sizeof(float);
+        SFI_TRY(cu(cudaMemcpy2DAsync(out, orow, reinterpret_cast<const char*>(c->wout) + (step % W) * orow, W * orow,
+                                     orow, (size_t)s.B * s.Hkv, cudaMemcpyDeviceToDevice, main)));
+      }
     }
     SFI_TRY(cu(cudaEventRecord(c->ev_dense[layer], main)));
     cudaStream_t side = c->side;
@@ -217,7 +272,7 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
     if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
     const int rows = slow_map.count(B) * s.Hq;   // logical rows of the Selector
     SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                              c->stats, side, slow_map));
+                              c->stats, side, slow_map, wmask));
     SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
     // the scratch is laid out for the whole batch whatever the rows of this
     // step, so its zero-state histograms stay where the last call cleared them
@@ -261,6 +316,8 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   size_t probe = 0;
   SFI_TRY(sfi_workspace_size(shape, params, &probe));
   if (n_layers < 1) return SFI_ERR_INVALID_ARG;
+  // the window's queries are the heads of one dense launch: at most 16 per group
+  if (evidence_window(*params) * (shape->Hq / shape->Hkv) > 16) return SFI_ERR_UNSUPPORTED;
   auto* c = new sfi_ctx();
   c->s = *shape;
   c->p = *params;
@@ -275,6 +332,8 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->packed_seen.assign(n_layers, nullptr);
   c->last_slow.assign(shape->B, 0);
   c->row_slow.assign(shape->B, 0);
+  c->win = evidence_window(*params);
+  c->slot_step.assign((size_t)n_layers * c->win, -1);
   for (int i = 0; i < n_layers && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
@@ -303,13 +362,13 @@ sfi_status sfi_ctx_destroy(sfi_ctx* c) {
 
 sfi_status sfi_ctx_workspace_size(const sfi_ctx* c, size_t* bytes) {
   if (!c || !bytes) return SFI_ERR_INVALID_ARG;
-  *bytes = ctx_layout(c->s, c->p).total;
+  *bytes = ctx_layout(c->s, c->p, c->n_layers).total;
   return SFI_OK;
 }
 
 sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   if (!c || !ws) return SFI_ERR_INVALID_ARG;
-  const CtxLayout l = ctx_layout(c->s, c->p);
+  const CtxLayout l = ctx_layout(c->s, c->p, c->n_layers);
   if (bytes < l.total) return SFI_ERR_WORKSPACE;
   char* w = static_cast<char*>(ws);
   // the counters in the workspace (attention work counter, combine and top-K
@@ -322,17 +381,20 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   c->ld = (int64_t)c->s.max_pages * kPage;
   for (int i = 0; i < 2; ++i) {
     c->logits[i] = reinterpret_cast<float*>(w + l.logit_off + i * l.logit_bytes);
-    c->lse_cand[i] =
-        reinterpret_cast<float*>(w + l.lsec_off + i * align_up((size_t)c->s.B * c->s.Hq * sizeof(float), 256));
+    c->lse_cand[i] = reinterpret_cast<float*>(w + l.lsec_off + i * l.lsec_bytes);
   }
+  c->ring = w + l.ring_off;
+  c->ring_layer_bytes = l.ring_layer_bytes;
+  c->wout = reinterpret_cast<float*>(w + l.wout_off);
   c->stats = w + l.stat_off;
   c->scores = reinterpret_cast<float*>(w + l.score_off);
   c->bits = reinterpret_cast<uint32_t*>(w + l.bits_off);
   c->bits_ld = l.bits_ld;
   c->cmp = compact_scratch(w + l.tc_off, c->s, c->p);
   c->topk_ws = w + l.tk_off;
-  // a new workspace holds no previous-selection state
+  // a new workspace holds no previous-selection state and no queries
   std::fill(c->packed_seen.begin(), c->packed_seen.end(), nullptr);
+  std::fill(c->slot_step.begin(), c->slot_step.end(), -1);
   return SFI_OK;
 }
 

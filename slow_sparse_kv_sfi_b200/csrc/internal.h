@@ -73,6 +73,8 @@ int fast_chunks(const sfi_shape& s, int p_max, int n_recent, int k_est);
 size_t attn_part_bytes(int n_items, int G, int D);
 int packed_rows_capacity(const sfi_shape& s, const sfi_params& p);
 int budget_k(const sfi_params& p, int L);   // -1 if |C| < 1
+// queries whose attention distributions the Selector's evidence averages
+inline int evidence_window(const sfi_params& p) { return p.evidence_window > 1 ? p.evidence_window : 1; }
 
 // Tensor maps of one layer's paged cache and packed buffer, kept by the
 // decode-step driver so that a launch does not encode them again (a host
@@ -133,7 +135,8 @@ sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st, const RowMap& rows = RowMap());
+                             cudaStream_t st, const RowMap& rows = RowMap(),
+                             uint32_t window_mask = 0xffffffffu);
 // Scratch of the top-K kernels for `rows` rows of n scores (topk.cu).  ghist
 // and done must be zero before the first call; every call leaves them zero.
 struct TopkScratch {

@@ -128,6 +128,11 @@ struct ScoreArgs {
   float* scores;         // logical rows of the launch
   int64_t ld_s;
   RowMap rows;
+  // evidence window: logits / lse_cand hold nq query slots of G heads per
+  // group; the slots in qmask are averaged (weight inv_nq each)
+  int nq;
+  uint32_t qmask;
+  float inv_nq;
 };
 
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes the log-score
@@ -154,15 +159,44 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
   const float inv_z = (float)(1.0 / reduce_parts(pbg, a.nch, 1, &bc));
   const float* nrm = a.norms + ((size_t)b * a.Hkv + g) * a.norm_ld;
   const float lam = a.lam;
-  const size_t row0 = (size_t)b * a.Hq + (size_t)g * G;
+  // logits rows of the group: nq query slots of G heads (nq = 1: row b * Hq + g * G + h)
+  const size_t row0 = ((size_t)b * a.Hkv + g) * (size_t)(a.nq * G);
   const float* z0 = a.logits + row0 * a.ld + a.lo;
   const float nan = __int_as_float(0x7fc00000);
   float lsec[GM];
 #pragma unroll
   for (int h = 0; h < GM; ++h) lsec[h] = (h < G) ? a.lse_cand[row0 + h] : 0.f;
+  if (a.nq > 1) {
+    // evidence window: the mean of the slots' restricted distributions
+    for (int k = threadIdx.x; k < W; k += blockDim.x) {
+      const int c = c0 - a.w + k;
+      if (c < 0 || c >= a.nC) {
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h < G) ell[h * W + k] = nan;
+        continue;
+      }
+      const int j = a.lo + c;
+      const float r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * inv_z;
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          float ft = 0.f;
+          for (int i = 0; i < a.nq; ++i) {
+            if ((a.qmask >> i) & 1u) {
+              const size_t row = (size_t)i * G + h;
+              ft += fast_exp2((z0[row * a.ld + c] - a.lse_cand[row0 + row]) * kLog2e);
+            }
+          }
+          const float sv = (1.f - lam) * (ft * a.inv_nq) + lam * r;
+          ell[h * W + k] = logf(sv + 1e-30f);
+        }
+      }
+    }
+  }
   // kU positions per thread and round: all their loads are issued first
   constexpr int kU = GM >= 8 ? 2 : 4;
-  for (int k0 = threadIdx.x; k0 < W; k0 += kU * blockDim.x) {
+  for (int k0 = threadIdx.x; a.nq == 1 && k0 < W; k0 += kU * blockDim.x) {
     float nv[kU], zv[kU][GM];
     bool in[kU];
 #pragma unroll
@@ -315,10 +349,13 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st, const RowMap& rows) {
+                             cudaStream_t st, const RowMap& rows, uint32_t window_mask) {
   const int G = s.Hq / s.Hkv;
   const int nb = rows.count(s.B);
   if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
+  const int nq = evidence_window(p);
+  const uint32_t qmask = window_mask & (nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u));
+  if (qmask == 0u) return SFI_ERR_INVALID_ARG;
   const int lo = p.n_sink, hi = L - p.n_recent;
   const int nC = hi - lo;
   double* part = reinterpret_cast<double*>(stat_ws);
@@ -343,6 +380,9 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.stat_part = part; a.nch = nch;
   a.scores = scores; a.ld_s = ld_s;
   a.rows = rows;
+  a.nq = nq;
+  a.qmask = qmask;
+  a.inv_nq = 1.f / (float)__builtin_popcount(qmask);
   const size_t smem = score_smem(G, a.tile, a.w);
   dim3 grid((nC + a.tile - 1) / a.tile, nb * s.Hkv);
   if (G <= 1) return launch_scores<1>(a, grid, smem, st);

@@ -45,7 +45,8 @@ class Params(C.Structure):
     _fields_ = [("n_sink", C.c_int32), ("n_recent", C.c_int32), ("k_fixed", C.c_int32),
                 ("budget_frac", C.c_double), ("lam", C.c_float), ("lambda_clip", C.c_float),
                 ("alpha_soft", C.c_float), ("alpha_cross", C.c_float),
-                ("nms_window", C.c_int32), ("refresh_budget", C.c_int32)]
+                ("nms_window", C.c_int32), ("refresh_budget", C.c_int32),
+                ("evidence_window", C.c_int32)]
 
 
 class PagedKV(C.Structure):
@@ -139,9 +140,9 @@ def make_shape(B, Hq, Hkv, D, max_pages, num_pages) -> Shape:
 
 
 def make_params(n_sink, n_recent, k_fixed, budget_frac, lam, lam_clip, alpha_soft, alpha_cross,
-                nms_window, refresh_budget) -> Params:
+                nms_window, refresh_budget, evidence_window=1) -> Params:
     return Params(n_sink, n_recent, k_fixed, budget_frac, lam, lam_clip, alpha_soft, alpha_cross,
-                  nms_window, refresh_budget)
+                  nms_window, refresh_budget, evidence_window)
 
 
 def make_kv(k_pool, v_pool, page_table, key_norms=None, err=None) -> PagedKV:

@@ -21,7 +21,7 @@ def shape_of(cfg: SFIConfig) -> S.Shape:
 def params_of(cfg: SFIConfig) -> S.Params:
     return S.make_params(cfg.n_sink, cfg.n_recent, cfg.k_fixed, cfg.budget_frac, cfg.lam,
                          cfg.lam_clip, cfg.alpha_soft, cfg.alpha_cross, cfg.nms_window,
-                         cfg.refresh_budget)
+                         cfg.refresh_budget, cfg.evidence_window)
 
 
 @dataclasses.dataclass

@@ -62,6 +62,7 @@ class SFIConfig:
     alpha_cross: float = 0.5
     nms_window: int = 32
     refresh_budget: int = 32
+    evidence_window: int = 1           # queries whose attention the Selector's evidence averages
     boundary_mode: str = "bernoulli"   # "none" | "bernoulli" | "slow_prefix"
     boundary_p: float = 1.0 / 16.0
     slow_prefix: int = 0               # "slow_prefix": steps [0, slow_prefix) are slow

@@ -80,10 +80,11 @@ def ambiguous_positions(ell: np.ndarray, ell1: np.ndarray, window: int, G: int) 
     return amb
 
 
-def oracle_selector_detail(f: np.ndarray, norms: np.ndarray, L: int, cfg):
-    """Oracle scores of one group plus the intermediate ell, ell' (float64)."""
+def oracle_selector_detail(f: np.ndarray, norms: np.ndarray, L: int, cfg, f_window=None):
+    """Oracle scores of one group plus the intermediate ell, ell' (float64).
+    f_window: the window's distributions (the query's own first), if any."""
     lo, hi = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
-    ft = O.evidence(f, lo, hi)
+    ft = O.evidence(f, lo, hi) if f_window is None else O.evidence_window(f_window, lo, hi)
     r = O.prior(norms, L, lo, hi)
     s = O.fuse(ft, r, cfg.lam, cfg.lam_clip)
     ell = O.log_score(s)

@@ -289,6 +289,27 @@ def test_compact_incremental_is_the_union_with_stable_slots(keep):
         prev_pos, prev_sel = pos, sel
 
 
+def test_evidence_window_hand_worked():
+    g = _golden("evidence_window_example.json")
+    lo, hi = g["C"]
+    got = O.evidence_window([np.array(f) for f in g["f"]], lo, hi)
+    np.testing.assert_allclose(got, g["evidence"], rtol=1e-12)
+
+
+def test_evidence_window_special_cases():
+    rng = np.random.default_rng(12)
+    fs = [rng.dirichlet(np.ones(50), size=3) for _ in range(4)]
+    lo, hi = 5, 40
+    # one query: the single-query evidence; repeated queries: the same
+    np.testing.assert_allclose(O.evidence_window(fs[:1], lo, hi), O.evidence(fs[0], lo, hi), rtol=1e-14)
+    np.testing.assert_allclose(O.evidence_window([fs[1]] * 3, lo, hi), O.evidence(fs[1], lo, hi), rtol=1e-14)
+    # a distribution over C per head, inside the hull of the members
+    ew = O.evidence_window(fs, lo, hi)
+    np.testing.assert_allclose(ew.sum(axis=1), 1.0, rtol=1e-12)
+    members = np.stack([O.evidence(f, lo, hi) for f in fs])
+    assert np.all(ew <= members.max(axis=0) + 1e-15) and np.all(ew >= members.min(axis=0) - 1e-15)
+
+
 def test_trigger_rows_hand_worked():
     g = _golden("trigger_rows_example.json")
     got = O.trigger_rows(np.array(g["boundary"], np.int8), g["M"])
