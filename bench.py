@@ -438,8 +438,11 @@ def run_sfi(args, cfg, rank, world, dist_on):
                 "peak_source": f"{peak_kind} hbm_gbs"}
     value = aggregate_rate(world, tokens, args.steps, t_sfi)
     # fast layer-step: attention (with the append) + combine; slow: the same
-    # two, then 2 statistics + scores + top-K + 3 compaction kernels (side stream)
-    launches_per_run = NL * (n_slow * 9 + (T - n_slow) * 2)
+    # two, then 2 statistics + scores + 5 top-K kernels, then the compaction:
+    # 3 kernels when step 0 builds the packed buffers, 5 when a later slow
+    # step refreshes them incrementally (side stream)
+    n_fresh = 1 if slows and slows[0] else 0
+    launches_per_run = NL * (n_fresh * 13 + (n_slow - n_fresh) * 15 + (T - n_slow) * 2)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000 * t_sfi / args.steps, "higher_is_better": True,
