@@ -457,7 +457,8 @@ def run_sfi(args, cfg, rank, world, dist_on):
         "config": {"workload": cfg.name, "B": B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": D,
                    "context": cfg.context, "layers": NL, "decode_steps": T, "budget": cfg.budget_frac,
                    "sink": cfg.n_sink, "recent": R, "trigger": f"bernoulli(1/16), M={cfg.refresh_budget}",
-                   "slow_steps": n_slow, "parallelism": "replicas" if world > 1 else "single",
+                   "slow_steps": n_slow, "evidence_window": cfg.evidence_window,
+                   "parallelism": "replicas" if world > 1 else "single",
                    "l2": "inputs larger than L2 (KV cache %.1f GB)" %
                          (NL * 2 * cfg.num_pages * cfg.Hkv * 16 * D * 2 / 1e9)},
         "roofline": roof,
@@ -527,10 +528,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layer-probe", type=int, default=0,
                     help="only run this many slow+fast layer-steps of one layer (profiler captures)")
+    ap.add_argument("--evidence-window", type=int, default=0,
+                    help="average the Selector's evidence over this many queries (default: the workload's)")
     args = ap.parse_args()
     cfg = W.CONFIG_BY_NAME[args.config]
     if args.decode_steps:
         cfg = cfg.replace(steps=args.decode_steps)
+    if args.evidence_window:
+        cfg = cfg.replace(evidence_window=args.evidence_window)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
