@@ -103,3 +103,33 @@ def test_context_rejects_bad_calls(S):
     h = C.c_void_p()
     st = S.lib().sfi_ctx_create(C.byref(sh), C.byref(p), 0, 1, C.byref(h))
     assert st == 1
+
+
+@pytest.mark.parametrize("window,code", [(0, 0), (1, 0), (4, 0), (33, 1), (65, 1), (-1, 1)])
+def test_evidence_window_validation(S, window, code):
+    """W in [0, 32] (0 and 1: the slow step's query alone) and W <= n_recent."""
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8, window)
+    n = C.c_size_t()
+    assert S.lib().sfi_workspace_size(C.byref(sh), C.byref(p), C.byref(n)) == code
+
+
+def test_new_entry_points_reject_bad_arguments(S):
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    p = S.make_params(4, 64, 128, 0.2, 0.2, 0.5, 0.5, 0.5, 32, 8)
+    kv = S.PagedKV(16, 16, 16, 16, None)
+    lib = S.lib()
+    # incremental compaction: no packed buffer / no selection
+    assert lib.sfi_compact_incremental(C.byref(sh), C.byref(p), C.byref(kv), 100, None, 3, 3, None, 0, None, 0,
+                                       None) == 1
+    pk = S.Packed(16, 16, 16, 16, 16, 64)
+    assert lib.sfi_compact_incremental(C.byref(sh), C.byref(p), C.byref(kv), 100, None, 3, 3, C.byref(pk), 0,
+                                       None, 0, None) == 1
+    # a packed buffer below the row capacity is refused (the refresh keeps slots up to it)
+    cap = S.sfi_packed_rows(sh, p)
+    if cap > 64:
+        assert lib.sfi_compact_incremental(C.byref(sh), C.byref(p), C.byref(kv), 100, 16, 3, 3, C.byref(pk), 0,
+                                           None, 0, None) == 2
+    # the driver's per-sequence step and compaction switch without a context
+    assert lib.sfi_decode_step_rows(None, 0, 0, None, 100, None, None, None, None, None, None, None, None) == 7
+    assert lib.sfi_ctx_set_compaction(None, 1) == 1
