@@ -16,10 +16,10 @@ Within-Sentence Support Stability" (arXiv 2603.12038), cited as
   [ZH] gist.science/zh/paper/2603.12038, technical summary
 
 Where the pages leave a step open, the plainest reading is taken and marked
-READING below.  Floating-point comparisons that decide an integer (soft-NMS
-dominance, the cross-head owner, the top-K order) are taken on values
-rounded to float32, the precision the CUDA path decides in; the arithmetic
-itself stays in float64.
+READING below.  Comparisons that decide an integer (soft-NMS dominance, the
+cross-head owner) are decided as real arithmetic decides them: from the
+terms of the fused score (see _score_diff and owner), never from the last
+bit of a rounded sum.  The top-K order is that of the float64 scores.
 
 Pins: every function here is checked in tests/test_oracle_*.py against
 closed forms, library routines, brute force or hand-worked fixtures.  Parity
@@ -217,11 +217,51 @@ def log_score(s: np.ndarray) -> np.ndarray:
     return np.log(np.asarray(s, np.float64) + LOG_EPS)
 
 
-def _f32(x):
-    return np.asarray(x, np.float64).astype(np.float32)
+def _score_diff(ell: np.ndarray, mixture, a: slice, b: slice) -> np.ndarray:
+    """l[:, a] - l[:, b] for two equally long column ranges, with the sign of
+    the exact difference.
+
+    Without a mixture the log-scores are compared as they are.  With the
+    mixture (f~, r, lambda) that l = ln(s + eps) was built from, ln is
+    monotone and eps is common, so the sign of l_i - l_j is the sign of
+    s_i - s_j = lambda (r_i - r_j) + (1 - lambda)(f~_i - f~_j), formed term
+    by term.  Rounding s itself would let its last bit decide comparisons
+    that real arithmetic decides by an evidence term far below it (where the
+    prior dominates, the group's heads share s to every digit of float64)."""
+    if mixture is None:
+        return ell[:, a] - ell[:, b]
+    ft, r, lam = mixture
+    return lam * (r[None, a] - r[None, b]) + (1.0 - lam) * (ft[:, a] - ft[:, b])
 
 
-def soft_nms(ell: np.ndarray, alpha_soft: float, window: int) -> np.ndarray:
+def soft_nms_distance(ell: np.ndarray, window: int, mixture=None) -> np.ndarray:
+    """Distance to the nearest dominating neighbour within w = window // 2
+    (0: none), for every (head, candidate) of ell [G, nC]:
+      i dominates j  <=>  l_i > l_j  or  (l_i == l_j and i < j),
+    with l_i vs l_j decided exactly (see _score_diff)."""
+    ell = np.asarray(ell, np.float64)
+    w = window // 2
+    G, n = ell.shape
+    dist = np.zeros((G, n), np.int64)
+    for d in range(w, 0, -1):      # descending: the nearest hit is written last
+        hit = np.zeros((G, n), bool)
+        # left neighbour i = j - d dominates j when l_i >= l_j
+        hit[:, d:] |= _score_diff(ell, mixture, slice(0, n - d), slice(d, n)) >= 0
+        # right neighbour i = j + d dominates j when l_i > l_j
+        hit[:, :n - d] |= _score_diff(ell, mixture, slice(d, n), slice(0, n - d)) > 0
+        dist = np.where(hit, d, dist)
+    return dist
+
+
+def soft_nms_weight(dist: np.ndarray, window: int) -> np.ndarray:
+    """Penalty weight of a nearest dominator at distance d: 1 - (d - 1) / w,
+    and 0 where there is none (d = 0)."""
+    w = window // 2
+    d = np.asarray(dist, np.float64)
+    return np.where(d > 0, 1.0 - (d - 1.0) / w, 0.0)
+
+
+def soft_nms(ell: np.ndarray, alpha_soft: float, window: int, mixture=None) -> np.ndarray:
     """Soft non-maximum suppression within each head: penalise tokens whose
     neighbours score higher ([FR] "B. Le Sélecteur", Suppression Non-Maximum
     Douce; [ZH] "2.2", Soft-NMS).
@@ -230,39 +270,53 @@ def soft_nms(ell: np.ndarray, alpha_soft: float, window: int) -> np.ndarray:
       N(j) = {i in C : 1 <= |i - j| <= w}
       i dominates j  <=>  l_i > l_j  or  (l_i == l_j and i < j)
       l'_j = l_j - alpha_soft * max_{i in N(j), i dominates j} (1 - (|i-j| - 1) / w)
-    with max over the empty set = 0.  Dominance is decided on float32 values.
-    ell: [G, nC] over the candidate positions in order.
+    with max over the empty set = 0.  The weight falls with distance, so the
+    max is the weight of the nearest dominator.  ell: [G, nC] over the
+    candidate positions in order; mixture: see _score_diff.
     """
     ell = np.asarray(ell, np.float64)
-    w = window // 2
-    G, n = ell.shape
-    e32 = _f32(ell)
-    pen = np.zeros_like(ell)
-    for d in range(1, w + 1):
-        weight = 1.0 - (d - 1) / w
-        # left neighbour i = j - d dominates j when e[i] >= e[j] (i < j)
-        dom_left = np.zeros((G, n), bool)
-        dom_left[:, d:] = e32[:, :-d] >= e32[:, d:]
-        # right neighbour i = j + d dominates j when e[i] > e[j] (i > j)
-        dom_right = np.zeros((G, n), bool)
-        dom_right[:, :-d] = e32[:, d:] > e32[:, :-d]
-        hit = dom_left | dom_right
-        pen = np.where(hit, np.maximum(pen, weight), pen)
-    return ell - alpha_soft * pen
+    return ell - alpha_soft * soft_nms_weight(soft_nms_distance(ell, window, mixture), window)
 
 
-def cross_head(ell1: np.ndarray, alpha_cross: float) -> np.ndarray:
+def owner(ell1: np.ndarray, dist=None, ft=None, lam=None) -> np.ndarray:
+    """owner(j) = argmax_h l'_{h,j}, ties to the lowest head: a scan over
+    the heads in order, a head replacing the best so far only when its l' is
+    strictly larger.
+
+    l'_a vs l'_b is decided exactly.  With the soft-NMS distances and the
+    evidence given, two heads with the same penalty compare as l_a vs l_b,
+    whose sign is that of (1 - lambda)(f~_a - f~_b): the prior is common to
+    the KV group.  Heads with different penalties compare by l' itself (the
+    penalties differ by at least alpha_soft / w)."""
+    ell1 = np.asarray(ell1, np.float64)
+    G, n = ell1.shape
+    cols = np.arange(n)
+    best = np.zeros(n, np.int64)
+    for h in range(1, G):
+        wins = ell1[h] > ell1[best, cols]
+        if dist is not None:
+            same = np.asarray(dist)[h] == np.asarray(dist)[best, cols]
+            if lam >= 1.0:
+                by_ev = np.zeros(n, bool)
+            else:
+                by_ev = np.asarray(ft, np.float64)[h] > np.asarray(ft, np.float64)[best, cols]
+            wins = np.where(same, by_ev, wins)
+        best = np.where(wins, h, best)
+    return best
+
+
+def cross_head(ell1: np.ndarray, alpha_cross: float, dist=None, ft=None, lam=None) -> np.ndarray:
     """Cross-head exclusivity within one KV group: discourage the group's
     query heads from choosing the same positions ([FR] "B. Le Sélecteur",
     Exclusivité inter-têtes; [ZH] "2.2", 跨头互斥).
 
-    READING: owner(j) = argmax_h l'_{h,j} (ties to the lowest h, decided on
-    float32 values); l''_{h,j} = l'_{h,j} - alpha_cross * [h != owner(j)].
+    READING: owner(j) = argmax_h l'_{h,j} (ties to the lowest h, see
+    `owner`); l''_{h,j} = l'_{h,j} - alpha_cross * [h != owner(j)].
     """
     ell1 = np.asarray(ell1, np.float64)
-    owner = np.argmax(_f32(ell1), axis=0)
+    own = owner(ell1, dist, ft, lam)
     G = ell1.shape[0]
-    not_owner = np.arange(G)[:, None] != owner[None, :]
+    not_owner = np.arange(G)[:, None] != own[None, :]
     return ell1 - alpha_cross * not_owner
 
 
@@ -271,15 +325,34 @@ def topk(scores: np.ndarray, K: int) -> np.ndarray:
     Top-K 选择): the K largest scores of each row.
 
     READING: ties go to the lower index; the result is sorted ascending.
-    The order is decided on float32 values.  scores: [G, n] -> [G, K]."""
-    s32 = _f32(scores)
-    G, n = s32.shape
+    scores: [G, n] -> [G, K]."""
+    s = np.asarray(scores, np.float64)
+    G, n = s.shape
     out = np.empty((G, K), np.int64)
     idx = np.arange(n)
     for h in range(G):
-        order = np.lexsort((idx, -s32[h]))
+        order = np.lexsort((idx, -s[h]))
         out[h] = np.sort(order[:K])
     return out
+
+
+def selector_detail(ft: np.ndarray, r: np.ndarray, lam: float, lam_clip: float,
+                    alpha_soft: float, alpha_cross: float, window: int) -> dict:
+    """Every step of the Selector for one KV group from the evidence f~
+    [G, nC] and the prior r [nC], in the order the pages give: fusion, log,
+    soft-NMS, cross-head.  Returns the intermediates: s, ell (l), dist (the
+    soft-NMS nearest-dominator distances), ell1 (l'), owner, ell2 (l'')."""
+    lam_eff = min(max(lam, 0.0), lam_clip)
+    ft = np.asarray(ft, np.float64)
+    r = np.asarray(r, np.float64)
+    s = fuse(ft, r, lam, lam_clip)
+    ell = log_score(s)
+    mixture = (ft, r, lam_eff)
+    dist = soft_nms_distance(ell, window, mixture)
+    ell1 = ell - alpha_soft * soft_nms_weight(dist, window)
+    own = owner(ell1, dist, ft, lam_eff)
+    ell2 = ell1 - alpha_cross * (np.arange(ft.shape[0])[:, None] != own[None, :])
+    return {"lam_eff": lam_eff, "s": s, "ell": ell, "dist": dist, "ell1": ell1, "owner": own, "ell2": ell2}
 
 
 def selector_scores(f: np.ndarray, norms: np.ndarray, L: int, n_sink: int,
@@ -291,10 +364,7 @@ def selector_scores(f: np.ndarray, norms: np.ndarray, L: int, n_sink: int,
     lo, hi = candidate_range(L, n_sink, n_recent)
     ft = evidence(f, lo, hi)
     r = prior(norms, L, lo, hi)
-    s = fuse(ft, r, lam, lam_clip)
-    ell = log_score(s)
-    ell1 = soft_nms(ell, alpha_soft, window)
-    return cross_head(ell1, alpha_cross)
+    return selector_detail(ft, r, lam, lam_clip, alpha_soft, alpha_cross, window)["ell2"]
 
 
 def select(f: np.ndarray, norms: np.ndarray, L: int, n_sink: int, n_recent: int,

@@ -3,7 +3,9 @@
 The fusion is pinned by its closed form and by an independent numerical
 minimisation of the KL objective the pages state; top-K by Python's sorted();
 soft-NMS, cross-head exclusivity, the prior, compaction and the trigger by
-hand-worked fixtures under tests/golden/ and by their special cases.
+hand-worked fixtures under tests/golden/ and by their special cases; the
+Selector's decisions by a brute-force evaluation in 80-digit decimal
+arithmetic.
 """
 import json
 import math
@@ -162,6 +164,109 @@ def test_cross_head_special_cases():
     np.testing.assert_array_equal(O.cross_head(e[:1], 0.7), e[:1])    # G = 1
     out = O.cross_head(e, 0.5)
     assert np.all(np.sum(out == e, axis=0) == 1)                       # one owner per column
+
+
+# ---------------------------------------------------------------- exact decisions
+def _selector_decimal(ft, r, lam, alpha_soft, alpha_cross, window, K, prec=80):
+    """The Selector's steps (fusion, log, soft-NMS, cross-head, top-K) in
+    80-digit decimal arithmetic, by brute force over every pair: the reference
+    the float64 oracle's decisions must agree with."""
+    from decimal import Decimal as Dc, localcontext
+    with localcontext() as ctx:
+        ctx.prec = prec
+        G, n = ft.shape
+        lam_d, one = Dc(lam), Dc(1)
+        eps = Dc(O.LOG_EPS)
+        ell = [[((one - lam_d) * Dc(ft[h, j]) + lam_d * Dc(r[j]) + eps).ln() for j in range(n)] for h in range(G)]
+        w = window // 2
+        ell1 = []
+        for h in range(G):
+            row = []
+            for j in range(n):
+                wt = Dc(0)
+                for d in range(1, w + 1):
+                    left = j - d >= 0 and ell[h][j - d] >= ell[h][j]
+                    right = j + d < n and ell[h][j + d] > ell[h][j]
+                    if left or right:
+                        wt = one - Dc(d - 1) / Dc(w)
+                        break
+                row.append(ell[h][j] - Dc(alpha_soft) * wt)
+            ell1.append(row)
+        sel = []
+        ell2 = [[None] * n for _ in range(G)]
+        for j in range(n):
+            best = 0
+            for h in range(1, G):
+                if ell1[h][j] > ell1[best][j]:
+                    best = h
+            for h in range(G):
+                ell2[h][j] = ell1[h][j] - (Dc(alpha_cross) if h != best else Dc(0))
+        for h in range(G):
+            sel.append(sorted(sorted(range(n), key=lambda j: (-ell2[h][j], j))[:K]))
+        return np.array(sel)
+
+
+def _prior_dominated_case(seed, n=72, G=3, tiny=1e-24):
+    """Evidence many orders of magnitude below the prior (the regime of most
+    candidates on the long-context workloads), with a damped prior shape."""
+    rng = np.random.default_rng(seed)
+    L = n + 20
+    kappa = np.minimum(1.0, rng.lognormal(0.0, 0.5, size=n) ** -1 * 1.1)
+    pi = np.log1p(L - np.arange(n, dtype=np.float64))
+    r = kappa * pi / np.sum(kappa * pi)
+    ft = tiny * rng.lognormal(0.0, 2.0, size=(G, n))
+    return ft, r
+
+
+@pytest.mark.parametrize("seed,tiny", [(0, 1e-24), (1, 1e-18), (2, 1e-12), (3, 1e-3), (4, 1.0)])
+def test_selector_decisions_agree_with_80_digit_arithmetic(seed, tiny):
+    ft, r = _prior_dominated_case(seed, tiny=tiny)
+    lam, a_s, a_c, window, K = 0.2, 0.5, 0.5, 8, 20
+    det = O.selector_detail(ft, r, lam, 0.5, a_s, a_c, window)
+    got = O.topk(det["ell2"], K)
+    ref = _selector_decimal(ft, r, lam, a_s, a_c, window, K)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_rounded_decisions_would_break_exact_arithmetic():
+    """Why the oracle never decides on a rounded s: where the prior dominates,
+    every head's s is the same float64 (and float32) number, so a decision
+    taken on the rounded values hands every position to head 0, while real
+    arithmetic gives it to the head with the most evidence."""
+    ft, r = _prior_dominated_case(0, tiny=1e-24)
+    lam, a_s, a_c, window, K = 0.2, 0.5, 0.5, 8, 20
+    ref = _selector_decimal(ft, r, lam, a_s, a_c, window, K)
+    ell = O.log_score(O.fuse(ft, r, lam, 0.5))
+    for cast in (np.float64, np.float32):
+        e = ell.astype(cast).astype(np.float64)
+        rounded = O.topk(O.cross_head(O.soft_nms(e, a_s, window), a_c), K)
+        assert not np.array_equal(rounded, ref)
+
+
+def test_owner_exact_special_cases():
+    # equal penalties, the prior common: the head with the largest evidence owns
+    ell1 = np.zeros((3, 2))
+    dist = np.ones((3, 2), np.int64)
+    ft = np.array([[1e-30, 5e-31], [3e-30, 1e-31], [2e-30, 7e-31]])
+    np.testing.assert_array_equal(O.owner(ell1, dist, ft, 0.2), [1, 2])
+    # lambda = 1: the evidence has no weight, ties go to the lowest head
+    np.testing.assert_array_equal(O.owner(ell1, dist, ft, 1.0), [0, 0])
+    # different penalties: l' decides, not the evidence
+    ell1 = np.array([[0.0], [-0.5]])
+    np.testing.assert_array_equal(O.owner(ell1, np.array([[1], [2]]), np.array([[1e-30], [1.0]]), 0.2), [0])
+
+
+def test_soft_nms_exact_dominance_under_equal_prior():
+    # two neighbours share the prior; the right one has the larger (tiny)
+    # evidence, so it dominates the left one, although their float64 s is equal
+    ft = np.array([[1e-30, 2e-30, 0.0]])
+    r = np.array([0.5, 0.5, 0.0])
+    ell = O.log_score(O.fuse(ft, r, 0.5, 1.0))
+    assert ell[0, 0] == ell[0, 1]
+    d = O.soft_nms_distance(ell, 2, (ft, r, 0.5))
+    assert d[0, 0] == 1 and d[0, 1] == 0
+    # without the mixture the rounded tie makes the left one dominate instead
+    assert O.soft_nms_distance(ell, 2)[0, 1] == 1
 
 
 # ---------------------------------------------------------------- top-K
