@@ -281,74 +281,142 @@ def _group_rows(layer_or_li, b, g, L, device_tensors=True):
     return sub_k, sub_v, sub_pt
 
 
-def oracle_sample(cfg, layer, q_t, slow_frac):
-    """Times the CPU oracle, as it stands, on one slow and one fast layer-step
-    of one layer (all (sequence, KV head) groups); returns tok/s per attention
-    layer for the run's slow/fast mix, seconds spent and the BLAS threads."""
-    from oracle import sfi_oracle as O
+def host_cores():
+    """CPU threads this process may run on (its affinity), and the machine's count."""
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
-    except Exception:
-        cores = 1
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:
+        aff = os.cpu_count() or 1
+    return aff, os.cpu_count() or aff
+
+
+FAST_SAMPLE = 8     # fast layer-steps per sampled group
+
+
+def oracle_sample(cfg, layer, q_t, slow_frac, budget_s=20.0):
+    """Times the CPU oracle, as it stands, on one slow layer-step (dense
+    attention + Selector) and FAST_SAMPLE fast layer-steps (sparse attention
+    over the slow step's sets) of layer 0, group by group until about
+    budget_s seconds are spent, and scales to all (sequence, KV head) groups.
+    Returns tok/s per attention layer for the run's slow/fast mix, the
+    seconds spent, the groups sampled, the groups in all, and the seconds per
+    slow and per fast layer-step."""
+    from oracle import sfi_oracle as O
     G = cfg.G
     L = cfg.seq_len(0)
     groups = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
-    subs = {bg: _group_rows(layer, bg[0], bg[1], L) for bg in groups}
     qh = q_t.float().cpu().numpy().astype(np.float64)
-    t0 = time.perf_counter()
-    sels = {}
+    t_slow = t_fast = 0.0
+    done = 0
     for (b, g) in groups:
-        sk, sv, spt = subs[(b, g)]
+        sk, sv, spt = _group_rows(layer, b, g, L)
+        qg = qh[b, g * G:(g + 1) * G]
+        t0 = time.perf_counter()
         K = O.gather_cache(sk, spt, 0, 0, L)
         V = O.gather_cache(sv, spt, 0, 0, L)
-        o, f, _, _ = O.dense_attention(qh[b, g * G:(g + 1) * G], K, V)
-        sels[(b, g)] = O.select(f, O.key_norms(K), L, cfg.n_sink, cfg.n_recent, cfg.k_fixed,
-                                cfg.budget_frac, cfg.lam, cfg.lam_clip, cfg.alpha_soft,
-                                cfg.alpha_cross, cfg.nms_window)
-    t_slow = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    for (b, g) in groups:
-        sk, sv, spt = subs[(b, g)]
-        K = O.gather_cache(sk, spt, 0, 0, L)
-        V = O.gather_cache(sv, spt, 0, 0, L)
-        sets = O.sparse_sets(L, cfg.n_sink, cfg.n_recent, list(sels[(b, g)]))
-        O.sparse_attention(qh[b, g * G:(g + 1) * G], K, V, sets)
-    t_fast = time.perf_counter() - t0
-    per_layer_step = slow_frac * t_slow + (1 - slow_frac) * t_fast
-    return cfg.B / per_layer_step, t_slow + t_fast, cores, t_slow, t_fast
+        _, f, _, _ = O.dense_attention(qg, K, V)
+        sel = O.select(f, O.key_norms(K), L, cfg.n_sink, cfg.n_recent, cfg.k_fixed, cfg.budget_frac, cfg.lam,
+                       cfg.lam_clip, cfg.alpha_soft, cfg.alpha_cross, cfg.nms_window)
+        t1 = time.perf_counter()
+        for _ in range(FAST_SAMPLE):
+            K = O.gather_cache(sk, spt, 0, 0, L)
+            V = O.gather_cache(sv, spt, 0, 0, L)
+            O.sparse_attention(qg, K, V, O.sparse_sets(L, cfg.n_sink, cfg.n_recent, list(sel)))
+        t2 = time.perf_counter()
+        t_slow += t1 - t0
+        t_fast += (t2 - t1) / FAST_SAMPLE
+        done += 1
+        if t_slow + FAST_SAMPLE * t_fast >= budget_s:
+            break
+    scale = len(groups) / done
+    slow_step, fast_step = scale * t_slow, scale * t_fast
+    per_layer_step = slow_frac * slow_step + (1 - slow_frac) * fast_step
+    spent = t_slow + FAST_SAMPLE * t_fast
+    return cfg.B / per_layer_step, spent, done, len(groups), slow_step, fast_step
+
+
+def cpu_baseline_line(value, spent, done, n_groups, slow_step, fast_step, slow_frac):
+    cores, nproc = host_cores()
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"layer 0: one slow and {FAST_SAMPLE} fast layer-steps of {done} of the {n_groups} "
+                      f"(sequence, KV head) groups ({spent:.1f} s), scaled to all groups: "
+                      f"{slow_step:.1f} s per slow and {fast_step:.2f} s per fast layer-step, weighted by the "
+                      f"run's slow fraction {slow_frac:.3f}; {cores} of {nproc} host threads available",
+            "nproc": nproc}
+
+
+def config_dict(cfg, n_slow, world):
+    """The workload description both arms print."""
+    D = cfg.D
+    cache = cfg.n_layers * 2 * cfg.num_pages * cfg.Hkv * 16 * D * 2
+    if cfg.boundary_mode == "bernoulli":
+        trig = f"bernoulli({cfg.boundary_p:g}), M={cfg.refresh_budget}"
+    elif cfg.boundary_mode == "slow_prefix":
+        trig = f"slow steps 0..{cfg.slow_prefix - 1}, then fast"
+    else:
+        trig = f"every {cfg.refresh_budget} steps"
+    return {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": D,
+            "context": cfg.context, "layers": cfg.n_layers, "decode_steps": cfg.steps,
+            "budget": cfg.budget_frac if cfg.k_fixed <= 0 else f"K={cfg.k_fixed}",
+            "sink": cfg.n_sink, "recent": cfg.n_recent, "trigger": trig, "slow_steps": int(n_slow),
+            "evidence_window": cfg.evidence_window,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": ("inputs larger than L2 (KV cache %.1f GB)" if cache > 126e6 else
+                   "inputs fit in L2, no flush (KV cache %.3f GB)") % (cache / 1e9)}
 
 
 # ---------------------------------------------------------------- arms
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return
+    from oracle import sfi_oracle as O
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     li = W.make_layer(cfg.replace(n_layers=1), 0, dev)
-    slow_frac = float(np.mean(__import__("oracle.sfi_oracle", fromlist=["trigger"]).trigger(
-        W.boundary_stream(cfg), cfg.refresh_budget)))
+    slow = O.trigger(W.boundary_stream(cfg), cfg.refresh_budget)
+    slow_frac = float(np.mean(slow))
     vals, secs = [], []
-    cores = 1
+    last = None
     for i in range(args.warmup + args.steps):
-        v, s, cores, _, _ = oracle_sample(cfg, li, li.q[0], slow_frac)
+        last = oracle_sample(cfg, li, li.q[0], slow_frac, budget_s=args.cpu_budget)
         if i >= args.warmup:
-            vals.append(v)
-            secs.append(s)
+            vals.append(last[0])
+            secs.append(last[1])
     value = float(np.mean(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * float(np.mean(secs)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
-                   "context": cfg.context, "layers": cfg.n_layers, "decode_steps": cfg.steps},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": "per step: one slow and one fast layer-step of layer 0, all "
-                                   f"{cfg.B * cfg.Hkv} (sequence, KV head) groups, weighted by the "
-                                   f"run's slow fraction {slow_frac:.3f}"},
+        "config": config_dict(cfg, int(slow.sum()), world),
+        "cpu_baseline": cpu_baseline_line(value, *last[1:], slow_frac),
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, the nominal figure
+
+
+def step_bytes(cfg, L, packed_rows, slow, moved_rows=None):
+    """Algorithmic bytes of one layer-step (what the method must move).
+    Fast: the packed and recent rows of every (sequence, KV head), the
+    queries and the outputs.  Slow: the whole cache, the logits written and
+    read once by the Selector, the candidates' key norms, and the packed rows
+    the refresh copies (read and written; all of them when the buffer is
+    built, moved_rows when it is refreshed in place)."""
+    B, Hq, Hkv, D, R = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.n_recent
+    row = 4 * D
+    qo = B * Hq * D * (2 + 4)
+    if not slow:
+        return float((packed_rows.astype(np.float64) + R).sum()) * row + qo
+    nC = L - R - cfg.n_sink
+    copied = float(packed_rows.sum()) if moved_rows is None else float(moved_rows)
+    return (B * Hkv * L * row + B * Hq * L * 4 + B * Hq * nC * 4 + B * Hkv * nC * 4 + 2 * copied * row + qo)
+
+
+def frac_entry(bytes_, seconds, peak):
+    gbs = bytes_ / seconds / 1e9 if seconds > 0 else 0.0
+    return {"GBps": gbs, "frac_measured": gbs / peak, "frac_nominal": gbs / NOMINAL_HBM_GBS}
 
 
 def run_sfi(args, cfg, rank, world, dist_on):
@@ -364,22 +432,32 @@ def run_sfi(args, cfg, rank, world, dist_on):
     torch.cuda.synchronize()
     n_slow = sum(slows)
     D = cfg.D
-    row_bytes = 4 * D
     R = cfg.n_recent
-    # algorithmic bytes of the attention launches whose durations are sampled:
-    # layers 0, TIMING_STRIDE, ... of every step
+    # algorithmic bytes: of the attention launches whose durations are sampled
+    # (layers 0, TIMING_STRIDE, ...), and of every layer-step of the run
     sampled = range(0, NL, TIMING_STRIDE)
     fast_bytes = 0.0
+    run_fast_bytes = run_slow_bytes = 0.0
     union_rows = []
     cur = None
+    first = True
     for t in range(T):
+        L = cfg.seq_len(t)
         if slows[t]:
             cur = [x.cpu().numpy() for x in probe[t]]
             union_rows.extend([float(x.mean()) for x in cur])
+            # the refresh after the first slow step copies few rows (not
+            # counted: the incremental refresh moves well under 1 % of them)
+            for l in range(NL):
+                run_slow_bytes += step_bytes(cfg, L, cur[l], True, None if first else 0)
+            first = False
         else:
-            for l in sampled:
-                fast_bytes += float((cur[l].astype(np.float64) + R).sum()) * row_bytes + B * cfg.Hq * D * 2
-    dense_bytes_slow = sum(float(B * cfg.Hkv * cfg.seq_len(t) * row_bytes + B * cfg.Hq * cfg.seq_len(t) * 4)
+            for l in range(NL):
+                b_ = step_bytes(cfg, L, cur[l], False)
+                run_fast_bytes += b_
+                if l in sampled:
+                    fast_bytes += b_
+    dense_bytes_slow = sum(float(B * cfg.Hkv * cfg.seq_len(t) * 4 * D + B * cfg.Hq * cfg.seq_len(t) * 4)
                            for t in range(T) if slows[t]) * len(sampled)
     # timed region: SFI mixed decode, with kernel and step events
     clocks = Clocks(torch.cuda.current_device())
@@ -397,7 +475,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
         bench.run_sfi(step_events=step_ev[k])
     e1.record()
     _sync_barrier(dist_on)
-    clk = clocks.stop()
+    clk_sfi = clocks.stop()
     t_sfi = _max_over_ranks(e0.elapsed_time(e1) / 1000.0, dist_on)
     fast_ms, fast_n = bench.ctx.timing(0, reset=True)
     dense_ms, dense_n = bench.ctx.timing(1, reset=True)
@@ -412,7 +490,10 @@ def run_sfi(args, cfg, rank, world, dist_on):
             prev = step_ev[k][t]
     # dense full-KV baseline on the same cache
     bench.run_dense()
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
     t_dense = _timed(bench.run_dense, args.steps, dist_on)
+    clk_dense = clocks.stop()
     # end to end through host buffers
     hq = bench.q.cpu().pin_memory()
     hk = bench.kn.cpu().pin_memory()
@@ -420,7 +501,10 @@ def run_sfi(args, cfg, rank, world, dist_on):
     hout = torch.empty((T,) + tuple(bench.out.shape), dtype=torch.float32).pin_memory()
     dq, dk, dv = torch.empty_like(bench.q[0]), torch.empty_like(bench.kn[0]), torch.empty_like(bench.vn[0])
     bench.run_e2e(hq, hk, hv, hout, dq, dk, dv)
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
     t_e2e = _timed(lambda: bench.run_e2e(hq, hk, hv, hout, dq, dk, dv), args.steps, dist_on)
+    clk_e2e = clocks.stop()
     h2d = (hq[0].numel() * 2 + hk[0].numel() * 2 + hv[0].numel() * 2) * T
     d2h = hout[0].numel() * 4 * T
     # roofline of the dominant kernel, with launches measured in the timed region
@@ -430,19 +514,34 @@ def run_sfi(args, cfg, rank, world, dist_on):
     ach_dense = (dense_bytes_slow * k / 1e9) / (dense_ms / 1e3) if dense_ms > 0 else 0.0
     dominant = "fast" if fast_ms >= dense_ms else "dense"
     if dominant == "fast":
-        roof = {"kernel": "attn_kernel<128,1,kFast> (fast step)", "bound": "hbm", "achieved": ach_fast,
+        roof = {"kernel": f"attn_kernel<{D},*,kFast> (fast step)", "bound": "hbm", "achieved": ach_fast,
                 "peak": peak, "unit": "GB/s", "frac": ach_fast / peak,
                 "traffic": kernel_traffic("fast_attn_bytes_per_launch"),
                 "algorithmic_bytes_per_launch": fast_bytes / max(fast_n / k, 1),
                 "launches": fast_n, "avg_launch_us": 1000 * fast_ms / max(fast_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
     else:
-        roof = {"kernel": "attn_kernel<128,1,kDenseExtras> (slow step)", "bound": "hbm", "achieved": ach_dense,
+        roof = {"kernel": f"attn_kernel<{D},*,kDenseExtras> (slow step)", "bound": "hbm", "achieved": ach_dense,
                 "peak": peak, "unit": "GB/s", "frac": ach_dense / peak,
                 "traffic": kernel_traffic("dense_attn_bytes_per_launch"),
                 "algorithmic_bytes_per_launch": dense_bytes_slow / max(dense_n / k, 1),
                 "launches": dense_n, "avg_launch_us": 1000 * dense_ms / max(dense_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
+    roof["frac_nominal"] = roof["achieved"] / NOMINAL_HBM_GBS
+    # every step type as a fraction of the HBM roofline: algorithmic bytes of
+    # the run's fast (slow) layer-steps over the main stream's fast (slow)
+    # step time, the whole run's bytes over the whole run's time, and the
+    # dense baseline's cache bytes over its time
+    n_fast = T - n_slow
+    dense_run_bytes = sum(float(B * cfg.Hkv * cfg.seq_len(t) * 4 * D + B * cfg.Hq * D * 6) for t in range(T)) * NL
+    roof["steps"] = {
+        "fast": frac_entry(run_fast_bytes / max(n_fast, 1), statistics.mean(st_fast) / 1e3, peak) if st_fast else None,
+        "slow": frac_entry(run_slow_bytes / max(n_slow, 1), statistics.mean(st_slow) / 1e3, peak) if st_slow else None,
+        "mix": frac_entry(run_fast_bytes + run_slow_bytes, t_sfi / args.steps, peak),
+        "dense_baseline": frac_entry(dense_run_bytes, t_dense / args.steps, peak),
+        "bytes": "fast: (packed + recent rows) x 4D + q, o; slow: cache + logits written and read once + "
+                 "candidate norms + rows copied by the refresh (all at the first slow step); per layer-step",
+    }
     value = aggregate_rate(world, tokens, args.steps, t_sfi)
     # fast layer-step: attention (with the append) + combine; slow: the same
     # two, then 2 statistics + scores + 5 top-K kernels, then the compaction:
@@ -450,17 +549,17 @@ def run_sfi(args, cfg, rank, world, dist_on):
     # step refreshes them incrementally (side stream)
     n_fresh = 1 if slows and slows[0] else 0
     launches_per_run = NL * (n_fresh * 13 + (n_slow - n_fresh) * 15 + (T - n_slow) * 2)
+    legs = {"sfi": clk_sfi, "dense": clk_dense, "e2e": clk_e2e}
+    mhz = [v["sm_mhz"] for v in legs.values() if v.get("sm_mhz")]
+    clk = {"sm_mhz": statistics.median(mhz) if mhz else None,
+           "sm_max_mhz": max([v["sm_max_mhz"] for v in legs.values() if v.get("sm_max_mhz")] or [0]) or None,
+           "reasons": sorted(set(r for v in legs.values() for r in v.get("reasons", []))),
+           "legs": legs}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000 * t_sfi / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": cfg.name, "B": B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": D,
-                   "context": cfg.context, "layers": NL, "decode_steps": T, "budget": cfg.budget_frac,
-                   "sink": cfg.n_sink, "recent": R, "trigger": f"bernoulli(1/16), M={cfg.refresh_budget}",
-                   "slow_steps": n_slow, "evidence_window": cfg.evidence_window,
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (KV cache %.1f GB)" %
-                         (NL * 2 * cfg.num_pages * cfg.Hkv * 16 * D * 2 / 1e9)},
+        "config": config_dict(cfg, n_slow, world),
         "roofline": roof,
         "e2e": {"value": aggregate_rate(world, tokens, args.steps, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -471,6 +570,8 @@ def run_sfi(args, cfg, rank, world, dist_on):
             "speedup_vs_dense": t_dense / t_sfi,
             "fast_step_tok_s": B * NL / (statistics.mean(st_fast) / 1e3) if st_fast else None,
             "slow_step_tok_s": B * NL / (statistics.mean(st_slow) / 1e3) if st_slow else None,
+            "slow_layer_step_us": 1000 * statistics.mean(st_slow) / NL if st_slow else None,
+            "fast_layer_step_us": 1000 * statistics.mean(st_fast) / NL if st_fast else None,
             "fast_attn_GBps": ach_fast, "dense_attn_GBps": ach_dense,
             "timed_layers": f"every {TIMING_STRIDE}th layer ({len(range(0, NL, TIMING_STRIDE))} of {NL})",
             "fast_attn_ms_sampled": fast_ms, "dense_attn_ms_sampled": dense_ms,
@@ -480,13 +581,9 @@ def run_sfi(args, cfg, rank, world, dist_on):
         },
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        li0 = bench.layers[0]
         slow_frac = n_slow / T
-        v, secs, cores, ts, tf = oracle_sample(cfg, li0, bench.q[0, 0], slow_frac)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"one slow ({ts:.1f} s) and one fast ({tf:.1f} s) layer-step of "
-                                          f"layer 0, all {B * cfg.Hkv} (sequence, KV head) groups, "
-                                          f"weighted by the run's slow fraction {slow_frac:.3f}"}
+        res = oracle_sample(cfg, bench.layers[0], bench.q[0, 0], slow_frac, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline_line(*res, slow_frac)
     if rank == 0:
         print(json.dumps(line), flush=True)
     bench.ctx.close()
@@ -526,6 +623,8 @@ def main():
     ap.add_argument("--impl", default="sfi", choices=["sfi", "reference"])
     ap.add_argument("--decode-steps", type=int, default=0, help="override the workload's decode steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work per CPU-baseline sample")
     ap.add_argument("--layer-probe", type=int, default=0,
                     help="only run this many slow+fast layer-steps of one layer (profiler captures)")
     ap.add_argument("--evidence-window", type=int, default=0,

@@ -12,6 +12,16 @@
 //   exclusivity l'' = l' - alpha_cross * [h != argmax_h' l'_{h',j}]
 //   top-K      K largest l'' per query head, ties to the lower position.
 //
+// Comparisons that decide an integer follow real arithmetic, not the last bit
+// of a rounded sum: l_i vs l_j has the sign of s_i - s_j (ln is monotone),
+// with s = (1 - lambda) f~ + lambda r formed in fp64 from an fp64 prior and
+// rounded once to fp32 (where the prior dominates, neighbouring candidates
+// differ in r by ~1e-6 relative, far above that rounding); two heads with the
+// same soft-NMS penalty compare by their evidence, since r is common to the
+// group (their s agree to every digit where the prior dominates).  The
+// evidence is compared through its logarithm x = z - lse_C, which does not
+// underflow.  With lambda = 0 the dominance is decided on x as well.
+//
 // Kernels: stats_norm / stats_prior (per (b, kv head) and chunk of C: fp64
 // partial sums of the norms and of kappa pi; every consumer reduces the
 // partials in the same fixed order), select_scores (one CTA per (b, kv group,
@@ -62,13 +72,17 @@ __device__ __forceinline__ double reduce_parts(const double* part, int nch, int 
   return r;
 }
 
-__device__ __forceinline__ float kappa_of(float nbar, float n) {
-  return n > 0.f ? fminf(1.f, nbar / n) : 1.f;
+// Prior factors in fp64 (the stored norms are fp32): kappa_j = min(1, nbar /
+// n_j) (1 for a zero key), pi_j = ln(1 + L - j).  stats_prior and
+// select_scores evaluate them with the same code, so the normaliser is the
+// sum of exactly the values the scores use.
+__device__ __forceinline__ double kappa_of(double nbar, float n) {
+  return n > 0.f ? fmin(1.0, nbar / (double)n) : 1.0;
 }
 
-__device__ __forceinline__ float pi_of(int L, int j) { return logf((float)(1 + L - j)); }
+__device__ __forceinline__ double pi_of(int L, int j) { return log((double)(1 + L - j)); }
 
-__device__ __forceinline__ float nbar_of(double sum_norms, int nC) { return (float)(sum_norms / (double)nC); }
+__device__ __forceinline__ double nbar_of(double sum_norms, int nC) { return sum_norms / (double)nC; }
 
 // Key-norm row of the launch's logical (row, kv head) bgl.
 __device__ __forceinline__ const float* norm_row(const float* norms, int64_t norm_ld, const RowMap& rows, int Hkv,
@@ -103,13 +117,13 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
   __shared__ double bc;
   const int bg = blockIdx.y;
   double* pbg = part + (size_t)bg * nch * 2;
-  const float nbar = nbar_of(reduce_parts(pbg, nch, 0, &bc), nC);
+  const double nbar = nbar_of(reduce_parts(pbg, nch, 0, &bc), nC);
   const float* n = norm_row(norms, norm_ld, rows, Hkv, bg);
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double z = 0.0;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
     const int j = lo + c;
-    z += (double)(kappa_of(nbar, n[j]) * pi_of(L, j));
+    z += kappa_of(nbar, n[j]) * pi_of(L, j);
   }
   const double t = block_sum_d(z, red);
   if (threadIdx.x == 0) pbg[blockIdx.x * 2 + 1] = t;
@@ -117,7 +131,8 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
 
 struct ScoreArgs {
   int L, lo, nC, Hq, Hkv, G, w, tile;
-  float lam, alpha_soft, alpha_cross;
+  double lam, one_minus_lam;    // lambda_eff and 1 - lambda_eff
+  float alpha_soft, alpha_cross;
   const float* logits;
   int64_t ld;
   const float* lse_cand;
@@ -135,17 +150,20 @@ struct ScoreArgs {
   float inv_nq;
 };
 
-// One CTA per (b, KV group, tile of candidates).  Phase 1 writes the log-score
-// of every head of the group over the tile plus a halo of w on each side to
-// shared memory (NaN outside C: a NaN never dominates).  Phase 2 finds every
-// head's nearest dominator (two passes, below), then the thread of a position
-// applies soft-NMS to every head, picks the owner and writes l''.
+// One CTA per (b, KV group, tile of candidates).  Phase 1 writes, for every
+// head of the group over the tile plus a halo of w on each side, the
+// dominance key (s rounded once to fp32, or x when lambda = 0; NaN outside C:
+// a NaN never dominates) and, over the tile, the log-evidence x.  Phase 2
+// finds every head's nearest dominator (two passes, below).  Phase 3: the
+// thread of a position applies soft-NMS to every head, picks the owner and
+// writes l''.
 template <int GM>
-__global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
+__global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
   grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
-  float* ell = sm;                    // [G][W]
+  float* key = sm;                    // [G][W] dominance key
+  float* xo = key + a.G * W;          // [G][tile] log-evidence
   const int bg = blockIdx.y;                        // logical (row, kv head)
   const int bl = bg / a.Hkv, g = bg - bl * a.Hkv;
   const int b = a.rows.phys(bl);                    // the sequence
@@ -155,10 +173,11 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
   __shared__ double bc;
   __shared__ int qn;
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
-  const float nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
-  const float inv_z = (float)(1.0 / reduce_parts(pbg, a.nch, 1, &bc));
+  const double nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
+  const double inv_z = 1.0 / reduce_parts(pbg, a.nch, 1, &bc);
   const float* nrm = a.norms + ((size_t)b * a.Hkv + g) * a.norm_ld;
-  const float lam = a.lam;
+  const bool by_x = a.lam <= 0.0;          // lambda = 0: s = f~, decided on x
+  const double lam_r = a.lam * inv_z;      // lambda / Z
   // logits rows of the group: nq query slots of G heads (nq = 1: row b * Hq + g * G + h)
   const size_t row0 = ((size_t)b * a.Hkv + g) * (size_t)(a.nq * G);
   const float* z0 = a.logits + row0 * a.ld + a.lo;
@@ -167,29 +186,38 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
 #pragma unroll
   for (int h = 0; h < GM; ++h) lsec[h] = (h < G) ? a.lse_cand[row0 + h] : 0.f;
   if (a.nq > 1) {
-    // evidence window: the mean of the slots' restricted distributions
+    // evidence window: f~ = the mean of the slots' restricted distributions,
+    // x = ln f~ = m + ln(mean exp(x_i - m)), m the largest x_i
     for (int k = threadIdx.x; k < W; k += blockDim.x) {
       const int c = c0 - a.w + k;
+      const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (c < 0 || c >= a.nC) {
 #pragma unroll
         for (int h = 0; h < GM; ++h)
-          if (h < G) ell[h * W + k] = nan;
+          if (h < G) key[h * W + k] = nan;
         continue;
       }
       const int j = a.lo + c;
-      const float r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * inv_z;
+      const double r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * lam_r;   // lambda r_j
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
-          float ft = 0.f;
-          for (int i = 0; i < a.nq; ++i) {
+          float m = -INFINITY;
+          for (int i = 0; i < a.nq; ++i)
             if ((a.qmask >> i) & 1u) {
               const size_t row = (size_t)i * G + h;
-              ft += fast_exp2((z0[row * a.ld + c] - a.lse_cand[row0 + row]) * kLog2e);
+              m = fmaxf(m, z0[row * a.ld + c] - a.lse_cand[row0 + row]);
             }
-          }
-          const float sv = (1.f - lam) * (ft * a.inv_nq) + lam * r;
-          ell[h * W + k] = logf(sv + 1e-30f);
+          float acc = 0.f;
+          for (int i = 0; i < a.nq; ++i)
+            if ((a.qmask >> i) & 1u) {
+              const size_t row = (size_t)i * G + h;
+              acc += fast_exp2((z0[row * a.ld + c] - a.lse_cand[row0 + row] - m) * kLog2e);
+            }
+          const float x = m + logf(acc * a.inv_nq);
+          const float ft = fast_exp2(x * kLog2e);
+          key[h * W + k] = by_x ? x : (float)fma(a.one_minus_lam, (double)ft, r);
+          if (tile_k) xo[h * a.tile + k - a.w] = x;
         }
       }
     }
@@ -212,25 +240,25 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
     for (int u = 0; u < kU; ++u) {
       const int k = k0 + u * blockDim.x;
       if (k >= W) continue;
+      const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (in[u]) {
         const int j = a.lo + c0 - a.w + k;
-        const float r = kappa_of(nbar, nv[u]) * pi_of(a.L, j) * inv_z;
+        const double r = kappa_of(nbar, nv[u]) * pi_of(a.L, j) * lam_r;   // lambda r_j
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
           if (h < G) {
             // exp through the hardware's base-2 approximation (relative
-            // error ~1e-7); the log stays the accurate one, since the
-            // selection compares scores that can sit an ulp apart and an
-            // approximate log does not keep their order
-            const float ft = fast_exp2((zv[u][h] - lsec[h]) * kLog2e);
-            const float sv = (1.f - lam) * ft + lam * r;
-            ell[h * W + k] = logf(sv + 1e-30f);
+            // error ~1e-7, below the error of the logits themselves)
+            const float x = zv[u][h] - lsec[h];
+            const float ft = fast_exp2(x * kLog2e);
+            key[h * W + k] = by_x ? x : (float)fma(a.one_minus_lam, (double)ft, r);
+            if (tile_k) xo[h * a.tile + k - a.w] = x;
           }
         }
       } else {
 #pragma unroll
         for (int h = 0; h < GM; ++h)
-          if (h < G) ell[h * W + k] = nan;
+          if (h < G) key[h * W + k] = nan;
       }
     }
   }
@@ -241,8 +269,8 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
   // still undecided go to a queue.  2b: the queue, scanned to w with all lanes
   // busy.  dom = distance of the nearest dominator, 0: none within w.
   constexpr int kNear = 4;
-  uint16_t* dom = reinterpret_cast<uint16_t*>(ell + G * W);            // [G][tile]
-  uint32_t* queue = reinterpret_cast<uint32_t*>(dom + G * a.tile);     // [tile]
+  uint16_t* dom = reinterpret_cast<uint16_t*>(xo + G * a.tile);          // [G][tile]
+  uint32_t* queue = reinterpret_cast<uint32_t*>(dom + G * a.tile);       // [tile]
   const int lane = threadIdx.x & 31;
   for (int k0 = 0; k0 < tile_n; k0 += blockDim.x) {
     const int k = k0 + threadIdx.x;
@@ -251,7 +279,7 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
-          const float* row = ell + h * W + a.w + k;
+          const float* row = key + h * W + a.w + k;
           const float e = row[0];
           int d_hit = 0;
 #pragma unroll
@@ -273,15 +301,15 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
     }
   }
   __syncthreads();
-  const int nq = qn;
-  for (int qi = threadIdx.x; qi < nq; qi += blockDim.x) {
+  const int nqueue = qn;
+  for (int qi = threadIdx.x; qi < nqueue; qi += blockDim.x) {
     const uint32_t ent = queue[qi];
     const int k = (int)(ent & 0xffffu);
     uint32_t open = ent >> 16;
     while (open) {
       const int h = __ffs(open) - 1;
       open &= open - 1u;
-      const float* row = ell + h * W + a.w + k;
+      const float* row = key + h * W + a.w + k;
       const float e = row[0];
       int d_hit = 0;
       for (int d = kNear + 1; d <= a.w; ++d) {
@@ -294,26 +322,42 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
     }
   }
   __syncthreads();
+  // Phase 3: l' = ln(s + 1e-30) - alpha_soft * weight(d); the owner scans the
+  // heads in order (ties to the lowest): equal distances compare by x (never
+  // when lambda = 1: the evidence has no weight), others by l'.
   const float inv_w = 1.f / (float)a.w;
+  const bool ev_counts = a.one_minus_lam > 0.0;
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
-    float l1[GM];
+    float l1[GM], xv[GM];
+    int dv[GM];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       l1[h] = -INFINITY;
+      xv[h] = 0.f;
+      dv[h] = 0;
       if (h < G) {
         const int d = dom[h * a.tile + k];
         const float pen = d > 0 ? 1.f - (float)(d - 1) * inv_w : 0.f;
-        l1[h] = ell[h * W + a.w + k] - a.alpha_soft * pen;
+        xv[h] = xo[h * a.tile + k];
+        const float sv = by_x ? fast_exp2(xv[h] * kLog2e) : key[h * W + a.w + k];
+        l1[h] = logf(sv + 1e-30f) - a.alpha_soft * pen;
+        dv[h] = d;
       }
     }
-    int owner = 0;
-    float best = l1[0];
+    int owner = 0, bd = dv[0];
+    float bx = xv[0], bl = l1[0];
 #pragma unroll
-    for (int h = 1; h < GM; ++h)
-      if (h < G && l1[h] > best) {
-        best = l1[h];
-        owner = h;
+    for (int h = 1; h < GM; ++h) {
+      if (h < G) {
+        const bool wins = dv[h] == bd ? (ev_counts && xv[h] > bx) : (l1[h] > bl);
+        if (wins) {
+          owner = h;
+          bd = dv[h];
+          bx = xv[h];
+          bl = l1[h];
+        }
       }
+    }
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
@@ -327,10 +371,11 @@ __global__ void __launch_bounds__(256) select_scores_kernel(const __grid_constan
 // ---------------------------------------------------------------- host
 int score_tile(int G) { return std::max(256, 4096 / G); }
 
-// log-scores with halo, nearest-dominator distances, queue of undecided positions
+// dominance keys with halo, log-evidence, nearest-dominator distances, queue
+// of undecided positions
 size_t score_smem(int G, int tile, int w) {
-  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(uint16_t) +
-         (size_t)tile * sizeof(uint32_t);
+  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(float) +
+         (size_t)G * tile * sizeof(uint16_t) + (size_t)tile * sizeof(uint32_t);
 }
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }
@@ -371,8 +416,9 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
   a.w = std::max(p.nms_window / 2, 1);
   a.tile = score_tile(G);
-  const float lam = std::min(std::max(p.lambda, 0.f), p.lambda_clip);
+  const double lam = std::min(std::max((double)p.lambda, 0.0), (double)p.lambda_clip);
   a.lam = lam;
+  a.one_minus_lam = 1.0 - lam;
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;

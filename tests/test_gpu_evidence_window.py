@@ -71,13 +71,12 @@ def _run(cfg, per_sequence):
                     fw = [f] + [O.dense_attention(H.to64(li.q[t - i, b, hs]), Kc, Vc)[1]
                                 for i in range(1, min(Wn, t + 1))]
                     n_slow_window += len(fw) > 1
-                    ell, ell1, ell2 = H.oracle_selector_detail(f, O.key_norms(Kc), L, cfg, f_window=fw)
-                    amb = H.ambiguous_positions(ell, ell1, cfg.nms_window, G)
-                    ora = O.topk(ell2, K) + lo
+                    qw = [H.to64(li.q[t - i, b, hs]) for i in range(len(fw))]
+                    bnd, _ = H.decode_selection_bounds(qw[0], Kc, f, L, cfg, f_window=fw, q_window=qw)
                     n = int(layer.n_rows[b, g])
                     sg = H.packed_sets(layer.pos[b, g].cpu().numpy(), layer.headmask[b, g].cpu().numpy(),
                                        n, cfg.n_sink, G)
-                    H.assert_selection_close(np.stack(sg), ora, ell2, amb, lo, what)
+                    H.check_selection(np.stack(sg), bnd, K, lo, what)
                     sets[b * cfg.Hkv + g] = sg
                 else:
                     o = O.sparse_attention(H.to64(li.q[t, b, hs]), Kc, Vc,
