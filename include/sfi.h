@@ -197,16 +197,17 @@ sfi_status sfi_dense_attn_append(const sfi_shape* shape, const sfi_paged_kv* kv,
 
 /* sfi_dense_attn without a workspace argument, for callers that cannot
  * allocate device memory where they call it: serving runtimes whose pool
- * hands the library only input and output tensors, plugin or embedded hosts
- * without access to the CUDA allocator, code that must not allocate during
- * CUDA graph capture.  The paper has no counterpart to this entry point.
- * Arguments and results are those of sfi_dense_attn.  The scratch (a work
+ * hands the library only input and output tensors, and plugin or embedded
+ * hosts without access to the CUDA allocator.  The paper has no counterpart
+ * to this entry point.  Arguments, their checks and results are those of
+ * sfi_dense_attn.  The scratch (a work
  * counter and the split-K partials) is a static 16 MiB device array that
  * every GPU loading the library holds until the process exits; a call whose
  * partials would not fit returns SFI_ERR_WORKSPACE and launches nothing.
  * Nothing is allocated.  The first call on each device looks up the array's
- * device address (cudaGetSymbolAddress), so make it before any stream
- * capture.  All calls share the one array and it keeps the last call's
+ * device address (cudaGetSymbolAddress) and keeps it for the process, which
+ * assumes the device's context is not reset meanwhile; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the last call's
  * contents (the counter is cleared at the start of every call): calls that
  * overlap on the GPU race, so order them (one stream, or events). */
 sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
@@ -253,14 +254,16 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
 /* Per-row top-K: the K largest of scores[r, 0:n] (finite values; ties ->
  * lower index), written ascending as idx[r, 0:K] = offset + column.  rows =
  * number of rows; scores row stride ld_s, idx row stride ld_i (elements);
- * n <= 262144.  ws: device scratch of sfi_topk_workspace_size(rows, n) bytes,
- * 16-byte aligned, zero-filled before its first use; every successful call
- * leaves it ready for the next one with the same rows (zero it again after an
- * error or before a call with another row count).  Exact radix select over
- * order-preserving 32-bit keys of the scores: three digit passes (12, 12 and
- * 8 bits; every row cut into slices of 8192 with one CTA each, the last CTA
- * of a row narrowing the threshold prefix), then a pass marking the scores
- * above the threshold and one taking the ties in position order. */
+ * n <= 262144, rows <= 65535.  The top-K keeps its state on chip and needs
+ * no scratch: sfi_topk_workspace_size reports 0 and ws may be null (a
+ * ws_bytes below the reported size is refused).  Exact radix select over
+ * order-preserving 32-bit keys of the scores, one thread-block cluster of up
+ * to 8 CTAs per row, each CTA holding its slice's keys in registers: the
+ * digit passes start at the highest bit where the row's smallest and largest
+ * keys differ (12 bits per pass), CTA histograms meet in distributed shared
+ * memory, and the ties at the threshold are taken in position order.  Not a
+ * step the pages describe in detail: the Top-K of gist.science/fr
+ * "B. Le Sélecteur" and gist.science/zh "2.2" (Top-K 选择). */
 sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes);
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
                     int32_t offset, int32_t* idx, int64_t ld_i, void* ws, size_t ws_bytes,

@@ -60,7 +60,9 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   off += w.part_bytes;
   const long nC = std::max<long>(Lmax - p.n_recent - p.n_sink, 1);
   w.stat_off = off;
-  w.stat_bytes = align_up((size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double), 256);
+  // per-chunk partial sums, then kappa * pi of every candidate
+  w.stat_bytes = align_up((size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double) +
+                          (size_t)bh * ((nC + 1) / 2 * 2) * sizeof(double), 256);
   off += w.stat_bytes;
   w.sel_off = off;
   w.sel_bytes = align_up((size_t)s.B * s.Hq * ((nC + 3) / 4 * 4) * sizeof(float), 256);
@@ -72,9 +74,6 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   w.bits_off = off;
   w.bits_bytes = align_up((size_t)s.B * s.Hq * w.bits_ld * sizeof(uint32_t), 256);
   off += w.bits_bytes;
-  w.tk_off = off;
-  w.tk_bytes = align_up(topk_scratch_bytes(s.B * s.Hq, (int)std::min<long>(nC, topk_max_n())), 256);
-  off += w.tk_bytes;
   w.total = off;
   return w;
 }
@@ -143,11 +142,12 @@ sfi_status check_packed(const sfi_shape* s, const sfi_params* p, const sfi_packe
     if (_r != SFI_OK) return _r;       \
   } while (0)
 
-// Shared bodies of the attention entry points with and without the fused
-// append of the step's token (tok == nullptr: none).
-sfi_status dense_attn_impl(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L, const StepToken* tok,
-                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras, void* ws,
-                           size_t ws_bytes, sfi_stream stream) {
+}  // namespace
+
+// Arguments of a dense-attention call (all but the scratch): shared by the
+// workspace and the allocation-free entry points.
+sfi_status check_dense_call(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L, const sfi_bf16* q,
+                            const float* out, const sfi_dense_extras* extras) {
   SFI_TRY(check_shape(shape));
   SFI_TRY(check_kv(kv));
   SFI_TRY(check_L(shape, L));
@@ -158,8 +158,19 @@ sfi_status dense_attn_impl(const sfi_shape* shape, const sfi_paged_kv* kv, int32
     if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
       return SFI_ERR_SHAPE;
   }
-  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
   if (!aligned16(q)) return SFI_ERR_INVALID_ARG;
+  return SFI_OK;
+}
+
+namespace {
+
+// Shared bodies of the attention entry points with and without the fused
+// append of the step's token (tok == nullptr: none).
+sfi_status dense_attn_impl(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L, const StepToken* tok,
+                           const sfi_bf16* q, float* out, const sfi_dense_extras* extras, void* ws,
+                           size_t ws_bytes, sfi_stream stream) {
+  SFI_TRY(check_dense_call(shape, kv, L, q, out, extras));
+  if (!ws || !aligned16(ws)) return SFI_ERR_WORKSPACE;
   const size_t part_bytes = ws_bytes > 256 ? ws_bytes - 256 : 0;
   return run_dense_attn(*shape, *kv, L, q, out, extras, static_cast<int*>(ws),
                         reinterpret_cast<float*>(static_cast<char*>(ws) + 256), part_bytes,
@@ -309,7 +320,7 @@ sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes) {
   if (!bytes) return SFI_ERR_INVALID_ARG;
   if (rows < 0 || n < 1) return SFI_ERR_SHAPE;
   if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  *bytes = topk_scratch_bytes(rows, n);
+  *bytes = 0;   // the top-K keeps its state on chip
   return SFI_OK;
 }
 
@@ -319,10 +330,9 @@ sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, 
   if (!scores || !idx) return SFI_ERR_INVALID_ARG;
   if (rows < 0 || n < 1 || K < 1 || K > n || ld_s < n || ld_i < K) return SFI_ERR_SHAPE;
   if (n > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  if (!ws || !aligned16(ws) || ws_bytes < topk_scratch_bytes(rows, n))
-    return SFI_ERR_WORKSPACE;
-  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, nullptr, 0, topk_scratch(ws, rows, n),
-                  (cudaStream_t)stream);
+  (void)ws;
+  (void)ws_bytes;
+  return run_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, nullptr, 0, (cudaStream_t)stream);
 }
 
 sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sfi_paged_kv* kv,
@@ -347,8 +357,7 @@ sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sf
   SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s,
                             static_cast<char*>(ws) + w.stat_off, st));
   const int rows = shape->B * shape->Hq;
-  SFI_TRY(run_topk(rows, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0,
-                   topk_scratch(static_cast<char*>(ws) + w.tk_off, rows, nC), st));
+  SFI_TRY(run_topk(rows, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0, st));
   if (K_out) *K_out = K;
   return SFI_OK;
 }

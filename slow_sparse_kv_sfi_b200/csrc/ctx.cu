@@ -53,7 +53,6 @@ struct sfi_ctx {
   float* scores = nullptr;
   uint32_t* bits = nullptr;
   int64_t bits_ld = 0;
-  char* topk_ws = nullptr;
   sfi::CompactScratch cmp;
   // compaction: incremental (rows that stay selected keep their slots) once
   // a layer's packed buffer holds this context's previous result
@@ -72,7 +71,7 @@ namespace {
 
 struct CtxLayout {
   size_t part_off, part_bytes, logit_off, logit_bytes, lsec_off, lsec_bytes, stat_off, stat_bytes, score_off,
-      score_bytes, bits_off, bits_bytes, tc_off, tc_bytes, tk_off, tk_bytes, ring_off, ring_layer_bytes,
+      score_bytes, bits_off, bits_bytes, tc_off, tc_bytes, ring_off, ring_layer_bytes,
       wout_off, total;
   int64_t bits_ld;
 };
@@ -114,9 +113,6 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p, int n_layers) {
   c.tc_off = off;
   c.tc_bytes = w.cmp_bytes;
   off += c.tc_bytes;
-  c.tk_off = off;
-  c.tk_bytes = w.tk_bytes;
-  off += c.tk_bytes;
   // evidence window: every layer's last W queries, [B][Hkv][W][G][D] bf16,
   // and the window launch's outputs [B][Hkv * W * G][D] fp32
   c.ring_off = off;
@@ -274,10 +270,7 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
     SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
                               c->stats, side, slow_map, wmask));
     SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-    // the scratch is laid out for the whole batch whatever the rows of this
-    // step, so its zero-state histograms stay where the last call cleared them
-    SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld,
-                     topk_scratch(c->topk_ws, B * s.Hq, nC), side));
+    SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, side));
     if (c->incremental && packed->p_max >= c->cmp.cap) {
       // step 0 starts a new decode: cache rows copied before may have changed
       const bool fresh = step == 0 || c->packed_seen[layer] != packed->pos;
@@ -391,7 +384,6 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   c->bits = reinterpret_cast<uint32_t*>(w + l.bits_off);
   c->bits_ld = l.bits_ld;
   c->cmp = compact_scratch(w + l.tc_off, c->s, c->p);
-  c->topk_ws = w + l.tk_off;
   // a new workspace holds no previous-selection state and no queries
   std::fill(c->packed_seen.begin(), c->packed_seen.end(), nullptr);
   std::fill(c->slot_step.begin(), c->slot_step.end(), -1);

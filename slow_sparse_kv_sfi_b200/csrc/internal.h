@@ -61,7 +61,6 @@ struct WsLayout {
   size_t stat_off, stat_bytes;
   size_t cmp_off, cmp_bytes;        // compaction tile counts
   size_t bits_off, bits_bytes;      // selection bitmaps [B*Hq][bits_ld]
-  size_t tk_off, tk_bytes;          // top-K scratch (zero before the first call)
   int64_t bits_ld;
   size_t total;
 };
@@ -114,6 +113,11 @@ struct StepToken {
   const sfi_bf16* v_new;
 };
 
+// Validation of a dense-attention call's shape, cache, length, query, output
+// and extras (api.cu); SFI_OK or the status the entry points return.
+sfi_status check_dense_call(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L, const sfi_bf16* q,
+                            const float* out, const sfi_dense_extras* extras);
+
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
@@ -137,22 +141,11 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
                              float* scores, int64_t ld_s, void* stat_ws,
                              cudaStream_t st, const RowMap& rows = RowMap(),
                              uint32_t window_mask = 0xffffffffu);
-// Scratch of the top-K kernels for `rows` rows of n scores (topk.cu).  ghist
-// and done must be zero before the first call; every call leaves them zero.
-struct TopkScratch {
-  int* ghist;         // [rows][4096] digit histogram
-  int* done;          // [rows] arrival counter of the digit kernels
-  int* info;          // [rows][4] threshold prefix, scores to take, digit mask
-  uint32_t* ties;     // [rows][words_ld] scores equal to the threshold
-  uint32_t* bits;     // [rows][words_ld] bitmap when the caller wants positions only
-  int64_t words_ld;
-};
-size_t topk_scratch_bytes(int rows, int n);
-TopkScratch topk_scratch(void* base, int rows, int n);
 // K largest of every row (ties to the lower index): bitmap bits[rows][ld_b]
-// and / or ascending positions idx[rows][ld_i] (+ offset).
+// and / or ascending positions idx[rows][ld_i] (+ offset).  No scratch: the
+// cluster kernel of topk.cu keeps its state on chip.
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
-                    int64_t ld_i, uint32_t* bits, int64_t ld_b, const TopkScratch& w, cudaStream_t st);
+                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st);
 int topk_max_n();
 // Compaction scratch (inside the workspace): per-tile counts of the full
 // compaction, and the incremental compaction's counts, previous-position

@@ -4,9 +4,8 @@
 // sfi_dense_attn needs scratch (a work counter and the split-K partials) and
 // takes it as a caller-allocated workspace.  Some callers have no way to
 // provide one: serving runtimes whose memory pool hands the library only the
-// input and output tensors, plugin or embedded hosts that have no access to
-// the CUDA allocator, and code that must not allocate while a CUDA graph is
-// being captured.  This entry point runs the same kernels with the scratch
+// input and output tensors, and plugin or embedded hosts that have no access
+// to the CUDA allocator.  This entry point runs the same kernels with the scratch
 // taken from g_noalloc_scratch, a file-scope device array of
 // kNoAllocScratchBytes that every GPU which loads the library holds until the
 // process exits.
@@ -27,7 +26,9 @@ std::mutex g_mu;
 void* g_addr[64] = {nullptr};
 
 // Device address of g_noalloc_scratch on the current device.  The first call
-// on a device looks it up (host code only holds a stand-in for the symbol).
+// on a device looks it up (host code only holds a stand-in for the symbol)
+// and keeps it for the life of the process: this assumes the device's
+// context is not reset (cudaDeviceReset) while the library is loaded.
 sfi_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SFI_ERR_CUDA;
@@ -46,8 +47,6 @@ __global__ void zero_counter_kernel(int* ctr) {
   ctr[0] = 0;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace sfi
 
@@ -56,24 +55,11 @@ using namespace sfi;
 extern "C" sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_paged_kv* kv, int32_t L,
                                              const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
                                              sfi_stream stream) {
-  if (!shape || !kv || !q || !out) return SFI_ERR_INVALID_ARG;
+  // the same argument checks as sfi_dense_attn
+  const sfi_status v = check_dense_call(shape, kv, L, q, out, extras);
+  if (v != SFI_OK) return v;
   const sfi_shape& s = *shape;
-  if (s.B < 1 || s.Hq < 1 || s.Hkv < 1 || s.Hq % s.Hkv != 0) return SFI_ERR_SHAPE;
   const int G = s.Hq / s.Hkv;
-  if (G > 16) return SFI_ERR_UNSUPPORTED;
-  if (s.D != 64 && s.D != 128) return SFI_ERR_UNSUPPORTED;
-  if (s.page_size != kPage) return SFI_ERR_UNSUPPORTED;
-  if (s.max_pages < 1 || s.num_pages < 1) return SFI_ERR_SHAPE;
-  if ((long long)s.num_pages * s.Hkv * kPage >= (1LL << 31)) return SFI_ERR_SHAPE;
-  if (L < 1 || L > s.max_pages * kPage) return SFI_ERR_SHAPE;
-  if (!kv->k_pool || !kv->v_pool || !kv->page_table) return SFI_ERR_INVALID_ARG;
-  if (!aligned16(kv->k_pool) || !aligned16(kv->v_pool) || !aligned16(q)) return SFI_ERR_INVALID_ARG;
-  if (extras) {
-    if ((extras->logits || extras->probs) && extras->ld < L) return SFI_ERR_SHAPE;
-    if (extras->probs && !extras->lse) return SFI_ERR_INVALID_ARG;
-    if (extras->lse_cand && (extras->cand_lo < 0 || extras->cand_hi > L || extras->cand_lo >= extras->cand_hi))
-      return SFI_ERR_SHAPE;
-  }
   // partials this call needs, against the static capacity
   const int T = (L + kPage - 1) / kPage;
   const int ct = dense_chunk_tiles(s, L);

@@ -107,10 +107,12 @@ __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC
   if (threadIdx.x == 0) part[((size_t)bg * nch + blockIdx.x) * 2] = t;
 }
 
-// part[bgl][chunk][1] = sum of kappa * pi over the chunk of C
+// part[bgl][chunk][1] = sum of kappa * pi over the chunk of C, and
+// kp[bgl][c] = kappa_j pi_j (j = lo + c) for the score kernel
 __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
                                                                    const float* __restrict__ norms,
                                                                    int64_t norm_ld, double* part, int nch, int Hkv,
+                                                                   double* __restrict__ kp, int64_t kp_ld,
                                                                    const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   __shared__ double red[32];
@@ -121,9 +123,12 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
   const float* n = norm_row(norms, norm_ld, rows, Hkv, bg);
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double z = 0.0;
+  double* kpr = kp + (size_t)bg * kp_ld;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
     const int j = lo + c;
-    z += kappa_of(nbar, n[j]) * pi_of(L, j);
+    const double v = kappa_of(nbar, n[j]) * pi_of(L, j);
+    kpr[c] = v;
+    z += v;
   }
   const double t = block_sum_d(z, red);
   if (threadIdx.x == 0) pbg[blockIdx.x * 2 + 1] = t;
@@ -136,10 +141,10 @@ struct ScoreArgs {
   const float* logits;
   int64_t ld;
   const float* lse_cand;
-  const float* norms;
-  int64_t norm_ld;
   const double* stat_part;   // [B*Hkv][nch][2]
   int nch;
+  const double* kp;          // [B*Hkv][kp_ld] kappa_j pi_j of the candidates
+  int64_t kp_ld;
   float* scores;         // logical rows of the launch
   int64_t ld_s;
   RowMap rows;
@@ -173,9 +178,8 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   __shared__ double bc;
   __shared__ int qn;
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
-  const double nbar = nbar_of(reduce_parts(pbg, a.nch, 0, &bc), a.nC);
   const double inv_z = 1.0 / reduce_parts(pbg, a.nch, 1, &bc);
-  const float* nrm = a.norms + ((size_t)b * a.Hkv + g) * a.norm_ld;
+  const double* kpr = a.kp + (size_t)bg * a.kp_ld;
   const bool by_x = a.lam <= 0.0;          // lambda = 0: s = f~, decided on x
   const double lam_r = a.lam * inv_z;      // lambda / Z
   // logits rows of the group: nq query slots of G heads (nq = 1: row b * Hq + g * G + h)
@@ -197,8 +201,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
           if (h < G) key[h * W + k] = nan;
         continue;
       }
-      const int j = a.lo + c;
-      const double r = kappa_of(nbar, nrm[j]) * pi_of(a.L, j) * lam_r;   // lambda r_j
+      const double r = kpr[c] * lam_r;   // lambda r_j
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
@@ -225,14 +228,15 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   // kU positions per thread and round: all their loads are issued first
   constexpr int kU = GM >= 8 ? 2 : 4;
   for (int k0 = threadIdx.x; a.nq == 1 && k0 < W; k0 += kU * blockDim.x) {
-    float nv[kU], zv[kU][GM];
+    double kv[kU];
+    float zv[kU][GM];
     bool in[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int c = c0 - a.w + k0 + u * blockDim.x;
       in[u] = k0 + u * blockDim.x < W && c >= 0 && c < a.nC;
       const int cc = in[u] ? c : 0;
-      nv[u] = in[u] ? nrm[a.lo + cc] : 1.f;
+      kv[u] = in[u] ? kpr[cc] : 0.0;
 #pragma unroll
       for (int h = 0; h < GM; ++h) zv[u][h] = (in[u] && h < G) ? z0[(size_t)h * a.ld + cc] : 0.f;
     }
@@ -242,8 +246,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
       if (k >= W) continue;
       const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (in[u]) {
-        const int j = a.lo + c0 - a.w + k;
-        const double r = kappa_of(nbar, nv[u]) * pi_of(a.L, j) * lam_r;   // lambda r_j
+        const double r = kv[u] * lam_r;   // lambda r_j
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
           if (h < G) {
@@ -409,8 +412,11 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   dim3 sgrid(nch, nb * s.Hkv);
   launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch,
            s.Hkv, rows);
+  // kappa * pi of every candidate follows the partial sums in the statistics area
+  double* kp = part + (size_t)nb * s.Hkv * nch * 2;
+  const int64_t kp_ld = (nC + 1) / 2 * 2;
   launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
-           s.Hkv, rows);
+           s.Hkv, kp, kp_ld, rows);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
@@ -422,8 +428,8 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;
-  a.norms = kv.key_norms; a.norm_ld = norm_ld;
   a.stat_part = part; a.nch = nch;
+  a.kp = kp; a.kp_ld = kp_ld;
   a.scores = scores; a.ld_s = ld_s;
   a.rows = rows;
   a.nq = nq;

@@ -3,116 +3,68 @@
 // highest score per query head), ties to the lower position.
 //
 // Exact MSB radix select on the order-preserving uint32 image of every fp32
-// score.  The rows are long (one score per candidate position) and few (one
-// per query head), so every row is cut into slices of kSlice scores with one
-// CTA per (slice, row):
-//   topk_digit<p>, p = 0, 1, 2: histogram of digit p (key bits 31-20, 19-8,
-//                7-0) over the scores whose higher digits equal the prefix
-//                found so far, added into the row's global histogram; the
-//                last CTA of the row to arrive (arrival counter) extends the
-//                prefix by the digit that holds the remaining k-th largest,
-//                lowers k by the scores in higher digits and clears the
-//                histogram for the next pass.  After pass 2 the prefix is the
-//                threshold key T and k the number of scores equal to T taken;
-//   topk_mark    scores above T are selected, scores equal to T are ties
-//                (both as bitmap words);
-//   topk_ties    one CTA per row: the first k ties in position order join the
-//                selection; then, if asked, the bitmap becomes K ascending
-//                positions.
-// The prior makes the scores of distant positions nearly equal (the position
-// factor ln(1 + L - j) flattens), so any binning by value range would pile
-// most of a row into one bin; the radix digits split such rows exactly.
+// score, one thread-block cluster per row.  The row is cut into slices of
+// T * 32 scores, one CTA of T threads each (up to 8 CTAs, cluster rank =
+// slice), and every thread keeps its 32 keys in registers for the whole
+// kernel, so the scores are read once:
+//   1. the cluster's smallest and largest key: their common leading bits are
+//      every key's, so the digit passes start at the highest bit where they
+//      differ (rows of log-scores share sign and exponent: two passes of 12
+//      and at most 11 bits instead of three);
+//   2. per digit pass: each CTA builds the histogram of its keys that match
+//      the prefix found so far in shared memory; after a cluster barrier CTA
+//      c sums bins [c * per, (c + 1) * per) over every CTA's histogram through
+//      distributed shared memory; after a second barrier every CTA reads the
+//      range totals and the reduced bins of the range holding the remaining
+//      k-th largest key, and extends the prefix by that bin;
+//   3. the prefix is now the threshold key T: keys above it are selected,
+//      keys equal to it are ties, taken in position order (a cluster-wide
+//      exclusive count of the ties in lower slices) until K are chosen.
+// Outputs: the selection bitmap (one bit per score) and / or the K positions
+// in ascending order.  The prior makes the scores of distant positions
+// nearly equal, so the digits (not a binning by value range) split such rows
+// exactly.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace sfi {
 
 namespace {
 
-constexpr int kSlice = 8192;          // scores per slice (a multiple of 128)
-constexpr int kTkThreads = 256;       // digit / mark / ties: 32 scores per thread
+constexpr int kKPT = 32;              // keys per thread: 8 loads of 4
+constexpr int kMaxCluster = 8;        // portable cluster size
 constexpr int kDigitBins = 4096;      // largest digit: 12 bits
-constexpr int kMaxWords = 8192;       // rows of at most 262144 scores
+constexpr int kMaxN = kMaxCluster * 1024 * kKPT;   // 262144
 
-struct Digit {
-  int shift, bits;
-};
-__host__ __device__ constexpr Digit digit_of(int pass) {
-  return pass == 0 ? Digit{20, 12} : (pass == 1 ? Digit{8, 12} : Digit{0, 8});
-}
-
-// The 32 scores of this thread in slice [s0, s0 + kSlice) of a row, as keys:
-// element e of load u is score s0 + (u * kTkThreads + tid) * 4 + e, so every
-// warp-wide load reads 512 consecutive bytes.  All eight loads are issued
-// before any is used.  Scores past n read as key 0 and are flagged by the
-// callers.
-struct SliceKeys {
-  uint32_t k[8][4];
+struct TopkArgs {
+  int rows, n, K, offset;
+  const float* scores;
+  int64_t ld_s;
+  bool vec;                  // rows 16-byte aligned: float4 loads
+  uint32_t* bits;            // [rows][ld_b] selection bitmap, or null
+  int64_t ld_b;
+  int32_t* idx;              // [rows][ld_i] ascending positions + offset, or null
+  int64_t ld_i;
 };
 
-__device__ __forceinline__ int pos_of(int s0, int u, int e) { return s0 + (u * kTkThreads + threadIdx.x) * 4 + e; }
-
-__device__ __forceinline__ void load_keys(const float* row, int n, int s0, bool vec, SliceKeys& x) {
-  if (vec && s0 + kSlice <= n) {
-    float4 f[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(row + pos_of(s0, u, 0)));
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      x.k[u][0] = float_key(f[u].x);
-      x.k[u][1] = float_key(f[u].y);
-      x.k[u][2] = float_key(f[u].z);
-      x.k[u][3] = float_key(f[u].w);
-    }
-  } else {
-    float f[8][4];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = pos_of(s0, u, e);
-        f[u][e] = j < n ? __ldg(row + j) : 0.f;
-      }
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x.k[u][e] = float_key(f[u][e]);
-  }
+// Element e of load u of thread t: score s0 + (u * T + t) * 4 + e, so every
+// warp-wide load reads 512 consecutive bytes.
+template <int T>
+__device__ __forceinline__ int pos_of(int s0, int u, int e) {
+  return s0 + (u * T + (int)threadIdx.x) * 4 + e;
 }
 
-// Reverse (suffix) inclusive scan of one value per thread across the block;
-// wtot holds 64 ints.
-__device__ __forceinline__ int suffix_incl(int v, int* wtot) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int sh = 1; sh < 32; sh <<= 1) {
-    const int y = __shfl_down_sync(0xffffffffu, x, sh);
-    if (lane + sh < 32) x += y;
-  }
-  if (lane == 0) wtot[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    const int nwarps = blockDim.x >> 5;
-    const int t = lane < nwarps ? wtot[lane] : 0;
-    int s = t;
-#pragma unroll
-    for (int sh = 1; sh < 32; sh <<= 1) {
-      const int y = __shfl_down_sync(0xffffffffu, s, sh);
-      if (lane + sh < 32) s += y;
-    }
-    wtot[32 + lane] = s - t;
-  }
-  __syncthreads();
-  const int r = x + wtot[32 + w];
-  __syncthreads();
-  return r;
-}
-
-// Exclusive prefix scan of one value per thread across the block.
-__device__ __forceinline__ int prefix_excl(int v, int* wtot) {
+// Exclusive prefix sum over the block (T threads) of one value per thread;
+// *total = the block's sum.  ws holds 33 ints.
+template <int T>
+__device__ __forceinline__ int block_excl(int v, int* ws, int* total) {
+  constexpr int kW = T / 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -120,274 +72,319 @@ __device__ __forceinline__ int prefix_excl(int v, int* wtot) {
     const int y = __shfl_up_sync(0xffffffffu, x, sh);
     if (lane >= sh) x += y;
   }
-  if (lane == 31) wtot[w] = x;
+  __syncthreads();
+  if (lane == 31) ws[w] = x;
   __syncthreads();
   if (w == 0) {
-    const int nwarps = blockDim.x >> 5;
-    const int t = lane < nwarps ? wtot[lane] : 0;
+    const int t = lane < kW ? ws[lane] : 0;
     int s = t;
 #pragma unroll
     for (int sh = 1; sh < 32; sh <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, sh);
       if (lane >= sh) s += y;
     }
-    wtot[32 + lane] = s - t;
+    ws[lane] = s - t;
+    if (lane == 31) ws[32] = s;
   }
   __syncthreads();
-  const int r = x - v + wtot[32 + w];
+  const int r = x - v + ws[w];
+  *total = ws[32];
+  return r;
+}
+
+template <int T>
+__device__ __forceinline__ uint32_t block_reduce_u32(uint32_t v, bool take_max, uint32_t* ws) {
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) {
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, v, sh);
+    v = take_max ? max(v, y) : min(v, y);
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) ws[w] = v;
+  __syncthreads();
+  uint32_t r = ws[0];
+  for (int i = 1; i < T / 32; ++i) r = take_max ? max(r, ws[i]) : min(r, ws[i]);
   __syncthreads();
   return r;
 }
 
-// The bin of `hist` (nb bins, a multiple of the block size) holding the k-th
-// largest element counted from the top: *bin, and *above = elements in
-// higher bins.
-__device__ __forceinline__ void find_bin(const int* hist, int nb, int k, int* wtot, int* s_bin, int* s_above) {
-  const int per = nb / blockDim.x;
-  const int b0 = threadIdx.x * per;
-  int mine = 0;
-  for (int i = 0; i < per; ++i) mine += hist[b0 + i];
-  int above = suffix_incl(mine, wtot) - mine;
-  for (int i = per - 1; i >= 0; --i) {
-    const int h = hist[b0 + i];
-    if (above < k && above + h >= k) {
-      *s_bin = b0 + i;
-      *s_above = above;
-    }
-    above += h;
-  }
-  __syncthreads();
-}
-
-struct TopkArgs {
-  int rows, n, K, offset;
-  const float* scores;
-  int64_t ld_s;
-  bool vec;                  // rows 16-byte aligned: float4 loads
-  int slices;
-  TopkScratch w;
-  uint32_t* bits;            // [rows][ld_b] selection bitmap (output)
-  int64_t ld_b;
-  int32_t* idx;              // [rows][ld_i] ascending positions + offset, or null
-  int64_t ld_i;
-};
-
-// Row state in w.info: [0] prefix of the threshold key, [1] scores still to
-// take (k), [2] mask of the digits fixed so far.
-template <int PASS>
-__global__ void __launch_bounds__(kTkThreads) topk_digit_kernel(const TopkArgs a) {
+template <int T>
+__global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__ TopkArgs a) {
   grid_dep_enter();
-  constexpr Digit dg = digit_of(PASS);
-  constexpr int kNb = 1 << dg.bits;
-  constexpr uint32_t kDm = (uint32_t)kNb - 1u;
-  __shared__ int hist[kNb];
-  __shared__ int wtot[64];
-  __shared__ int s_last, s_bin, s_above;
-  const int row = blockIdx.y, s0 = blockIdx.x * kSlice;
-  for (int i = threadIdx.x; i < kNb; i += kTkThreads) hist[i] = 0;
-  SliceKeys x;
-  load_keys(a.scores + (size_t)row * a.ld_s, a.n, s0, a.vec, x);
-  int* info = a.w.info + (size_t)row * 4;
-  const uint32_t prefix = PASS == 0 ? 0u : (uint32_t)info[0];
-  const uint32_t pmask = PASS == 0 ? 0u : (uint32_t)info[2];
-  const int k = PASS == 0 ? a.K : info[1];
-  __syncthreads();
-  // Neighbouring scores share digits, and the bins of a row's bulk are few:
-  // a lane whose 4 scores share one digit counts them as one, and a run of
-  // such lanes with one digit adds once (from its first lane); lanes with
-  // mixed digits add their scores one by one.
-  const int lane = threadIdx.x & 31;
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  const int row = blockIdx.y;
+  const int s0 = rank * T * kKPT;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int hist[kDigitBins];
+  __shared__ int red[kDigitBins];
+  __shared__ uint32_t selw[T], tiew[T];
+  __shared__ int ws[33];
+  __shared__ uint32_t wsu[32];
+  __shared__ int pub[4];            // published to the cluster: range total, ties, selected
+  __shared__ int s_pick[3];         // bin, keys above it, k
+  __shared__ uint32_t s_mm[2];
+
+  // ---- keys
+  const float* srow = a.scores + (size_t)row * a.ld_s;
+  uint32_t key[8][4];
+  if (a.vec && s0 + T * kKPT <= a.n) {
+    float4 f[8];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    int d[4];
+    for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(srow + pos_of<T>(s0, u, 0)));
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t key = x.k[u][e];
-      d[e] = (pos_of(s0, u, e) < a.n && (key & pmask) == prefix) ? (int)((key >> dg.shift) & kDm) : -1;
+    for (int u = 0; u < 8; ++u) {
+      key[u][0] = float_key(f[u].x);
+      key[u][1] = float_key(f[u].y);
+      key[u][2] = float_key(f[u].z);
+      key[u][3] = float_key(f[u].w);
     }
-    const bool uni = d[0] == d[1] && d[0] == d[2] && d[0] == d[3];
-    const int dl = uni ? d[0] : -2;
-    const int dprev = __shfl_up_sync(0xffffffffu, dl, 1);
-    const bool head = lane == 0 || dprev != dl;
-    const unsigned heads = __ballot_sync(0xffffffffu, head);
-    if (uni) {
-      if (head && dl >= 0) {
-        const unsigned later = heads & ~((2u << lane) - 1u);   // run heads after this lane
-        const int next = later ? __ffs(later) - 1 : 32;
-        atomicAdd(&hist[dl], 4 * (next - lane));
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = pos_of<T>(s0, u, e);
+        key[u][e] = j < a.n ? float_key(__ldg(srow + j)) : 0u;
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (d[e] >= 0) atomicAdd(&hist[d[e]], 1);
-    }
   }
-  __syncthreads();
-  int* gh = a.w.ghist + (size_t)row * kDigitBins;
-  for (int i = threadIdx.x; i < kNb; i += kTkThreads)
-    if (hist[i]) atomicAdd(&gh[i], hist[i]);
-  // the last CTA of the row to arrive fixes this digit
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&a.w.done[row], 1) == a.slices - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  {
-    // every load in flight before any store (the row's histogram, from L2)
-    constexpr int kPer = kNb / kTkThreads;
-    int v[kPer];
+  // ---- 1. common leading bits of the whole row
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) v[i] = __ldcg(&gh[i * kTkThreads + threadIdx.x]);
+  for (int u = 0; u < 8; ++u)
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      hist[i * kTkThreads + threadIdx.x] = v[i];
-      gh[i * kTkThreads + threadIdx.x] = 0;   // cleared for the next pass / call
-    }
-  }
-  __syncthreads();
-  find_bin(hist, kNb, k, wtot, &s_bin, &s_above);
+    for (int e = 0; e < 4; ++e)
+      if (pos_of<T>(s0, u, e) < a.n) {
+        kmin = min(kmin, key[u][e]);
+        kmax = max(kmax, key[u][e]);
+      }
+  kmin = block_reduce_u32<T>(kmin, false, wsu);
+  kmax = block_reduce_u32<T>(kmax, true, wsu);
   if (threadIdx.x == 0) {
-    info[0] = (int)(prefix | ((uint32_t)s_bin << dg.shift));
-    info[1] = k - s_above;
-    info[2] = (int)(pmask | (kDm << dg.shift));
-    a.w.done[row] = 0;
+    s_mm[0] = kmin;
+    s_mm[1] = kmax;
   }
-}
+  cl.sync();
+  if (threadIdx.x == 0) {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int c = 0; c < cs; ++c) {
+      const uint32_t* r = cl.map_shared_rank(s_mm, c);
+      lo = min(lo, r[0]);
+      hi = max(hi, r[1]);
+    }
+    wsu[0] = lo;
+    wsu[1] = hi;
+  }
+  __syncthreads();
+  const uint32_t gmin = wsu[0], gmax = wsu[1];
+  // hb: highest bit where the row's keys differ (-1: all equal)
+  const int hb = gmin == gmax ? -1 : 31 - __clz((int)(gmin ^ gmax));
+  uint32_t pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
+  uint32_t prefix = gmax & pmask;
+  int k = a.K;
 
-// Bitmap words of the slice: scores above T selected, scores equal to T ties.
-__global__ void __launch_bounds__(kTkThreads) topk_mark_kernel(const TopkArgs a) {
-  grid_dep_enter();
-  const int row = blockIdx.y, s0 = blockIdx.x * kSlice;
-  const int lane = threadIdx.x & 31;
-  SliceKeys x;
-  load_keys(a.scores + (size_t)row * a.ld_s, a.n, s0, a.vec, x);
-  const uint32_t T = (uint32_t)a.w.info[(size_t)row * 4];
-  uint32_t* brow = a.bits + (size_t)row * a.ld_b;
-  uint32_t* trow = a.w.ties + (size_t)row * a.w.words_ld;
-  const int nw = (a.n + 31) / 32;
+  // ---- 2. digit passes over bits hb .. 0
+  int done_bits = 0;
+  while (done_bits < hb + 1) {
+    const int nbits = min(12, hb + 1 - done_bits);
+    const int shift = hb + 1 - done_bits - nbits;
+    const int nb = 1 << nbits;
+    const uint32_t dm = (uint32_t)nb - 1u;
+    for (int i = threadIdx.x; i < nb; i += T) hist[i] = 0;
+    __syncthreads();
+    // a lane whose 4 keys share one digit counts them as one, and a run of
+    // such lanes with one digit adds once (from its first lane)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      int d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t kk = key[u][e];
+        d[e] = (pos_of<T>(s0, u, e) < a.n && (kk & pmask) == prefix) ? (int)((kk >> shift) & dm) : -1;
+      }
+      const bool uni = d[0] == d[1] && d[0] == d[2] && d[0] == d[3];
+      const int dl = uni ? d[0] : -2;
+      const int dprev = __shfl_up_sync(0xffffffffu, dl, 1);
+      const bool head = lane == 0 || dprev != dl;
+      const unsigned heads = __ballot_sync(0xffffffffu, head);
+      if (uni) {
+        if (head && dl >= 0) {
+          const unsigned later = heads & ~((2u << lane) - 1u);
+          const int next = later ? __ffs(later) - 1 : 32;
+          atomicAdd(&hist[dl], 4 * (next - lane));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (d[e] >= 0) atomicAdd(&hist[d[e]], 1);
+      }
+    }
+    cl.sync();   // every histogram of the cluster complete
+    // this CTA's bin range, summed over the cluster
+    const int per = (nb + cs - 1) / cs;
+    const int r0 = rank * per;
+    int mine = 0;
+    for (int i = threadIdx.x; i < per; i += T) {
+      const int bin = r0 + i;
+      int s = 0;
+      if (bin < nb)
+        for (int c = 0; c < cs; ++c) s += cl.map_shared_rank(hist, c)[bin];
+      red[i] = s;
+      mine += s;
+    }
+    int tot;
+    block_excl<T>(mine, ws, &tot);
+    if (threadIdx.x == 0) pub[0] = tot;
+    cl.sync();   // every range reduced
+    // the range holding the k-th largest key (ranges of higher bins first),
+    // then the bin inside it: every CTA does this on the same data
+    if (threadIdx.x == 0) {
+      int above = 0, c = cs - 1;
+      for (; c > 0; --c) {
+        const int t = cl.map_shared_rank(pub, c)[0];
+        if (above + t >= k) break;
+        above += t;
+      }
+      s_pick[0] = c;
+      s_pick[1] = above;
+    }
+    __syncthreads();
+    const int cr = s_pick[0];
+    const int above_r = s_pick[1];
+    const int* rred = cl.map_shared_rank(red, cr);
+    const int nr = min(per, nb - cr * per);
+    // thread t takes bins [t * bp, (t + 1) * bp) of the range; suffix counts
+    const int bp = (nr + T - 1) / T;
+    const int b0 = threadIdx.x * bp;
+    int part = 0;
+    for (int i = 0; i < bp; ++i)
+      if (b0 + i < nr) part += rred[b0 + i];
+    int sum_all;
+    const int before = block_excl<T>(part, ws, &sum_all);   // bins below this thread's
+    int above = above_r + (sum_all - before - part);         // keys in higher bins of the range
+    for (int i = bp - 1; i >= 0; --i) {
+      if (b0 + i >= nr) continue;
+      const int h = rred[b0 + i];
+      if (above < k && above + h >= k) {
+        s_pick[0] = cr * per + b0 + i;
+        s_pick[2] = above;
+      }
+      above += h;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_pick[0] << shift;
+    pmask |= dm << shift;
+    k -= s_pick[2];
+    done_bits += nbits;
+    __syncthreads();
+  }
+  // ---- 3. keys above the threshold, ties in position order
+  const uint32_t thr = hb < 0 ? gmin : prefix;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    // this warp's 128 scores of load u: lane l holds 4l .. 4l + 3
-    const int jb = pos_of(s0, u, 0);
+    const int jb = pos_of<T>(s0, u, 0);
     uint32_t up = 0u, eq = 0u;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (jb + e < a.n) {
-        up |= (x.k[u][e] > T ? 1u : 0u) << e;
-        eq |= (x.k[u][e] == T ? 1u : 0u) << e;
+        up |= (key[u][e] > thr ? 1u : 0u) << e;
+        eq |= (key[u][e] == thr ? 1u : 0u) << e;
       }
     }
-    // bitmap word of lanes 8q .. 8q + 7: nibble (l & 7) of word q
+    // the word of lanes 8q .. 8q + 7: nibble (lane & 7) of word q
     uint32_t wu = up << (4 * (lane & 7)), we = eq << (4 * (lane & 7));
 #pragma unroll
     for (int sh = 1; sh <= 4; sh <<= 1) {
       wu |= __shfl_xor_sync(0xffffffffu, wu, sh);
       we |= __shfl_xor_sync(0xffffffffu, we, sh);
     }
-    const int wi = jb >> 5;
-    if ((lane & 7) == 0 && wi < nw) {
-      brow[wi] = wu;
-      trow[wi] = we;
+    if ((lane & 7) == 0) {
+      const int wi = (u * T + warp * 32) / 8 + (lane >> 3);
+      selw[wi] = wu;
+      tiew[wi] = we;
     }
   }
-}
-
-// One CTA per row: the first k ties in position order join the selection;
-// then the selection as ascending positions, if wanted.  Thread t owns the
-// bitmap words [t * per, (t + 1) * per), held in registers.
-constexpr int kMaxPer = kMaxWords / kTkThreads;
-
-__global__ void __launch_bounds__(kTkThreads) topk_ties_kernel(const TopkArgs a) {
-  grid_dep_enter();
-  __shared__ int wtot[64];
-  const int row = blockIdx.x, tid = threadIdx.x;
+  __syncthreads();
+  // thread i owns word i of the slice (words are in position order)
+  const int i = threadIdx.x;
+  const uint32_t tw = tiew[i];
+  int ties_tot;
+  const int tie_before_local = block_excl<T>(__popc(tw), ws, &ties_tot);
+  if (threadIdx.x == 0) pub[1] = ties_tot;
+  cl.sync();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int c = 0; c < rank; ++c) s += cl.map_shared_rank(pub, c)[1];
+    s_pick[1] = s;
+  }
+  __syncthreads();
+  int rk = s_pick[1] + tie_before_local;
+  uint32_t t = tw, take = 0u;
+  while (t && rk < k) {
+    const uint32_t lowbit = t & (~t + 1u);
+    take |= lowbit;
+    t ^= lowbit;
+    ++rk;
+  }
+  const uint32_t sw = selw[i] | take;
+  const int word = rank * T + i;
   const int nw = (a.n + 31) / 32;
-  const int k = a.w.info[(size_t)row * 4 + 1];
-  uint32_t* brow = a.bits + (size_t)row * a.ld_b;
-  const uint32_t* trow = a.w.ties + (size_t)row * a.w.words_ld;
-  const int per = (nw + kTkThreads - 1) / kTkThreads;
-  const int w0 = tid * per;
-  uint32_t tw[kMaxPer], sw[kMaxPer];
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    const bool in = i < per && w0 + i < nw;
-    tw[i] = in ? trow[w0 + i] : 0u;
-    sw[i] = in ? brow[w0 + i] : 0u;
-  }
-  int mine = 0;
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) mine += __popc(tw[i]);
-  int before = prefix_excl(mine, wtot);
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    uint32_t t = tw[i];
-    uint32_t take = 0u;
-    while (t && before < k) {
-      const uint32_t lowbit = t & (~t + 1u);
-      take |= lowbit;
-      t ^= lowbit;
-      ++before;
+  if (a.bits && word < nw) a.bits[(size_t)row * a.ld_b + word] = sw;
+  if (a.idx) {
+    int sel_tot;
+    const int sel_before_local = block_excl<T>(__popc(sw), ws, &sel_tot);
+    if (threadIdx.x == 0) pub[2] = sel_tot;
+    cl.sync();
+    if (threadIdx.x == 0) {
+      int s = 0;
+      for (int c = 0; c < rank; ++c) s += cl.map_shared_rank(pub, c)[2];
+      s_pick[1] = s;
     }
-    if (take) {
-      sw[i] |= take;
-      brow[w0 + i] = sw[i];   // this thread owns the word
-    }
-  }
-  if (!a.idx) return;
-  mine = 0;
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) mine += __popc(sw[i]);
-  int at = prefix_excl(mine, wtot);
-  int32_t* out = a.idx + (size_t)row * a.ld_i;
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    uint32_t t = sw[i];
-    while (t) {
-      const int bpos = __ffs(t) - 1;
-      t &= t - 1u;
-      if (at < a.K) out[at] = a.offset + (w0 + i) * 32 + bpos;
+    __syncthreads();
+    int at = s_pick[1] + sel_before_local;
+    int32_t* out = a.idx + (size_t)row * a.ld_i;
+    uint32_t x = sw;
+    while (x) {
+      const int bpos = __ffs(x) - 1;
+      x &= x - 1u;
+      if (at < a.K) out[at] = a.offset + word * 32 + bpos;
       ++at;
     }
   }
+  cl.sync();   // no CTA leaves while another may still read its shared memory
+}
+
+template <int T>
+sfi_status launch_topk(const TopkArgs& a, int cs, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, a.rows);
+  cfg.blockDim = dim3(T);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T>, a);
+  return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 }  // namespace
 
-int topk_max_n() { return kMaxWords * 32; }
-
-// Layout: the state that must stay zero between calls (histograms, arrival
-// counters) first, at offsets that depend on `rows` only, then the per-call
-// arrays.
-size_t topk_scratch_bytes(int rows, int n) {
-  const size_t nw = (size_t)(n + 31) / 32;
-  size_t b = 0;
-  b += align_up((size_t)rows * kDigitBins * sizeof(int), 256);   // ghist
-  b += align_up((size_t)rows * 5 * sizeof(int), 256);            // done, info
-  b += 2 * align_up((size_t)rows * nw * sizeof(uint32_t), 256);  // ties, bitmap
-  return b;
-}
-
-TopkScratch topk_scratch(void* base, int rows, int n) {
-  const size_t nw = (size_t)(n + 31) / 32;
-  char* p = static_cast<char*>(base);
-  TopkScratch w{};
-  w.ghist = reinterpret_cast<int*>(p);
-  p += align_up((size_t)rows * kDigitBins * sizeof(int), 256);
-  w.done = reinterpret_cast<int*>(p);
-  w.info = w.done + rows;
-  p += align_up((size_t)rows * 5 * sizeof(int), 256);
-  w.ties = reinterpret_cast<uint32_t*>(p);
-  p += align_up((size_t)rows * nw * sizeof(uint32_t), 256);
-  w.bits = reinterpret_cast<uint32_t*>(p);
-  w.words_ld = (int64_t)nw;
-  return w;
-}
+int topk_max_n() { return kMaxN; }
 
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
-                    int64_t ld_i, uint32_t* bits, int64_t ld_b, const TopkScratch& w, cudaStream_t st) {
+                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st) {
   if (rows <= 0) return SFI_OK;
   if (n > topk_max_n() || n < 1 || K < 1 || K > n) return SFI_ERR_UNSUPPORTED;
+  if (rows > 65535) return SFI_ERR_UNSUPPORTED;
   TopkArgs a{};
   a.rows = rows;
   a.n = n;
@@ -396,19 +393,16 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
   a.scores = scores;
   a.ld_s = ld_s;
   a.vec = (ld_s % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
-  a.slices = (n + kSlice - 1) / kSlice;
-  a.w = w;
-  a.bits = bits ? bits : w.bits;
-  a.ld_b = bits ? ld_b : w.words_ld;
+  a.bits = bits;
+  a.ld_b = ld_b;
   a.idx = idx;
   a.ld_i = ld_i;
-  const dim3 sgrid(a.slices, rows);
-  launch_k(topk_digit_kernel<0>, sgrid, dim3(kTkThreads), 0, st, a);
-  launch_k(topk_digit_kernel<1>, sgrid, dim3(kTkThreads), 0, st, a);
-  launch_k(topk_digit_kernel<2>, sgrid, dim3(kTkThreads), 0, st, a);
-  launch_k(topk_mark_kernel, sgrid, dim3(kTkThreads), 0, st, a);
-  launch_k(topk_ties_kernel, dim3(rows), dim3(kTkThreads), 0, st, a);
-  return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+  // slices of T * 32 scores: at most 8 per row, the fewest threads that cover it
+  const int cs = std::min(kMaxCluster, (n + 256 * kKPT - 1) / (256 * kKPT));
+  const int need = (n + cs * kKPT - 1) / (cs * kKPT);   // threads per slice
+  if (need <= 256) return launch_topk<256>(a, cs, st);
+  if (need <= 512) return launch_topk<512>(a, cs, st);
+  return launch_topk<1024>(a, cs, st);
 }
 
 }  // namespace sfi

@@ -241,9 +241,9 @@ def sfi_topk_workspace_size(rows, n) -> int:
 
 
 def sfi_topk(rows, n, scores, ld_s, K, offset, idx, ld_i, ws, stream=None):
-    """ws: zero-filled scratch of sfi_topk_workspace_size(rows, n) bytes (left zero-filled)."""
+    """ws: scratch of sfi_topk_workspace_size(rows, n) bytes (0: none needed; ws may be None)."""
     _check(lib().sfi_topk(rows, n, _p(scores), ld_s, K, offset, _p(idx), ld_i, _p(ws),
-                          ws.numel() * ws.element_size(), _stream(stream)), "sfi_topk")
+                          0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)), "sfi_topk")
 
 
 def sfi_select(shape, params, kv, L, logits, ld, lse_cand, sel_idx, sel_ld, ws, stream=None) -> int:

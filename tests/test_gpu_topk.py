@@ -1,8 +1,10 @@
 """sfi_topk against the oracle's top-K (K largest, ties to the lower index,
-ascending) on inputs that reach every path of the sliced kernels: several
-slices with a ragged last one, rows that are not 16-byte aligned, exact ties
-at the threshold, a boundary bin too full for the candidate buffer, constant
-rows, K = 1 and K = n, and one workspace reused by calls of different sizes."""
+ascending) on inputs that reach every path of the cluster kernel: one to
+eight slices per row with a ragged last one and slices holding no score,
+256, 512 and 1024 threads per slice (n up to the 262144 maximum), rows that
+are not 16-byte aligned, exact ties at the threshold, rows whose keys share
+no leading bit or all of them (constant rows), K = 1 and K = n, and calls of
+different sizes in a row."""
 import numpy as np
 import pytest
 import torch
@@ -45,6 +47,9 @@ def _check(x, K, **kw):
     (4, 777, 1),            # K = 1
     (2, 1000, 1000),        # K = n
     (64, 20000, 3000),
+    (1, 262144, 50000),     # eight slices of 1024 threads
+    (2, 200001, 7),         # 1024 threads, ragged
+    (3, 70000, 9000),       # 512 threads, the last slices hold no score
 ])
 def test_topk_random(rows, n, K):
     rng = np.random.default_rng(n + K)
@@ -74,6 +79,10 @@ def test_topk_full_boundary_bin_and_constant_rows():
     x[1, :5] = [1e4, -1e4, 2e4, -2e4, 3e4]       # outliers squeeze the rest into one bin
     x[2] = np.where(rng.random(n) < 0.5, 0.25, 0.75).astype(np.float32)
     _check(x, 30000)
+    # signs differ: the passes start at the top bit
+    y = rng.standard_normal((2, 5000)).astype(np.float32)
+    y[0, 17] = -np.float32(3e38)
+    _check(y, 2500)
 
 
 def test_topk_workspace_reused_across_sizes():

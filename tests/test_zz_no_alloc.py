@@ -1,7 +1,6 @@
 """sfi_dense_attn_noalloc: dense attention for callers that cannot allocate
 device memory at the call (runtimes that hand the library only input and
-output tensors, hosts without access to the CUDA allocator, code running
-during graph capture).  Its scratch is a static device array inside the
+output tensors, hosts without access to the CUDA allocator).  Its scratch is a static device array inside the
 library.  Checked through the C ABI against sfi_dense_attn, which takes a
 caller-allocated workspace, on two calls in a row (the static area keeps the
 previous call's contents), and for the clear rejection of a shape whose
