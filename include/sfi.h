@@ -147,7 +147,8 @@ const char* sfi_version(void);
  * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes
  * (16-byte aligned).  Ownership stays with the caller.  The scratch must be
  * zero-filled before its first use (the first 256 bytes hold a work counter
- * of the attention kernels, other parts the top-K histograms); every
+ * of the attention kernels, another part the incremental compaction's
+ * previous-position bitmap); every
  * successful call leaves it ready for the next one (after an error, zero it
  * again).  Calls that share one ws must not run concurrently. */
 sfi_status sfi_workspace_size(const sfi_shape* shape, const sfi_params* params, size_t* bytes);
@@ -307,6 +308,24 @@ sfi_status sfi_compact_incremental(const sfi_shape* shape, const sfi_params* par
 
 /* Read the latched device error word of kv (synchronous), then clear it. */
 sfi_status sfi_poll_error(const sfi_paged_kv* kv, int32_t* code);
+
+/* Limit, in nanoseconds, of every device-side pipeline wait of the library's
+ * kernels (process-wide; read at each launch; default 2e9).  A wait that
+ * reaches it latches SFI_ERR_TIMEOUT with its site into the cache's error
+ * word, stops waiting and lets its kernel return (copies in flight are
+ * drained first, under a fixed 2 s limit), so the context stays usable.  The
+ * limit must exceed the longest legitimate wait (milliseconds under heavy
+ * load).  ns outside [1e5, 6e10]: SFI_ERR_INVALID_ARG.  Failure detection
+ * has no counterpart in the pages. */
+sfi_status sfi_set_wait_limit(int64_t ns);
+sfi_status sfi_get_wait_limit(int64_t* ns);
+
+/* Runs the library's bounded wait on a barrier that nothing completes, with
+ * the given limit (ns in [1e3, 6e10]): the wait expires, SFI_ERR_TIMEOUT |
+ * (11 << 8) is latched into kv->err (which must be non-NULL; no other field
+ * is used) and the kernel returns.  For checking the expiry path on a healthy
+ * GPU; asynchronous on stream.  No counterpart in the pages. */
+sfi_status sfi_selftest_wait(const sfi_paged_kv* kv, int64_t limit_ns, sfi_stream stream);
 
 /* ------------------------------------------------------------------------
  * Decode-step driver ([ES] §2 trigger, §3 item 1 asynchronous pipeline;

@@ -64,6 +64,7 @@ struct AttnArgs {
   int p_max;
   int rec_lo;           // L - n_recent
   int* err;
+  unsigned long long wait_ns;   // limit of every pipeline wait
   // the step's token, appended at L - 1 by the item holding the last tile
   // (k_new == nullptr: already in the cache)
   const __nv_bfloat16* k_new;
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
         if (!drawn && st >= nst - 2) draw_next();
         bool good = true;
         if (lane == 0) {
-          good = !*abort_flag && mbar_wait(&empty[slot], phase ^ 1, a.err, kSiteAttnProducer);
+          good = !*abort_flag && mbar_wait(&empty[slot], phase ^ 1, a.err, kSiteAttnProducer, a.wait_ns);
           if (good) {
             StageMeta& m = smeta[slot];
             if (item >= a.n_items) {
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
           slot = kStages - 1;
           phase ^= 1;
         }
-        mbar_wait(&full[slot], phase, nullptr, 0);
+        mbar_wait(&full[slot], phase, nullptr, 0);   // own copies: the fixed 2 s limit, whatever wait_ns is
       }
     }
     return;
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
   float mrun[NT][2], lrun[NT][2], lcand[NT][2];
   int cur_b = 0, cur_g = 0;
   for (;;) {
-    if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer)) {
+    if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer, a.wait_ns)) {
       *abort_flag = 1;
       break;
     }
@@ -1057,6 +1058,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   a.scale = 1.0f / sqrtf((float)s.D);
   a.scale_log2 = kLog2e * a.scale;
   a.err = kv.err;
+  a.wait_ns = wait_limit_ns();
   set_token(a, s, kv, tok);
   const bool extras = ex && (ex->logits || ex->probs || ex->lse_cand);
   float* zbuf = nullptr;
@@ -1117,6 +1119,7 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   a.p_max = pk.p_max;
   a.rec_lo = std::max(L - p.n_recent, 0);
   a.err = kv.err;
+  a.wait_ns = wait_limit_ns();
   set_token(a, s, kv, tok);
   if (ev_begin) cudaEventRecord(ev_begin, st);
   sfi_status r = launch_attn<kFast>(s.D, G, maps, a, st);

@@ -34,13 +34,13 @@ __device__ __forceinline__ void grid_dep_enter() {
 constexpr int kPage = 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default limit of one wait: 2 s
 
 // Device error word layout: low byte = sfi_status, next byte = site id.
 enum ErrSite : int {
   kSiteAppend = 1, kSiteNorms = 2, kSiteAttnProducer = 3, kSiteAttnConsumer = 4,
   kSiteAttnPage = 5, kSiteAttnRows = 6, kSiteCompactIdx = 7, kSiteCompactPage = 8,
-  kSiteSelectPage = 9, kSiteCompactRows = 10,
+  kSiteSelectPage = 9, kSiteCompactRows = 10, kSiteSelfTest = 11,
 };
 
 __device__ __forceinline__ void latch_error(int* err, int status, int site) {
@@ -98,13 +98,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: true when the phase with the given parity completed, false
-// (after latching SFI_ERR_TIMEOUT) when kWaitLimitNs elapsed first.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int site) {
+// (after latching SFI_ERR_TIMEOUT) when limit_ns elapsed first.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) {
       latch_error(err, SFI_ERR_TIMEOUT, site);
       return false;
     }

@@ -15,6 +15,10 @@ namespace sfi {
 // Streaming-multiprocessor count of the current device (cached per device).
 int num_sms();
 
+// Limit of every device-side pipeline wait, in nanoseconds (sfi_set_wait_limit;
+// default 2 s), passed to each launch.
+unsigned long long wait_limit_ns();
+
 // Per-device one-time flag (up to 64 devices).
 struct DeviceOnce {
   std::atomic<uint64_t> bits{0};

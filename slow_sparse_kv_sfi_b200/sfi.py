@@ -88,6 +88,9 @@ def _declare(L):
         "sfi_compact": (C.c_int, [P, P, P, I32, P, I32, I32, P, P, SZ, P]),
         "sfi_compact_incremental": (C.c_int, [P, P, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "sfi_poll_error": (C.c_int, [P, C.POINTER(I32)]),
+        "sfi_set_wait_limit": (C.c_int, [C.c_int64]),
+        "sfi_get_wait_limit": (C.c_int, [C.POINTER(C.c_int64)]),
+        "sfi_selftest_wait": (C.c_int, [P, C.c_int64, P]),
         "sfi_ctx_create": (C.c_int, [P, P, I32, I32, C.POINTER(P)]),
         "sfi_ctx_destroy": (C.c_int, [P]),
         "sfi_ctx_workspace_size": (C.c_int, [P, C.POINTER(SZ)]),
@@ -109,7 +112,8 @@ EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_r
             "sfi_append_kv", "sfi_key_norms", "sfi_dense_attn", "sfi_dense_attn_append",
             "sfi_dense_attn_noalloc", "sfi_attn_probs", "sfi_fast_attn", "sfi_fast_attn_append",
             "sfi_select_scores", "sfi_topk_workspace_size", "sfi_topk", "sfi_select", "sfi_compact",
-            "sfi_compact_incremental", "sfi_poll_error",
+            "sfi_compact_incremental", "sfi_poll_error", "sfi_set_wait_limit", "sfi_get_wait_limit",
+            "sfi_selftest_wait",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
             "sfi_decode_step", "sfi_decode_step_rows", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_compaction",
             "sfi_ctx_timing"]
@@ -270,6 +274,20 @@ def sfi_poll_error(kv) -> int:
     code = C.c_int32(0)
     _check(lib().sfi_poll_error(C.byref(kv), C.byref(code)), "sfi_poll_error")
     return code.value
+
+
+def sfi_set_wait_limit(ns: int):
+    _check(lib().sfi_set_wait_limit(int(ns)), "sfi_set_wait_limit")
+
+
+def sfi_get_wait_limit() -> int:
+    v = C.c_int64(0)
+    _check(lib().sfi_get_wait_limit(C.byref(v)), "sfi_get_wait_limit")
+    return v.value
+
+
+def sfi_selftest_wait(kv, limit_ns: int, stream=None):
+    _check(lib().sfi_selftest_wait(C.byref(kv), int(limit_ns), _stream(stream)), "sfi_selftest_wait")
 
 
 class Context:

@@ -94,6 +94,11 @@ def test_null_pointers_rejected_before_any_launch(S):
     assert lib.sfi_topk_workspace_size(4, 10, C.byref(need)) == 0 and need.value == 0
     assert lib.sfi_topk(70000, 10, 16, 10, 3, 0, 16, 3, None, 0, None) == 3
     assert lib.sfi_ctx_set_workspace(None, None, 0) == 1
+    # wait limits outside their range, a self-test without an error word
+    assert lib.sfi_set_wait_limit(10) == 1 and lib.sfi_set_wait_limit(10 ** 12) == 1
+    got = C.c_int64(0)
+    assert lib.sfi_get_wait_limit(C.byref(got)) == 0 and got.value == 2_000_000_000
+    assert lib.sfi_selftest_wait(C.byref(S.PagedKV(None, None, None, None, None)), 50_000, None) == 1
 
 
 def test_context_rejects_bad_calls(S):
@@ -132,3 +137,34 @@ def test_new_entry_points_reject_bad_arguments(S):
     # the driver's per-sequence step and compaction switch without a context
     assert lib.sfi_decode_step_rows(None, 0, 0, None, 100, None, None, None, None, None, None, None, None) == 7
     assert lib.sfi_ctx_set_compaction(None, 1) == 1
+
+
+def test_noalloc_rejects_bad_arguments_like_the_workspace_call(S):
+    """sfi_dense_attn_noalloc shares sfi_dense_attn's argument checks: every
+    refusal below happens on the host, before the scratch address is looked up
+    or anything is launched, with the status sfi_dense_attn returns."""
+    lib = S.lib()
+    f = lib.sfi_dense_attn_noalloc
+    sh = S.make_shape(1, 4, 2, 64, 10, 10)
+    kv = S.PagedKV(16, 16, 16, None, None)
+    cases = [
+        (None, kv, 100, 16, 16, None, 1),                          # no shape
+        (sh, None, 100, 16, 16, None, 1),                          # no cache
+        (sh, kv, 100, None, 16, None, 1),                          # no query
+        (sh, kv, 100, 16, None, None, 1),                          # no output
+        (sh, kv, 100, 24, 16, None, 1),                            # query not 16-byte aligned
+        (sh, S.PagedKV(8, 16, 16, None, None), 100, 16, 16, None, 1),   # pool not aligned
+        (sh, kv, 161, 16, 16, None, 2),                            # longer than the cache
+        (S.make_shape(1, 34, 1, 64, 10, 10), kv, 100, 16, 16, None, 2),  # G > 32
+        (S.make_shape(1, 32, 1, 64, 10, 10), kv, 100, 16, 16, None, 3),  # G = 32 > 16
+        (S.make_shape(1, 4, 2, 96, 10, 10), kv, 100, 16, 16, None, 3),   # D not 64 / 128
+        (sh, kv, 100, 16, 16, S.DenseExtras(None, 16, None, 50, None, 0, 0), 2),          # ld < L
+        (sh, kv, 100, 16, 16, S.DenseExtras(None, None, None, 0, 16, 60, 40), 2),         # empty candidate range
+        (sh, kv, 100, 16, 16, S.DenseExtras(None, None, 16, 100, None, 0, 0), 1),         # probs without lse
+    ]
+    for shape, kvv, L, q, out, extras, code in cases:
+        args = [None if shape is None else C.byref(shape), None if kvv is None else C.byref(kvv), L, q, out,
+                None if extras is None else C.byref(extras), None]
+        assert f(*args) == code, (shape, L, q, out, code)
+        wsargs = args[:6] + [16, 1 << 20, None]
+        assert lib.sfi_dense_attn(*wsargs) == code
