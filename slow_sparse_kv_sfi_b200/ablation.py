@@ -81,7 +81,10 @@ def _selected(layer, cfg: W.SFIConfig) -> List[set]:
     return out
 
 
-def run_setting(cfg: W.SFIConfig, device) -> Dict[str, float]:
+def run_setting(cfg: W.SFIConfig, device, detail: bool = False) -> Dict[str, float]:
+    """Decodes one layer of cfg and returns the sweep's measurements; with
+    detail, also every fast step's recall per (sequence, query head) and every
+    slow step's stability per (sequence, query head), keyed by step."""
     shape, params = shape_of(cfg), params_of(cfg)
     li = W.make_layer(cfg, 0, device)
     layer = alloc_layer(cfg, li, device)
@@ -94,6 +97,7 @@ def run_setting(cfg: W.SFIConfig, device) -> Dict[str, float]:
     probs = torch.empty(cfg.B, cfg.Hq, ld, device=device)
     lse = torch.empty(cfg.B, cfg.Hq, device=device)
     recalls, reach, overlaps = [], [], []
+    per_step_recall, per_step_stability = {}, {}
     prev = None
     n_slow = 0
     L_slow = cfg.seq_len(0)
@@ -107,7 +111,9 @@ def run_setting(cfg: W.SFIConfig, device) -> Dict[str, float]:
             L_slow = L
             cur = _selected(layer, cfg)
             if prev is not None:
-                overlaps.extend(len(a & b) / max(len(a), 1) for a, b in zip(cur, prev))
+                st = [len(a & b) / max(len(a), 1) for a, b in zip(cur, prev)]
+                overlaps.extend(st)
+                per_step_stability[t] = st
             prev = cur
             continue
         ex = S.DenseExtras(lse.data_ptr(), None, probs.data_ptr(), ld, None, 0, 0)
@@ -121,18 +127,24 @@ def run_setting(cfg: W.SFIConfig, device) -> Dict[str, float]:
         cover[: max(L_slow - cfg.n_recent, 0)] = True
         cover[max(L - cfg.n_recent, 0):] = True
         recalls.append(r.flatten())
+        if detail:
+            per_step_recall[t] = r.flatten().cpu().tolist()
         reach.append((r / (f * cover).sum(dim=2)).flatten())
     torch.cuda.synchronize()
     assert S.sfi_poll_error(layer.kv) == 0
     ctx.close()
     rec = torch.cat(recalls) if recalls else torch.zeros(1, device=device)
     rea = torch.cat(reach) if reach else torch.zeros(1, device=device)
-    return {
+    res = {
         "fast_steps": len(recalls), "slow_steps": n_slow,
         "recall_mean": float(rec.mean()), "recall_p10": float(rec.quantile(0.10)), "recall_min": float(rec.min()),
         "recall_of_reachable_mean": float(rea.mean()), "recall_of_reachable_min": float(rea.min()),
         "stability_mean": float(sum(overlaps) / len(overlaps)) if overlaps else float("nan"),
     }
+    if detail:
+        res["recall_steps"] = per_step_recall
+        res["stability_steps"] = per_step_stability
+    return res
 
 
 def main():

@@ -28,8 +28,10 @@ DEV = "cuda"
 CASES = [
     # (workload, steps, overrides, sampled (b, kv head) groups)
     ("qwen3-4b-32k", 3, {}, [(0, 0), (5, 7)]),
-    ("qwen3-4b-128k-36l", 4, {}, [(0, 3), (1, 6)]),
-    ("qwen3-235b-a22b-64k", 4, {"slow_prefix": 2}, [(3, 1), (15, 3)]),   # G = 16
+    # slow steps 0 and 3: a full build, fast steps, an incremental refresh, a fast step
+    ("qwen3-4b-128k-36l", 5, {"boundary_mode": "none", "refresh_budget": 3}, [(0, 3), (1, 6)]),
+    # G = 16 Selector stress: nine slow steps in a row (eight incremental refreshes), then fast
+    ("qwen3-235b-a22b-64k", 10, {"slow_prefix": 9}, [(3, 1), (15, 3)]),
 ]
 
 
