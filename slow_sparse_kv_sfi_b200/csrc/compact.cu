@@ -15,8 +15,12 @@
 // compact_copy then copies the K and V rows, one warp per row, eight rows in
 // flight per warp, over fixed 128-row blocks (the selection is far from
 // uniform over positions, so per-tile copying would be imbalanced).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace sfi {
 
@@ -255,29 +259,32 @@ int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
 //   * the i-th mover is copied from the pages into the i-th hole.
 // Only movers are copied: with a stable support that is a few percent of the
 // rows.  A fresh buffer (no previous rows) gets sinks and U in ascending
-// order, the layout of the full compaction.  Five launches per slow step:
-//   inc_old    previous rows: mark their positions, keep or drop them;
-//   inc_count  per bitmap tile: |U| and the entering count;
-//   inc_slots  per slot tile: holes and kept rows past n_new;
-//   inc_list   the mover list (entering positions, then moved rows) and the
-//              hole list; clears the previous-position bitmap again;
-//   inc_copy   the movers' rows into the holes, zero rows up to the next
-//              multiple of 16, sinks of a fresh buffer, n_rows.
-constexpr int kSTile = 1024;        // slots per slot tile (4 per thread)
-
-int inc_slot_tiles(int cap) { return (cap + kSTile - 1) / kSTile; }
+// order: the full compaction above.
+//
+// One launch: a cluster of kIncCluster CTAs per (sequence, KV head).  The
+// previous rows' positions are marked in a bitmap over the candidates that
+// lives in the CTAs' shared memory, each CTA holding a slice of words (remote
+// bits land through distributed shared memory), so no global state has to
+// be cleared between calls.  The phases, each ended by a cluster barrier:
+//   1. previous rows (split over the CTAs): head mask rewritten (0: the row
+//      leaves), position marked in the bitmap;
+//   2. each CTA's bitmap words: |U| and the entering positions U & ~old;
+//   3. each CTA's slots of [n_sink, max(n_old, n_new)): kept, hole, moved
+//      (kept rows at or past n_new);
+//   4. the mover and hole lists, in the order of the rule (cluster-wide
+//      exclusive counts from the phases above);
+//   5. the copy: the i-th mover into the i-th hole, zero rows from n_new to
+//      the next multiple of 16, n_rows.
+constexpr int kIncThreads = 512;
+constexpr int kIncCluster = 8;
+constexpr int kIncMaxWords = 1024;       // candidate bitmap words per CTA (|C| <= 262144)
+constexpr int kIncMaxSlotWords = 2048;   // slot words per CTA (packed capacity <= 524288)
 
 struct IncArgs {
   CompactArgs c;        // bitmaps, pages, packed buffer, error word
   int cap;              // packed rows any selection can need (multiple of 16)
-  int n_stiles;
-  int fresh;            // 1: ignore the previous rows
-  int32_t* wcounts;     // [BH][n_tiles][2]  |U|, entering
-  int32_t* scounts;     // [BH][n_stiles][2] holes, moved
-  uint32_t* oldbits;    // [BH][nw] positions of the previous rows (zero between calls)
   int32_t* mover_pos;   // [BH][cap]
   int32_t* hole_slot;   // [BH][cap]
-  int32_t* info;        // [BH][4] previous rows taken into account, n_new, holes, movers
 };
 
 template <int GM>
@@ -289,298 +296,288 @@ __device__ __forceinline__ uint32_t head_bits_at(const CompactArgs& a, int b, in
   return m;
 }
 
-// Exclusive block prefix of two counts packed as lo + (hi << 16) (each at
-// most blockDim.x per call); returns the prefix, *total the block sum.
-__device__ __forceinline__ int block_scan2(int x, int* sh, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int v = x;
+// Exclusive prefix sum over the CTA of one value per thread; *total: the sum.
+__device__ __forceinline__ int inc_block_excl(int v, int* ws, int* total) {
+  constexpr int kW = kIncThreads / 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
 #pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, v, d);
-    if (lane >= d) v += y;
+  for (int sh = 1; sh < 32; sh <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, sh);
+    if (lane >= sh) x += y;
   }
   __syncthreads();
-  if (lane == 31) sh[warp] = v;
+  if (lane == 31) ws[w] = x;
   __syncthreads();
-  int before = 0, all = 0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-    const int t = sh[w];
-    if (w < warp) before += t;
-    all += t;
-  }
-  *total = all;
-  return before + v - x;
-}
-
-__device__ __forceinline__ int n_old_of(const IncArgs& a, int bgp) {
-  if (a.fresh) return 0;
-  const int n = a.c.n_rows[bgp];
-  return (n < a.c.n_sink || n > a.cap) ? 0 : n;
-}
-
-template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_old_kernel(const __grid_constant__ IncArgs a) {
-  grid_dep_enter();
-  const int bg = blockIdx.y;                    // logical (row, kv head)
-  const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
-  const int bp = a.c.rows.phys(b);                // the sequence
-  const int bgp = bp * a.c.Hkv + g;
-  const int n_old = n_old_of(a, bgp);
-  if (blockIdx.x == 0 && threadIdx.x == 0) a.info[bg * 4] = n_old;
-  const int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
-  uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
-  uint32_t* ob = a.oldbits + (size_t)bg * a.c.nw;
-  constexpr int kPer = kSTile / kCThreads;
-  int c[kPer];
+  if (w == 0) {
+    const int t = lane < kW ? ws[lane] : 0;
+    int s = t;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {   // all position loads first
-    const int s = blockIdx.x * kSTile + i * kCThreads + threadIdx.x;
-    c[i] = (s >= a.c.n_sink && s < n_old) ? pos[s] - a.c.lo : -1;
-  }
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int s = blockIdx.x * kSTile + i * kCThreads + threadIdx.x;
-    if (s < a.c.n_sink || s >= n_old) continue;
-    uint32_t m = 0u;
-    if (c[i] >= 0 && c[i] < a.c.nC) {
-      atomicOr(ob + (c[i] >> 5), 1u << (c[i] & 31));
-      m = head_bits_at<GM>(a.c, b, g, c[i]);
+    for (int sh = 1; sh < 32; sh <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, sh);
+      if (lane >= sh) s += y;
     }
-    hm[s] = m;   // 0: the row leaves
+    ws[lane] = s - t;
+    if (lane == 31) ws[32] = s;
   }
+  __syncthreads();
+  const int r = x - v + ws[w];
+  *total = ws[32];
+  return r;
 }
 
-template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_count_kernel(const __grid_constant__ IncArgs a) {
-  grid_dep_enter();
-  __shared__ int sh[kCThreads / 32];
-  const int bg = blockIdx.y;
-  const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
-  const int w = blockIdx.x * kCWords + threadIdx.x;
-  uint32_t hw[GM];
-  const uint32_t u = union_word<GM>(a.c, b, g, w, hw);
-  const uint32_t o = w < a.c.nw ? a.oldbits[(size_t)bg * a.c.nw + w] : 0u;
-  int total;
-  block_scan2(__popc(u) + (__popc(u & ~o) << 16), sh, &total);
-  if (threadIdx.x == 0) {
-    int32_t* wc = a.wcounts + ((size_t)bg * a.c.n_tiles + blockIdx.x) * 2;
-    wc[0] = total & 0xffff;
-    wc[1] = total >> 16;
-  }
-}
-
-// Totals over the tiles before `upto` (and over all of them) of one count.
-__device__ __forceinline__ void tile_prefix(const int32_t* cnt, int n, int upto, int which, int* before,
-                                            int* all) {
-  int s0 = 0, s1 = 0;
-  for (int t = threadIdx.x & 31; t < n; t += 32) {
-    const int v = cnt[t * 2 + which];
-    s1 += v;
-    if (t < upto) s0 += v;
-  }
-#pragma unroll
-  for (int sh = 16; sh >= 1; sh >>= 1) {
-    s0 += __shfl_xor_sync(0xffffffffu, s0, sh);
-    s1 += __shfl_xor_sync(0xffffffffu, s1, sh);
-  }
-  *before = s0;
-  *all = s1;
-}
-
-__device__ __forceinline__ int n_new_of(const IncArgs& a, int bg) {
-  int before, all;
-  tile_prefix(a.wcounts + (size_t)bg * a.c.n_tiles * 2, a.c.n_tiles, 0, 0, &before, &all);
-  return a.c.n_sink + all;
-}
-
-__global__ void __launch_bounds__(kCThreads) inc_slots_kernel(const __grid_constant__ IncArgs a) {
-  grid_dep_enter();
-  __shared__ int sh[kCThreads / 32];
-  const int bg = blockIdx.y;                    // logical (row, kv head)
-  const int bgp = a.c.rows.phys(bg / a.c.Hkv) * a.c.Hkv + bg % a.c.Hkv;
-  const int n_old = a.info[bg * 4];
-  const int n_new = min(n_new_of(a, bg), a.cap);
-  const uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
-  int x = 0;
-#pragma unroll
-  for (int i = 0; i < kSTile / kCThreads; ++i) {
-    const int s = blockIdx.x * kSTile + i * kCThreads + threadIdx.x;
-    const bool kept = s >= a.c.n_sink && s < n_old && hm[s] != 0u;
-    x += (s >= a.c.n_sink && s < n_new && !kept) ? 1 : 0;
-    x += (s >= n_new && kept) ? (1 << 16) : 0;
-  }
-  int total;
-  block_scan2(x, sh, &total);
-  if (threadIdx.x == 0) {
-    int32_t* sc = a.scounts + ((size_t)bg * a.n_stiles + blockIdx.x) * 2;
-    sc[0] = total & 0xffff;
-    sc[1] = total >> 16;
-  }
-}
-
-template <int GM>
-__global__ void __launch_bounds__(kCThreads) inc_list_kernel(const __grid_constant__ IncArgs a) {
-  grid_dep_enter();
-  __shared__ int sh[kCThreads / 32];
-  const int bg = blockIdx.y;                    // logical (row, kv head)
-  const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
-  const int bp = a.c.rows.phys(b);                // the sequence
-  const int bgp = bp * a.c.Hkv + g;
-  int32_t* mv = a.mover_pos + (size_t)bg * a.cap;
-  const int32_t* wc = a.wcounts + (size_t)bg * a.c.n_tiles * 2;
-  if ((int)blockIdx.x < a.c.n_tiles) {
-    // entering positions of this bitmap tile, ascending
-    const int w = blockIdx.x * kCWords + threadIdx.x;
-    uint32_t hw[GM];
-    const uint32_t u = union_word<GM>(a.c, b, g, w, hw);
-    uint32_t* ob = a.oldbits + (size_t)bg * a.c.nw;
-    const uint32_t o = w < a.c.nw ? ob[w] : 0u;
-    if (w < a.c.nw && o) ob[w] = 0u;          // back to the zero state
-    int before, all, total;
-    tile_prefix(wc, a.c.n_tiles, blockIdx.x, 1, &before, &all);
-    uint32_t e = u & ~o;
-    int r = before + block_scan2(__popc(e), sh, &total);
-    while (e) {
-      const int bit = __ffs(e) - 1;
-      e &= e - 1u;
-      if (r < a.cap) mv[r] = a.c.lo + w * 32 + bit;
-      ++r;
-    }
-    return;
-  }
-  // moved rows and holes of this slot tile, in slot order
-  const int t = blockIdx.x - a.c.n_tiles;
-  const int n_old = a.info[bg * 4];
-  int e_before, e_all, h_before, h_all, m_before, m_all;
-  tile_prefix(wc, a.c.n_tiles, 0, 1, &e_before, &e_all);
-  const int n_want = n_new_of(a, bg);
-  const int n_new = min(n_want, a.cap);
-  const int32_t* sc = a.scounts + (size_t)bg * a.n_stiles * 2;
-  tile_prefix(sc, a.n_stiles, t, 0, &h_before, &h_all);
-  tile_prefix(sc, a.n_stiles, t, 1, &m_before, &m_all);
-  if (t == 0 && threadIdx.x == 0) {
-    // totals for the copy; n_new > cap is reported there
-    a.info[bg * 4 + 1] = n_want;
-    a.info[bg * 4 + 2] = h_all;
-    a.info[bg * 4 + 3] = e_all + m_all;
-  }
-  const int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
-  const uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
-  int32_t* hs = a.hole_slot + (size_t)bg * a.cap;
-  int hr = h_before, mr = e_all + m_before;
-#pragma unroll 1
-  for (int i = 0; i < kSTile / kCThreads; ++i) {
-    const int s = t * kSTile + i * kCThreads + threadIdx.x;
-    const bool kept = s >= a.c.n_sink && s < n_old && hm[s] != 0u;
-    const bool hole = s >= a.c.n_sink && s < n_new && !kept;
-    const bool moved = s >= n_new && kept;
-    int total;
-    const int pre = block_scan2((hole ? 1 : 0) + (moved ? 1 << 16 : 0), sh, &total);
-    if (hole && hr + (pre & 0xffff) < a.cap) hs[hr + (pre & 0xffff)] = s;
-    if (moved && mr + (pre >> 16) < a.cap) mv[mr + (pre >> 16)] = pos[s];
-    hr += total & 0xffff;
-    mr += total >> 16;
-  }
+// Bits i of a 32-slot word starting at slot s0 with s0 + i < x.
+__device__ __forceinline__ uint32_t below(int s0, int x) {
+  if (x <= s0) return 0u;
+  if (x >= s0 + 32) return 0xffffffffu;
+  return (1u << (x - s0)) - 1u;
 }
 
 template <int D, int GM>
-__global__ void __launch_bounds__(kCopyWarps * 32) inc_copy_kernel(const __grid_constant__ IncArgs a) {
+__global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter();
-  constexpr int kUnits = D / 8;
-  constexpr int kRowUnits = 2 * kUnits;
-  constexpr int kRowsPerPass = 32 / kRowUnits;
-  constexpr int kRowsPerWarp = kCopyRows / kCopyWarps;
-  constexpr int kIn = 8;
-  __shared__ long long src[kCopyRows];
-  __shared__ int dst[kCopyRows];
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const CompactArgs& c = a.c;
+  constexpr int T = kIncThreads;
   const int bg = blockIdx.y;                    // logical (row, kv head)
-  const int b = bg / a.c.Hkv, g = bg - b * a.c.Hkv;
-  const int bp = a.c.rows.phys(b);                // the sequence
-  const int bgp = bp * a.c.Hkv + g;
-  const int4 inf = *reinterpret_cast<const int4*>(a.info + bg * 4);
-  const int n_want = inf.y;
+  const int b = bg / c.Hkv, g = bg - b * c.Hkv;
+  const int bp = c.rows.phys(b);                // the sequence
+  const int bgp = bp * c.Hkv + g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ uint32_t oldw[kIncMaxWords];       // this CTA's slice of the previous positions
+  __shared__ uint32_t entw[kIncMaxWords];       // its entering positions
+  __shared__ uint32_t keptw[kIncMaxSlotWords];  // its slots holding a kept row
+  __shared__ int pub[4];                        // published: |U|, entering, holes, moved
+  __shared__ int ws[33];
+  __shared__ int tot[8];
+  int32_t* pos = c.pos + (size_t)bgp * c.p_max;
+  uint32_t* hm = c.headmask + (size_t)bgp * c.p_max;
+  const int nw = c.nw;
+  const int Wc = (nw + cs - 1) / cs;
+  const int w0 = min(nw, rank * Wc), w1 = min(nw, w0 + Wc);
+  for (int i = tid; i < Wc; i += T) oldw[i] = 0u;
+  // previous rows; a count outside [n_sink, cap] means no usable buffer: the
+  // sinks are written again and every selected row enters
+  const int n_raw = c.n_rows[bgp];
+  const bool valid = n_raw >= c.n_sink && n_raw <= a.cap;
+  const int n_old = valid ? n_raw : c.n_sink;
+  cl.sync();   // every slice cleared before any remote bit lands
+
+  // ---- 1. previous rows
+  {
+    const int n1 = n_old - c.n_sink;
+    const int per1 = (n1 + cs - 1) / cs;
+    const int lo1 = c.n_sink + rank * per1, hi1 = min(n_old, lo1 + per1);
+    for (int s = lo1 + tid; s < hi1; s += T) {
+      const int ci = pos[s] - c.lo;
+      uint32_t m = 0u;
+      if ((unsigned)ci < (unsigned)c.nC) {
+        m = head_bits_at<GM>(c, b, g, ci);
+        const int wd = ci >> 5, owner = wd / Wc;
+        atomicOr(cl.map_shared_rank(oldw, owner) + (wd - owner * Wc), 1u << (ci & 31));
+      }
+      hm[s] = m;   // 0: the row leaves
+    }
+  }
+  cl.sync();
+
+  // ---- 2. this CTA's bitmap words
+  {
+    int cu = 0, ce = 0;
+    for (int w = w0 + tid; w < w1; w += T) {
+      uint32_t hw[GM];
+      const uint32_t u = union_word<GM>(c, b, g, w, hw);
+      const uint32_t e = u & ~oldw[w - w0];
+      entw[w - w0] = e;
+      cu += __popc(u);
+      ce += __popc(e);
+    }
+    int tu, te;
+    inc_block_excl(cu, ws, &tu);
+    inc_block_excl(ce, ws, &te);
+    if (tid == 0) {
+      pub[0] = tu;
+      pub[1] = te;
+    }
+  }
+  cl.sync();
+  if (tid == 0) {
+    int U = 0, E = 0, Eb = 0;
+    for (int r = 0; r < cs; ++r) {
+      const int* pr = cl.map_shared_rank(pub, r);
+      U += pr[0];
+      E += pr[1];
+      if (r < rank) Eb += pr[1];
+    }
+    tot[0] = U;
+    tot[1] = E;
+    tot[2] = Eb;
+  }
+  __syncthreads();
+  const int n_want = c.n_sink + tot[0];
   const int n_new = min(n_want, a.cap);
-  const int n_holes = inf.z, n_mov = inf.w;
-  const bool fresh = inf.x == 0;
+  const int E_tot = tot[1], E_before = tot[2];
+
+  // ---- 3. this CTA's slots: kept rows (one ballot per 32 slots), holes, moved
+  const int hi3 = max(n_old, n_new);
+  const int per3 = ((hi3 - c.n_sink + cs - 1) / cs + 31) / 32 * 32;
+  const int lo3 = c.n_sink + rank * per3, up3 = min(hi3, lo3 + per3);
+  const int nsw = up3 > lo3 ? (up3 - lo3 + 31) / 32 : 0;
+  for (int k = warp; k < nsw; k += T / 32) {
+    const int s = lo3 + k * 32 + lane;
+    const bool kept = s < up3 && s < n_old && hm[s] != 0u;
+    const uint32_t bw = __ballot_sync(0xffffffffu, kept);
+    if (lane == 0) keptw[k] = bw;
+  }
+  __syncthreads();
+  const int cw = (nsw + T - 1) / T;   // slot words per thread, contiguous
+  const int k0 = min(nsw, tid * cw), k1 = min(nsw, k0 + cw);
+  int hc = 0, mc = 0;
+  for (int k = k0; k < k1; ++k) {
+    const int s0 = lo3 + k * 32;
+    const uint32_t in = below(s0, up3), lt = below(s0, n_new), kw = keptw[k];
+    hc += __popc(in & lt & ~kw);
+    mc += __popc(in & ~lt & kw);
+  }
+  int th, tm;
+  const int h_local = inc_block_excl(hc, ws, &th);
+  const int m_local = inc_block_excl(mc, ws, &tm);
+  if (tid == 0) {
+    pub[2] = th;
+    pub[3] = tm;
+  }
+  cl.sync();
+  if (tid == 0) {
+    int H = 0, Hb = 0, M = 0, Mb = 0;
+    for (int r = 0; r < cs; ++r) {
+      const int* pr = cl.map_shared_rank(pub, r);
+      H += pr[2];
+      M += pr[3];
+      if (r < rank) {
+        Hb += pr[2];
+        Mb += pr[3];
+      }
+    }
+    tot[3] = H;
+    tot[4] = Hb;
+    tot[5] = M;
+    tot[6] = Mb;
+  }
+  __syncthreads();
+  const int H_tot = tot[3], M_tot = E_tot + tot[5];
+
+  // ---- 4. the lists
+  int32_t* mv = a.mover_pos + (size_t)bg * a.cap;
+  int32_t* hs = a.hole_slot + (size_t)bg * a.cap;
+  {
+    int hr = tot[4] + h_local, mr = E_tot + tot[6] + m_local;
+    for (int k = k0; k < k1; ++k) {
+      const int s0 = lo3 + k * 32;
+      const uint32_t in = below(s0, up3), lt = below(s0, n_new), kw = keptw[k];
+      uint32_t hole = in & lt & ~kw, moved = in & ~lt & kw;
+      while (hole) {
+        const int i = __ffs(hole) - 1;
+        hole &= hole - 1u;
+        if (hr < a.cap) hs[hr] = s0 + i;
+        ++hr;
+      }
+      while (moved) {
+        const int i = __ffs(moved) - 1;
+        moved &= moved - 1u;
+        if (mr < a.cap) mv[mr] = pos[s0 + i];
+        ++mr;
+      }
+    }
+    // entering positions of this CTA's bitmap words, ascending
+    const int nwc = w1 - w0;
+    const int cwe = (nwc + T - 1) / T;
+    const int e0 = min(nwc, tid * cwe), e1 = min(nwc, e0 + cwe);
+    int ec = 0;
+    for (int k = e0; k < e1; ++k) ec += __popc(entw[k]);
+    int te;
+    int er = E_before + inc_block_excl(ec, ws, &te);
+    for (int k = e0; k < e1; ++k) {
+      uint32_t e = entw[k];
+      while (e) {
+        const int i = __ffs(e) - 1;
+        e &= e - 1u;
+        if (er < a.cap) mv[er] = c.lo + (w0 + k) * 32 + i;
+        ++er;
+      }
+    }
+  }
+  cl.sync();   // every list entry written
+
+  // ---- 5. the copy
+  if (rank == 0 && tid == 0) {
+    c.n_rows[bgp] = n_new;
+    if (n_want > a.cap || M_tot != H_tot) latch_error(c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
+  }
+  const int n_hole = min(H_tot, a.cap);
+  const int n_mov = min(M_tot, a.cap);
   const int pad_end = min((n_new + kPage - 1) / kPage * kPage, a.cap);
   const int n_pad = pad_end - n_new;
-  const int n_sf = fresh ? a.c.n_sink : 0;
-  const int items = n_holes + n_pad + n_sf;
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    a.c.n_rows[bgp] = n_new;
-    if (n_want > a.cap || n_mov < n_holes) latch_error(a.c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactRows);
-  }
-  int32_t* pos = a.c.pos + (size_t)bgp * a.c.p_max;
-  uint32_t* hm = a.c.headmask + (size_t)bgp * a.c.p_max;
-  // 128-item chunks, strided over the blocks of this (b, KV head)
-  for (int i0 = blockIdx.x * kCopyRows; i0 < items; i0 += gridDim.x * kCopyRows) {
-    const int nr = min(kCopyRows, items - i0);
-    __syncthreads();   // src/dst of the previous chunk consumed
-    if (threadIdx.x < kCopyRows) {
-      const int i = i0 + threadIdx.x;
-      long long off = -1;
-      int slot = -1;
-      if (threadIdx.x < nr) {
-        int p = -1;
-        uint32_t m = 0u;
-        if (i < n_holes) {
-          slot = a.hole_slot[(size_t)bg * a.cap + i];
-          if (i < n_mov) {
-            p = a.mover_pos[(size_t)bg * a.cap + i];
-            m = head_bits_at<GM>(a.c, b, g, p - a.c.lo);
-          }
-        } else if (i < n_holes + n_pad) {
-          slot = n_new + (i - n_holes);
+  const int n_sf = valid ? 0 : c.n_sink;
+  const int items = n_hole + n_pad + n_sf;
+  const int per5 = (items + cs - 1) / cs;
+  const int i_lo = rank * per5, i_hi = min(items, i_lo + per5);
+  constexpr int kUnits = D / 8;                 // 16-byte units of one K (or V) row
+  constexpr int kRowUnits = 2 * kUnits;         // K then V
+  constexpr int kRowsPerPass = 32 / kRowUnits;  // rows one warp moves per pass
+  constexpr int kIn = 4;                        // passes in flight
+  const int sub = lane / kRowUnits;
+  const int u = lane % kRowUnits;
+  const bool isv = u >= kUnits;
+  const int cu = isv ? u - kUnits : u;
+  const uint4* from = isv ? c.vpool : c.kpool;
+  uint4* to = isv ? c.pv : c.pk;
+  const size_t base = (size_t)bgp * c.p_max * kUnits + cu;
+  const uint32_t all = c.G >= 32 ? 0xffffffffu : ((1u << c.G) - 1u);
+  for (int i0 = i_lo + warp * kIn * kRowsPerPass; i0 < i_hi; i0 += (T / 32) * kIn * kRowsPerPass) {
+    uint4 v[kIn];
+    int slot[kIn];
+#pragma unroll
+    for (int k = 0; k < kIn; ++k) {
+      const int i = i0 + k * kRowsPerPass + sub;
+      slot[k] = -1;
+      v[k] = make_uint4(0, 0, 0, 0);
+      if (i >= i_hi) continue;
+      int p = -1;
+      uint32_t m = 0u;
+      if (i < n_hole) {
+        slot[k] = hs[i];
+        if (i < n_mov) {
+          p = mv[i];
+          m = head_bits_at<GM>(c, b, g, p - c.lo);
+        }
+      } else if (i < n_hole + n_pad) {
+        slot[k] = n_new + (i - n_hole);
+      } else {
+        slot[k] = i - n_hole - n_pad;
+        p = slot[k];
+        m = all;
+      }
+      if (u == 0) {
+        pos[slot[k]] = p;
+        hm[slot[k]] = m;
+      }
+      if (p >= 0) {
+        const int pi = p / kPage;
+        int page = -1;
+        if (pi < c.max_pages) page = __ldg(c.pt + (size_t)bp * c.max_pages + pi);
+        if ((unsigned)page >= (unsigned)c.num_pages) {
+          if (u == 0) latch_error(c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
         } else {
-          slot = i - n_holes - n_pad;
-          p = slot;
-          m = a.c.G >= 32 ? 0xffffffffu : ((1u << a.c.G) - 1u);
-        }
-        pos[slot] = p;
-        hm[slot] = m;
-        if (p >= 0) {
-          const int pi = p / kPage;
-          int page = -1;
-          if (pi < a.c.max_pages) page = __ldg(a.c.pt + (size_t)bp * a.c.max_pages + pi);
-          if ((unsigned)page >= (unsigned)a.c.num_pages) latch_error(a.c.err, SFI_ERR_DEVICE_CHECK, kSiteCompactPage);
-          else off = ((long long)(page * a.c.Hkv + g) * kPage + p % kPage) * kUnits;
+          v[k] = __ldg(from + ((long long)(page * c.Hkv + g) * kPage + p % kPage) * kUnits + cu);
         }
       }
-      src[threadIdx.x] = off;
-      dst[threadIdx.x] = slot;
     }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int sub = lane / kRowUnits;
-    const int u = lane % kRowUnits;
-    const bool isv = u >= kUnits;
-    const int cu = isv ? u - kUnits : u;
-    const uint4* from = isv ? a.c.vpool : a.c.kpool;
-    uint4* to = isv ? a.c.pv : a.c.pk;
-    const size_t base = (size_t)bgp * a.c.p_max * kUnits + cu;
 #pragma unroll
-    for (int i0r = 0; i0r < kRowsPerWarp; i0r += kIn * kRowsPerPass) {
-      uint4 v[kIn];
-#pragma unroll
-      for (int k = 0; k < kIn; ++k) {
-        const int r = warp * kRowsPerWarp + i0r + k * kRowsPerPass + sub;
-        const long long off = (r < nr) ? src[r] : -1;
-        v[k] = off >= 0 ? __ldg(from + off + cu) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int k = 0; k < kIn; ++k) {
-        const int r = warp * kRowsPerWarp + i0r + k * kRowsPerPass + sub;
-        if (r < nr) to[base + (size_t)dst[r] * kUnits] = v[k];
-      }
-    }
+    for (int k = 0; k < kIn; ++k)
+      if (slot[k] >= 0) to[base + (size_t)slot[k] * kUnits] = v[k];
   }
-}
-
-// Blocks of inc_copy per (b, KV head): enough for a large move to reach the
-// copy bandwidth, few enough that a small one is not a launch of idle blocks.
-int inc_copy_blocks(int cap, int n_sink, int BH, int sms) {
-  const int chunks = (cap + kPage + n_sink + kCopyRows - 1) / kCopyRows;
-  return std::max(1, std::min(chunks, (4 * sms + BH - 1) / BH));
+  cl.sync();   // no CTA leaves while another may still read its shared memory
 }
 
 size_t compact_scratch_bytes(const sfi_shape& s, const sfi_params& p) {
@@ -589,9 +586,7 @@ size_t compact_scratch_bytes(const sfi_shape& s, const sfi_params& p) {
   const int nC = std::max(Lmax - p.n_recent - p.n_sink, 1);
   const int cap = packed_rows_capacity(s, p);
   return align_up((size_t)bh * compact_tiles(nC) * 2 * sizeof(int32_t), 256) +
-         align_up((size_t)bh * inc_slot_tiles(cap) * 2 * sizeof(int32_t), 256) +
-         align_up((size_t)bh * ((nC + 31) / 32) * sizeof(uint32_t), 256) +
-         2 * align_up((size_t)bh * cap * sizeof(int32_t), 256) + align_up((size_t)bh * 4 * sizeof(int32_t), 256);
+         2 * align_up((size_t)bh * cap * sizeof(int32_t), 256);
 }
 
 CompactScratch compact_scratch(void* base, const sfi_shape& s, const sfi_params& p) {
@@ -605,29 +600,34 @@ CompactScratch compact_scratch(void* base, const sfi_shape& s, const sfi_params&
   c.wcounts = reinterpret_cast<int32_t*>(w);
   c.wcount_bytes = align_up((size_t)bh * compact_tiles(nC) * 2 * sizeof(int32_t), 256);
   w += c.wcount_bytes;
-  c.scounts = reinterpret_cast<int32_t*>(w);
-  w += align_up((size_t)bh * inc_slot_tiles(cap) * 2 * sizeof(int32_t), 256);
-  c.oldbits = reinterpret_cast<uint32_t*>(w);
-  w += align_up((size_t)bh * ((nC + 31) / 32) * sizeof(uint32_t), 256);
   c.mover_pos = reinterpret_cast<int32_t*>(w);
   w += align_up((size_t)bh * cap * sizeof(int32_t), 256);
   c.hole_slot = reinterpret_cast<int32_t*>(w);
-  w += align_up((size_t)bh * cap * sizeof(int32_t), 256);
-  c.info = reinterpret_cast<int32_t*>(w);
   return c;
+}
+
+template <int D, int GM>
+sfi_status launch_inc_t(const IncArgs& a, int BH, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kIncCluster, BH);
+  cfg.blockDim = dim3(kIncThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kIncCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, inc_refresh_kernel<D, GM>, a) == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 template <int GM>
 sfi_status launch_inc(const IncArgs& a, int BH, cudaStream_t st) {
-  const dim3 sgrid(a.n_stiles, BH), wgrid(a.c.n_tiles, BH);
-  launch_k(inc_old_kernel<GM>, sgrid, dim3(kCThreads), 0, st, a);
-  launch_k(inc_count_kernel<GM>, wgrid, dim3(kCThreads), 0, st, a);
-  launch_k(inc_slots_kernel, sgrid, dim3(kCThreads), 0, st, a);
-  launch_k(inc_list_kernel<GM>, dim3(a.c.n_tiles + a.n_stiles, BH), dim3(kCThreads), 0, st, a);
-  const dim3 cgrid(inc_copy_blocks(a.cap, a.c.n_sink, BH, num_sms()), BH);
-  if (a.c.D == 128) launch_k(inc_copy_kernel<128, GM>, cgrid, dim3(kCopyWarps * 32), 0, st, a);
-  else launch_k(inc_copy_kernel<64, GM>, cgrid, dim3(kCopyWarps * 32), 0, st, a);
-  return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+  return a.c.D == 128 ? launch_inc_t<128, GM>(a, BH, st) : launch_inc_t<64, GM>(a, BH, st);
 }
 
 template <int GM>
@@ -688,17 +688,16 @@ sfi_status run_compact_inc(const sfi_shape& s, const sfi_params& p, const sfi_pa
                            int L_slow, bool fresh, cudaStream_t st, const RowMap& rows) {
   const int nb = rows.count(s.B);
   if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
+  if (fresh)   // sinks and the union in ascending order: the full compaction
+    return run_compact_bits(s, p, kv, bits, ld_b, pk, cs, L_slow, st, rows);
   IncArgs a{};
   a.c = compact_args(s, p, kv, bits, ld_b, pk, L_slow);
   a.c.rows = rows;
   a.cap = cs.cap;
   if (a.cap % kPage != 0 || pk.p_max < a.cap) return SFI_ERR_SHAPE;
-  a.n_stiles = inc_slot_tiles(a.cap);
-  if (fresh)   // same layout as the full compaction, which copies faster
-    return run_compact_bits(s, p, kv, bits, ld_b, pk, cs, L_slow, st, rows);
-  a.fresh = 0;
-  a.wcounts = cs.wcounts; a.scounts = cs.scounts; a.oldbits = cs.oldbits;
-  a.mover_pos = cs.mover_pos; a.hole_slot = cs.hole_slot; a.info = cs.info;
+  if (a.c.nw > kIncCluster * kIncMaxWords || a.cap > kIncCluster * kIncMaxSlotWords * 32) return SFI_ERR_UNSUPPORTED;
+  a.mover_pos = cs.mover_pos;
+  a.hole_slot = cs.hole_slot;
   const int BH = nb * s.Hkv;
   if (a.c.G <= 1) return launch_inc<1>(a, BH, st);
   if (a.c.G <= 2) return launch_inc<2>(a, BH, st);

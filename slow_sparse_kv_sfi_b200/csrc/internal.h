@@ -152,16 +152,12 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
                     int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st);
 int topk_max_n();
 // Compaction scratch (inside the workspace): per-tile counts of the full
-// compaction, and the incremental compaction's counts, previous-position
-// bitmap (zero between calls), mover and hole lists.
+// compaction, and the incremental refresh's mover and hole lists.
 struct CompactScratch {
   int32_t* wcounts = nullptr;   // [BH][n_tiles][2]
   size_t wcount_bytes = 0;
-  int32_t* scounts = nullptr;   // [BH][slot tiles][2]
-  uint32_t* oldbits = nullptr;  // [BH][nw]
   int32_t* mover_pos = nullptr; // [BH][cap]
   int32_t* hole_slot = nullptr; // [BH][cap]
-  int32_t* info = nullptr;      // [BH][4]
   int cap = 0;                  // packed_rows_capacity
 };
 size_t compact_scratch_bytes(const sfi_shape& s, const sfi_params& p);
