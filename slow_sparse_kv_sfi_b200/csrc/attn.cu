@@ -65,6 +65,10 @@ struct AttnArgs {
   int rec_lo;           // L - n_recent
   int* err;
   unsigned long long wait_ns;   // limit of every pipeline wait
+  // 1: let the dependent launches be scheduled only once this CTA has no
+  // work item left (a persistent grid that signals at its start has the next
+  // kernel's CTAs take every SM it frees, ahead of other streams' kernels)
+  int late_trigger;
   // the step's token, appended at L - 1 by the item holding the last tile
   // (k_new == nullptr: already in the cache)
   const __nv_bfloat16* k_new;
@@ -214,7 +218,8 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     fence_barrier_init();
   }
   __syncthreads();
-  grid_dep_enter();
+  grid_dep_wait();
+  if (!a.late_trigger) grid_dep_launch();
 
   // ------------------------------------------------------------ producer warp
   if (warp == kConsumerWarps) {
@@ -402,6 +407,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
       }
       if (item >= a.n_items) break;
     }
+    if (a.late_trigger) grid_dep_launch();   // no item left for this CTA
     if (!ok && lane == 0) {
       // Drain: wait (bounded) for the copies of stages still in flight so no
       // TMA write lands after this CTA has left the SM.
@@ -434,11 +440,15 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
   for (;;) {
     if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer, a.wait_ns)) {
       *abort_flag = 1;
+      if (a.late_trigger) grid_dep_launch();
       break;
     }
     const StageMeta& m = smeta[slot];
     const int item = m.item;
-    if (item < 0) break;
+    if (item < 0) {
+      if (a.late_trigger) grid_dep_launch();
+      break;
+    }
     const int flags = m.flags;
     if (flags & 1) {
       // first stage of an item: the group's queries (B operand of S^T) and a fresh state
@@ -1033,7 +1043,7 @@ void set_token(AttnArgs& a, const sfi_shape& s, const sfi_paged_kv& kv, const St
 sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, const sfi_bf16* q,
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
-                          const StepToken* tok, AttnMapCache* cache, const RowMap& rmap) {
+                          const StepToken* tok, AttnMapCache* cache, const RowMap& rmap, bool late_trigger) {
   const int G = s.Hq / s.Hkv;
   if (rmap.count(s.B) < 1 || rmap.count(s.B) > s.B) return SFI_ERR_SHAPE;
   Maps maps;
@@ -1059,6 +1069,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   a.scale_log2 = kLog2e * a.scale;
   a.err = kv.err;
   a.wait_ns = wait_limit_ns();
+  a.late_trigger = late_trigger ? 1 : 0;
   set_token(a, s, kv, tok);
   const bool extras = ex && (ex->logits || ex->probs || ex->lse_cand);
   float* zbuf = nullptr;

@@ -4,17 +4,25 @@
 // Pipeline Asynchrone; [ZH] "2.3" 异步流水线).
 //
 // On a slow step the main stream runs dense attention for layer i (also
-// writing the logits and the candidate log-sum-exp into one of two ping-pong
+// writing the logits and the candidate log-sum-exp into one of a ring of
 // buffers) and moves on to layer i+1; the Selector and the compaction of
 // layer i run on the context's side stream after an event.  The next step of
 // layer i waits for that refresh before it touches the layer's cache or
 // packed buffer.  A logits buffer is rewritten only after the side stream has
-// finished reading it.
+// finished reading it.  The side stream has the highest priority, and the
+// dense launches let the next kernel be scheduled only when their CTAs run
+// out of work, so the Selector kernels take the SMs freed in the attention's
+// tail instead of queueing behind the next layer's whole grid.
 #include <algorithm>
 #include <vector>
 
 #include "common.cuh"
 #include "internal.h"
+
+// Logits buffers the slow steps of consecutive layers rotate through: layer
+// i's dense launch waits until the Selector of layer i - kLogitBufs has read
+// its buffer, so a Selector may lag that many layers behind the attention.
+constexpr int kLogitBufs = 4;
 
 struct sfi_ctx {
   sfi_shape s;
@@ -26,7 +34,7 @@ struct sfi_ctx {
   cudaStream_t side = nullptr;
   std::vector<cudaEvent_t> ev_dense, ev_sel;
   std::vector<uint8_t> pending;
-  cudaEvent_t ev_buf_free[2] = {nullptr, nullptr};
+  cudaEvent_t ev_buf_free[kLogitBufs] = {};
   int cur_step = -1;
   // per-sequence trigger state: the last slow step of every sequence and the
   // decision of the current step (layer 0 decides, the other layers reuse it)
@@ -46,8 +54,8 @@ struct sfi_ctx {
   size_t ws_bytes = 0;
   float* part = nullptr;
   size_t part_bytes = 0;
-  float* logits[2] = {nullptr, nullptr};
-  float* lse_cand[2] = {nullptr, nullptr};
+  float* logits[kLogitBufs] = {};
+  float* lse_cand[kLogitBufs] = {};
   int64_t ld = 0;
   void* stats = nullptr;
   float* scores = nullptr;
@@ -96,10 +104,10 @@ CtxLayout ctx_layout(const sfi_shape& s, const sfi_params& p, int n_layers) {
   off += c.part_bytes;
   c.logit_off = off;
   c.logit_bytes = align_up((size_t)s.B * sw.Hq * Lmax * sizeof(float), 256);
-  off += 2 * c.logit_bytes;
+  off += kLogitBufs * c.logit_bytes;
   c.lsec_off = off;
   c.lsec_bytes = align_up((size_t)s.B * sw.Hq * sizeof(float), 256);
-  off += 2 * c.lsec_bytes;
+  off += kLogitBufs * c.lsec_bytes;
   c.stat_off = off;
   c.stat_bytes = w.stat_bytes;
   off += c.stat_bytes;
@@ -232,7 +240,7 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
       if (ss[i] >= 0 && ss[i] > step - W) wmask |= 1u << i;
   }
   if (c->n_slow > 0) {
-    const int buf = layer & 1;
+    const int buf = layer % kLogitBufs;
     SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
     sfi_dense_extras ex{};
     ex.logits = c->logits[buf];
@@ -245,14 +253,14 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
       timing_events(c, 1, layer, &b, &e);
       if (W == 1) {
         SFI_TRY(run_dense_attn(s, *kv, L, q, out, &ex, reinterpret_cast<int*>(c->ws), c->part, c->part_bytes,
-                               main, b, e, &tok, &c->maps[layer], slow_map));
+                               main, b, e, &tok, &c->maps[layer], slow_map, c->overlap != 0));
       } else {
         // one pass over the cache for the group's last W queries (Hkv * W * G
         // heads); the outputs of the step's own queries are copied out
         const sfi_shape sw = window_shape(s, p);
         SFI_TRY(run_dense_attn(sw, *kv, L, reinterpret_cast<const sfi_bf16*>(ring), c->wout, &ex,
                                reinterpret_cast<int*>(c->ws), c->part, c->part_bytes, main, b, e, &tok,
-                               &c->maps[layer], slow_map));
+                               &c->maps[layer], slow_map, c->overlap != 0));
         const size_t orow = (size_t)G * s.D * sizeof(float);
         SFI_TRY(cu(cudaMemcpy2DAsync(out, orow, reinterpret_cast<const char*>(c->wout) + (step % W) * orow, W * orow,
                                      orow, (size_t)s.B * s.Hkv, cudaMemcpyDeviceToDevice, main)));
@@ -317,7 +325,11 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->n_layers = n_layers;
   c->overlap = overlap ? 1 : 0;
   cudaGetDevice(&c->device);
-  bool ok = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking) == cudaSuccess;
+  // the side stream gets the highest priority: its Selector kernels take the
+  // SMs that the main stream's attention frees in its tail
+  int least = 0, greatest = 0;
+  bool ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
+            cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, greatest) == cudaSuccess;
   c->ev_dense.resize(n_layers, nullptr);
   c->ev_sel.resize(n_layers, nullptr);
   c->pending.assign(n_layers, 0);
@@ -330,7 +342,7 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   for (int i = 0; i < n_layers && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
-  for (int i = 0; i < 2 && ok; ++i)
+  for (int i = 0; i < kLogitBufs && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_buf_free[i], cudaEventDisableTiming) == cudaSuccess;
   if (!ok) {
     sfi_ctx_destroy(c);
@@ -372,7 +384,7 @@ sfi_status sfi_ctx_set_workspace(sfi_ctx* c, void* ws, size_t bytes) {
   c->part = reinterpret_cast<float*>(w + l.part_off);
   c->part_bytes = l.part_bytes;
   c->ld = (int64_t)c->s.max_pages * kPage;
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < kLogitBufs; ++i) {
     c->logits[i] = reinterpret_cast<float*>(w + l.logit_off + i * l.logit_bytes);
     c->lse_cand[i] = reinterpret_cast<float*>(w + l.lsec_off + i * l.lsec_bytes);
   }

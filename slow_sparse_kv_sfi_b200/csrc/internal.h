@@ -126,7 +126,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
                           float* out, const sfi_dense_extras* ex, int* ctr, float* part,
                           size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin, cudaEvent_t ev_end,
                           const StepToken* tok = nullptr, AttnMapCache* maps = nullptr,
-                          const RowMap& rows = RowMap());
+                          const RowMap& rows = RowMap(), bool late_trigger = false);
 sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                          const sfi_bf16* q, const sfi_packed& pk, float* out, float* lse, int* ctr,
                          float* part, size_t part_bytes, cudaStream_t st, cudaEvent_t ev_begin,
