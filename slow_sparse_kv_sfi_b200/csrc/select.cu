@@ -347,17 +347,17 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
         dv[h] = d;
       }
     }
-    int owner = 0, bd = dv[0];
-    float bx = xv[0], bl = l1[0];
+    int owner = 0, best_d = dv[0];
+    float best_x = xv[0], best_l1 = l1[0];
 #pragma unroll
     for (int h = 1; h < GM; ++h) {
       if (h < G) {
-        const bool wins = dv[h] == bd ? (ev_counts && xv[h] > bx) : (l1[h] > bl);
+        const bool wins = dv[h] == best_d ? (ev_counts && xv[h] > best_x) : (l1[h] > best_l1);
         if (wins) {
           owner = h;
-          bd = dv[h];
-          bx = xv[h];
-          bl = l1[h];
+          best_d = dv[h];
+          best_x = xv[h];
+          best_l1 = l1[h];
         }
       }
     }
