@@ -261,14 +261,16 @@ int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
 // rows.  A fresh buffer (no previous rows) gets sinks and U in ascending
 // order: the full compaction above.
 //
-// One launch: a cluster of kIncCluster CTAs per (sequence, KV head).  The
-// previous rows' positions are marked in a bitmap over the candidates that
-// lives in the CTAs' shared memory, each CTA holding a slice of words (remote
-// bits land through distributed shared memory), so no global state has to
-// be cleared between calls.  The phases, each ended by a cluster barrier:
+// One launch: a cluster of kIncCluster CTAs per (sequence, KV head).  Each CTA
+// marks the positions of its share of the previous rows in a bitmap over the
+// candidates in its own shared memory (local atomics), so no global state
+// has to be cleared between calls.  The phases, each ended by a cluster
+// barrier:
 //   1. previous rows (split over the CTAs): head mask rewritten (0: the row
-//      leaves), position marked in the bitmap;
-//   2. each CTA's bitmap words: |U| and the entering positions U & ~old;
+//      leaves), position marked in the CTA's bitmap;
+//   2. each CTA's slice of bitmap words: the previous positions (the OR of
+//      every CTA's bitmap, read through distributed shared memory), |U| and
+//      the entering positions U & ~old;
 //   3. each CTA's slots of [n_sink, max(n_old, n_new)): kept, hole, moved
 //      (kept rows at or past n_new);
 //   4. the mover and hole lists, in the order of the rule (cluster-wide
@@ -277,7 +279,7 @@ int compact_tiles(int nC) { return ((nC + 31) / 32 + kCWords - 1) / kCWords; }
 //      the next multiple of 16, n_rows.
 constexpr int kIncThreads = 512;
 constexpr int kIncCluster = 8;
-constexpr int kIncMaxWords = 1024;       // candidate bitmap words per CTA (|C| <= 262144)
+constexpr int kIncMaxWords = 8192;       // candidate bitmap words (|C| <= 262144)
 constexpr int kIncMaxSlotWords = 2048;   // slot words per CTA (packed capacity <= 524288)
 
 struct IncArgs {
@@ -345,8 +347,8 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
   const int bp = c.rows.phys(b);                // the sequence
   const int bgp = bp * c.Hkv + g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ uint32_t oldw[kIncMaxWords];       // this CTA's slice of the previous positions
-  __shared__ uint32_t entw[kIncMaxWords];       // its entering positions
+  __shared__ uint32_t oldw[kIncMaxWords];       // positions of this CTA's share of the previous rows
+  __shared__ uint32_t entw[kIncMaxWords / kIncCluster];   // entering positions of its word slice
   __shared__ uint32_t keptw[kIncMaxSlotWords];  // its slots holding a kept row
   __shared__ int pub[4];                        // published: |U|, entering, holes, moved
   __shared__ int ws[33];
@@ -356,13 +358,13 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
   const int nw = c.nw;
   const int Wc = (nw + cs - 1) / cs;
   const int w0 = min(nw, rank * Wc), w1 = min(nw, w0 + Wc);
-  for (int i = tid; i < Wc; i += T) oldw[i] = 0u;
+  for (int i = tid; i < nw; i += T) oldw[i] = 0u;
   // previous rows; a count outside [n_sink, cap] means no usable buffer: the
   // sinks are written again and every selected row enters
   const int n_raw = c.n_rows[bgp];
   const bool valid = n_raw >= c.n_sink && n_raw <= a.cap;
   const int n_old = valid ? n_raw : c.n_sink;
-  cl.sync();   // every slice cleared before any remote bit lands
+  __syncthreads();
 
   // ---- 1. previous rows
   {
@@ -374,8 +376,7 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
       uint32_t m = 0u;
       if ((unsigned)ci < (unsigned)c.nC) {
         m = head_bits_at<GM>(c, b, g, ci);
-        const int wd = ci >> 5, owner = wd / Wc;
-        atomicOr(cl.map_shared_rank(oldw, owner) + (wd - owner * Wc), 1u << (ci & 31));
+        atomicOr(&oldw[ci >> 5], 1u << (ci & 31));
       }
       hm[s] = m;   // 0: the row leaves
     }
@@ -388,7 +389,9 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
     for (int w = w0 + tid; w < w1; w += T) {
       uint32_t hw[GM];
       const uint32_t u = union_word<GM>(c, b, g, w, hw);
-      const uint32_t e = u & ~oldw[w - w0];
+      uint32_t old = 0u;
+      for (int r = 0; r < cs; ++r) old |= cl.map_shared_rank(oldw, r)[w];
+      const uint32_t e = u & ~old;
       entw[w - w0] = e;
       cu += __popc(u);
       ce += __popc(e);
@@ -695,7 +698,7 @@ sfi_status run_compact_inc(const sfi_shape& s, const sfi_params& p, const sfi_pa
   a.c.rows = rows;
   a.cap = cs.cap;
   if (a.cap % kPage != 0 || pk.p_max < a.cap) return SFI_ERR_SHAPE;
-  if (a.c.nw > kIncCluster * kIncMaxWords || a.cap > kIncCluster * kIncMaxSlotWords * 32) return SFI_ERR_UNSUPPORTED;
+  if (a.c.nw > kIncMaxWords || a.cap > kIncCluster * kIncMaxSlotWords * 32) return SFI_ERR_UNSUPPORTED;
   a.mover_pos = cs.mover_pos;
   a.hole_slot = cs.hole_slot;
   const int BH = nb * s.Hkv;

@@ -92,13 +92,20 @@ __device__ __forceinline__ const float* norm_row(const float* norms, int64_t nor
 }
 
 // part[bgl][chunk][0] = sum of key norms over the chunk of C (bgl: logical
-// (row, kv head) of the launch)
-__global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC, const float* __restrict__ norms,
+// (row, kv head) of the launch); the CTAs of row 0 also write the position
+// factor pi[c] = ln(1 + L - (lo + c)) of their chunk, shared by every row
+__global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int L, int lo, int nC,
+                                                                  const float* __restrict__ norms,
                                                                   int64_t norm_ld, double* part, int nch, int Hkv,
+                                                                  double* __restrict__ pitab,
                                                                   const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   __shared__ double red[32];
   const int bg = blockIdx.y;
+  if (bg == 0) {
+    const int c1 = min(nC, (int)(blockIdx.x + 1) * kStatChunk);
+    for (int c = blockIdx.x * kStatChunk + threadIdx.x; c < c1; c += blockDim.x) pitab[c] = pi_of(L, lo + c);
+  }
   const float* n = norm_row(norms, norm_ld, rows, Hkv, bg) + lo;
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double sacc = 0.0;
@@ -112,6 +119,7 @@ __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int lo, int nC
 __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
                                                                    const float* __restrict__ norms,
                                                                    int64_t norm_ld, double* part, int nch, int Hkv,
+                                                                   const double* __restrict__ pitab,
                                                                    double* __restrict__ kp, int64_t kp_ld,
                                                                    const __grid_constant__ RowMap rows) {
   grid_dep_enter();
@@ -126,7 +134,7 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
   double* kpr = kp + (size_t)bg * kp_ld;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
     const int j = lo + c;
-    const double v = kappa_of(nbar, n[j]) * pi_of(L, j);
+    const double v = kappa_of(nbar, n[j]) * pitab[c];
     kpr[c] = v;
     z += v;
   }
@@ -410,13 +418,15 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   const int nch = stat_chunks(nC);
   const int64_t norm_ld = (int64_t)s.max_pages * kPage;
   dim3 sgrid(nch, nb * s.Hkv);
-  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, lo, nC, kv.key_norms, norm_ld, part, nch,
-           s.Hkv, rows);
-  // kappa * pi of every candidate follows the partial sums in the statistics area
-  double* kp = part + (size_t)nb * s.Hkv * nch * 2;
+  // the statistics area: partial sums, then the position factors, then
+  // kappa * pi of every candidate of every row
   const int64_t kp_ld = (nC + 1) / 2 * 2;
+  double* pitab = part + (size_t)nb * s.Hkv * nch * 2;
+  double* kp = pitab + kp_ld;
+  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
+           s.Hkv, pitab, rows);
   launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
-           s.Hkv, kp, kp_ld, rows);
+           s.Hkv, pitab, kp, kp_ld, rows);
   if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;

@@ -30,7 +30,7 @@ def pytest_terminal_summary(terminalreporter):
     logit error seen, relative to sum |q k| / sqrt(D)."""
     import helpers
     rec = helpers.SELECTION_RECORD
-    if not rec and not helpers.LOGIT_RECORD:
+    if not rec and not helpers.LOGIT_RECORD and not helpers.LSE_RECORD:
         return
     tr = terminalreporter
     tr.section("selection parity")
@@ -53,3 +53,5 @@ def pytest_terminal_summary(terminalreporter):
     if helpers.LOGIT_RECORD:
         tr.write_line(f"logit error: at most {max(helpers.LOGIT_RECORD):.3e} x sum|q k|/sqrt(D) "
                       f"(bound {helpers.C_Z:.3e})")
+    if helpers.LSE_RECORD:
+        tr.write_line(f"candidate lse error: at most {max(helpers.LSE_RECORD):.3f} of its bound")

@@ -57,13 +57,19 @@ def assert_attn_close(o, ref, what=""):
 
 # Error budget of the CUDA path's Selector inputs (see selection_bounds).
 # Logits from the dense kernel: |z_gpu - z| <= C_Z * sum_d |q_d k_d| / sqrt(D)
-# (bf16 products accumulated in fp32 on the tensor cores), checked element by
-# element in the dense-attention parity test; the candidate lse adds the
-# largest of those bounds over C and LSE_SUM_ERR for its fp32 sum.
-C_Z = 2.0 ** -18
-LSE_SUM_ERR = 1e-5
-# The prior from fp32-stored norms: relative error of r.
-EPS_R_FP32_NORMS = 2.0 ** -21
+# (bf16 products accumulated in fp32 on the tensor cores; the largest ratio
+# measured on the dense parity cases is 1.8e-7, a fifth of C_Z), checked
+# element by element in the dense-attention parity test.  The candidate lse
+# moves by the softmax-weighted mean of the logit errors, sum_j f~_j bound_j,
+# plus LSE_SUM_ERR for its fp32 sum; checked there too.
+C_Z = 2.0 ** -20
+LSE_SUM_ERR = 2e-6
+# The prior from fp32-stored norms: the normaliser sum_C kappa pi is off by at
+# most EPS_Z (relative, common to every candidate, so it never changes which
+# of two priors is larger); kappa_j = min(1, nbar / n_j) by at most EPS_KAPPA
+# where n_j is at or above the mean (elsewhere kappa = 1 exactly).
+EPS_Z = 2.0 ** -22
+EPS_KAPPA = 2.0 ** -22
 # Undecided candidates allowed per head, as a share of K (and at least this many).
 MAX_UNDECIDED_SHARE = 0.01
 MIN_UNDECIDED_ALLOWED = 2
@@ -74,6 +80,8 @@ MIN_OVERLAP = 0.999
 SELECTION_RECORD = []
 # largest observed |z_gpu - z| / (sum_d |q_d k_d| / sqrt(D)) per dense-attention check
 LOGIT_RECORD = []
+# largest observed candidate-lse error as a share of its bound
+LSE_RECORD = []
 _CURRENT_TEST = {"name": ""}
 
 
@@ -85,13 +93,20 @@ def logit_error_bound(q: np.ndarray, K: np.ndarray) -> np.ndarray:
     return C_Z * (q @ K.T) / np.sqrt(q.shape[-1])
 
 
-def evidence_error_from_logits(zb: np.ndarray, lo: int, hi: int) -> np.ndarray:
-    """[G, |C|] bound of the error of x = z - lse_C, given the logit bound zb."""
+def lse_error_bound(zb: np.ndarray, ft: np.ndarray) -> np.ndarray:
+    """[G] bound of the error of lse over C: the f~-weighted mean of the logit
+    bounds zb [G, |C|] (first order in the errors), plus the fp32 sum's."""
+    return np.sum(ft * zb, axis=1) + LSE_SUM_ERR
+
+
+def evidence_error_from_logits(zb: np.ndarray, ft: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """[G, |C|] bound of the error of x = z - lse_C, given the logit bound zb
+    [G, L] and the evidence ft [G, |C|] the lse is taken over."""
     zc = zb[:, lo:hi]
-    return zc + zc.max(axis=1, keepdims=True) + LSE_SUM_ERR
+    return zc + lse_error_bound(zc, ft)[:, None]
 
 
-def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps_r, x=None):
+def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps_r, x=None, eps_r_common=0.0):
     """Intervals of l'' that the CUDA Selector can produce for one KV group.
 
     The kernel computes x = z - lse_C in fp32 (error eps_x, absolute: the
@@ -104,8 +119,10 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     heads that can own a position, and finally [lo, hi] of l'' per (head,
     candidate), widened by the fp32 rounding of the kernel's l''.
 
-    ft [G, n], r [n] (oracle float64), eps_x scalar or [G, n], eps_r scalar,
-    x: the oracle's log-evidence (default ln ft)."""
+    ft [G, n], r [n] (oracle float64), eps_x scalar or [G, n], eps_r scalar
+    or [n]: independent relative error of each r_j, eps_r_common: relative
+    error common to every r_j (it scales both sides of a comparison between
+    candidates), x: the oracle's log-evidence (default ln ft)."""
     ft = np.asarray(ft, np.float64)
     r = np.asarray(r, np.float64)
     G, n = ft.shape
@@ -120,7 +137,9 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     x = np.asarray(x, np.float64)
     tiny = 2.0 ** -126 * 4                      # the kernel's exp flushes below fp32's normal range
     ev_err = (1.0 - lam) * (ft * np.expm1(eps_x + 2.0 ** -21) + tiny)
-    ds = ev_err + lam * r[None, :] * eps_r + 2.0 ** -24 * s
+    eps_r = np.broadcast_to(np.asarray(eps_r, np.float64), (n,))
+    ds = ev_err + lam * (r * eps_r)[None, :] + 2.0 ** -24 * s      # independent part
+    ds_all = ds + lam * r[None, :] * eps_r_common
     by_x = lam <= 0.0
     if by_x:
         key_err = eps_x + 2.0 ** -24 * np.abs(x)
@@ -129,7 +148,7 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
         if by_x:
             return x[:, a] - x[:, b], key_err[:, a] + key_err[:, b]
         d = lam * (r[None, a] - r[None, b]) + (1.0 - lam) * (ft[:, a] - ft[:, b])
-        return d, ds[:, a] + ds[:, b]
+        return d, ds[:, a] + ds[:, b] + lam * np.abs(r[None, a] - r[None, b]) * eps_r_common
 
     INF = w + 1
     d_lo = np.full((G, n), INF, np.int64)      # nearest possible dominator
@@ -153,7 +172,7 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     pen_lo = weight[np.where(d_hi > w, 0, d_hi)]
     ell = det["ell"]
     with np.errstate(divide="ignore", invalid="ignore"):
-        dl_rel = np.where(s > 0, ds / s, np.inf)
+        dl_rel = np.where(s > 0, ds_all / s, np.inf)
     dell = dl_rel + 2.0 ** -22 * np.abs(ell) + 1e-7
     if by_x:
         dell = key_err * ft / (ft + O.LOG_EPS) + 2.0 ** -22 * np.abs(ell) + 1e-7
@@ -294,11 +313,16 @@ def decode_selection_bounds(q, Kc, f, L, cfg, f_window=None, q_window=None):
     logits come from the dense kernel (error bound logit_error_bound), the
     prior from fp32 norms.  q [G, D] the step's queries, Kc [L, D] the
     cache; q_window: the window's queries (with f_window)."""
-    ft, r, lam_eff, lo, hi = oracle_group_parts(f, O.key_norms(Kc), L, cfg, f_window)
+    norms = O.key_norms(Kc)
+    ft, r, lam_eff, lo, hi = oracle_group_parts(f, norms, L, cfg, f_window)
+    nc = norms[lo:hi]
+    eps_r = np.where(nc >= nc.mean() * (1.0 - 2.0 ** -21), EPS_KAPPA, 0.0)
     qs = [q] if q_window is None else q_window
-    ex = np.max([evidence_error_from_logits(logit_error_bound(qq, Kc), lo, hi) for qq in qs], axis=0)
+    fs = [f] if f_window is None else f_window
+    ex = np.max([evidence_error_from_logits(logit_error_bound(qq, Kc), O.evidence(ff, lo, hi), lo, hi)
+                 for qq, ff in zip(qs, fs)], axis=0)
     return selection_bounds(ft, r, lam_eff, cfg.alpha_soft, cfg.alpha_cross, cfg.nms_window, ex,
-                            EPS_R_FP32_NORMS), lo
+                            eps_r, eps_r_common=EPS_Z), lo
 
 
 def packed_sets(pos: np.ndarray, hm: np.ndarray, n_rows: int, n_sink: int, G: int):

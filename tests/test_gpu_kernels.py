@@ -83,7 +83,9 @@ def test_dense_attention_parity(B, Hq, Hkv, D, L):
             H.LOGIT_RECORD.append(float((dz / zb).max()) * H.C_Z)
             assert np.all(dz <= zb), f"logit error beyond its bound: {(dz / zb).max():.3f} x the bound"
             dl = np.abs(lsec[b, sl].cpu().numpy().astype(np.float64) - lc)
-            assert np.all(dl <= zb[:, lo:hi].max(axis=1) + H.LSE_SUM_ERR), f"candidate lse error {dl.max():.3e}"
+            lb = H.lse_error_bound(zb[:, lo:hi], O.evidence(f, lo, hi))
+            H.LSE_RECORD.append(float((dl / lb).max()))
+            assert np.all(dl <= lb), f"candidate lse error {dl.max():.3e} beyond its bound"
 
 
 def test_dense_attention_masks_garbage_beyond_L():
