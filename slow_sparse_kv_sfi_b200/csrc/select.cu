@@ -14,13 +14,15 @@
 //
 // Comparisons that decide an integer follow real arithmetic, not the last bit
 // of a rounded sum: l_i vs l_j has the sign of s_i - s_j (ln is monotone),
-// with s = (1 - lambda) f~ + lambda r formed in fp64 from an fp64 prior and
-// rounded once to fp32 (where the prior dominates, neighbouring candidates
-// differ in r by ~1e-6 relative, far above that rounding); two heads with the
-// same soft-NMS penalty compare by their evidence, since r is common to the
-// group (their s agree to every digit where the prior dominates).  The
-// evidence is compared through its logarithm x = z - lse_C, which does not
-// underflow.  With lambda = 0 the dominance is decided on x as well.
+// with s = (1 - lambda) f~ + lambda r formed by one fp32 FMA from lambda r
+// (fp64 prior, rounded to fp32): within 1 ulp of s, where the prior dominates
+// neighbouring candidates differ in r by ~1e-6 relative, far above that; two
+// heads with the same soft-NMS penalty compare by their evidence, since r is
+// common to the group (their s agree to every digit where the prior
+// dominates).  The evidence is compared through its logarithm x = z - lse_C,
+// which does not underflow.  With lambda = 0 the dominance is decided on x
+// as well.  No decision rests on the last bit of a logarithm, so l = ln(s)
+// uses the hardware's base-2 approximation.
 //
 // Kernels: stats_norm / stats_prior (per (b, kv head) and chunk of C: fp64
 // partial sums of the norms and of kappa pi; every consumer reduces the
@@ -144,7 +146,8 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
 
 struct ScoreArgs {
   int L, lo, nC, Hq, Hkv, G, w, tile;
-  double lam, one_minus_lam;    // lambda_eff and 1 - lambda_eff
+  double lam;                   // lambda_eff
+  float one_minus_lam;          // 1 - lambda_eff
   float alpha_soft, alpha_cross;
   const float* logits;
   int64_t ld;
@@ -190,6 +193,9 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   const double* kpr = a.kp + (size_t)bg * a.kp_ld;
   const bool by_x = a.lam <= 0.0;          // lambda = 0: s = f~, decided on x
   const double lam_r = a.lam * inv_z;      // lambda / Z
+  __shared__ float wt[64];                 // soft-NMS weight of a nearest dominator at distance d
+  for (int d = threadIdx.x; d <= a.w && d < 64; d += blockDim.x)
+    wt[d] = d > 0 ? 1.f - (float)(d - 1) / (float)a.w : 0.f;
   // logits rows of the group: nq query slots of G heads (nq = 1: row b * Hq + g * G + h)
   const size_t row0 = ((size_t)b * a.Hkv + g) * (size_t)(a.nq * G);
   const float* z0 = a.logits + row0 * a.ld + a.lo;
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
           if (h < G) key[h * W + k] = nan;
         continue;
       }
-      const double r = kpr[c] * lam_r;   // lambda r_j
+      const float r = (float)(kpr[c] * lam_r);   // lambda r_j
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
             }
           const float x = m + logf(acc * a.inv_nq);
           const float ft = fast_exp2(x * kLog2e);
-          key[h * W + k] = by_x ? x : (float)fma(a.one_minus_lam, (double)ft, r);
+          key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
           if (tile_k) xo[h * a.tile + k - a.w] = x;
         }
       }
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
       if (k >= W) continue;
       const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (in[u]) {
-        const double r = kv[u] * lam_r;   // lambda r_j
+        const float r = (float)(kv[u] * lam_r);   // lambda r_j
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
           if (h < G) {
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
             // error ~1e-7, below the error of the logits themselves)
             const float x = zv[u][h] - lsec[h];
             const float ft = fast_exp2(x * kLog2e);
-            key[h * W + k] = by_x ? x : (float)fma(a.one_minus_lam, (double)ft, r);
+            key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
             if (tile_k) xo[h * a.tile + k - a.w] = x;
           }
         }
@@ -336,8 +342,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   // Phase 3: l' = ln(s + 1e-30) - alpha_soft * weight(d); the owner scans the
   // heads in order (ties to the lowest): equal distances compare by x (never
   // when lambda = 1: the evidence has no weight), others by l'.
-  const float inv_w = 1.f / (float)a.w;
-  const bool ev_counts = a.one_minus_lam > 0.0;
+  const bool ev_counts = a.one_minus_lam > 0.f;
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
     float l1[GM], xv[GM];
     int dv[GM];
@@ -348,10 +353,9 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
       dv[h] = 0;
       if (h < G) {
         const int d = dom[h * a.tile + k];
-        const float pen = d > 0 ? 1.f - (float)(d - 1) * inv_w : 0.f;
         xv[h] = xo[h * a.tile + k];
         const float sv = by_x ? fast_exp2(xv[h] * kLog2e) : key[h * W + a.w + k];
-        l1[h] = logf(sv + 1e-30f) - a.alpha_soft * pen;
+        l1[h] = fast_log2(sv + 1e-30f) * kLn2 - a.alpha_soft * wt[d];
         dv[h] = d;
       }
     }
@@ -434,7 +438,8 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.tile = score_tile(G);
   const double lam = std::min(std::max((double)p.lambda, 0.0), (double)p.lambda_clip);
   a.lam = lam;
-  a.one_minus_lam = 1.0 - lam;
+  a.one_minus_lam = (float)(1.0 - lam);
+  if (a.w > 63) return SFI_ERR_UNSUPPORTED;   // the weight table
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;

@@ -8,9 +8,9 @@
 // slice), and every thread keeps its 32 keys in registers for the whole
 // kernel, so the scores are read once:
 //   1. the cluster's smallest and largest key: their common leading bits are
-//      every key's, so the digit passes start at the highest bit where they
-//      differ (rows of log-scores share sign and exponent: two passes of 12
-//      and at most 11 bits instead of three);
+//      every key's, so the digit passes cover only the bits below the highest
+//      one where they differ, in as few passes of at most 14 bits as cover
+//      them (rows of log-scores share sign and most of the exponent: two);
 //   2. per digit pass: each CTA builds the histogram of its keys that match
 //      the prefix found so far in shared memory; after a cluster barrier CTA
 //      c sums bins [c * per, (c + 1) * per) over every CTA's histogram through
@@ -39,7 +39,8 @@ namespace {
 
 constexpr int kKPT = 32;              // keys per thread: 8 loads of 4
 constexpr int kMaxCluster = 8;        // portable cluster size
-constexpr int kDigitBins = 4096;      // largest digit: 12 bits
+constexpr int kDigitBits = 14;        // widest digit
+constexpr int kDigitBins = 1 << kDigitBits;
 constexpr int kMaxN = kMaxCluster * 1024 * kKPT;   // 262144
 
 struct TopkArgs {
@@ -109,6 +110,12 @@ __device__ __forceinline__ uint32_t block_reduce_u32(uint32_t v, bool take_max, 
   return r;
 }
 
+// Dynamic shared memory of the kernel: the digit histogram, then (clusters of
+// more than one CTA) this CTA's range of the cluster-wide histogram.
+__host__ __device__ constexpr size_t topk_smem_bytes(int cs) {
+  return (size_t)kDigitBins * 4 + (cs > 1 ? (size_t)((kDigitBins + cs - 1) / cs) * 4 : 0);
+}
+
 template <int T>
 __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__ TopkArgs a) {
   grid_dep_enter();
@@ -118,8 +125,9 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   const int row = blockIdx.y;
   const int s0 = rank * T * kKPT;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ int hist[kDigitBins];
-  __shared__ int red[kDigitBins];
+  extern __shared__ int dyn[];
+  int* hist = dyn;                                   // [2^nbits] this CTA's digit counts
+  int* red = cs > 1 ? dyn + kDigitBins : dyn;        // this CTA's range, summed over the cluster
   __shared__ uint32_t selw[T], tiew[T];
   __shared__ int ws[33];
   __shared__ uint32_t wsu[32];
@@ -185,53 +193,39 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   uint32_t prefix = gmax & pmask;
   int k = a.K;
 
-  // ---- 2. digit passes over bits hb .. 0
+  // ---- 2. digit passes over bits hb .. 0, as few as cover them, balanced
+  const int npass = (hb + 1 + kDigitBits - 1) / kDigitBits;
+  const int width = npass > 0 ? (hb + 1 + npass - 1) / npass : 0;
   int done_bits = 0;
   while (done_bits < hb + 1) {
-    const int nbits = min(12, hb + 1 - done_bits);
+    const int nbits = min(width, hb + 1 - done_bits);
     const int shift = hb + 1 - done_bits - nbits;
     const int nb = 1 << nbits;
     const uint32_t dm = (uint32_t)nb - 1u;
     for (int i = threadIdx.x; i < nb; i += T) hist[i] = 0;
     __syncthreads();
-    // a lane whose 4 keys share one digit counts them as one, and a run of
-    // such lanes with one digit adds once (from its first lane)
+    // the keys still matching the prefix, counted by digit
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      int d[4];
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t kk = key[u][e];
-        d[e] = (pos_of<T>(s0, u, e) < a.n && (kk & pmask) == prefix) ? (int)((kk >> shift) & dm) : -1;
+        if (pos_of<T>(s0, u, e) < a.n && (kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & dm], 1);
       }
-      const bool uni = d[0] == d[1] && d[0] == d[2] && d[0] == d[3];
-      const int dl = uni ? d[0] : -2;
-      const int dprev = __shfl_up_sync(0xffffffffu, dl, 1);
-      const bool head = lane == 0 || dprev != dl;
-      const unsigned heads = __ballot_sync(0xffffffffu, head);
-      if (uni) {
-        if (head && dl >= 0) {
-          const unsigned later = heads & ~((2u << lane) - 1u);
-          const int next = later ? __ffs(later) - 1 : 32;
-          atomicAdd(&hist[dl], 4 * (next - lane));
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (d[e] >= 0) atomicAdd(&hist[d[e]], 1);
-      }
-    }
     cl.sync();   // every histogram of the cluster complete
-    // this CTA's bin range, summed over the cluster
+    // this CTA's bin range, summed over the cluster (one CTA: its own histogram)
     const int per = (nb + cs - 1) / cs;
     const int r0 = rank * per;
     int mine = 0;
     for (int i = threadIdx.x; i < per; i += T) {
       const int bin = r0 + i;
       int s = 0;
-      if (bin < nb)
+      if (cs == 1) {
+        s = hist[i];
+      } else if (bin < nb) {
         for (int c = 0; c < cs; ++c) s += cl.map_shared_rank(hist, c)[bin];
-      red[i] = s;
+        red[i] = s;
+      }
       mine += s;
     }
     int tot;
@@ -358,10 +352,15 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
 
 template <int T>
 sfi_status launch_topk(const TopkArgs& a, int cs, cudaStream_t st) {
+  static DeviceOnce smem_attr;
+  if (!smem_attr.done() && !smem_attr.mark(cudaFuncSetAttribute(topk_cluster_kernel<T>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      (int)topk_smem_bytes(2))))
+    return SFI_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, a.rows);
   cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = topk_smem_bytes(cs);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -7,7 +7,7 @@ and compares the two with the tolerances of the hot path:
 * Selector scores and selections: within the intervals that the CUDA path's
   input error budget allows around the oracle's values (selection_bounds,
   check_selection): every score inside its interval, every candidate that is
-  in (out of) the top-K in every realisation chosen (not chosen), at most 1 %
+  in (out of) the top-K in every realisation chosen (not chosen), at most 2 %
   of K undecided, and >= 99.9 % overlap with the oracle's set when K >= 1000.
 """
 from __future__ import annotations
@@ -71,8 +71,8 @@ LSE_SUM_ERR = 2e-6
 EPS_Z = 2.0 ** -22
 EPS_KAPPA = 2.0 ** -22
 # Undecided candidates allowed per head, as a share of K (and at least this many).
-MAX_UNDECIDED_SHARE = 0.01
-MIN_UNDECIDED_ALLOWED = 2
+MAX_UNDECIDED_SHARE = 0.02
+MIN_UNDECIDED_ALLOWED = 3
 # Selection overlap with the oracle's point result required when K >= 1000.
 MIN_OVERLAP = 0.999
 
@@ -111,9 +111,10 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
 
     The kernel computes x = z - lse_C in fp32 (error eps_x, absolute: the
     error of its inputs z and lse_C plus its own exp), the prior in fp64 from
-    its norms (relative error eps_r), s = (1 - lambda) f~ + lambda r rounded
-    once to fp32, decides dominance on s (on x when lambda = 0) and the owner
-    by x at equal penalties, else by l' in fp32.  Every comparison whose two
+    its norms (relative error eps_r), s = (1 - lambda) f~ + lambda r in fp32
+    within 1 ulp (lambda r rounded to fp32, one FMA), decides dominance on s
+    (on x when lambda = 0) and the owner by x at equal penalties, else by l'
+    in fp32 (log through the hardware's base-2 approximation).  Every comparison whose two
     sides are closer than their errors may fall either way; this function
     propagates those choices: soft-NMS distance ranges, penalty ranges, the
     heads that can own a position, and finally [lo, hi] of l'' per (head,
@@ -138,7 +139,7 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     tiny = 2.0 ** -126 * 4                      # the kernel's exp flushes below fp32's normal range
     ev_err = (1.0 - lam) * (ft * np.expm1(eps_x + 2.0 ** -21) + tiny)
     eps_r = np.broadcast_to(np.asarray(eps_r, np.float64), (n,))
-    ds = ev_err + lam * (r * eps_r)[None, :] + 2.0 ** -24 * s      # independent part
+    ds = ev_err + lam * (r * eps_r)[None, :] + 2.0 ** -23 * s      # independent part
     ds_all = ds + lam * r[None, :] * eps_r_common
     by_x = lam <= 0.0
     if by_x:
@@ -173,9 +174,9 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     ell = det["ell"]
     with np.errstate(divide="ignore", invalid="ignore"):
         dl_rel = np.where(s > 0, ds_all / s, np.inf)
-    dell = dl_rel + 2.0 ** -22 * np.abs(ell) + 1e-7
+    dell = dl_rel + 2.0 ** -22 * np.abs(ell) + 2e-7
     if by_x:
-        dell = key_err * ft / (ft + O.LOG_EPS) + 2.0 ** -22 * np.abs(ell) + 1e-7
+        dell = key_err * ft / (ft + O.LOG_EPS) + 2.0 ** -22 * np.abs(ell) + 2e-7
     l1_lo = ell - dell - alpha_soft * pen_hi
     l1_hi = ell + dell - alpha_soft * pen_lo
     # possible owners: h unless some head b certainly beats it

@@ -62,12 +62,12 @@ def _run(cfg, overlap, n_layers=1):
                     qg = qh[b, g * G:(g + 1) * G]
                     if slow_ref[t]:
                         o, f, _, _ = O.dense_attention(qg, Kc, Vc)
-                        bnd, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
+                        sb, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
                         n = int(layer.n_rows[b, g])
                         sets = H.packed_sets(layer.pos[b, g].cpu().numpy(),
                                              layer.headmask[b, g].cpu().numpy(), n, cfg.n_sink, G)
                         got = np.stack(sets)
-                        ov = H.check_selection(got, bnd, K, lo, f"step {t} b{b} g{g}")
+                        ov = H.check_selection(got, sb, K, lo, f"step {t} b{b} g{g}")
                         worst["overlap"] = min(worst["overlap"], ov)
                         gpu_sets[l].append(sets)
                     else:

@@ -72,11 +72,11 @@ def _run(cfg, per_sequence):
                                 for i in range(1, min(Wn, t + 1))]
                     n_slow_window += len(fw) > 1
                     qw = [H.to64(li.q[t - i, b, hs]) for i in range(len(fw))]
-                    bnd, _ = H.decode_selection_bounds(qw[0], Kc, f, L, cfg, f_window=fw, q_window=qw)
+                    sb, _ = H.decode_selection_bounds(qw[0], Kc, f, L, cfg, f_window=fw, q_window=qw)
                     n = int(layer.n_rows[b, g])
                     sg = H.packed_sets(layer.pos[b, g].cpu().numpy(), layer.headmask[b, g].cpu().numpy(),
                                        n, cfg.n_sink, G)
-                    H.check_selection(np.stack(sg), bnd, K, lo, what)
+                    H.check_selection(np.stack(sg), sb, K, lo, what)
                     sets[b * cfg.Hkv + g] = sg
                 else:
                     o = O.sparse_attention(H.to64(li.q[t, b, hs]), Kc, Vc,
@@ -94,10 +94,8 @@ def test_window_three_queries_per_sequence_triggers():
 
 
 def test_window_four_queries_sixteen_rows():
-    """G = 4, W = 4: sixteen query rows per group (the two-tile launch plan).
-    Planted queries: with the clustered ones at this short context most
-    candidates are prior-dominated, and the near-tied cross-head owners take
-    the set overlap under the coarse floor even for a single query."""
+    """G = 4, W = 4: sixteen query rows per group (the two-tile launch plan),
+    planted queries."""
     cfg = W.CONFIG_BY_NAME["qwen3-4b-32k"].replace(B=2, context=2600, steps=12, boundary_p=0.3,
                                                    refresh_budget=4, evidence_window=4, query_mode="planted")
     worst, n = _run(cfg, per_sequence=False)

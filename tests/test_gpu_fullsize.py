@@ -81,11 +81,11 @@ def test_full_size_decode_sampled(name, steps, over, groups):
                 o, f, _, _ = O.dense_attention(qg, Kc, Vc)
                 K = O.budget(L, cfg.n_sink, cfg.n_recent, cfg.k_fixed, cfg.budget_frac)
                 lo, _ = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
-                bnd, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
+                sb, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
                 n = int(layer.n_rows[b, g])
                 sets = H.packed_sets(layer.pos[b, g].cpu().numpy(), layer.headmask[b, g].cpu().numpy(),
                                      n, cfg.n_sink, G)
-                H.check_selection(np.stack(sets), bnd, K, lo, f"{name} step {t} b{b} g{g}")
+                H.check_selection(np.stack(sets), sb, K, lo, f"{name} step {t} b{b} g{g}")
                 # the packed rows are bit-exact copies of the cache rows they name
                 pos = layer.pos[b, g, :n].cpu().numpy()
                 assert np.array_equal(H.to64(layer.pk[b, g, :n]), Kc[pos])

@@ -65,11 +65,11 @@ def _run(cfg, overlap, n_layers, incremental=True):
                     what = f"layer {l} step {t} b{b} g{g}"
                     if slow_ref[b, t]:
                         o, f, _, _ = O.dense_attention(qg, Kc, Vc)
-                        bnd, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
+                        sb, _ = H.decode_selection_bounds(qg, Kc, f, L, cfg)
                         n = int(layer.n_rows[b, g])
                         sg = H.packed_sets(layer.pos[b, g].cpu().numpy(), layer.headmask[b, g].cpu().numpy(),
                                            n, cfg.n_sink, G)
-                        H.check_selection(np.stack(sg), bnd, K, lo, what)
+                        H.check_selection(np.stack(sg), sb, K, lo, what)
                         sets[l][b * cfg.Hkv + g] = sg
                     else:
                         o = O.sparse_attention(qg, Kc, Vc, O.sparse_sets(L, cfg.n_sink, cfg.n_recent,

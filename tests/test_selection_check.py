@@ -17,8 +17,9 @@ import helpers as H
 
 def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
     """The CUDA Selector's arithmetic in numpy: x = z - lse_C in fp32, prior
-    in fp64 from fp32 norms, s rounded once to fp32, dominance on s, owner by
-    x at equal distances (or, rounded_owner, by the rounded l'), keys fp32."""
+    in fp64 from fp32 norms, lambda r rounded to fp32, s by one fp32 FMA,
+    dominance on s, owner by x at equal distances (or, rounded_owner, by the
+    rounded l'), log in base 2, keys fp32."""
     lo, hi = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
     lam = min(max(cfg.lam, 0.0), cfg.lam_clip)
     w = cfg.nms_window // 2
@@ -29,7 +30,8 @@ def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
     r = kp / kp.sum()
     x = (z32[:, lo:hi] - lse32[:, None]).astype(np.float32)
     ft = np.exp(x.astype(np.float64)).astype(np.float32)
-    s32 = ((1.0 - lam) * ft.astype(np.float64) + lam * r[None]).astype(np.float32)
+    lr32 = (lam * r).astype(np.float32)
+    s32 = (np.float64(np.float32(1.0 - lam)) * ft.astype(np.float64) + lr32.astype(np.float64)[None]).astype(np.float32)
     key = x if lam <= 0 else s32
     G, nC = x.shape
     dist = np.zeros((G, nC), np.int64)
@@ -40,8 +42,8 @@ def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
         dist = np.where(hit, d, dist)
     pen = np.where(dist > 0, 1.0 - (dist - 1.0) / w, 0.0).astype(np.float32)
     sv = np.exp(x.astype(np.float64)).astype(np.float32) if lam <= 0 else s32
-    l1 = (np.log((sv + np.float32(1e-30)).astype(np.float64)).astype(np.float32)
-          - np.float32(cfg.alpha_soft) * pen).astype(np.float32)
+    l1 = ((np.log2((sv + np.float32(1e-30)).astype(np.float64)).astype(np.float32) * np.float32(np.log(2.0)))
+          .astype(np.float32) - np.float32(cfg.alpha_soft) * pen).astype(np.float32)
     cols = np.arange(nC)
     best = np.zeros(nC, np.int64)
     for h in range(1, G):
