@@ -16,10 +16,10 @@ Within-Sentence Support Stability" (arXiv 2603.12038), cited as
   [ZH] gist.science/zh/paper/2603.12038, technical summary
 
 Where the pages leave a step open, the plainest reading is taken and marked
-READING below.  Comparisons that decide an integer (soft-NMS dominance, the
-cross-head owner) are decided as real arithmetic decides them: from the
-terms of the fused score (see _score_diff and owner), never from the last
-bit of a rounded sum.  The top-K order is that of the float64 scores.
+READING below.  Soft-NMS dominance is decided as real arithmetic decides it,
+from the terms of the fused score (see _score_diff), never from the last bit
+of a rounded sum; the cross-head owner treats scores equal to six digits as
+tied (see owner); the top-K order is that of the float64 scores.
 
 Pins: every function here is checked in tests/test_oracle_*.py against
 closed forms, library routines, brute force or hand-worked fixtures.  Parity
@@ -278,43 +278,36 @@ def soft_nms(ell: np.ndarray, alpha_soft: float, window: int, mixture=None) -> n
     return ell - alpha_soft * soft_nms_weight(soft_nms_distance(ell, window, mixture), window)
 
 
-def owner(ell1: np.ndarray, dist=None, ft=None, lam=None) -> np.ndarray:
-    """owner(j) = argmax_h l'_{h,j}, ties to the lowest head: a scan over
-    the heads in order, a head replacing the best so far only when its l' is
-    strictly larger.
+OWNER_TIE = 1e-6
 
-    l'_a vs l'_b is decided exactly.  With the soft-NMS distances and the
-    evidence given, two heads with the same penalty compare as l_a vs l_b,
-    whose sign is that of (1 - lambda)(f~_a - f~_b): the prior is common to
-    the KV group.  Heads with different penalties compare by l' itself (the
-    penalties differ by at least alpha_soft / w)."""
+
+def owner(ell1: np.ndarray, tie: float = OWNER_TIE) -> np.ndarray:
+    """owner(j): the lowest-indexed head whose l'_{h,j} is within a relative
+    `tie` of the group's largest, M_j = max_h l'_{h,j}:
+      owner(j) = min { h : l'_{h,j} >= M_j - tie * max(1, |M_j|) }.
+
+    READING (the pages name the argmax but no tie rule): heads whose refined
+    scores agree to six digits are tied and the lowest one owns the position.
+    Where the prior dominates, the group's heads share s to some twenty
+    digits; a plain argmax would hand each such position to whichever head
+    has the most evidence there, a difference far below anything the scores
+    represent, and the ownership of most candidates would then follow it."""
     ell1 = np.asarray(ell1, np.float64)
-    G, n = ell1.shape
-    cols = np.arange(n)
-    best = np.zeros(n, np.int64)
-    for h in range(1, G):
-        wins = ell1[h] > ell1[best, cols]
-        if dist is not None:
-            same = np.asarray(dist)[h] == np.asarray(dist)[best, cols]
-            if lam >= 1.0:
-                by_ev = np.zeros(n, bool)
-            else:
-                by_ev = np.asarray(ft, np.float64)[h] > np.asarray(ft, np.float64)[best, cols]
-            wins = np.where(same, by_ev, wins)
-        best = np.where(wins, h, best)
-    return best
+    M = ell1.max(axis=0)
+    thr = M - tie * np.maximum(1.0, np.abs(M))
+    return np.argmax(ell1 >= thr[None, :], axis=0)
 
 
-def cross_head(ell1: np.ndarray, alpha_cross: float, dist=None, ft=None, lam=None) -> np.ndarray:
+def cross_head(ell1: np.ndarray, alpha_cross: float) -> np.ndarray:
     """Cross-head exclusivity within one KV group: discourage the group's
     query heads from choosing the same positions ([FR] "B. Le Sélecteur",
     Exclusivité inter-têtes; [ZH] "2.2", 跨头互斥).
 
-    READING: owner(j) = argmax_h l'_{h,j} (ties to the lowest h, see
-    `owner`); l''_{h,j} = l'_{h,j} - alpha_cross * [h != owner(j)].
+    READING: owner(j) as `owner` gives it (the argmax of l', near-ties to the
+    lowest head); l''_{h,j} = l'_{h,j} - alpha_cross * [h != owner(j)].
     """
     ell1 = np.asarray(ell1, np.float64)
-    own = owner(ell1, dist, ft, lam)
+    own = owner(ell1)
     G = ell1.shape[0]
     not_owner = np.arange(G)[:, None] != own[None, :]
     return ell1 - alpha_cross * not_owner
@@ -350,7 +343,7 @@ def selector_detail(ft: np.ndarray, r: np.ndarray, lam: float, lam_clip: float,
     mixture = (ft, r, lam_eff)
     dist = soft_nms_distance(ell, window, mixture)
     ell1 = ell - alpha_soft * soft_nms_weight(dist, window)
-    own = owner(ell1, dist, ft, lam_eff)
+    own = owner(ell1)
     ell2 = ell1 - alpha_cross * (np.arange(ft.shape[0])[:, None] != own[None, :])
     return {"lam_eff": lam_eff, "s": s, "ell": ell, "dist": dist, "ell1": ell1, "owner": own, "ell2": ell2}
 

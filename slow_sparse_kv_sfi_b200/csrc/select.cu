@@ -9,20 +9,20 @@
 //   log-score  l = ln(s + 1e-30)
 //   soft-NMS   l' = l - alpha_soft * (1 - (d - 1) / w), d = distance to the
 //              nearest dominating neighbour within w (none: no penalty)
-//   exclusivity l'' = l' - alpha_cross * [h != argmax_h' l'_{h',j}]
+//   exclusivity l'' = l' - alpha_cross * [h != owner(j)], owner(j) = the
+//              lowest head whose l' is within 1e-6 * max(1, |M_j|) of the
+//              group's largest, M_j (near-ties go to the lowest head)
 //   top-K      K largest l'' per query head, ties to the lower position.
 //
-// Comparisons that decide an integer follow real arithmetic, not the last bit
-// of a rounded sum: l_i vs l_j has the sign of s_i - s_j (ln is monotone),
-// with s = (1 - lambda) f~ + lambda r formed by one fp32 FMA from lambda r
-// (fp64 prior, rounded to fp32): within 1 ulp of s, where the prior dominates
-// neighbouring candidates differ in r by ~1e-6 relative, far above that; two
-// heads with the same soft-NMS penalty compare by their evidence, since r is
-// common to the group (their s agree to every digit where the prior
-// dominates).  The evidence is compared through its logarithm x = z - lse_C,
-// which does not underflow.  With lambda = 0 the dominance is decided on x
-// as well.  No decision rests on the last bit of a logarithm, so l = ln(s)
-// uses the hardware's base-2 approximation.
+// The soft-NMS dominance follows real arithmetic, not the last bit of a
+// rounded sum: l_i vs l_j has the sign of s_i - s_j (ln is monotone), with
+// s = (1 - lambda) f~ + lambda r formed by one fp32 FMA from lambda r (fp64
+// prior, rounded to fp32): within 1 ulp of s, where the prior dominates
+// neighbouring candidates differ in r by ~1e-6 relative, far above that.
+// With lambda = 0 the dominance is decided on the log-evidence x = z - lse_C,
+// which does not underflow.  l = ln(s) is the accurate logf (1 ulp), so the
+// owner's tie tolerance (~1e-5 absolute) stays several times the kernel's
+// error on l'.
 //
 // Kernels: stats_norm / stats_prior (per (b, kv head) and chunk of C: fp64
 // partial sums of the norms and of kappa pi; every consumer reduces the
@@ -38,6 +38,7 @@
 namespace sfi {
 
 constexpr int kStatThreads = 256;
+constexpr float kOwnerTie = 1e-6f;   // relative tie tolerance of the cross-head owner
 constexpr int kStatChunk = 4096;
 
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
@@ -168,18 +169,16 @@ struct ScoreArgs {
 
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes, for every
 // head of the group over the tile plus a halo of w on each side, the
-// dominance key (s rounded once to fp32, or x when lambda = 0; NaN outside C:
-// a NaN never dominates) and, over the tile, the log-evidence x.  Phase 2
-// finds every head's nearest dominator (two passes, below).  Phase 3: the
-// thread of a position applies soft-NMS to every head, picks the owner and
-// writes l''.
+// dominance key (s in fp32, or x when lambda = 0; NaN outside C: a NaN never
+// dominates).  Phase 2 finds every head's nearest dominator (two passes,
+// below).  Phase 3: the thread of a position applies soft-NMS to every head,
+// picks the owner and writes l''.
 template <int GM>
 __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
   grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
   float* key = sm;                    // [G][W] dominance key
-  float* xo = key + a.G * W;          // [G][tile] log-evidence
   const int bg = blockIdx.y;                        // logical (row, kv head)
   const int bl = bg / a.Hkv, g = bg - bl * a.Hkv;
   const int b = a.rows.phys(bl);                    // the sequence
@@ -208,7 +207,6 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
     // x = ln f~ = m + ln(mean exp(x_i - m)), m the largest x_i
     for (int k = threadIdx.x; k < W; k += blockDim.x) {
       const int c = c0 - a.w + k;
-      const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (c < 0 || c >= a.nC) {
 #pragma unroll
         for (int h = 0; h < GM; ++h)
@@ -234,7 +232,6 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
           const float x = m + logf(acc * a.inv_nq);
           const float ft = fast_exp2(x * kLog2e);
           key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
-          if (tile_k) xo[h * a.tile + k - a.w] = x;
         }
       }
     }
@@ -258,7 +255,6 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
     for (int u = 0; u < kU; ++u) {
       const int k = k0 + u * blockDim.x;
       if (k >= W) continue;
-      const bool tile_k = k >= a.w && k < a.w + a.tile;
       if (in[u]) {
         const float r = (float)(kv[u] * lam_r);   // lambda r_j
 #pragma unroll
@@ -269,7 +265,6 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
             const float x = zv[u][h] - lsec[h];
             const float ft = fast_exp2(x * kLog2e);
             key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
-            if (tile_k) xo[h * a.tile + k - a.w] = x;
           }
         }
       } else {
@@ -286,7 +281,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   // still undecided go to a queue.  2b: the queue, scanned to w with all lanes
   // busy.  dom = distance of the nearest dominator, 0: none within w.
   constexpr int kNear = 4;
-  uint16_t* dom = reinterpret_cast<uint16_t*>(xo + G * a.tile);          // [G][tile]
+  uint16_t* dom = reinterpret_cast<uint16_t*>(key + G * W);              // [G][tile]
   uint32_t* queue = reinterpret_cast<uint32_t*>(dom + G * a.tile);       // [tile]
   const int lane = threadIdx.x & 31;
   for (int k0 = 0; k0 < tile_n; k0 += blockDim.x) {
@@ -339,40 +334,27 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
     }
   }
   __syncthreads();
-  // Phase 3: l' = ln(s + 1e-30) - alpha_soft * weight(d); the owner scans the
-  // heads in order (ties to the lowest): equal distances compare by x (never
-  // when lambda = 1: the evidence has no weight), others by l'.
-  const bool ev_counts = a.one_minus_lam > 0.f;
+  // Phase 3: l' = ln(s + 1e-30) - alpha_soft * weight(d); the owner is the
+  // lowest head within the tie tolerance of the largest l'.
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
-    float l1[GM], xv[GM];
-    int dv[GM];
+    float l1[GM];
+    float M = -INFINITY;
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       l1[h] = -INFINITY;
-      xv[h] = 0.f;
-      dv[h] = 0;
       if (h < G) {
         const int d = dom[h * a.tile + k];
-        xv[h] = xo[h * a.tile + k];
-        const float sv = by_x ? fast_exp2(xv[h] * kLog2e) : key[h * W + a.w + k];
-        l1[h] = fast_log2(sv + 1e-30f) * kLn2 - a.alpha_soft * wt[d];
-        dv[h] = d;
+        const float kv = key[h * W + a.w + k];
+        const float sv = by_x ? fast_exp2(kv * kLog2e) : kv;
+        l1[h] = logf(sv + 1e-30f) - a.alpha_soft * wt[d];
+        M = fmaxf(M, l1[h]);
       }
     }
-    int owner = 0, best_d = dv[0];
-    float best_x = xv[0], best_l1 = l1[0];
+    const float thr = M - kOwnerTie * fmaxf(1.f, fabsf(M));
+    int owner = GM;
 #pragma unroll
-    for (int h = 1; h < GM; ++h) {
-      if (h < G) {
-        const bool wins = dv[h] == best_d ? (ev_counts && xv[h] > best_x) : (l1[h] > best_l1);
-        if (wins) {
-          owner = h;
-          best_d = dv[h];
-          best_x = xv[h];
-          best_l1 = l1[h];
-        }
-      }
-    }
+    for (int h = GM - 1; h >= 0; --h)
+      if (h < G && l1[h] >= thr) owner = h;
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
@@ -386,11 +368,11 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
 // ---------------------------------------------------------------- host
 int score_tile(int G) { return std::max(256, 4096 / G); }
 
-// dominance keys with halo, log-evidence, nearest-dominator distances, queue
-// of undecided positions
+// dominance keys with halo, nearest-dominator distances, queue of undecided
+// positions
 size_t score_smem(int G, int tile, int w) {
-  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(float) +
-         (size_t)G * tile * sizeof(uint16_t) + (size_t)tile * sizeof(uint32_t);
+  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(uint16_t) +
+         (size_t)tile * sizeof(uint32_t);
 }
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }

@@ -113,8 +113,8 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     error of its inputs z and lse_C plus its own exp), the prior in fp64 from
     its norms (relative error eps_r), s = (1 - lambda) f~ + lambda r in fp32
     within 1 ulp (lambda r rounded to fp32, one FMA), decides dominance on s
-    (on x when lambda = 0) and the owner by x at equal penalties, else by l'
-    in fp32 (log through the hardware's base-2 approximation).  Every comparison whose two
+    (on x when lambda = 0) and the owner with its tie tolerance on l' in fp32
+    (logf, within 1 ulp).  Every comparison whose two
     sides are closer than their errors may fall either way; this function
     propagates those choices: soft-NMS distance ranges, penalty ranges, the
     heads that can own a position, and finally [lo, hi] of l'' per (head,
@@ -174,31 +174,27 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     ell = det["ell"]
     with np.errstate(divide="ignore", invalid="ignore"):
         dl_rel = np.where(s > 0, ds_all / s, np.inf)
-    dell = dl_rel + 2.0 ** -22 * np.abs(ell) + 2e-7
+    ulp = np.spacing(np.abs(ell).astype(np.float32)).astype(np.float64)   # fp32 ulp of l
+    dell = dl_rel + 1.5 * ulp + 1e-7
     if by_x:
-        dell = key_err * ft / (ft + O.LOG_EPS) + 2.0 ** -22 * np.abs(ell) + 2e-7
+        dell = key_err * ft / (ft + O.LOG_EPS) + 1.5 * ulp + 1e-7
     l1_lo = ell - dell - alpha_soft * pen_hi
     l1_hi = ell + dell - alpha_soft * pen_lo
-    # possible owners: h unless some head b certainly beats it
-    d_set = possible.copy()
-    d_set[INF] = d_hi > w                     # "no dominator" is possible when none is certain
-    for d in range(1, w + 1):
-        d_set[d] &= d <= d_hi                 # nothing beyond the nearest certain one
-    cert_eq = d_lo == d_hi
-    can_be_owner = np.ones((G, n), bool)
-    xe = eps_x + 2.0 ** -24 * np.abs(x) + 2.0 ** -21
-    for h in range(G):
-        for b in range(G):
-            if b == h:
-                continue
-            can_equal = np.any(d_set[:, b] & d_set[:, h], axis=0)
-            can_differ = ~(cert_eq[b] & cert_eq[h] & (d_lo[b] == d_lo[h]))
-            if lam >= 1.0:
-                ev_beats = np.full(n, b < h)
-            else:
-                ev_beats = (x[b] - x[h]) > (xe[b] + xe[h])
-            beats = (~can_equal | ev_beats) & (~can_differ | (l1_lo[b] > l1_hi[h]))
-            can_be_owner[h] &= ~beats
+    # possible owners under the tie rule (owner = the lowest head with
+    # l' >= M - tie * max(1, |M|)): h can own j if it may clear the threshold
+    # while no lower head certainly clears it; the threshold moves with M and
+    # with the fp32 rounding of the kernel's threshold
+    M_lo, M_hi = l1_lo.max(axis=0), l1_hi.max(axis=0)
+
+    def thr(M):
+        return M - O.OWNER_TIE * np.maximum(1.0, np.abs(M))
+
+    tpad = np.spacing(np.maximum(np.abs(M_lo), np.abs(M_hi)).astype(np.float32)).astype(np.float64)
+    t_lo, t_hi = thr(M_lo) - tpad, thr(M_hi) + tpad
+    certain_q = l1_lo >= t_hi[None, :]
+    possible_q = l1_hi >= t_lo[None, :]
+    lower_certain = np.cumsum(certain_q, axis=0) - certain_q
+    can_be_owner = possible_q & (lower_certain == 0)
     n_poss = can_be_owner.sum(axis=0)
     sure_owner = can_be_owner & (n_poss == 1)[None, :]
     lo2 = np.where(sure_owner, l1_lo, l1_lo - alpha_cross)

@@ -5,7 +5,7 @@ minimisation of the KL objective the pages state; top-K by Python's sorted();
 soft-NMS, cross-head exclusivity, the prior, compaction and the trigger by
 hand-worked fixtures under tests/golden/ and by their special cases; the
 Selector's decisions by a brute-force evaluation in 80-digit decimal
-arithmetic.
+arithmetic (with the owner's tie tolerance).
 """
 import json
 import math
@@ -194,11 +194,11 @@ def _selector_decimal(ft, r, lam, alpha_soft, alpha_cross, window, K, prec=80):
             ell1.append(row)
         sel = []
         ell2 = [[None] * n for _ in range(G)]
+        tie = Dc(O.OWNER_TIE)
         for j in range(n):
-            best = 0
-            for h in range(1, G):
-                if ell1[h][j] > ell1[best][j]:
-                    best = h
+            M = max(ell1[h][j] for h in range(G))
+            thr = M - tie * max(one, abs(M))
+            best = min(h for h in range(G) if ell1[h][j] >= thr)
             for h in range(G):
                 ell2[h][j] = ell1[h][j] - (Dc(alpha_cross) if h != best else Dc(0))
         for h in range(G):
@@ -228,32 +228,22 @@ def test_selector_decisions_agree_with_80_digit_arithmetic(seed, tiny):
     np.testing.assert_array_equal(got, ref)
 
 
-def test_rounded_decisions_would_break_exact_arithmetic():
-    """Why the oracle never decides on a rounded s: where the prior dominates,
-    every head's s is the same float64 (and float32) number, so a decision
-    taken on the rounded values hands every position to head 0, while real
-    arithmetic gives it to the head with the most evidence."""
-    ft, r = _prior_dominated_case(0, tiny=1e-24)
-    lam, a_s, a_c, window, K = 0.2, 0.5, 0.5, 8, 20
-    ref = _selector_decimal(ft, r, lam, a_s, a_c, window, K)
-    ell = O.log_score(O.fuse(ft, r, lam, 0.5))
-    for cast in (np.float64, np.float32):
-        e = ell.astype(cast).astype(np.float64)
-        rounded = O.topk(O.cross_head(O.soft_nms(e, a_s, window), a_c), K)
-        assert not np.array_equal(rounded, ref)
-
-
-def test_owner_exact_special_cases():
-    # equal penalties, the prior common: the head with the largest evidence owns
-    ell1 = np.zeros((3, 2))
-    dist = np.ones((3, 2), np.int64)
-    ft = np.array([[1e-30, 5e-31], [3e-30, 1e-31], [2e-30, 7e-31]])
-    np.testing.assert_array_equal(O.owner(ell1, dist, ft, 0.2), [1, 2])
-    # lambda = 1: the evidence has no weight, ties go to the lowest head
-    np.testing.assert_array_equal(O.owner(ell1, dist, ft, 1.0), [0, 0])
-    # different penalties: l' decides, not the evidence
-    ell1 = np.array([[0.0], [-0.5]])
-    np.testing.assert_array_equal(O.owner(ell1, np.array([[1], [2]]), np.array([[1e-30], [1.0]]), 0.2), [0])
+def test_owner_tie_tolerance():
+    # heads whose l' agree to twenty digits: tied, the lowest head owns
+    base = -13.0
+    ell1 = np.array([[base], [base + 1e-14], [base + 2e-14]])
+    np.testing.assert_array_equal(O.owner(ell1), [0])
+    # six digits apart (13 * 1e-6 = 1.3e-5): still tied; clearly above: the max owns
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1.0e-5]])), [0])
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 2.0e-5]])), [1])
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1e-3], [base + 0.5]])), [2])
+    # a plain argmax would take the largest: the tolerance is what differs
+    ell1 = np.array([[base, -0.5], [base + 1e-9, -0.5 + 2e-6]])
+    np.testing.assert_array_equal(O.owner(ell1), [0, 1])       # |M| < 1: the tolerance is 1e-6 absolute
+    assert list(np.argmax(ell1, axis=0)) == [1, 1]
+    # cross_head penalises everyone but the owner
+    out = O.cross_head(np.array([[base], [base + 1e-14]]), 0.5)
+    np.testing.assert_allclose(out[:, 0], [base, base + 1e-14 - 0.5])
 
 
 def test_soft_nms_exact_dominance_under_equal_prior():

@@ -2,7 +2,7 @@
 on the CPU: a float32 emulation of the CUDA Selector's arithmetic passes it on
 seeded workload groups, with few undecided candidates, and planted mistakes
 fail it: a swapped pick, a score moved by a cross-head penalty, and owners
-decided on rounded scores (which hand prior-dominated positions to head 0)."""
+taken by a plain argmax of the rounded scores (no tie tolerance)."""
 import math
 
 import numpy as np
@@ -18,8 +18,8 @@ import helpers as H
 def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
     """The CUDA Selector's arithmetic in numpy: x = z - lse_C in fp32, prior
     in fp64 from fp32 norms, lambda r rounded to fp32, s by one fp32 FMA,
-    dominance on s, owner by x at equal distances (or, rounded_owner, by the
-    rounded l'), log in base 2, keys fp32."""
+    dominance on s, owner with the tie tolerance on l' (or, rounded_owner, a
+    plain argmax of the fp32 l'), keys fp32."""
     lo, hi = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
     lam = min(max(cfg.lam, 0.0), cfg.lam_clip)
     w = cfg.nms_window // 2
@@ -42,17 +42,15 @@ def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
         dist = np.where(hit, d, dist)
     pen = np.where(dist > 0, 1.0 - (dist - 1.0) / w, 0.0).astype(np.float32)
     sv = np.exp(x.astype(np.float64)).astype(np.float32) if lam <= 0 else s32
-    l1 = ((np.log2((sv + np.float32(1e-30)).astype(np.float64)).astype(np.float32) * np.float32(np.log(2.0)))
-          .astype(np.float32) - np.float32(cfg.alpha_soft) * pen).astype(np.float32)
+    l1 = (np.log((sv + np.float32(1e-30)).astype(np.float64)).astype(np.float32)
+          - np.float32(cfg.alpha_soft) * pen).astype(np.float32)
     cols = np.arange(nC)
-    best = np.zeros(nC, np.int64)
-    for h in range(1, G):
-        if rounded_owner:
-            wins = l1[h] > l1[best, cols]
-        else:
-            same = dist[h] == dist[best, cols]
-            wins = np.where(same, (lam < 1.0) & (x[h] > x[best, cols]), l1[h] > l1[best, cols])
-        best = np.where(wins, h, best)
+    if rounded_owner:      # a plain argmax on the fp32 scores
+        best = np.argmax(l1, axis=0)
+    else:                  # the lowest head within the tie tolerance of the largest
+        M = l1.max(axis=0)
+        thr = (M - np.float32(O.OWNER_TIE) * np.maximum(np.float32(1.0), np.abs(M))).astype(np.float32)
+        best = np.argmax(l1 >= thr[None, :], axis=0)
     sc = (l1 - np.float32(cfg.alpha_cross) * (np.arange(G)[:, None] != best[None]).astype(np.float32)).astype(np.float32)
     sel = np.stack([np.sort(np.lexsort((cols, -sc[h]))[:K]) for h in range(G)]) + lo
     return sel, sc
@@ -129,7 +127,7 @@ def test_planted_mistakes_fail():
     sc2[1, 10] += cfg.alpha_cross
     with pytest.raises(AssertionError):
         H.check_selection(sel, b, K, lo, "moved score", gpu_scores=sc2)
-    # owners decided on the rounded scores
+    # owners by a plain argmax of the rounded scores
     sel3, sc3 = _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=True)
     with pytest.raises(AssertionError):
         H.check_selection(sel3, b, K, lo, "rounded owner", gpu_scores=sc3)
