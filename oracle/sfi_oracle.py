@@ -18,8 +18,8 @@ Within-Sentence Support Stability" (arXiv 2603.12038), cited as
 Where the pages leave a step open, the plainest reading is taken and marked
 READING below.  Soft-NMS dominance is decided as real arithmetic decides it,
 from the terms of the fused score (see _score_diff), never from the last bit
-of a rounded sum; the cross-head owner treats scores equal to six digits as
-tied (see owner); the top-K order is that of the float64 scores.
+of a rounded sum; the cross-head owner treats log-scores within 1e-3 of each
+other as tied (see owner); the top-K order is that of the float64 scores.
 
 Pins: every function here is checked in tests/test_oracle_*.py against
 closed forms, library routines, brute force or hand-worked fixtures.  Parity
@@ -278,24 +278,25 @@ def soft_nms(ell: np.ndarray, alpha_soft: float, window: int, mixture=None) -> n
     return ell - alpha_soft * soft_nms_weight(soft_nms_distance(ell, window, mixture), window)
 
 
-OWNER_TIE = 1e-6
+OWNER_TIE = 1e-3
 
 
 def owner(ell1: np.ndarray, tie: float = OWNER_TIE) -> np.ndarray:
-    """owner(j): the lowest-indexed head whose l'_{h,j} is within a relative
-    `tie` of the group's largest, M_j = max_h l'_{h,j}:
-      owner(j) = min { h : l'_{h,j} >= M_j - tie * max(1, |M_j|) }.
+    """owner(j): the lowest-indexed head whose l'_{h,j} is within `tie` of the
+    group's largest, M_j = max_h l'_{h,j}:
+      owner(j) = min { h : l'_{h,j} >= M_j - tie }.
 
     READING (the pages name the argmax but no tie rule): heads whose refined
-    scores agree to six digits are tied and the lowest one owns the position.
+    log-scores agree within 1e-3 (their fused scores within 0.1 %) are tied
+    and the lowest one owns the position; the tolerance is thirty times
+    below the smallest step of the soft-NMS penalty (alpha_soft / w).
     Where the prior dominates, the group's heads share s to some twenty
     digits; a plain argmax would hand each such position to whichever head
     has the most evidence there, a difference far below anything the scores
     represent, and the ownership of most candidates would then follow it."""
     ell1 = np.asarray(ell1, np.float64)
     M = ell1.max(axis=0)
-    thr = M - tie * np.maximum(1.0, np.abs(M))
-    return np.argmax(ell1 >= thr[None, :], axis=0)
+    return np.argmax(ell1 >= (M - tie)[None, :], axis=0)
 
 
 def cross_head(ell1: np.ndarray, alpha_cross: float) -> np.ndarray:

@@ -187,7 +187,7 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     M_lo, M_hi = l1_lo.max(axis=0), l1_hi.max(axis=0)
 
     def thr(M):
-        return M - O.OWNER_TIE * np.maximum(1.0, np.abs(M))
+        return M - O.OWNER_TIE
 
     tpad = np.spacing(np.maximum(np.abs(M_lo), np.abs(M_hi)).astype(np.float32)).astype(np.float64)
     t_lo, t_hi = thr(M_lo) - tpad, thr(M_hi) + tpad

@@ -197,7 +197,7 @@ def _selector_decimal(ft, r, lam, alpha_soft, alpha_cross, window, K, prec=80):
         tie = Dc(O.OWNER_TIE)
         for j in range(n):
             M = max(ell1[h][j] for h in range(G))
-            thr = M - tie * max(one, abs(M))
+            thr = M - tie
             best = min(h for h in range(G) if ell1[h][j] >= thr)
             for h in range(G):
                 ell2[h][j] = ell1[h][j] - (Dc(alpha_cross) if h != best else Dc(0))
@@ -231,16 +231,16 @@ def test_selector_decisions_agree_with_80_digit_arithmetic(seed, tiny):
 def test_owner_tie_tolerance():
     # heads whose l' agree to twenty digits: tied, the lowest head owns
     base = -13.0
-    ell1 = np.array([[base], [base + 1e-14], [base + 2e-14]])
-    np.testing.assert_array_equal(O.owner(ell1), [0])
-    # six digits apart (13 * 1e-6 = 1.3e-5): still tied; clearly above: the max owns
-    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1.0e-5]])), [0])
-    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 2.0e-5]])), [1])
-    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1e-3], [base + 0.5]])), [2])
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1e-14], [base + 2e-14]])), [0])
+    # within the tolerance (1e-3): tied; clearly above it: the largest owns
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 0.9e-3]])), [0])
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 1.1e-3]])), [1])
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 0.01], [base + 0.5]])), [2])
+    # two heads tie with each other above a third: the lower of the two owns
+    np.testing.assert_array_equal(O.owner(np.array([[base], [base + 0.5], [base + 0.5 + 1e-4]])), [1])
     # a plain argmax would take the largest: the tolerance is what differs
-    ell1 = np.array([[base, -0.5], [base + 1e-9, -0.5 + 2e-6]])
-    np.testing.assert_array_equal(O.owner(ell1), [0, 1])       # |M| < 1: the tolerance is 1e-6 absolute
-    assert list(np.argmax(ell1, axis=0)) == [1, 1]
+    ell1 = np.array([[base], [base + 1e-9]])
+    assert list(np.argmax(ell1, axis=0)) == [1] and list(O.owner(ell1)) == [0]
     # cross_head penalises everyone but the owner
     out = O.cross_head(np.array([[base], [base + 1e-14]]), 0.5)
     np.testing.assert_allclose(out[:, 0], [base, base + 1e-14 - 0.5])

@@ -49,7 +49,7 @@ def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
         best = np.argmax(l1, axis=0)
     else:                  # the lowest head within the tie tolerance of the largest
         M = l1.max(axis=0)
-        thr = (M - np.float32(O.OWNER_TIE) * np.maximum(np.float32(1.0), np.abs(M))).astype(np.float32)
+        thr = (M - np.float32(O.OWNER_TIE)).astype(np.float32)
         best = np.argmax(l1 >= thr[None, :], axis=0)
     sc = (l1 - np.float32(cfg.alpha_cross) * (np.arange(G)[:, None] != best[None]).astype(np.float32)).astype(np.float32)
     sel = np.stack([np.sort(np.lexsort((cols, -sc[h]))[:K]) for h in range(G)]) + lo
