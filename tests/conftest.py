@@ -36,8 +36,10 @@ def pytest_terminal_summary(terminalreporter):
     tr.section("selection parity")
     agg = OrderedDict()
     for test, _what, _h, K, und, ov, diff in rec:
-        a = agg.setdefault(test, {"checks": 0, "K": set(), "und": 0, "share": 0.0, "ov": 1.0, "diff": 0})
+        a = agg.setdefault(test, {"checks": 0, "K": set(), "und": 0, "share": 0.0, "ov": 1.0, "diff": 0,
+                                  "sum": 0.0})
         a["checks"] += 1
+        a["sum"] += und / K
         a["K"].add(K)
         a["und"] = max(a["und"], und)
         a["share"] = max(a["share"], und / K)
@@ -46,10 +48,11 @@ def pytest_terminal_summary(terminalreporter):
     for test, a in agg.items():
         ks = sorted(a["K"])
         tr.write_line(f"{test}: {a['checks']} head checks, K {ks[0]}..{ks[-1]}, max undecided {a['und']} "
-                      f"({100 * a['share']:.3f} % of K), min overlap {a['ov']:.6f}, max differing picks {a['diff']}")
+                      f"({100 * a['share']:.3f} % of K; mean {100 * a['sum'] / a['checks']:.3f} %), min overlap {a['ov']:.6f}, max differing picks {a['diff']}")
     if rec:
         tr.write_line(f"all: {len(rec)} head checks, max undecided share "
-                      f"{100 * max(r[4] / r[3] for r in rec):.3f} %, min overlap {min(r[5] for r in rec):.6f}")
+                      f"{100 * max(r[4] / r[3] for r in rec):.3f} % (mean {100 * sum(r[4] / r[3] for r in rec) / len(rec):.3f} %), "
+                      f"min overlap {min(r[5] for r in rec):.6f}")
     if helpers.LOGIT_RECORD:
         tr.write_line(f"logit error: at most {max(helpers.LOGIT_RECORD):.3e} x sum|q k|/sqrt(D) "
                       f"(bound {helpers.C_Z:.3e})")
