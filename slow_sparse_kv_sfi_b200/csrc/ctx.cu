@@ -32,7 +32,7 @@ struct sfi_ctx {
   int device;
   int p_max_ws;
   cudaStream_t side = nullptr;
-  std::vector<cudaEvent_t> ev_dense, ev_sel;
+  std::vector<cudaEvent_t> ev_pre, ev_dense, ev_sel;
   std::vector<uint8_t> pending;
   cudaEvent_t ev_buf_free[kLogitBufs] = {};
   int cur_step = -1;
@@ -242,6 +242,12 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
   if (c->n_slow > 0) {
     const int buf = layer % kLogitBufs;
     SFI_TRY(cu(cudaStreamWaitEvent(main, c->ev_buf_free[buf], 0)));
+    // the prior's statistics read key norms only (the step's appended token
+    // is in the recent window, never a candidate): on the side stream, beside
+    // this layer's attention
+    SFI_TRY(cu(cudaEventRecord(c->ev_pre[layer], main)));
+    SFI_TRY(cu(cudaStreamWaitEvent(c->side, c->ev_pre[layer], 0)));
+    SFI_TRY(run_select_stats(s, p, *kv, L, c->stats, c->side, slow_map));
     sfi_dense_extras ex{};
     ex.logits = c->logits[buf];
     ex.ld = c->ld;
@@ -276,7 +282,7 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
     if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
     const int rows = slow_map.count(B) * s.Hq;   // logical rows of the Selector
     SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                              c->stats, side, slow_map, wmask));
+                              c->stats, side, slow_map, wmask, false));
     SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
     SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, side));
     if (c->incremental && packed->p_max >= c->cmp.cap) {
@@ -330,6 +336,7 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   int least = 0, greatest = 0;
   bool ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
             cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, greatest) == cudaSuccess;
+  c->ev_pre.resize(n_layers, nullptr);
   c->ev_dense.resize(n_layers, nullptr);
   c->ev_sel.resize(n_layers, nullptr);
   c->pending.assign(n_layers, 0);
@@ -340,7 +347,8 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->win = evidence_window(*params);
   c->slot_step.assign((size_t)n_layers * c->win, -1);
   for (int i = 0; i < n_layers && ok; ++i)
-    ok = cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
+    ok = cudaEventCreateWithFlags(&c->ev_pre[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&c->ev_dense[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&c->ev_sel[i], cudaEventDisableTiming) == cudaSuccess;
   for (int i = 0; i < kLogitBufs && ok; ++i)
     ok = cudaEventCreateWithFlags(&c->ev_buf_free[i], cudaEventDisableTiming) == cudaSuccess;
@@ -355,6 +363,7 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
 sfi_status sfi_ctx_destroy(sfi_ctx* c) {
   if (!c) return SFI_OK;
   if (c->side) cudaStreamSynchronize(c->side);
+  for (auto e : c->ev_pre) if (e) cudaEventDestroy(e);
   for (auto e : c->ev_dense) if (e) cudaEventDestroy(e);
   for (auto e : c->ev_sel) if (e) cudaEventDestroy(e);
   for (auto e : c->ev_buf_free) if (e) cudaEventDestroy(e);

@@ -140,11 +140,17 @@ sfi_status run_append(const sfi_shape& s, const sfi_paged_kv& kv, int L, const s
 sfi_status run_key_norms(const sfi_shape& s, const sfi_paged_kv& kv, int lo, int hi,
                          cudaStream_t st);
 
+// The prior's statistics of a slow step at context L (key norms only: they
+// may run before the step's attention, whose appended token is never a
+// candidate) into stat_ws; then the scores, which read them.  with_stats:
+// run_select_scores launches the statistics itself first.
+sfi_status run_select_stats(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
+                            void* stat_ws, cudaStream_t st, const RowMap& rows = RowMap());
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
                              cudaStream_t st, const RowMap& rows = RowMap(),
-                             uint32_t window_mask = 0xffffffffu);
+                             uint32_t window_mask = 0xffffffffu, bool with_stats = true);
 // K largest of every row (ties to the lower index): bitmap bits[rows][ld_b]
 // and / or ascending positions idx[rows][ld_i] (+ offset).  No scratch: the
 // cluster kernel of topk.cu keeps its state on chip.

@@ -37,7 +37,8 @@
 namespace sfi {
 
 constexpr int kStatThreads = 256;
-constexpr float kOwnerTie = 1e-3f;   // tie tolerance of the cross-head owner (log-score units)
+constexpr float kOwnerTie = 1e-3f;
+constexpr double kMaxProductPenalty = 18.0;   // tie tolerance of the cross-head owner (log-score units)
 constexpr int kStatChunk = 4096;
 
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
@@ -387,32 +388,62 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
+namespace {
+
+// The statistics area: partial sums, then the position factors, then
+// kappa * pi of every candidate of every row.
+struct StatLayout {
+  int nb, nC, nch;
+  int64_t kp_ld;
+  double *part, *pitab, *kp;
+  StatLayout(const sfi_shape& s, const sfi_params& p, int L, const RowMap& rows, void* ws) {
+    nb = rows.count(s.B);
+    nC = L - p.n_recent - p.n_sink;
+    nch = stat_chunks(nC);
+    kp_ld = (nC + 1) / 2 * 2;
+    part = reinterpret_cast<double*>(ws);
+    pitab = part + (size_t)nb * s.Hkv * nch * 2;
+    kp = pitab + kp_ld;
+  }
+};
+
+}  // namespace
+
+sfi_status run_select_stats(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
+                            void* stat_ws, cudaStream_t st, const RowMap& rows) {
+  const StatLayout sl(s, p, L, rows, stat_ws);
+  if (sl.nb < 1 || sl.nb > s.B) return SFI_ERR_SHAPE;
+  const int lo = p.n_sink;
+  const int64_t norm_ld = (int64_t)s.max_pages * kPage;
+  dim3 sgrid(sl.nch, sl.nb * s.Hkv);
+  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, sl.nC, kv.key_norms, norm_ld, sl.part,
+           sl.nch, s.Hkv, sl.pitab, rows);
+  launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, sl.nC, kv.key_norms, norm_ld, sl.part,
+           sl.nch, s.Hkv, sl.pitab, sl.kp, sl.kp_ld, rows);
+  return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+}
+
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st, const RowMap& rows, uint32_t window_mask) {
+                             cudaStream_t st, const RowMap& rows, uint32_t window_mask, bool with_stats) {
   const int G = s.Hq / s.Hkv;
   const int nb = rows.count(s.B);
   if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
   const int nq = evidence_window(p);
   const uint32_t qmask = window_mask & (nq >= 32 ? 0xffffffffu : ((1u << nq) - 1u));
   if (qmask == 0u) return SFI_ERR_INVALID_ARG;
-  const int lo = p.n_sink, hi = L - p.n_recent;
-  const int nC = hi - lo;
-  double* part = reinterpret_cast<double*>(stat_ws);
-  const int nch = stat_chunks(nC);
-  const int64_t norm_ld = (int64_t)s.max_pages * kPage;
-  dim3 sgrid(nch, nb * s.Hkv);
-  // the statistics area: partial sums, then the position factors, then
-  // kappa * pi of every candidate of every row
-  const int64_t kp_ld = (nC + 1) / 2 * 2;
-  double* pitab = part + (size_t)nb * s.Hkv * nch * 2;
-  double* kp = pitab + kp_ld;
-  launch_k(stats_norm_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
-           s.Hkv, pitab, rows);
-  launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, nC, kv.key_norms, norm_ld, part, nch,
-           s.Hkv, pitab, kp, kp_ld, rows);
-  if (cudaPeekAtLastError() != cudaSuccess) return SFI_ERR_CUDA;
+  const int lo = p.n_sink;
+  const StatLayout sl(s, p, L, rows, stat_ws);
+  const int nC = sl.nC, nch = sl.nch;
+  if (std::max(p.nms_window / 2, 1) > 63) return SFI_ERR_UNSUPPORTED;   // the weight table
+  if (with_stats) {
+    const sfi_status r = run_select_stats(s, p, kv, L, stat_ws, st, rows);
+    if (r != SFI_OK) return r;
+  }
+  double* part = sl.part;
+  double* kp = sl.kp;
+  const int64_t kp_ld = sl.kp_ld;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;
   a.w = std::max(p.nms_window / 2, 1);
@@ -420,7 +451,6 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   const double lam = std::min(std::max((double)p.lambda, 0.0), (double)p.lambda_clip);
   a.lam = lam;
   a.one_minus_lam = (float)(1.0 - lam);
-  if (a.w > 63) return SFI_ERR_UNSUPPORTED;   // the weight table
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;

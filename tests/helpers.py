@@ -70,6 +70,9 @@ LSE_SUM_ERR = 2e-6
 # where n_j is at or above the mean (elsewhere kappa = 1 exactly).
 EPS_Z = 2.0 ** -23
 EPS_KAPPA = 2.0 ** -23
+# Rounding of the kernel's fused score s (relative, per element): lambda r
+# rounded to fp32, then one FMA.
+S_ROUND = 2.0 ** -23
 # Undecided candidates allowed per head, as a share of K (and at least this
 # many).  The count is a property of the input, not of the kernel (whose
 # choices are checked candidate by candidate against the sure-in / sure-out
@@ -149,7 +152,7 @@ def selection_bounds(ft, r, lam_eff, alpha_soft, alpha_cross, window, eps_x, eps
     tiny = 2.0 ** -126 * 4                      # the kernel's exp flushes below fp32's normal range
     ev_err = (1.0 - lam) * (ft * np.expm1(eps_x + 2.0 ** -21) + tiny)
     eps_r = np.broadcast_to(np.asarray(eps_r, np.float64), (n,))
-    ds = ev_err + lam * (r * eps_r)[None, :] + 2.0 ** -23 * s      # independent part
+    ds = ev_err + lam * (r * eps_r)[None, :] + S_ROUND * s      # independent part
     ds_all = ds + lam * r[None, :] * eps_r_common
     by_x = lam <= 0.0
     if by_x:
