@@ -167,18 +167,83 @@ struct ScoreArgs {
   float inv_nq;
 };
 
-// One CTA per (b, KV group, tile of candidates).  Phase 1 writes, for every
-// head of the group over the tile plus a halo of w on each side, the
-// dominance key (s in fp32, or x when lambda = 0; NaN outside C: a NaN never
-// dominates).  Phase 2 finds every head's nearest dominator (two passes,
-// below).  Phase 3: the thread of a position applies soft-NMS to every head,
-// picks the owner and writes l''.
+// Phase 3 of one position: l' = ln(s + 1e-30) - alpha_soft * weight(d) of
+// every head (s = exp(x) when the key is x), the owner = the lowest head
+// within the tie tolerance of the largest l', and l'' = l' - alpha_cross off
+// the owner, written to outp[h * ld_s + k].
 template <int GM>
-__global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
+__device__ __forceinline__ void finish_position(const float (&kv)[GM], const int (&d)[GM], int G, bool by_x,
+                                                float alpha_soft, float alpha_cross, const float* wt,
+                                                float* outp, int64_t ld_s, int k) {
+  float l1[GM];
+  float M = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    l1[h] = -INFINITY;
+    if (h < G) {
+      const float sv = by_x ? fast_exp2(kv[h] * kLog2e) : kv[h];
+      l1[h] = logf(sv + 1e-30f) - alpha_soft * wt[d[h]];
+      M = fmaxf(M, l1[h]);
+    }
+  }
+  const float thr = M - kOwnerTie;
+  int owner = GM;
+#pragma unroll
+  for (int h = GM - 1; h >= 0; --h)
+    if (h < G && l1[h] >= thr) owner = h;
+#pragma unroll
+  for (int h = 0; h < GM; ++h)
+    if (h < G) outp[(size_t)h * ld_s + k] = l1[h] - (h != owner ? alpha_cross : 0.f);
+}
+
+// The GM keys of one position (16-byte loads for GM >= 4).
+template <int GM>
+__device__ __forceinline__ void load_keys(const float* p, float (&v)[GM]) {
+  if constexpr (GM >= 4) {
+#pragma unroll
+    for (int j = 0; j < GM / 4; ++j) {
+      const float4 t = reinterpret_cast<const float4*>(p)[j];
+      v[4 * j] = t.x;
+      v[4 * j + 1] = t.y;
+      v[4 * j + 2] = t.z;
+      v[4 * j + 3] = t.w;
+    }
+  } else if constexpr (GM == 2) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x;
+    v[1] = t.y;
+  } else {
+    v[0] = p[0];
+  }
+}
+
+template <int GM>
+__device__ __forceinline__ void store_keys(float* p, const float (&v)[GM]) {
+  if constexpr (GM >= 4) {
+#pragma unroll
+    for (int j = 0; j < GM / 4; ++j)
+      reinterpret_cast<float4*>(p)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else if constexpr (GM == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    p[0] = v[0];
+  }
+}
+
+// One CTA per (b, KV group, tile of candidates).  Phase 1 writes, for every
+// position of the tile plus a halo of w on each side, the dominance keys of
+// the group's heads side by side (s in fp32, or x when lambda = 0; NaN
+// outside C and for heads >= G: a NaN never dominates).  Phase 2: the thread
+// of a position finds every head's nearest dominator, distances 1..kNear for
+// all heads at once (one vector load per side and distance), then the
+// heads still without one alone, to w; phase 3 (finish_position) applies
+// soft-NMS, picks the owner and writes l''.
+template <int GM>
+__global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
   grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
-  float* key = sm;                    // [G][W] dominance key
+  float* key = sm;                    // [W][GM] dominance keys
   const int bg = blockIdx.y;                        // logical (row, kv head)
   const int bl = bg / a.Hkv, g = bg - bl * a.Hkv;
   const int b = a.rows.phys(bl);                    // the sequence
@@ -186,7 +251,6 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
   const int tile_n = min(a.tile, a.nC - c0);
   const int G = a.G;
   __shared__ double bc;
-  __shared__ int qn;
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
   const double inv_z = 1.0 / reduce_parts(pbg, a.nch, 1, &bc);
   const double* kpr = a.kp + (size_t)bg * a.kp_ld;
@@ -207,39 +271,39 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
     // x = ln f~ = m + ln(mean exp(x_i - m)), m the largest x_i
     for (int k = threadIdx.x; k < W; k += blockDim.x) {
       const int c = c0 - a.w + k;
-      if (c < 0 || c >= a.nC) {
+      float kv[GM];
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h < G) key[h * W + k] = nan;
-        continue;
-      }
-      const float r = (float)(kpr[c] * lam_r);   // lambda r_j
+      for (int h = 0; h < GM; ++h) kv[h] = nan;
+      if (c >= 0 && c < a.nC) {
+        const float r = (float)(kpr[c] * lam_r);   // lambda r_j
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-          float m = -INFINITY;
-          for (int i = 0; i < a.nq; ++i)
-            if ((a.qmask >> i) & 1u) {
-              const size_t row = (size_t)i * G + h;
-              m = fmaxf(m, z0[row * a.ld + c] - a.lse_cand[row0 + row]);
-            }
-          float acc = 0.f;
-          for (int i = 0; i < a.nq; ++i)
-            if ((a.qmask >> i) & 1u) {
-              const size_t row = (size_t)i * G + h;
-              acc += fast_exp2((z0[row * a.ld + c] - a.lse_cand[row0 + row] - m) * kLog2e);
-            }
-          const float x = m + logf(acc * a.inv_nq);
-          const float ft = fast_exp2(x * kLog2e);
-          key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
+        for (int h = 0; h < GM; ++h) {
+          if (h < G) {
+            float m = -INFINITY;
+            for (int i = 0; i < a.nq; ++i)
+              if ((a.qmask >> i) & 1u) {
+                const size_t row = (size_t)i * G + h;
+                m = fmaxf(m, z0[row * a.ld + c] - a.lse_cand[row0 + row]);
+              }
+            float acc = 0.f;
+            for (int i = 0; i < a.nq; ++i)
+              if ((a.qmask >> i) & 1u) {
+                const size_t row = (size_t)i * G + h;
+                acc += fast_exp2((z0[row * a.ld + c] - a.lse_cand[row0 + row] - m) * kLog2e);
+              }
+            const float x = m + logf(acc * a.inv_nq);
+            const float ft = fast_exp2(x * kLog2e);
+            kv[h] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
+          }
         }
       }
+      store_keys<GM>(key + (size_t)k * GM, kv);
     }
   }
   // kU positions per thread and round: all their loads are issued first
   constexpr int kU = GM >= 8 ? 2 : 4;
   for (int k0 = threadIdx.x; a.nq == 1 && k0 < W; k0 += kU * blockDim.x) {
-    double kv[kU];
+    double kp[kU];
     float zv[kU][GM];
     bool in[kU];
 #pragma unroll
@@ -247,7 +311,7 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
       const int c = c0 - a.w + k0 + u * blockDim.x;
       in[u] = k0 + u * blockDim.x < W && c >= 0 && c < a.nC;
       const int cc = in[u] ? c : 0;
-      kv[u] = in[u] ? kpr[cc] : 0.0;
+      kp[u] = in[u] ? kpr[cc] : 0.0;
 #pragma unroll
       for (int h = 0; h < GM; ++h) zv[u][h] = (in[u] && h < G) ? z0[(size_t)h * a.ld + cc] : 0.f;
     }
@@ -255,124 +319,68 @@ __global__ void __launch_bounds__(256, 2) select_scores_kernel(const __grid_cons
     for (int u = 0; u < kU; ++u) {
       const int k = k0 + u * blockDim.x;
       if (k >= W) continue;
-      if (in[u]) {
-        const float r = (float)(kv[u] * lam_r);   // lambda r_j
-#pragma unroll
-        for (int h = 0; h < GM; ++h) {
-          if (h < G) {
-            // exp through the hardware's base-2 approximation (relative
-            // error ~1e-7, below the error of the logits themselves)
-            const float x = zv[u][h] - lsec[h];
-            const float ft = fast_exp2(x * kLog2e);
-            key[h * W + k] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h < G) key[h * W + k] = nan;
-      }
-    }
-  }
-  if (threadIdx.x == 0) qn = 0;
-  __syncthreads();
-  // Phase 2a: distances 1..kNear of every head for every position (no early
-  // exit, so a warp does not wait for its local maxima); positions with a head
-  // still undecided go to a queue.  2b: the queue, scanned to w with all lanes
-  // busy.  dom = distance of the nearest dominator, 0: none within w.
-  constexpr int kNear = 4;
-  uint16_t* dom = reinterpret_cast<uint16_t*>(key + G * W);              // [G][tile]
-  uint32_t* queue = reinterpret_cast<uint32_t*>(dom + G * a.tile);       // [tile]
-  const int lane = threadIdx.x & 31;
-  for (int k0 = 0; k0 < tile_n; k0 += blockDim.x) {
-    const int k = k0 + threadIdx.x;
-    uint32_t open = 0u;
-    if (k < tile_n) {
+      float kv[GM];
+      const float r = (float)(kp[u] * lam_r);   // lambda r_j
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-          const float* row = key + h * W + a.w + k;
-          const float e = row[0];
-          int d_hit = 0;
-#pragma unroll
-          for (int d = kNear; d >= 1; --d) {   // descending: the nearest hit stays
-            const int dd = min(d, a.w);
-            if (d <= a.w && (row[-dd] >= e || row[dd] > e)) d_hit = d;   // NaN compares false
-          }
-          dom[h * a.tile + k] = (uint16_t)d_hit;
-          if (d_hit == 0 && a.w > kNear) open |= 1u << h;
-        }
+        // exp through the hardware's base-2 approximation (relative error
+        // ~1e-7, below the error of the logits themselves)
+        const float x = zv[u][h] - lsec[h];
+        const float ft = fast_exp2(x * kLog2e);
+        kv[h] = (in[u] && h < G) ? (by_x ? x : fmaf(a.one_minus_lam, ft, r)) : nan;
       }
-    }
-    const unsigned ball = __ballot_sync(0xffffffffu, open != 0u);
-    if (ball) {
-      int base = 0;
-      if (lane == 0) base = atomicAdd(&qn, __popc(ball));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (open) queue[base + __popc(ball & ((1u << lane) - 1u))] = (uint32_t)k | (open << 16);
+      store_keys<GM>(key + (size_t)k * GM, kv);
     }
   }
   __syncthreads();
-  const int nqueue = qn;
-  for (int qi = threadIdx.x; qi < nqueue; qi += blockDim.x) {
-    const uint32_t ent = queue[qi];
-    const int k = (int)(ent & 0xffffu);
-    uint32_t open = ent >> 16;
-    while (open) {
-      const int h = __ffs(open) - 1;
-      open &= open - 1u;
-      const float* row = key + h * W + a.w + k;
-      const float e = row[0];
-      int d_hit = 0;
-      for (int d = kNear + 1; d <= a.w; ++d) {
-        if (row[-d] >= e || row[d] > e) {
-          d_hit = d;
-          break;
-        }
-      }
-      dom[h * a.tile + k] = (uint16_t)d_hit;
-    }
-  }
-  __syncthreads();
-  // Phase 3: l' = ln(s + 1e-30) - alpha_soft * weight(d); the owner is the
-  // lowest head within the tie tolerance of the largest l'.
+  // Phases 2 and 3.  dh = distance of the nearest dominator, 0: none within w.
+  constexpr int kNear = 4;
+  const int near = min(kNear, a.w);
+  float* outp = a.scores + ((size_t)bl * a.Hq + (size_t)g * G) * a.ld_s + c0;
   for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
-    float l1[GM];
-    float M = -INFINITY;
+    const float* row = key + (size_t)(a.w + k) * GM;
+    float e[GM];
+    int dh[GM];
+    load_keys<GM>(row, e);
 #pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      l1[h] = -INFINITY;
-      if (h < G) {
-        const int d = dom[h * a.tile + k];
-        const float kv = key[h * W + a.w + k];
-        const float sv = by_x ? fast_exp2(kv * kLog2e) : kv;
-        l1[h] = logf(sv + 1e-30f) - a.alpha_soft * wt[d];
-        M = fmaxf(M, l1[h]);
+    for (int h = 0; h < GM; ++h) dh[h] = 0;
+#pragma unroll
+    for (int d = 1; d <= kNear; ++d) {
+      if (d > near) break;
+      float lv[GM], rv[GM];
+      load_keys<GM>(row - d * GM, lv);
+      load_keys<GM>(row + d * GM, rv);
+#pragma unroll
+      for (int h = 0; h < GM; ++h)   // a left neighbour dominates on ties; NaN compares false
+        if (dh[h] == 0 && (lv[h] >= e[h] || rv[h] > e[h])) dh[h] = d;
+    }
+    if (a.w > kNear) {
+      // the heads still without a dominator (about 1 % of positions): alone, to w
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G && dh[h] == 0) {
+          for (int d = kNear + 1; d <= a.w; ++d) {
+            if (row[h - d * GM] >= e[h] || row[h + d * GM] > e[h]) {
+              dh[h] = d;
+              break;
+            }
+          }
+        }
       }
     }
-    const float thr = M - kOwnerTie;
-    int owner = GM;
-#pragma unroll
-    for (int h = GM - 1; h >= 0; --h)
-      if (h < G && l1[h] >= thr) owner = h;
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      if (h < G) {
-        const float v = l1[h] - (h != owner ? a.alpha_cross : 0.f);
-        a.scores[((size_t)bl * a.Hq + (size_t)g * G + h) * a.ld_s + c0 + k] = v;
-      }
-    }
+    finish_position<GM>(e, dh, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
   }
 }
 
 // ---------------------------------------------------------------- host
 int score_tile(int G) { return std::max(256, 4096 / G); }
 
-// dominance keys with halo, nearest-dominator distances, queue of undecided
-// positions
+// dominance keys of the tile with its halo, GM (G rounded up to a power of
+// two) per position
 size_t score_smem(int G, int tile, int w) {
-  return (size_t)G * (tile + 2 * w) * sizeof(float) + (size_t)G * tile * sizeof(uint16_t) +
-         (size_t)tile * sizeof(uint32_t);
+  int gm = 1;
+  while (gm < G) gm *= 2;
+  return (size_t)gm * (tile + 2 * w) * sizeof(float);
 }
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }

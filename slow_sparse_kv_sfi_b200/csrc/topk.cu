@@ -4,19 +4,22 @@
 //
 // Exact MSB radix select on the order-preserving uint32 image of every fp32
 // score, one thread-block cluster per row.  The row is cut into slices of
-// T * 32 scores, one CTA of T threads each (up to 8 CTAs, cluster rank =
-// slice), and every thread keeps its 32 keys in registers for the whole
+// T * 32 scores, one CTA of T threads each (1, 2, 4 or 8 CTAs, cluster rank
+// = slice), and every thread keeps its 32 keys in registers for the whole
 // kernel, so the scores are read once:
-//   1. the cluster's smallest and largest key: their common leading bits are
-//      every key's, so the digit passes cover only the bits below the highest
-//      one where they differ, in as few passes of at most 14 bits as cover
-//      them (rows of log-scores share sign and most of the exponent: two);
+//   1. the cluster's smallest and largest key: the passes work on the offset
+//      key - smallest, whose bits above the highest bit of (largest -
+//      smallest) are zero, in as few passes of at most 14 bits as cover the
+//      rest (a row of log-scores spans about 2^26 keys: two passes, where the
+//      keys' own leading bits would need three once the scores straddle a
+//      power of two);
 //   2. per digit pass: each CTA builds the histogram of its keys that match
 //      the prefix found so far in shared memory; after a cluster barrier CTA
 //      c sums bins [c * per, (c + 1) * per) over every CTA's histogram through
-//      distributed shared memory; after a second barrier every CTA reads the
-//      range totals and the reduced bins of the range holding the remaining
-//      k-th largest key, and extends the prefix by that bin;
+//      distributed shared memory (the CS loads of a bin issued together);
+//      after a second barrier every CTA reads the range totals (one lane per
+//      CTA), copies the reduced bins of the range holding the remaining k-th
+//      largest key and extends the prefix by that bin;
 //   3. the prefix is now the threshold key T: keys above it are selected,
 //      keys equal to it are ties, taken in position order (a cluster-wide
 //      exclusive count of the ties in lower slices) until K are chosen.
@@ -116,24 +119,47 @@ __host__ __device__ constexpr size_t topk_smem_bytes(int cs) {
   return (size_t)kDigitBins * 4 + (cs > 1 ? (size_t)((kDigitBins + cs - 1) / cs) * 4 : 0);
 }
 
-template <int T>
+// Reads one int that every CTA of the cluster published at `pub` (lanes c <
+// CS of the calling warp read CTA c's) and returns this lane's value; lanes
+// >= CS get 0.
+template <int CS>
+__device__ __forceinline__ int read_published(cg::cluster_group& cl, int* pub, int lane) {
+  if (lane >= CS) return 0;
+  if constexpr (CS > 1) return cl.map_shared_rank(pub, lane)[0];
+  return pub[0];
+}
+
+// Sum of the values published by the CTAs of ranks below `rank` (warp 0).
+template <int CS>
+__device__ __forceinline__ int published_before(cg::cluster_group& cl, int* pub, int lane, int rank) {
+  int v = read_published<CS>(cl, pub, lane);
+  v = lane < rank ? v : 0;
+#pragma unroll
+  for (int sh = 16; sh >= 1; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
+  return v;
+}
+
+template <int T, int CS>
 __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__ TopkArgs a) {
   grid_dep_enter();
   cg::cluster_group cl = cg::this_cluster();
-  const int cs = (int)cl.num_blocks();
-  const int rank = (int)cl.block_rank();
+  const int rank = CS > 1 ? (int)cl.block_rank() : 0;
   const int row = blockIdx.y;
   const int s0 = rank * T * kKPT;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   extern __shared__ int dyn[];
-  int* hist = dyn;                                   // [2^nbits] this CTA's digit counts
-  int* red = cs > 1 ? dyn + kDigitBins : dyn;        // this CTA's range, summed over the cluster
+  int* hist = dyn;                  // [2^nbits] this CTA's digit counts; then a copy of the chosen range
+  int* red = dyn + kDigitBins;      // this CTA's range, summed over the cluster (CS > 1)
   __shared__ uint32_t selw[T], tiew[T];
   __shared__ int ws[33];
   __shared__ uint32_t wsu[32];
-  __shared__ int pub[4];            // published to the cluster: range total, ties, selected
-  __shared__ int s_pick[3];         // bin, keys above it, k
+  __shared__ int pub[3];            // published to the cluster: range total, ties, selected
+  __shared__ int s_pick[3];         // range / bin, keys above it, k
   __shared__ uint32_t s_mm[2];
+  auto csync = [&]() {
+    if constexpr (CS > 1) cl.sync();
+    else __syncthreads();
+  };
 
   // ---- keys
   const float* srow = a.scores + (size_t)row * a.ld_s;
@@ -158,7 +184,7 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
         key[u][e] = j < a.n ? float_key(__ldg(srow + j)) : 0u;
       }
   }
-  // ---- 1. common leading bits of the whole row
+  // ---- 1. smallest and largest key of the row
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int u = 0; u < 8; ++u)
@@ -174,24 +200,38 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     s_mm[0] = kmin;
     s_mm[1] = kmax;
   }
-  cl.sync();
-  if (threadIdx.x == 0) {
+  csync();
+  if (warp == 0) {
     uint32_t lo = 0xffffffffu, hi = 0u;
-    for (int c = 0; c < cs; ++c) {
-      const uint32_t* r = cl.map_shared_rank(s_mm, c);
-      lo = min(lo, r[0]);
-      hi = max(hi, r[1]);
+    if (lane < CS) {
+      const uint32_t* r = s_mm;
+      if constexpr (CS > 1) r = cl.map_shared_rank(s_mm, lane);
+      lo = r[0];
+      hi = r[1];
     }
-    wsu[0] = lo;
-    wsu[1] = hi;
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, sh));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, sh));
+    }
+    if (lane == 0) {
+      wsu[0] = lo;
+      wsu[1] = hi;
+    }
   }
   __syncthreads();
   const uint32_t gmin = wsu[0], gmax = wsu[1];
-  // hb: highest bit where the row's keys differ (-1: all equal)
-  const int hb = gmin == gmax ? -1 : 31 - __clz((int)(gmin ^ gmax));
+  // the passes work on off = key - gmin in [0, gmax - gmin]; hb: its highest
+  // bit that can be set (-1: all keys equal)
+  const uint32_t span = gmax - gmin;
+  const int hb = span == 0u ? -1 : 31 - __clz((int)span);
   uint32_t pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
-  uint32_t prefix = gmax & pmask;
+  uint32_t prefix = 0u;
   int k = a.K;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) key[u][e] -= gmin;
 
   // ---- 2. digit passes over bits hb .. 0, as few as cover them, balanced
   const int npass = (hb + 1 + kDigitBits - 1) / kDigitBits;
@@ -209,58 +249,81 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     for (int u = 0; u < 8; ++u)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint32_t kk = key[u][e];
-        if (pos_of<T>(s0, u, e) < a.n && (kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & dm], 1);
+        const uint32_t off = key[u][e];
+        if (pos_of<T>(s0, u, e) < a.n && (off & pmask) == prefix) atomicAdd(&hist[(off >> shift) & dm], 1);
       }
-    cl.sync();   // every histogram of the cluster complete
-    // this CTA's bin range, summed over the cluster (one CTA: its own histogram)
-    const int per = (nb + cs - 1) / cs;
-    const int r0 = rank * per;
+    csync();   // every histogram of the cluster complete
+    // this CTA's bin range, summed over the cluster: the CS loads of a bin
+    // are issued together
+    const int per = (nb + CS - 1) / CS;
     int mine = 0;
-    for (int i = threadIdx.x; i < per; i += T) {
-      const int bin = r0 + i;
-      int s = 0;
-      if (cs == 1) {
-        s = hist[i];
-      } else if (bin < nb) {
-        for (int c = 0; c < cs; ++c) s += cl.map_shared_rank(hist, c)[bin];
-        red[i] = s;
+    if constexpr (CS == 1) {
+      for (int i = threadIdx.x; i < nb; i += T) mine += hist[i];
+    } else {
+      const int* hs[CS];
+#pragma unroll
+      for (int c = 0; c < CS; ++c) hs[c] = cl.map_shared_rank(hist, c);
+      const int r0 = rank * per;
+      for (int i = threadIdx.x; i < per; i += T) {
+        const int bin = r0 + i;
+        int sum = 0;
+        if (bin < nb) {
+          int v[CS];
+#pragma unroll
+          for (int c = 0; c < CS; ++c) v[c] = hs[c][bin];
+#pragma unroll
+          for (int c = 0; c < CS; ++c) sum += v[c];
+        }
+        red[i] = sum;
+        mine += sum;
       }
-      mine += s;
     }
     int tot;
     block_excl<T>(mine, ws, &tot);
     if (threadIdx.x == 0) pub[0] = tot;
-    cl.sync();   // every range reduced
-    // the range holding the k-th largest key (ranges of higher bins first),
-    // then the bin inside it: every CTA does this on the same data
-    if (threadIdx.x == 0) {
-      int above = 0, c = cs - 1;
-      for (; c > 0; --c) {
-        const int t = cl.map_shared_rank(pub, c)[0];
-        if (above + t >= k) break;
-        above += t;
+    csync();   // every range reduced and published
+    // the range holding the k-th largest key (ranges of higher bins first):
+    // the highest rank whose suffix total reaches k
+    if (warp == 0) {
+      const int t = read_published<CS>(cl, pub, lane);
+      int suf = t;
+#pragma unroll
+      for (int sh = 1; sh < 32; sh <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, suf, sh);
+        if (lane + sh < 32) suf += y;
       }
-      s_pick[0] = c;
-      s_pick[1] = above;
+      const unsigned bal = __ballot_sync(0xffffffffu, lane < CS && suf >= k);
+      const int c = bal ? 31 - __clz((int)bal) : 0;
+      const int above = __shfl_sync(0xffffffffu, suf - t, c);
+      if (lane == 0) {
+        s_pick[0] = c;
+        s_pick[1] = above;
+      }
     }
     __syncthreads();
     const int cr = s_pick[0];
     const int above_r = s_pick[1];
-    const int* rred = cl.map_shared_rank(red, cr);
-    const int nr = min(per, nb - cr * per);
+    const int nr = CS == 1 ? nb : min(per, nb - cr * per);
+    if constexpr (CS > 1) {
+      // every CTA is past its reads of this CTA's histogram: the chosen
+      // range is copied into it
+      const int* src = cl.map_shared_rank(red, cr);
+#pragma unroll 4
+      for (int i = threadIdx.x; i < nr; i += T) hist[i] = src[i];
+      __syncthreads();
+    }
     // thread t takes bins [t * bp, (t + 1) * bp) of the range; suffix counts
     const int bp = (nr + T - 1) / T;
     const int b0 = threadIdx.x * bp;
     int part = 0;
     for (int i = 0; i < bp; ++i)
-      if (b0 + i < nr) part += rred[b0 + i];
+      if (b0 + i < nr) part += hist[b0 + i];
     int sum_all;
     const int before = block_excl<T>(part, ws, &sum_all);   // bins below this thread's
     int above = above_r + (sum_all - before - part);         // keys in higher bins of the range
     for (int i = bp - 1; i >= 0; --i) {
       if (b0 + i >= nr) continue;
-      const int h = rred[b0 + i];
+      const int h = hist[b0 + i];
       if (above < k && above + h >= k) {
         s_pick[0] = cr * per + b0 + i;
         s_pick[2] = above;
@@ -274,8 +337,9 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     done_bits += nbits;
     __syncthreads();
   }
-  // ---- 3. keys above the threshold, ties in position order
-  const uint32_t thr = hb < 0 ? gmin : prefix;
+  // ---- 3. keys above the threshold, ties in position order (offset keys:
+  // the threshold is the prefix; all keys equal: every key is a tie)
+  const uint32_t thr = prefix;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int jb = pos_of<T>(s0, u, 0);
@@ -283,8 +347,9 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (jb + e < a.n) {
-        up |= (key[u][e] > thr ? 1u : 0u) << e;
-        eq |= (key[u][e] == thr ? 1u : 0u) << e;
+        const uint32_t off = key[u][e];
+        up |= (off > thr ? 1u : 0u) << e;
+        eq |= (off == thr ? 1u : 0u) << e;
       }
     }
     // the word of lanes 8q .. 8q + 7: nibble (lane & 7) of word q
@@ -307,11 +372,10 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   int ties_tot;
   const int tie_before_local = block_excl<T>(__popc(tw), ws, &ties_tot);
   if (threadIdx.x == 0) pub[1] = ties_tot;
-  cl.sync();
-  if (threadIdx.x == 0) {
-    int s = 0;
-    for (int c = 0; c < rank; ++c) s += cl.map_shared_rank(pub, c)[1];
-    s_pick[1] = s;
+  csync();
+  if (warp == 0) {
+    const int sb = published_before<CS>(cl, pub + 1, lane, rank);
+    if (lane == 0) s_pick[1] = sb;
   }
   __syncthreads();
   int rk = s_pick[1] + tie_before_local;
@@ -330,11 +394,10 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     int sel_tot;
     const int sel_before_local = block_excl<T>(__popc(sw), ws, &sel_tot);
     if (threadIdx.x == 0) pub[2] = sel_tot;
-    cl.sync();
-    if (threadIdx.x == 0) {
-      int s = 0;
-      for (int c = 0; c < rank; ++c) s += cl.map_shared_rank(pub, c)[2];
-      s_pick[1] = s;
+    csync();
+    if (warp == 0) {
+      const int sb = published_before<CS>(cl, pub + 2, lane, rank);
+      if (lane == 0) s_pick[1] = sb;
     }
     __syncthreads();
     int at = s_pick[1] + sel_before_local;
@@ -347,32 +410,39 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
       ++at;
     }
   }
-  cl.sync();   // no CTA leaves while another may still read its shared memory
+  if constexpr (CS > 1) cl.sync();   // no CTA leaves while another may still read its shared memory
 }
 
-template <int T>
-sfi_status launch_topk(const TopkArgs& a, int cs, cudaStream_t st) {
+template <int T, int CS>
+sfi_status launch_topk(const TopkArgs& a, cudaStream_t st) {
   static DeviceOnce smem_attr;
-  if (!smem_attr.done() && !smem_attr.mark(cudaFuncSetAttribute(topk_cluster_kernel<T>,
+  if (!smem_attr.done() && !smem_attr.mark(cudaFuncSetAttribute(topk_cluster_kernel<T, CS>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      (int)topk_smem_bytes(2))))
+                                                      (int)topk_smem_bytes(CS))))
     return SFI_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs, a.rows);
+  cfg.gridDim = dim3(CS, a.rows);
   cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = topk_smem_bytes(cs);
+  cfg.dynamicSmemBytes = topk_smem_bytes(CS);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.x = CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T>, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T, CS>, a);
   return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+}
+
+template <int CS>
+sfi_status launch_topk_cs(const TopkArgs& a, int threads, cudaStream_t st) {
+  if (threads <= 256) return launch_topk<256, CS>(a, st);
+  if (threads <= 512) return launch_topk<512, CS>(a, st);
+  return launch_topk<1024, CS>(a, st);
 }
 
 }  // namespace
@@ -396,12 +466,20 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
   a.ld_b = ld_b;
   a.idx = idx;
   a.ld_i = ld_i;
-  // slices of T * 32 scores: at most 8 per row, the fewest threads that cover it
-  const int cs = std::min(kMaxCluster, (n + 256 * kKPT - 1) / (256 * kKPT));
+  // slices of T * 32 scores: the fewest CTAs of up to 1024 threads that
+  // cover the row, a power of two of them, at most 4 while that suffices.
+  // A cluster's CTAs land on distinct SMs of one GPC and a CTA of 1024
+  // threads fills an SM's registers, so clusters of 4 run about twice as
+  // many at once as clusters of 8 of 512-thread CTAs.
+  int cs = 1;
+  while (cs < kMaxCluster && cs * 1024 * kKPT < n) cs *= 2;
   const int need = (n + cs * kKPT - 1) / (cs * kKPT);   // threads per slice
-  if (need <= 256) return launch_topk<256>(a, cs, st);
-  if (need <= 512) return launch_topk<512>(a, cs, st);
-  return launch_topk<1024>(a, cs, st);
+  switch (cs) {
+    case 1: return launch_topk_cs<1>(a, need, st);
+    case 2: return launch_topk_cs<2>(a, need, st);
+    case 4: return launch_topk_cs<4>(a, need, st);
+    default: return launch_topk_cs<8>(a, need, st);
+  }
 }
 
 }  // namespace sfi

@@ -85,7 +85,9 @@ S_ROUND = 2.0 ** -23
 MAX_UNDECIDED_SHARE = 0.06
 MIN_UNDECIDED_ALLOWED = 3
 # Picks allowed to differ from the oracle's point selection: this share of K,
-# and at least MIN_DIFFERING_ALLOWED.
+# at least MIN_DIFFERING_ALLOWED, and at least a quarter of the head's
+# undecided candidates (a differing pick is always an undecided candidate,
+# and at most half of them can differ: as many leave the set as enter it).
 MAX_DIFFERING_SHARE = 0.001
 MIN_DIFFERING_ALLOWED = 3
 
@@ -253,8 +255,8 @@ def check_selection(gpu_sel, bounds, K: int, lo: int, what: str = "", gpu_scores
         comparisons fall is chosen, and none that is out either way;
       * undecided candidates are at most MAX_UNDECIDED_SHARE of K (at least
         MIN_UNDECIDED_ALLOWED);
-      * at most max(MAX_DIFFERING_SHARE * K, MIN_DIFFERING_ALLOWED) picks
-        differ from the oracle's own selection;
+      * at most max(MAX_DIFFERING_SHARE * K, MIN_DIFFERING_ALLOWED, undecided
+        / 4) picks differ from the oracle's own selection;
       * (gpu_scores given) every GPU score lies in its interval.
     Records (undecided, overlap, differing picks) in SELECTION_RECORD and
     returns the worst overlap."""
@@ -287,7 +289,7 @@ def check_selection(gpu_sel, bounds, K: int, lo: int, what: str = "", gpu_scores
         SELECTION_RECORD.append((_CURRENT_TEST["name"], what, h, K, undecided, ov, K - common))
         cap = max(int(MAX_UNDECIDED_SHARE * K), MIN_UNDECIDED_ALLOWED)
         assert undecided <= cap, f"{what}: head {h}: {undecided} undecided candidates (cap {cap})"
-        allowed = max(int(np.ceil(MAX_DIFFERING_SHARE * K)), MIN_DIFFERING_ALLOWED)
+        allowed = max(int(np.ceil(MAX_DIFFERING_SHARE * K)), MIN_DIFFERING_ALLOWED, undecided // 4)
         assert K - common <= allowed, f"{what}: head {h}: {K - common} picks differ from the oracle's (allowed {allowed})"
     return worst
 

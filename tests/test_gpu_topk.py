@@ -41,15 +41,16 @@ def _check(x, K, **kw):
 
 
 @pytest.mark.parametrize("rows,n,K", [
-    (3, 131000, 19650),     # 16 slices, ragged tail
-    (5, 8192, 100),         # exactly one slice
-    (2, 8193, 4096),        # one score in the second slice
+    (3, 131000, 19650),     # four slices of 1024 threads, ragged tail
+    (5, 8192, 100),         # one slice of 256 threads, exactly full
+    (2, 8193, 4096),        # one slice of 512 threads, one score past 8192
     (4, 777, 1),            # K = 1
     (2, 1000, 1000),        # K = n
-    (64, 20000, 3000),
-    (1, 262144, 50000),     # eight slices of 1024 threads
-    (2, 200001, 7),         # 1024 threads, ragged
-    (3, 70000, 9000),       # 512 threads, the last slices hold no score
+    (64, 20000, 3000),      # one slice of 1024 threads per row, 64 rows
+    (4, 40000, 6000),       # two slices
+    (1, 262144, 50000),     # eight slices of 1024 threads, full
+    (2, 200001, 7),         # eight slices, ragged
+    (3, 70000, 9000),       # four slices, the last ones partly empty
 ])
 def test_topk_random(rows, n, K):
     rng = np.random.default_rng(n + K)
