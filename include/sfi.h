@@ -138,12 +138,16 @@ typedef struct {
   int32_t cand_lo, cand_hi;
 } sfi_dense_extras;
 
+/* Text of a status code (static storage).  A utility of this library, no
+ * step of the pages. */
 const char* sfi_status_str(sfi_status s);
 
-/* Library version string (static storage). */
+/* Library version string (static storage).  A utility, no step of the pages. */
 const char* sfi_version(void);
 
-/* Bytes of scratch the per-op calls below need for contexts up to
+/* Sizing calls (this and the next two): no step of the pages, they size the
+ * caller's allocations for the steps below.
+ * Bytes of scratch the per-op calls below need for contexts up to
  * L_max = max_pages * 16 tokens.  Pass at least that much as ws/ws_bytes
  * (16-byte aligned).  Ownership stays with the caller.  The scratch must be
  * zero-filled before its first use (the first 256 bytes hold a work counter
@@ -215,7 +219,10 @@ sfi_status sfi_dense_attn_noalloc(const sfi_shape* shape, const sfi_paged_kv* kv
                                   const sfi_bf16* q, float* out, const sfi_dense_extras* extras,
                                   sfi_stream stream);
 
-/* f = exp(logits - lse) over j < L for every (b, hq) row. */
+/* f = exp(logits - lse) over j < L for every (b, hq) row: the attention
+ * distribution itself, which [ZH] §2.2 names as the Selector's input (this
+ * library's Selector reads the logits and lse_cand instead).  For callers
+ * that want f; not on the decode path. */
 sfi_status sfi_attn_probs(const sfi_shape* shape, int32_t L, const float* logits, int64_t ld,
                           const float* lse, float* probs, sfi_stream stream);
 
@@ -258,13 +265,13 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
  * n <= 262144, rows <= 65535.  The top-K keeps its state on chip and needs
  * no scratch: sfi_topk_workspace_size reports 0 and ws may be null (a
  * ws_bytes below the reported size is refused).  Exact radix select over
- * order-preserving 32-bit keys of the scores, one thread-block cluster of up
- * to 8 CTAs per row, each CTA holding its slice's keys in registers: the
- * digit passes start at the highest bit where the row's smallest and largest
- * keys differ (12 bits per pass), CTA histograms meet in distributed shared
- * memory, and the ties at the threshold are taken in position order.  Not a
- * step the pages describe in detail: the Top-K of gist.science/fr
- * "B. Le Sélecteur" and gist.science/zh "2.2" (Top-K 选择). */
+ * order-preserving 32-bit keys of the scores, one thread-block cluster of 1,
+ * 2, 4 or 8 CTAs (of up to 1024 threads) per row, each CTA holding its
+ * slice's keys in registers: the digit passes run over key - smallest key,
+ * from the highest bit of (largest - smallest), at most 14 bits per pass; CTA
+ * histograms meet in distributed shared memory, and the ties at the
+ * threshold are taken in position order.  The pages name the step and give
+ * no method: the Top-K of [FR] "B. Le Sélecteur" and [ZH] §2.2. */
 sfi_status sfi_topk_workspace_size(int32_t rows, int32_t n, size_t* bytes);
 sfi_status sfi_topk(int32_t rows, int32_t n, const float* scores, int64_t ld_s, int32_t K,
                     int32_t offset, int32_t* idx, int64_t ld_i, void* ws, size_t ws_bytes,
