@@ -117,13 +117,14 @@ __global__ void __launch_bounds__(kStatThreads) stats_norm_kernel(int L, int lo,
   if (threadIdx.x == 0) part[((size_t)bg * nch + blockIdx.x) * 2] = t;
 }
 
-// part[bgl][chunk][1] = sum of kappa * pi over the chunk of C, and
-// kp[bgl][c] = kappa_j pi_j (j = lo + c) for the score kernel
+// part[bgl][chunk][1] = sum of kappa * pi over the chunk of C (fp64), and
+// kp[bgl][c] = kappa_j pi_j (j = lo + c) rounded once to fp32 for the score
+// kernel, which multiplies it by lambda / Z in fp32
 __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo, int nC,
                                                                    const float* __restrict__ norms,
                                                                    int64_t norm_ld, double* part, int nch, int Hkv,
                                                                    const double* __restrict__ pitab,
-                                                                   double* __restrict__ kp, int64_t kp_ld,
+                                                                   float* __restrict__ kp, int64_t kp_ld,
                                                                    const __grid_constant__ RowMap rows) {
   grid_dep_enter();
   __shared__ double red[32];
@@ -134,11 +135,11 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
   const float* n = norm_row(norms, norm_ld, rows, Hkv, bg);
   const int c0 = blockIdx.x * kStatChunk, c1 = min(nC, c0 + kStatChunk);
   double z = 0.0;
-  double* kpr = kp + (size_t)bg * kp_ld;
+  float* kpr = kp + (size_t)bg * kp_ld;
   for (int c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
     const int j = lo + c;
     const double v = kappa_of(nbar, n[j]) * pitab[c];
-    kpr[c] = v;
+    kpr[c] = (float)v;
     z += v;
   }
   const double t = block_sum_d(z, red);
@@ -155,7 +156,7 @@ struct ScoreArgs {
   const float* lse_cand;
   const double* stat_part;   // [B*Hkv][nch][2]
   int nch;
-  const double* kp;          // [B*Hkv][kp_ld] kappa_j pi_j of the candidates
+  const float* kp;           // [B*Hkv][kp_ld] kappa_j pi_j of the candidates (fp32)
   int64_t kp_ld;
   float* scores;         // logical rows of the launch
   int64_t ld_s;
@@ -253,9 +254,9 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
   __shared__ double bc;
   const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
   const double inv_z = 1.0 / reduce_parts(pbg, a.nch, 1, &bc);
-  const double* kpr = a.kp + (size_t)bg * a.kp_ld;
+  const float* kpr = a.kp + (size_t)bg * a.kp_ld;
   const bool by_x = a.lam <= 0.0;          // lambda = 0: s = f~, decided on x
-  const double lam_r = a.lam * inv_z;      // lambda / Z
+  const float lam_r = (float)(a.lam * inv_z);   // lambda / Z, rounded once
   __shared__ float wt[64];                 // soft-NMS weight of a nearest dominator at distance d
   for (int d = threadIdx.x; d <= a.w && d < 64; d += blockDim.x)
     wt[d] = d > 0 ? 1.f - (float)(d - 1) / (float)a.w : 0.f;
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
 #pragma unroll
       for (int h = 0; h < GM; ++h) kv[h] = nan;
       if (c >= 0 && c < a.nC) {
-        const float r = (float)(kpr[c] * lam_r);   // lambda r_j
+        const float r = kpr[c] * lam_r;   // lambda r_j
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
           if (h < G) {
@@ -303,7 +304,7 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
   // kU positions per thread and round: all their loads are issued first
   constexpr int kU = GM >= 8 ? 2 : 4;
   for (int k0 = threadIdx.x; a.nq == 1 && k0 < W; k0 += kU * blockDim.x) {
-    double kp[kU];
+    float kp[kU];
     float zv[kU][GM];
     bool in[kU];
 #pragma unroll
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
       const int c = c0 - a.w + k0 + u * blockDim.x;
       in[u] = k0 + u * blockDim.x < W && c >= 0 && c < a.nC;
       const int cc = in[u] ? c : 0;
-      kp[u] = in[u] ? kpr[cc] : 0.0;
+      kp[u] = in[u] ? kpr[cc] : 0.f;
 #pragma unroll
       for (int h = 0; h < GM; ++h) zv[u][h] = (in[u] && h < G) ? z0[(size_t)h * a.ld + cc] : 0.f;
     }
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
       const int k = k0 + u * blockDim.x;
       if (k >= W) continue;
       float kv[GM];
-      const float r = (float)(kp[u] * lam_r);   // lambda r_j
+      const float r = kp[u] * lam_r;   // lambda r_j
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         // exp through the hardware's base-2 approximation (relative error
@@ -399,11 +400,12 @@ sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_
 namespace {
 
 // The statistics area: partial sums, then the position factors, then
-// kappa * pi of every candidate of every row.
+// kappa * pi (fp32) of every candidate of every row.
 struct StatLayout {
   int nb, nC, nch;
   int64_t kp_ld;
-  double *part, *pitab, *kp;
+  double *part, *pitab;
+  float* kp;
   StatLayout(const sfi_shape& s, const sfi_params& p, int L, const RowMap& rows, void* ws) {
     nb = rows.count(s.B);
     nC = L - p.n_recent - p.n_sink;
@@ -411,7 +413,7 @@ struct StatLayout {
     kp_ld = (nC + 1) / 2 * 2;
     part = reinterpret_cast<double*>(ws);
     pitab = part + (size_t)nb * s.Hkv * nch * 2;
-    kp = pitab + kp_ld;
+    kp = reinterpret_cast<float*>(pitab + kp_ld);
   }
 };
 
@@ -450,7 +452,7 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
     if (r != SFI_OK) return r;
   }
   double* part = sl.part;
-  double* kp = sl.kp;
+  float* kp = sl.kp;
   const int64_t kp_ld = sl.kp_ld;
   ScoreArgs a{};
   a.L = L; a.lo = lo; a.nC = nC; a.Hq = s.Hq; a.Hkv = s.Hkv; a.G = G;

@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   __shared__ int ws[33];
   __shared__ uint32_t wsu[32];
   __shared__ int pub[3];            // published to the cluster: range total, ties, selected
-  __shared__ int s_pick[3];         // range / bin, keys above it, k
+  __shared__ int s_pick[4];         // range / bin, keys above it, k, keys in the bin
   __shared__ uint32_t s_mm[2];
   auto csync = [&]() {
     if constexpr (CS > 1) cl.sync();
@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
       if (above < k && above + h >= k) {
         s_pick[0] = cr * per + b0 + i;
         s_pick[2] = above;
+        s_pick[3] = h;
       }
       above += h;
     }
@@ -338,8 +339,11 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     __syncthreads();
   }
   // ---- 3. keys above the threshold, ties in position order (offset keys:
-  // the threshold is the prefix; all keys equal: every key is a tie)
+  // the threshold is the prefix; all keys equal: every key is a tie).  The
+  // last pass's bin holds exactly the keys equal to the threshold: when all
+  // of them are taken no cluster-wide count of ties is needed.
   const uint32_t thr = prefix;
+  const bool take_all_ties = (hb < 0 ? a.n : s_pick[3]) == k;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int jb = pos_of<T>(s0, u, 0);
@@ -369,22 +373,26 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   // thread i owns word i of the slice (words are in position order)
   const int i = threadIdx.x;
   const uint32_t tw = tiew[i];
-  int ties_tot;
-  const int tie_before_local = block_excl<T>(__popc(tw), ws, &ties_tot);
-  if (threadIdx.x == 0) pub[1] = ties_tot;
-  csync();
-  if (warp == 0) {
-    const int sb = published_before<CS>(cl, pub + 1, lane, rank);
-    if (lane == 0) s_pick[1] = sb;
-  }
-  __syncthreads();
-  int rk = s_pick[1] + tie_before_local;
-  uint32_t t = tw, take = 0u;
-  while (t && rk < k) {
-    const uint32_t lowbit = t & (~t + 1u);
-    take |= lowbit;
-    t ^= lowbit;
-    ++rk;
+  uint32_t take = tw;
+  if (!take_all_ties) {   // the same decision in every CTA of the cluster
+    int ties_tot;
+    const int tie_before_local = block_excl<T>(__popc(tw), ws, &ties_tot);
+    if (threadIdx.x == 0) pub[1] = ties_tot;
+    csync();
+    if (warp == 0) {
+      const int sb = published_before<CS>(cl, pub + 1, lane, rank);
+      if (lane == 0) s_pick[1] = sb;
+    }
+    __syncthreads();
+    int rk = s_pick[1] + tie_before_local;
+    uint32_t t = tw;
+    take = 0u;
+    while (t && rk < k) {
+      const uint32_t lowbit = t & (~t + 1u);
+      take |= lowbit;
+      t ^= lowbit;
+      ++rk;
+    }
   }
   const uint32_t sw = selw[i] | take;
   const int word = rank * T + i;

@@ -70,9 +70,10 @@ LSE_SUM_ERR = 2e-6
 # where n_j is at or above the mean (elsewhere kappa = 1 exactly).
 EPS_Z = 2.0 ** -23
 EPS_KAPPA = 2.0 ** -23
-# Rounding of the kernel's fused score s (relative, per element): lambda r
-# rounded to fp32, then one FMA.
-S_ROUND = 2.0 ** -23
+# Rounding of the kernel's fused score s (relative, per element): kappa pi
+# rounded to fp32, its product with lambda / Z (whose own rounding is common
+# and inside EPS_Z) rounded, then one FMA: three roundings of 2^-24.
+S_ROUND = 1.5 * 2.0 ** -23
 # Undecided candidates allowed per head, as a share of K (and at least this
 # many).  The count is a property of the input, not of the kernel (whose
 # choices are checked candidate by candidate against the sure-in / sure-out

@@ -16,8 +16,9 @@ import helpers as H
 
 
 def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
-    """The CUDA Selector's arithmetic in numpy: x = z - lse_C in fp32, prior
-    in fp64 from fp32 norms, lambda r rounded to fp32, s by one fp32 FMA,
+    """The CUDA Selector's arithmetic in numpy: x = z - lse_C in fp32, kappa pi
+    in fp64 from fp32 norms rounded to fp32, lambda r = that times lambda / Z
+    in fp32, s by one fp32 FMA,
     dominance on s, owner with the tie tolerance on l' (or, rounded_owner, a
     plain argmax of the fp32 l'), keys fp32."""
     lo, hi = O.candidate_range(L, cfg.n_sink, cfg.n_recent)
@@ -27,10 +28,10 @@ def _emulate(z32, lse32, norms32, L, cfg, K, rounded_owner=False):
     nbar = n.mean()
     kap = np.where(n > 0, np.minimum(1.0, nbar / np.where(n > 0, n, 1.0)), 1.0)
     kp = kap * np.log(1.0 + L - np.arange(lo, hi, dtype=np.float64))
-    r = kp / kp.sum()
+    lam_z = np.float32(lam / kp.sum())          # lambda / Z, rounded once
     x = (z32[:, lo:hi] - lse32[:, None]).astype(np.float32)
     ft = np.exp(x.astype(np.float64)).astype(np.float32)
-    lr32 = (lam * r).astype(np.float32)
+    lr32 = (kp.astype(np.float32) * lam_z).astype(np.float32)   # fp32 kappa pi times lambda / Z
     s32 = (np.float64(np.float32(1.0 - lam)) * ft.astype(np.float64) + lr32.astype(np.float64)[None]).astype(np.float32)
     key = x if lam <= 0 else s32
     G, nC = x.shape
