@@ -168,48 +168,61 @@ struct ScoreArgs {
   float inv_nq;
 };
 
-// Phase 3 of one position: l' = ln(s + 1e-30) - alpha_soft * weight(d) of
-// every head (s = exp(x) when the key is x), the owner = the lowest head
-// within the tie tolerance of the largest l', and l'' = l' - alpha_cross off
-// the owner, written to outp[h * ld_s + k].
+// How a CTA of the score kernel spreads a group's GM heads: kHPT heads per
+// thread, kTPP consecutive lanes per position.
 template <int GM>
-__device__ __forceinline__ void finish_position(const float (&kv)[GM], const int (&d)[GM], int G, bool by_x,
-                                                float alpha_soft, float alpha_cross, const float* wt,
+struct ScoreLanes {
+  static constexpr int kHPT = GM < 4 ? GM : 4;
+  static constexpr int kTPP = GM / kHPT;
+};
+
+// Phase 3 of one position, by its kTPP threads, this one holding heads h0 ..
+// h0 + kHPT - 1: l' = ln(s + 1e-30) - alpha_soft * weight(d) of every head
+// (s = exp(x) when the key is x), the owner = the lowest head within the tie
+// tolerance of the largest l' (both found across the position's threads),
+// and l'' = l' - alpha_cross off the owner, written to outp[h * ld_s + k].
+// Every lane of the warp calls it (act: the lane holds a position).
+template <int GM>
+__device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>::kHPT],
+                                                const int (&d)[ScoreLanes<GM>::kHPT], int h0, bool act, int G,
+                                                bool by_x, float alpha_soft, float alpha_cross, const float* wt,
                                                 float* outp, int64_t ld_s, int k) {
-  float l1[GM];
+  constexpr int H = ScoreLanes<GM>::kHPT, P = ScoreLanes<GM>::kTPP;
+  float l1[H];
   float M = -INFINITY;
 #pragma unroll
-  for (int h = 0; h < GM; ++h) {
-    l1[h] = -INFINITY;
-    if (h < G) {
-      const float sv = by_x ? fast_exp2(kv[h] * kLog2e) : kv[h];
-      l1[h] = logf(sv + 1e-30f) - alpha_soft * wt[d[h]];
-      M = fmaxf(M, l1[h]);
+  for (int j = 0; j < H; ++j) {
+    l1[j] = -INFINITY;
+    if (act && h0 + j < G) {
+      const float sv = by_x ? fast_exp2(kv[j] * kLog2e) : kv[j];
+      l1[j] = logf(sv + 1e-30f) - alpha_soft * wt[d[j]];
+      M = fmaxf(M, l1[j]);
     }
   }
+#pragma unroll
+  for (int sh = 1; sh < P; sh <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
   const float thr = M - kOwnerTie;
   int owner = GM;
 #pragma unroll
-  for (int h = GM - 1; h >= 0; --h)
-    if (h < G && l1[h] >= thr) owner = h;
+  for (int j = H - 1; j >= 0; --j)
+    if (act && h0 + j < G && l1[j] >= thr) owner = h0 + j;
 #pragma unroll
-  for (int h = 0; h < GM; ++h)
-    if (h < G) outp[(size_t)h * ld_s + k] = l1[h] - (h != owner ? alpha_cross : 0.f);
+  for (int sh = 1; sh < P; sh <<= 1) owner = min(owner, __shfl_xor_sync(0xffffffffu, owner, sh));
+#pragma unroll
+  for (int j = 0; j < H; ++j)
+    if (act && h0 + j < G) outp[(size_t)(h0 + j) * ld_s + k] = l1[j] - (h0 + j != owner ? alpha_cross : 0.f);
 }
 
-// The GM keys of one position (16-byte loads for GM >= 4).
-template <int GM>
-__device__ __forceinline__ void load_keys(const float* p, float (&v)[GM]) {
-  if constexpr (GM >= 4) {
-#pragma unroll
-    for (int j = 0; j < GM / 4; ++j) {
-      const float4 t = reinterpret_cast<const float4*>(p)[j];
-      v[4 * j] = t.x;
-      v[4 * j + 1] = t.y;
-      v[4 * j + 2] = t.z;
-      v[4 * j + 3] = t.w;
-    }
-  } else if constexpr (GM == 2) {
+// N consecutive keys (16-byte loads for N = 4).
+template <int N>
+__device__ __forceinline__ void load_keys(const float* p, float (&v)[N]) {
+  if constexpr (N == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(p);
+    v[0] = t.x;
+    v[1] = t.y;
+    v[2] = t.z;
+    v[3] = t.w;
+  } else if constexpr (N == 2) {
     const float2 t = *reinterpret_cast<const float2*>(p);
     v[0] = t.x;
     v[1] = t.y;
@@ -218,13 +231,11 @@ __device__ __forceinline__ void load_keys(const float* p, float (&v)[GM]) {
   }
 }
 
-template <int GM>
-__device__ __forceinline__ void store_keys(float* p, const float (&v)[GM]) {
-  if constexpr (GM >= 4) {
-#pragma unroll
-    for (int j = 0; j < GM / 4; ++j)
-      reinterpret_cast<float4*>(p)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-  } else if constexpr (GM == 2) {
+template <int N>
+__device__ __forceinline__ void store_keys(float* p, const float (&v)[N]) {
+  if constexpr (N == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (N == 2) {
     *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
   } else {
     p[0] = v[0];
@@ -234,13 +245,14 @@ __device__ __forceinline__ void store_keys(float* p, const float (&v)[GM]) {
 // One CTA per (b, KV group, tile of candidates).  Phase 1 writes, for every
 // position of the tile plus a halo of w on each side, the dominance keys of
 // the group's heads side by side (s in fp32, or x when lambda = 0; NaN
-// outside C and for heads >= G: a NaN never dominates).  Phase 2: the thread
-// of a position finds every head's nearest dominator, distances 1..kNear for
-// all heads at once (one vector load per side and distance), then the
-// heads still without one alone, to w; phase 3 (finish_position) applies
-// soft-NMS, picks the owner and writes l''.
+// outside C and for heads >= G: a NaN never dominates).  Phase 2: the kTPP
+// threads of a position find the nearest dominator of their kHPT heads each,
+// distances 1..kNear for their heads at once (one vector load per side and
+// distance), then the heads still without one alone, to w; phase 3
+// (finish_position) applies soft-NMS, picks the owner and writes l''.
 template <int GM>
-__global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
+__global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
+  constexpr int H = ScoreLanes<GM>::kHPT, P = ScoreLanes<GM>::kTPP;
   grid_dep_enter();
   extern __shared__ float sm[];
   const int W = a.tile + 2 * a.w;     // haloed width
@@ -260,25 +272,29 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
   __shared__ float wt[64];                 // soft-NMS weight of a nearest dominator at distance d
   for (int d = threadIdx.x; d <= a.w && d < 64; d += blockDim.x)
     wt[d] = d > 0 ? 1.f - (float)(d - 1) / (float)a.w : 0.f;
+  // this thread's heads and its place among a position's threads
+  const int h0 = (int)(threadIdx.x % P) * H;
+  const int pstride = blockDim.x / P;      // positions per pass of the block
   // logits rows of the group: nq query slots of G heads (nq = 1: row b * Hq + g * G + h)
   const size_t row0 = ((size_t)b * a.Hkv + g) * (size_t)(a.nq * G);
   const float* z0 = a.logits + row0 * a.ld + a.lo;
   const float nan = __int_as_float(0x7fc00000);
-  float lsec[GM];
+  float lsec[H];
 #pragma unroll
-  for (int h = 0; h < GM; ++h) lsec[h] = (h < G) ? a.lse_cand[row0 + h] : 0.f;
+  for (int j = 0; j < H; ++j) lsec[j] = (h0 + j < G) ? a.lse_cand[row0 + h0 + j] : 0.f;
   if (a.nq > 1) {
     // evidence window: f~ = the mean of the slots' restricted distributions,
     // x = ln f~ = m + ln(mean exp(x_i - m)), m the largest x_i
-    for (int k = threadIdx.x; k < W; k += blockDim.x) {
+    for (int k = threadIdx.x / P; k < W; k += pstride) {
       const int c = c0 - a.w + k;
-      float kv[GM];
+      float kv[H];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) kv[h] = nan;
+      for (int j = 0; j < H; ++j) kv[j] = nan;
       if (c >= 0 && c < a.nC) {
         const float r = kpr[c] * lam_r;   // lambda r_j
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
+        for (int j = 0; j < H; ++j) {
+          const int h = h0 + j;
           if (h < G) {
             float m = -INFINITY;
             for (int i = 0; i < a.nq; ++i)
@@ -294,43 +310,43 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
               }
             const float x = m + logf(acc * a.inv_nq);
             const float ft = fast_exp2(x * kLog2e);
-            kv[h] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
+            kv[j] = by_x ? x : fmaf(a.one_minus_lam, ft, r);
           }
         }
       }
-      store_keys<GM>(key + (size_t)k * GM, kv);
+      store_keys<H>(key + (size_t)k * GM + h0, kv);
     }
   }
   // kU positions per thread and round: all their loads are issued first
-  constexpr int kU = GM >= 8 ? 2 : 4;
-  for (int k0 = threadIdx.x; a.nq == 1 && k0 < W; k0 += kU * blockDim.x) {
+  constexpr int kU = 4;
+  for (int k0 = threadIdx.x / P; a.nq == 1 && k0 < W; k0 += kU * pstride) {
     float kp[kU];
-    float zv[kU][GM];
+    float zv[kU][H];
     bool in[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int c = c0 - a.w + k0 + u * blockDim.x;
-      in[u] = k0 + u * blockDim.x < W && c >= 0 && c < a.nC;
+      const int c = c0 - a.w + k0 + u * pstride;
+      in[u] = k0 + u * pstride < W && c >= 0 && c < a.nC;
       const int cc = in[u] ? c : 0;
       kp[u] = in[u] ? kpr[cc] : 0.f;
 #pragma unroll
-      for (int h = 0; h < GM; ++h) zv[u][h] = (in[u] && h < G) ? z0[(size_t)h * a.ld + cc] : 0.f;
+      for (int j = 0; j < H; ++j) zv[u][j] = (in[u] && h0 + j < G) ? z0[(size_t)(h0 + j) * a.ld + cc] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      const int k = k0 + u * blockDim.x;
+      const int k = k0 + u * pstride;
       if (k >= W) continue;
-      float kv[GM];
+      float kv[H];
       const float r = kp[u] * lam_r;   // lambda r_j
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
+      for (int j = 0; j < H; ++j) {
         // exp through the hardware's base-2 approximation (relative error
         // ~1e-7, below the error of the logits themselves)
-        const float x = zv[u][h] - lsec[h];
+        const float x = zv[u][j] - lsec[j];
         const float ft = fast_exp2(x * kLog2e);
-        kv[h] = (in[u] && h < G) ? (by_x ? x : fmaf(a.one_minus_lam, ft, r)) : nan;
+        kv[j] = (in[u] && h0 + j < G) ? (by_x ? x : fmaf(a.one_minus_lam, ft, r)) : nan;
       }
-      store_keys<GM>(key + (size_t)k * GM, kv);
+      store_keys<H>(key + (size_t)k * GM + h0, kv);
     }
   }
   __syncthreads();
@@ -338,43 +354,50 @@ __global__ void __launch_bounds__(256, GM >= 16 ? 2 : 4) select_scores_kernel(co
   constexpr int kNear = 4;
   const int near = min(kNear, a.w);
   float* outp = a.scores + ((size_t)bl * a.Hq + (size_t)g * G) * a.ld_s + c0;
-  for (int k = threadIdx.x; k < tile_n; k += blockDim.x) {
-    const float* row = key + (size_t)(a.w + k) * GM;
-    float e[GM];
-    int dh[GM];
-    load_keys<GM>(row, e);
+  for (int base = 0; base < tile_n; base += pstride) {
+    const int k = base + (int)threadIdx.x / P;
+    const bool act = k < tile_n;
+    float e[H];
+    int dh[H];
 #pragma unroll
-    for (int h = 0; h < GM; ++h) dh[h] = 0;
-#pragma unroll
-    for (int d = 1; d <= kNear; ++d) {
-      if (d > near) break;
-      float lv[GM], rv[GM];
-      load_keys<GM>(row - d * GM, lv);
-      load_keys<GM>(row + d * GM, rv);
-#pragma unroll
-      for (int h = 0; h < GM; ++h)   // a left neighbour dominates on ties; NaN compares false
-        if (dh[h] == 0 && (lv[h] >= e[h] || rv[h] > e[h])) dh[h] = d;
+    for (int j = 0; j < H; ++j) {
+      e[j] = 0.f;
+      dh[j] = 0;
     }
-    if (a.w > kNear) {
-      // the heads still without a dominator (about 1 % of positions): alone, to w
+    if (act) {
+      const float* row = key + (size_t)(a.w + k) * GM + h0;
+      load_keys<H>(row, e);
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
-        if (h < G && dh[h] == 0) {
-          for (int d = kNear + 1; d <= a.w; ++d) {
-            if (row[h - d * GM] >= e[h] || row[h + d * GM] > e[h]) {
-              dh[h] = d;
-              break;
+      for (int d = 1; d <= kNear; ++d) {
+        if (d > near) break;
+        float lv[H], rv[H];
+        load_keys<H>(row - d * GM, lv);
+        load_keys<H>(row + d * GM, rv);
+#pragma unroll
+        for (int j = 0; j < H; ++j)   // a left neighbour dominates on ties; NaN compares false
+          if (dh[j] == 0 && (lv[j] >= e[j] || rv[j] > e[j])) dh[j] = d;
+      }
+      if (a.w > kNear) {
+        // the heads still without a dominator (about 1 % of positions): alone, to w
+#pragma unroll
+        for (int j = 0; j < H; ++j) {
+          if (h0 + j < G && dh[j] == 0) {
+            for (int d = kNear + 1; d <= a.w; ++d) {
+              if (row[j - d * GM] >= e[j] || row[j + d * GM] > e[j]) {
+                dh[j] = d;
+                break;
+              }
             }
           }
         }
       }
     }
-    finish_position<GM>(e, dh, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
+    finish_position<GM>(e, dh, h0, act, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
   }
 }
 
 // ---------------------------------------------------------------- host
-int score_tile(int G) { return std::max(256, 4096 / G); }
+int score_tile(int G) { return std::max(512, 4096 / G); }
 
 // dominance keys of the tile with its halo, GM (G rounded up to a power of
 // two) per position
