@@ -218,11 +218,30 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     fence_barrier_init();
   }
   __syncthreads();
-  grid_dep_wait();
-  if (!a.late_trigger) grid_dep_launch();
+  // The consumers wait for the previous kernel of the stream before anything
+  // else (they write the partials, which it may still read).  The producer
+  // issues its first copies at once: the query, the pages, the page table,
+  // the packed buffers and n_rows are written by no kernel of this library
+  // that lets its dependents start early (the append and the compaction
+  // signal them only at exit), so the copies overlap the previous kernel's
+  // tail.  The producer waits before it touches the work counter (reset by
+  // the previous combine) or appends the step's token.
+  if (warp != kConsumerWarps) {
+    grid_dep_wait();
+    if (!a.late_trigger) grid_dep_launch();
+  }
 
   // ------------------------------------------------------------ producer warp
   if (warp == kConsumerWarps) {
+    bool waited = false;
+    auto ensure_wait = [&]() {
+      if (!waited) {
+        grid_dep_wait();
+        if (!a.late_trigger) grid_dep_launch();
+        waited = true;
+      }
+    };
+
     if (lane == 0) {
       prefetch_tensormap(&maps.k);
       prefetch_tensormap(&maps.v);
@@ -271,6 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     // it cannot start soon, so CTAs that finish early take what remains.
     bool drawn = false;
     auto draw_next = [&]() {
+      ensure_wait();
       int v = 0;
       if (lane == 0) v = atomicAdd(a.ctr, 1) + (int)gridDim.x;
       nxt = __shfl_sync(0xffffffffu, v, 0);
@@ -300,6 +320,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
         // the item holding position L - 1 first appends the step's token
         // there (the whole warp), before any copy of that tile is issued
         if (a.k_new && it.t_begin < it.t_end && it.t_end == it.t_total) {
+          ensure_wait();
           const int pos = a.L - 1;
           append_row_warp<D>(lane, it.bg, it.g, pos, ptbuf[pos / kPage - p_lo], a.Hkv, a.num_pages, a.k_pool,
                              a.v_pool, a.k_new, a.v_new, a.norms, a.norm_ld, a.err);

@@ -18,17 +18,23 @@ namespace sfi {
 
 // Programmatic dependent launch.  The library launches its kernels with
 // programmatic stream serialization, so a kernel may be scheduled while the
-// previous kernel on its stream is still running.  Every kernel therefore
-// calls grid_dep_wait() before its first global-memory access (read or
-// write); it returns once the previous kernel has finished and its writes are
-// visible.  grid_dep_launch() lets the next kernel get scheduled early.  Both
-// are no-ops for a kernel launched the ordinary way.
+// previous kernel on its stream is still running.  A kernel calls
+// grid_dep_wait() before it touches global memory that the previous kernel
+// may write or read; it returns once the previous kernel has finished and its
+// writes are visible.  grid_dep_launch() lets the next kernel get scheduled
+// early; kernels that write the cache or the packed buffers (the append, the
+// key norms, the compaction) never call it, because the attention's producer
+// reads pages, packed rows and queries before its wait.  Both are no-ops for
+// a kernel launched the ordinary way.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_enter() {
   grid_dep_wait();
   grid_dep_launch();
 }
+// The start of a kernel that writes the cache or the packed buffers: wait,
+// and let the next kernel start only when this one has finished.
+__device__ __forceinline__ void grid_dep_enter_writer() { grid_dep_wait(); }
 
 
 constexpr int kPage = 16;

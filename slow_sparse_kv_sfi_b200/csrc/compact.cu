@@ -58,7 +58,7 @@ __device__ __forceinline__ uint32_t union_word(const CompactArgs& a, int b, int 
 
 template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const __grid_constant__ CompactArgs a) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   __shared__ int wsum[kCThreads / 32];
   const int bg = blockIdx.y;
   const int b = bg / a.Hkv, g = bg - b * a.Hkv;
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kCThreads) compact_count_kernel(const __grid_c
 
 template <int GM>
 __global__ void __launch_bounds__(kCThreads) compact_gather_kernel(const __grid_constant__ CompactArgs a) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   __shared__ int wtot[kCThreads / 32 + 1];
   __shared__ int base_s, total_s;
   const int bg = blockIdx.y;                    // logical (row, kv head)
@@ -169,7 +169,7 @@ constexpr int kCopyWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kCopyWarps * 32) compact_copy_kernel(const __grid_constant__ CompactArgs a) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   constexpr int kUnits = D / 8;                 // 16-byte units of one K (or V) row
   constexpr int kRowUnits = 2 * kUnits;         // K then V
   constexpr int kRowsPerPass = 32 / kRowUnits;  // rows one warp moves per pass
@@ -337,7 +337,7 @@ __device__ __forceinline__ uint32_t below(int s0, int x) {
 
 template <int D, int GM>
 __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_constant__ IncArgs a) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   cg::cluster_group cl = cg::this_cluster();
   const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
   const CompactArgs& c = a.c;

@@ -15,7 +15,7 @@ __global__ void __launch_bounds__(128) append_kernel(int BH, int Hkv, int L, int
                                                      __nv_bfloat16* vpool, const __nv_bfloat16* __restrict__ knew,
                                                      const __nv_bfloat16* __restrict__ vnew, float* norms,
                                                      int64_t norm_ld, int* err) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   const int bg = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (bg >= BH) return;
   const int b = bg / Hkv, h = bg - b * Hkv;
@@ -31,7 +31,7 @@ __global__ void key_norms_kernel(int Hkv, int lo, int hi, int max_pages, int num
                                  const int32_t* __restrict__ pt,
                                  const __nv_bfloat16* __restrict__ kpool, float* norms,
                                  int64_t norm_ld, int* err) {
-  grid_dep_enter();
+  grid_dep_enter_writer();
   const int bg = blockIdx.y;
   const int b = bg / Hkv, h = bg - b * Hkv;
   const int lane = threadIdx.x & 31;
