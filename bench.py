@@ -544,11 +544,11 @@ def run_sfi(args, cfg, rank, world, dist_on):
     }
     value = aggregate_rate(world, tokens, args.steps, t_sfi)
     # fast layer-step: attention (with the append) + combine; slow: the same
-    # two, 2 statistics, scores and the top-K, then the compaction: 3 kernels
+    # two, 3 statistics, scores and the top-K, then the compaction: 3 kernels
     # when step 0 builds the packed buffers, 1 (the incremental refresh) when
     # a later slow step refreshes them (side stream)
     n_fresh = 1 if slows and slows[0] else 0
-    launches_per_run = NL * (n_fresh * 9 + (n_slow - n_fresh) * 7 + (T - n_slow) * 2)
+    launches_per_run = NL * (n_fresh * 10 + (n_slow - n_fresh) * 8 + (T - n_slow) * 2)
     legs = {"sfi": clk_sfi, "dense": clk_dense, "e2e": clk_e2e}
     mhz = [v["sm_mhz"] for v in legs.values() if v.get("sm_mhz")]
     clk = {"sm_mhz": statistics.median(mhz) if mhz else None,

@@ -61,10 +61,10 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   const long nC = std::max<long>(Lmax - p.n_recent - p.n_sink, 1);
   w.stat_off = off;
   // per-chunk partial sums and the position factors (fp64), kappa * pi of
-  // every candidate (fp32)
+  // every candidate and lambda / Z of every row (fp32)
   const size_t kp_ld = (size_t)((nC + 1) / 2 * 2);
   w.stat_bytes = align_up((size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double) + kp_ld * sizeof(double) +
-                          (size_t)bh * kp_ld * sizeof(float), 256);
+                          (size_t)bh * kp_ld * sizeof(float) + (size_t)bh * sizeof(float), 256);
   off += w.stat_bytes;
   w.sel_off = off;
   w.sel_bytes = align_up((size_t)s.B * s.Hq * ((nC + 3) / 4 * 4) * sizeof(float), 256);

@@ -146,6 +146,16 @@ __global__ void __launch_bounds__(kStatThreads) stats_prior_kernel(int L, int lo
   if (threadIdx.x == 0) pbg[blockIdx.x * 2 + 1] = t;
 }
 
+// lamz[bgl] = lambda / Z rounded once to fp32, Z = sum of kappa pi over C
+// (the chunk partials summed in a fixed order): one warp per (row, kv head).
+__global__ void __launch_bounds__(32) stats_final_kernel(const double* __restrict__ part, int nch, double lam,
+                                                         float* __restrict__ lamz) {
+  grid_dep_enter();
+  __shared__ double bc;
+  const double z = reduce_parts(part + (size_t)blockIdx.x * nch * 2, nch, 1, &bc);
+  if (threadIdx.x == 0) lamz[blockIdx.x] = (float)(lam / z);
+}
+
 struct ScoreArgs {
   int L, lo, nC, Hq, Hkv, G, w, tile;
   double lam;                   // lambda_eff
@@ -154,8 +164,7 @@ struct ScoreArgs {
   const float* logits;
   int64_t ld;
   const float* lse_cand;
-  const double* stat_part;   // [B*Hkv][nch][2]
-  int nch;
+  const float* lamz;         // [B*Hkv] lambda / Z
   const float* kp;           // [B*Hkv][kp_ld] kappa_j pi_j of the candidates (fp32)
   int64_t kp_ld;
   float* scores;         // logical rows of the launch
@@ -182,7 +191,7 @@ struct ScoreLanes {
 // tolerance of the largest l' (both found across the position's threads),
 // and l'' = l' - alpha_cross off the owner, written to outp[h * ld_s + k].
 // Every lane of the warp calls it (act: the lane holds a position).
-template <int GM>
+template <int GM, bool EXACT>
 __device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>::kHPT],
                                                 const int (&d)[ScoreLanes<GM>::kHPT], int h0, bool act, int G,
                                                 bool by_x, float alpha_soft, float alpha_cross, const float* wt,
@@ -193,7 +202,7 @@ __device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>
 #pragma unroll
   for (int j = 0; j < H; ++j) {
     l1[j] = -INFINITY;
-    if (act && h0 + j < G) {
+    if (act && (EXACT || h0 + j < G)) {
       const float sv = by_x ? fast_exp2(kv[j] * kLog2e) : kv[j];
       l1[j] = logf(sv + 1e-30f) - alpha_soft * wt[d[j]];
       M = fmaxf(M, l1[j]);
@@ -205,12 +214,12 @@ __device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>
   int owner = GM;
 #pragma unroll
   for (int j = H - 1; j >= 0; --j)
-    if (act && h0 + j < G && l1[j] >= thr) owner = h0 + j;
+    if (act && (EXACT || h0 + j < G) && l1[j] >= thr) owner = h0 + j;
 #pragma unroll
   for (int sh = 1; sh < P; sh <<= 1) owner = min(owner, __shfl_xor_sync(0xffffffffu, owner, sh));
 #pragma unroll
   for (int j = 0; j < H; ++j)
-    if (act && h0 + j < G) outp[(size_t)(h0 + j) * ld_s + k] = l1[j] - (h0 + j != owner ? alpha_cross : 0.f);
+    if (act && (EXACT || h0 + j < G)) outp[(size_t)(h0 + j) * ld_s + k] = l1[j] - (h0 + j != owner ? alpha_cross : 0.f);
 }
 
 // N consecutive keys (16-byte loads for N = 4).
@@ -250,7 +259,8 @@ __device__ __forceinline__ void store_keys(float* p, const float (&v)[N]) {
 // distances 1..kNear for their heads at once (one vector load per side and
 // distance), then the heads still without one alone, to w; phase 3
 // (finish_position) applies soft-NMS, picks the owner and writes l''.
-template <int GM>
+// EXACT: G == GM, so every lane's heads exist.
+template <int GM, bool EXACT>
 __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_constant__ ScoreArgs a) {
   constexpr int H = ScoreLanes<GM>::kHPT, P = ScoreLanes<GM>::kTPP;
   grid_dep_enter();
@@ -262,13 +272,10 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
   const int b = a.rows.phys(bl);                    // the sequence
   const int c0 = blockIdx.x * a.tile;
   const int tile_n = min(a.tile, a.nC - c0);
-  const int G = a.G;
-  __shared__ double bc;
-  const double* pbg = a.stat_part + (size_t)bg * a.nch * 2;
-  const double inv_z = 1.0 / reduce_parts(pbg, a.nch, 1, &bc);
+  const int G = EXACT ? GM : a.G;
   const float* kpr = a.kp + (size_t)bg * a.kp_ld;
   const bool by_x = a.lam <= 0.0;          // lambda = 0: s = f~, decided on x
-  const float lam_r = (float)(a.lam * inv_z);   // lambda / Z, rounded once
+  const float lam_r = a.lamz[bg];          // lambda / Z, rounded once
   __shared__ float wt[64];                 // soft-NMS weight of a nearest dominator at distance d
   for (int d = threadIdx.x; d <= a.w && d < 64; d += blockDim.x)
     wt[d] = d > 0 ? 1.f - (float)(d - 1) / (float)a.w : 0.f;
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
   const float nan = __int_as_float(0x7fc00000);
   float lsec[H];
 #pragma unroll
-  for (int j = 0; j < H; ++j) lsec[j] = (h0 + j < G) ? a.lse_cand[row0 + h0 + j] : 0.f;
+  for (int j = 0; j < H; ++j) lsec[j] = (EXACT || h0 + j < G) ? a.lse_cand[row0 + h0 + j] : 0.f;
   if (a.nq > 1) {
     // evidence window: f~ = the mean of the slots' restricted distributions,
     // x = ln f~ = m + ln(mean exp(x_i - m)), m the largest x_i
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
 #pragma unroll
         for (int j = 0; j < H; ++j) {
           const int h = h0 + j;
-          if (h < G) {
+          if (EXACT || h < G) {
             float m = -INFINITY;
             for (int i = 0; i < a.nq; ++i)
               if ((a.qmask >> i) & 1u) {
@@ -330,7 +337,7 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
       const int cc = in[u] ? c : 0;
       kp[u] = in[u] ? kpr[cc] : 0.f;
 #pragma unroll
-      for (int j = 0; j < H; ++j) zv[u][j] = (in[u] && h0 + j < G) ? z0[(size_t)(h0 + j) * a.ld + cc] : 0.f;
+      for (int j = 0; j < H; ++j) zv[u][j] = (in[u] && (EXACT || h0 + j < G)) ? z0[(size_t)(h0 + j) * a.ld + cc] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -344,7 +351,7 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
         // ~1e-7, below the error of the logits themselves)
         const float x = zv[u][j] - lsec[j];
         const float ft = fast_exp2(x * kLog2e);
-        kv[j] = (in[u] && h0 + j < G) ? (by_x ? x : fmaf(a.one_minus_lam, ft, r)) : nan;
+        kv[j] = (in[u] && (EXACT || h0 + j < G)) ? (by_x ? x : fmaf(a.one_minus_lam, ft, r)) : nan;
       }
       store_keys<H>(key + (size_t)k * GM + h0, kv);
     }
@@ -368,20 +375,20 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
       const float* row = key + (size_t)(a.w + k) * GM + h0;
       load_keys<H>(row, e);
 #pragma unroll
-      for (int d = 1; d <= kNear; ++d) {
-        if (d > near) break;
+      for (int d = kNear; d >= 1; --d) {   // descending: the nearest hit is written last
+        if (d > near) continue;
         float lv[H], rv[H];
         load_keys<H>(row - d * GM, lv);
         load_keys<H>(row + d * GM, rv);
 #pragma unroll
         for (int j = 0; j < H; ++j)   // a left neighbour dominates on ties; NaN compares false
-          if (dh[j] == 0 && (lv[j] >= e[j] || rv[j] > e[j])) dh[j] = d;
+          if (lv[j] >= e[j] || rv[j] > e[j]) dh[j] = d;
       }
       if (a.w > kNear) {
         // the heads still without a dominator (about 1 % of positions): alone, to w
 #pragma unroll
         for (int j = 0; j < H; ++j) {
-          if (h0 + j < G && dh[j] == 0) {
+          if ((EXACT || h0 + j < G) && dh[j] == 0) {
             for (int d = kNear + 1; d <= a.w; ++d) {
               if (row[j - d * GM] >= e[j] || row[j + d * GM] > e[j]) {
                 dh[j] = d;
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
         }
       }
     }
-    finish_position<GM>(e, dh, h0, act, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
+    finish_position<GM, EXACT>(e, dh, h0, act, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
   }
 }
 
@@ -409,15 +416,20 @@ size_t score_smem(int G, int tile, int w) {
 
 int stat_chunks(int nC) { return (nC + kStatChunk - 1) / kStatChunk; }
 
-template <int GM>
-sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+template <int GM, bool EXACT>
+sfi_status launch_scores_t(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
   static DeviceOnce attr;
   if (!attr.done() &&
-      !attr.mark(cudaFuncSetAttribute(select_scores_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      !attr.mark(cudaFuncSetAttribute(select_scores_kernel<GM, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       200 * 1024)))
     return SFI_ERR_CUDA;
-  launch_k(select_scores_kernel<GM>, dim3(grid), dim3(256), smem, st, a);
+  launch_k(select_scores_kernel<GM, EXACT>, dim3(grid), dim3(256), smem, st, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
+}
+
+template <int GM>
+sfi_status launch_scores(const ScoreArgs& a, dim3 grid, size_t smem, cudaStream_t st) {
+  return a.G == GM ? launch_scores_t<GM, true>(a, grid, smem, st) : launch_scores_t<GM, false>(a, grid, smem, st);
 }
 
 namespace {
@@ -429,6 +441,7 @@ struct StatLayout {
   int64_t kp_ld;
   double *part, *pitab;
   float* kp;
+  float* lamz;
   StatLayout(const sfi_shape& s, const sfi_params& p, int L, const RowMap& rows, void* ws) {
     nb = rows.count(s.B);
     nC = L - p.n_recent - p.n_sink;
@@ -437,6 +450,7 @@ struct StatLayout {
     part = reinterpret_cast<double*>(ws);
     pitab = part + (size_t)nb * s.Hkv * nch * 2;
     kp = reinterpret_cast<float*>(pitab + kp_ld);
+    lamz = kp + (size_t)nb * s.Hkv * kp_ld;
   }
 };
 
@@ -453,6 +467,8 @@ sfi_status run_select_stats(const sfi_shape& s, const sfi_params& p, const sfi_p
            sl.nch, s.Hkv, sl.pitab, rows);
   launch_k(stats_prior_kernel, dim3(sgrid), dim3(kStatThreads), 0, st, L, lo, sl.nC, kv.key_norms, norm_ld, sl.part,
            sl.nch, s.Hkv, sl.pitab, sl.kp, sl.kp_ld, rows);
+  const double lam = std::min(std::max((double)p.lambda, 0.0), (double)p.lambda_clip);
+  launch_k(stats_final_kernel, dim3(sl.nb * s.Hkv), dim3(32), 0, st, sl.part, sl.nch, lam, sl.lamz);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -468,13 +484,12 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   if (qmask == 0u) return SFI_ERR_INVALID_ARG;
   const int lo = p.n_sink;
   const StatLayout sl(s, p, L, rows, stat_ws);
-  const int nC = sl.nC, nch = sl.nch;
+  const int nC = sl.nC;
   if (std::max(p.nms_window / 2, 1) > 63) return SFI_ERR_UNSUPPORTED;   // the weight table
   if (with_stats) {
     const sfi_status r = run_select_stats(s, p, kv, L, stat_ws, st, rows);
     if (r != SFI_OK) return r;
   }
-  double* part = sl.part;
   float* kp = sl.kp;
   const int64_t kp_ld = sl.kp_ld;
   ScoreArgs a{};
@@ -487,7 +502,7 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.alpha_soft = p.nms_window / 2 >= 1 ? p.alpha_soft : 0.f;
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;
-  a.stat_part = part; a.nch = nch;
+  a.lamz = sl.lamz;
   a.kp = kp; a.kp_ld = kp_ld;
   a.scores = scores; a.ld_s = ld_s;
   a.rows = rows;
