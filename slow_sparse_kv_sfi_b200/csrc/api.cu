@@ -60,11 +60,13 @@ WsLayout ws_layout(const sfi_shape& s, const sfi_params& p) {
   off += w.part_bytes;
   const long nC = std::max<long>(Lmax - p.n_recent - p.n_sink, 1);
   w.stat_off = off;
-  // per-chunk partial sums and the position factors (fp64), kappa * pi of
-  // every candidate and lambda / Z of every row (fp32)
+  // the rows' score ranges for the top-K, per-chunk partial sums and the
+  // position factors (fp64), kappa * pi of every candidate and lambda / Z of
+  // every row (fp32)
   const size_t kp_ld = (size_t)((nC + 1) / 2 * 2);
-  w.stat_bytes = align_up((size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double) + kp_ld * sizeof(double) +
-                          (size_t)bh * kp_ld * sizeof(float) + (size_t)bh * sizeof(float), 256);
+  w.stat_bytes = align_up((size_t)s.B * s.Hq * 2 * sizeof(uint32_t) +
+                              (size_t)bh * stat_chunks((int)nC) * 2 * sizeof(double) + kp_ld * sizeof(double) +
+                              (size_t)bh * kp_ld * sizeof(float) + (size_t)bh * sizeof(float), 256);
   off += w.stat_bytes;
   w.sel_off = off;
   w.sel_bytes = align_up((size_t)s.B * s.Hq * ((nC + 3) / 4 * 4) * sizeof(float), 256);
@@ -356,10 +358,12 @@ sfi_status sfi_select(const sfi_shape* shape, const sfi_params* params, const sf
   const int ld_s = (nC + 3) / 4 * 4;
   cudaStream_t st = (cudaStream_t)stream;
   if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
-  SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s,
-                            static_cast<char*>(ws) + w.stat_off, st));
+  void* stat_ws = static_cast<char*>(ws) + w.stat_off;
+  SFI_TRY(run_select_scores(*shape, *params, *kv, L, logits, ld, lse_cand, scores, ld_s, stat_ws, st, RowMap(),
+                            0xffffffffu, true, true));
   const int rows = shape->B * shape->Hq;
-  SFI_TRY(run_topk(rows, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0, st));
+  SFI_TRY(run_topk(rows, nC, scores, ld_s, K, params->n_sink, sel_idx, sel_ld, nullptr, 0, st,
+                   select_row_range(*shape, *params, L, stat_ws)));
   if (K_out) *K_out = K;
   return SFI_OK;
 }

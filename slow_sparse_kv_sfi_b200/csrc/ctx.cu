@@ -282,9 +282,10 @@ sfi_status run_layer(sfi_ctx* c, int layer, int step, int L, const sfi_paged_kv*
     if (nC > topk_max_n()) return SFI_ERR_UNSUPPORTED;
     const int rows = slow_map.count(B) * s.Hq;   // logical rows of the Selector
     SFI_TRY(run_select_scores(s, p, *kv, L, c->logits[buf], c->ld, c->lse_cand[buf], c->scores, ld_s,
-                              c->stats, side, slow_map, wmask, false));
+                              c->stats, side, slow_map, wmask, false, true));
     SFI_TRY(cu(cudaEventRecord(c->ev_buf_free[buf], side)));
-    SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, side));
+    SFI_TRY(run_topk(rows, nC, c->scores, ld_s, K, p.n_sink, nullptr, 0, c->bits, c->bits_ld, side,
+                     select_row_range(s, p, L, c->stats)));
     if (c->incremental && packed->p_max >= c->cmp.cap) {
       // step 0 starts a new decode: cache rows copied before may have changed
       const bool fresh = step == 0 || c->packed_seen[layer] != packed->pos;

@@ -150,12 +150,20 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
                              cudaStream_t st, const RowMap& rows = RowMap(),
-                             uint32_t window_mask = 0xffffffffu, bool with_stats = true);
+                             uint32_t window_mask = 0xffffffffu, bool with_stats = true,
+                             bool row_range = false);
+// row_range: the score kernel also records every row's largest key and key
+// complement (the order the top-K uses) at select_row_range(...), [B*Hq][2]
+// uint32 at the start of the statistics area, which must be zero before the
+// scores and which the top-K given it zeroes again.
+uint32_t* select_row_range(const sfi_shape& s, const sfi_params& p, int L, void* stat_ws);
 // K largest of every row (ties to the lower index): bitmap bits[rows][ld_b]
 // and / or ascending positions idx[rows][ld_i] (+ offset).  No scratch: the
 // cluster kernel of topk.cu keeps its state on chip.
+// minmax: [rows][2] the largest key and largest key complement of every row
+// (see run_select_scores), zeroed again by the top-K; null: found by it.
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
-                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st);
+                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st, uint32_t* minmax = nullptr);
 int topk_max_n();
 // Compaction scratch (inside the workspace): per-tile counts of the full
 // compaction, and the incremental refresh's mover and hole lists.

@@ -165,6 +165,7 @@ struct ScoreArgs {
   int64_t ld;
   const float* lse_cand;
   const float* lamz;         // [B*Hkv] lambda / Z
+  uint32_t* minmax;          // [rows][2] largest key / complement of the row's l'' (atomic max), or null
   const float* kp;           // [B*Hkv][kp_ld] kappa_j pi_j of the candidates (fp32)
   int64_t kp_ld;
   float* scores;         // logical rows of the launch
@@ -195,7 +196,9 @@ template <int GM, bool EXACT>
 __device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>::kHPT],
                                                 const int (&d)[ScoreLanes<GM>::kHPT], int h0, bool act, int G,
                                                 bool by_x, float alpha_soft, float alpha_cross, const float* wt,
-                                                float* outp, int64_t ld_s, int k) {
+                                                float* outp, int64_t ld_s, int k,
+                                                uint32_t (&kmx)[ScoreLanes<GM>::kHPT],
+                                                uint32_t (&knx)[ScoreLanes<GM>::kHPT]) {
   constexpr int H = ScoreLanes<GM>::kHPT, P = ScoreLanes<GM>::kTPP;
   float l1[H];
   float M = -INFINITY;
@@ -219,7 +222,13 @@ __device__ __forceinline__ void finish_position(const float (&kv)[ScoreLanes<GM>
   for (int sh = 1; sh < P; sh <<= 1) owner = min(owner, __shfl_xor_sync(0xffffffffu, owner, sh));
 #pragma unroll
   for (int j = 0; j < H; ++j)
-    if (act && (EXACT || h0 + j < G)) outp[(size_t)(h0 + j) * ld_s + k] = l1[j] - (h0 + j != owner ? alpha_cross : 0.f);
+    if (act && (EXACT || h0 + j < G)) {
+      const float v = l1[j] - (h0 + j != owner ? alpha_cross : 0.f);
+      outp[(size_t)(h0 + j) * ld_s + k] = v;
+      const uint32_t key = float_key(v);   // the top-K's order
+      kmx[j] = max(kmx[j], key);
+      knx[j] = max(knx[j], ~key);
+    }
 }
 
 // N consecutive keys (16-byte loads for N = 4).
@@ -361,6 +370,9 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
   constexpr int kNear = 4;
   const int near = min(kNear, a.w);
   float* outp = a.scores + ((size_t)bl * a.Hq + (size_t)g * G) * a.ld_s + c0;
+  uint32_t kmx[H], knx[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) kmx[j] = knx[j] = 0u;
   for (int base = 0; base < tile_n; base += pstride) {
     const int k = base + (int)threadIdx.x / P;
     const bool act = k < tile_n;
@@ -399,7 +411,40 @@ __global__ void __launch_bounds__(256, 4) select_scores_kernel(const __grid_cons
         }
       }
     }
-    finish_position<GM, EXACT>(e, dh, h0, act, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k);
+    finish_position<GM, EXACT>(e, dh, h0, act, G, by_x, a.alpha_soft, a.alpha_cross, wt, outp, a.ld_s, k, kmx,
+                               knx);
+  }
+  if (a.minmax) {
+    // the rows' largest key and key complement over the CTA, then one atomic
+    // each: the top-K reads them instead of finding the range itself
+    __shared__ uint32_t mm[8][GM][2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < H; ++j)
+#pragma unroll
+      for (int sh = P; sh < 32; sh <<= 1) {
+        kmx[j] = max(kmx[j], __shfl_xor_sync(0xffffffffu, kmx[j], sh));
+        knx[j] = max(knx[j], __shfl_xor_sync(0xffffffffu, knx[j], sh));
+      }
+    if (lane < P) {
+#pragma unroll
+      for (int j = 0; j < H; ++j) {
+        mm[warp][h0 + j][0] = kmx[j];
+        mm[warp][h0 + j][1] = knx[j];
+      }
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < G) {
+      const int h = threadIdx.x;
+      uint32_t x = 0u, y = 0u;
+      for (int w8 = 0; w8 < (int)(blockDim.x >> 5); ++w8) {
+        x = max(x, mm[w8][h][0]);
+        y = max(y, mm[w8][h][1]);
+      }
+      uint32_t* mrow = a.minmax + ((size_t)bl * a.Hq + (size_t)g * G + h) * 2;
+      atomicMax(mrow, x);
+      atomicMax(mrow + 1, y);
+    }
   }
 }
 
@@ -439,6 +484,7 @@ namespace {
 struct StatLayout {
   int nb, nC, nch;
   int64_t kp_ld;
+  uint32_t* minmax;          // [B*Hq][2], at the same place for every row map
   double *part, *pitab;
   float* kp;
   float* lamz;
@@ -447,7 +493,8 @@ struct StatLayout {
     nC = L - p.n_recent - p.n_sink;
     nch = stat_chunks(nC);
     kp_ld = (nC + 1) / 2 * 2;
-    part = reinterpret_cast<double*>(ws);
+    minmax = reinterpret_cast<uint32_t*>(ws);
+    part = reinterpret_cast<double*>(minmax + (size_t)s.B * s.Hq * 2);
     pitab = part + (size_t)nb * s.Hkv * nch * 2;
     kp = reinterpret_cast<float*>(pitab + kp_ld);
     lamz = kp + (size_t)nb * s.Hkv * kp_ld;
@@ -455,6 +502,10 @@ struct StatLayout {
 };
 
 }  // namespace
+
+uint32_t* select_row_range(const sfi_shape& s, const sfi_params& p, int L, void* stat_ws) {
+  return StatLayout(s, p, L, RowMap(), stat_ws).minmax;
+}
 
 sfi_status run_select_stats(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv, int L,
                             void* stat_ws, cudaStream_t st, const RowMap& rows) {
@@ -475,7 +526,8 @@ sfi_status run_select_stats(const sfi_shape& s, const sfi_params& p, const sfi_p
 sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_paged_kv& kv,
                              int L, const float* logits, int64_t ld, const float* lse_cand,
                              float* scores, int64_t ld_s, void* stat_ws,
-                             cudaStream_t st, const RowMap& rows, uint32_t window_mask, bool with_stats) {
+                             cudaStream_t st, const RowMap& rows, uint32_t window_mask, bool with_stats,
+                             bool row_range) {
   const int G = s.Hq / s.Hkv;
   const int nb = rows.count(s.B);
   if (nb < 1 || nb > s.B) return SFI_ERR_SHAPE;
@@ -503,6 +555,7 @@ sfi_status run_select_scores(const sfi_shape& s, const sfi_params& p, const sfi_
   a.alpha_cross = p.alpha_cross;
   a.logits = logits; a.ld = ld; a.lse_cand = lse_cand;
   a.lamz = sl.lamz;
+  a.minmax = row_range ? sl.minmax : nullptr;
   a.kp = kp; a.kp_ld = kp_ld;
   a.scores = scores; a.ld_s = ld_s;
   a.rows = rows;

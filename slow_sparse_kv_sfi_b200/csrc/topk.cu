@@ -55,6 +55,10 @@ struct TopkArgs {
   int64_t ld_b;
   int32_t* idx;              // [rows][ld_i] ascending positions + offset, or null
   int64_t ld_i;
+  // [rows][2]: the largest key and the largest complement of a key of every
+  // row, found by the kernel that wrote the scores (zero between uses; this
+  // kernel zeroes them again), or null: the kernel finds them itself
+  uint32_t* minmax;
 };
 
 // Element e of load u of thread t: score s0 + (u * T + t) * 4 + e, so every
@@ -184,42 +188,48 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
         key[u][e] = j < a.n ? float_key(__ldg(srow + j)) : 0u;
       }
   }
-  // ---- 1. smallest and largest key of the row
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  // ---- 1. smallest and largest key of the row (given, or found here)
+  if (a.minmax == nullptr) {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if (pos_of<T>(s0, u, e) < a.n) {
-        kmin = min(kmin, key[u][e]);
-        kmax = max(kmax, key[u][e]);
+      for (int e = 0; e < 4; ++e)
+        if (pos_of<T>(s0, u, e) < a.n) {
+          kmin = min(kmin, key[u][e]);
+          kmax = max(kmax, key[u][e]);
+        }
+    kmin = block_reduce_u32<T>(kmin, false, wsu);
+    kmax = block_reduce_u32<T>(kmax, true, wsu);
+    if (threadIdx.x == 0) {
+      s_mm[0] = kmin;
+      s_mm[1] = kmax;
+    }
+    csync();
+    if (warp == 0) {
+      uint32_t lo = 0xffffffffu, hi = 0u;
+      if (lane < CS) {
+        const uint32_t* r = s_mm;
+        if constexpr (CS > 1) r = cl.map_shared_rank(s_mm, lane);
+        lo = r[0];
+        hi = r[1];
       }
-  kmin = block_reduce_u32<T>(kmin, false, wsu);
-  kmax = block_reduce_u32<T>(kmax, true, wsu);
-  if (threadIdx.x == 0) {
-    s_mm[0] = kmin;
-    s_mm[1] = kmax;
-  }
-  csync();
-  if (warp == 0) {
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    if (lane < CS) {
-      const uint32_t* r = s_mm;
-      if constexpr (CS > 1) r = cl.map_shared_rank(s_mm, lane);
-      lo = r[0];
-      hi = r[1];
-    }
 #pragma unroll
-    for (int sh = 16; sh >= 1; sh >>= 1) {
-      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, sh));
-      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, sh));
+      for (int sh = 16; sh >= 1; sh >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, sh));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, sh));
+      }
+      if (lane == 0) {
+        wsu[0] = lo;
+        wsu[1] = hi;
+      }
     }
-    if (lane == 0) {
-      wsu[0] = lo;
-      wsu[1] = hi;
-    }
+    __syncthreads();
+  } else if (threadIdx.x == 0) {
+    wsu[0] = ~a.minmax[(size_t)row * 2 + 1];
+    wsu[1] = a.minmax[(size_t)row * 2];
   }
-  __syncthreads();
+  if (a.minmax) __syncthreads();
   const uint32_t gmin = wsu[0], gmax = wsu[1];
   // the passes work on off = key - gmin in [0, gmax - gmin]; hb: its highest
   // bit that can be set (-1: all keys equal)
@@ -419,6 +429,11 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     }
   }
   if constexpr (CS > 1) cl.sync();   // no CTA leaves while another may still read its shared memory
+  // every CTA of the row has read the given range: zero it for the next use
+  if (a.minmax && rank == 0 && threadIdx.x == 0) {
+    a.minmax[(size_t)row * 2] = 0u;
+    a.minmax[(size_t)row * 2 + 1] = 0u;
+  }
 }
 
 template <int T, int CS>
@@ -458,7 +473,7 @@ sfi_status launch_topk_cs(const TopkArgs& a, int threads, cudaStream_t st) {
 int topk_max_n() { return kMaxN; }
 
 sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, int offset, int32_t* idx,
-                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st) {
+                    int64_t ld_i, uint32_t* bits, int64_t ld_b, cudaStream_t st, uint32_t* minmax) {
   if (rows <= 0) return SFI_OK;
   if (n > topk_max_n() || n < 1 || K < 1 || K > n) return SFI_ERR_UNSUPPORTED;
   if (rows > 65535) return SFI_ERR_UNSUPPORTED;
@@ -474,6 +489,7 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
   a.ld_b = ld_b;
   a.idx = idx;
   a.ld_i = ld_i;
+  a.minmax = minmax;
   // slices of T * 32 scores: the fewest CTAs of up to 1024 threads that
   // cover the row, a power of two of them, at most 4 while that suffices.
   // A cluster's CTAs land on distinct SMs of one GPC and a CTA of 1024
