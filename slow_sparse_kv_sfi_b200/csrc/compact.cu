@@ -339,7 +339,8 @@ template <int D, int GM>
 __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_constant__ IncArgs a) {
   grid_dep_enter_writer();
   cg::cluster_group cl = cg::this_cluster();
-  const int cs = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  constexpr int cs = kIncCluster;               // the launch's cluster size
+  const int rank = (int)cl.block_rank();
   const CompactArgs& c = a.c;
   constexpr int T = kIncThreads;
   const int bg = blockIdx.y;                    // logical (row, kv head)
@@ -389,8 +390,12 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
     for (int w = w0 + tid; w < w1; w += T) {
       uint32_t hw[GM];
       const uint32_t u = union_word<GM>(c, b, g, w, hw);
+      uint32_t ow[cs];   // the cluster's loads issued together
+#pragma unroll
+      for (int r = 0; r < cs; ++r) ow[r] = cl.map_shared_rank(oldw, r)[w];
       uint32_t old = 0u;
-      for (int r = 0; r < cs; ++r) old |= cl.map_shared_rank(oldw, r)[w];
+#pragma unroll
+      for (int r = 0; r < cs; ++r) old |= ow[r];
       const uint32_t e = u & ~old;
       entw[w - w0] = e;
       cu += __popc(u);
@@ -405,17 +410,25 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
     }
   }
   cl.sync();
-  if (tid == 0) {
-    int U = 0, E = 0, Eb = 0;
-    for (int r = 0; r < cs; ++r) {
-      const int* pr = cl.map_shared_rank(pub, r);
-      U += pr[0];
-      E += pr[1];
-      if (r < rank) Eb += pr[1];
+  if (warp == 0) {   // lane r reads CTA r's totals
+    int pu = 0, pe = 0;
+    if (lane < cs) {
+      const int* pr = cl.map_shared_rank(pub, lane);
+      pu = pr[0];
+      pe = pr[1];
     }
-    tot[0] = U;
-    tot[1] = E;
-    tot[2] = Eb;
+    int peb = lane < rank ? pe : 0;
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+      pu += __shfl_xor_sync(0xffffffffu, pu, sh);
+      pe += __shfl_xor_sync(0xffffffffu, pe, sh);
+      peb += __shfl_xor_sync(0xffffffffu, peb, sh);
+    }
+    if (lane == 0) {
+      tot[0] = pu;
+      tot[1] = pe;
+      tot[2] = peb;
+    }
   }
   __syncthreads();
   const int n_want = c.n_sink + tot[0];
@@ -451,21 +464,27 @@ __global__ void __launch_bounds__(kIncThreads) inc_refresh_kernel(const __grid_c
     pub[3] = tm;
   }
   cl.sync();
-  if (tid == 0) {
-    int H = 0, Hb = 0, M = 0, Mb = 0;
-    for (int r = 0; r < cs; ++r) {
-      const int* pr = cl.map_shared_rank(pub, r);
-      H += pr[2];
-      M += pr[3];
-      if (r < rank) {
-        Hb += pr[2];
-        Mb += pr[3];
-      }
+  if (warp == 0) {   // lane r reads CTA r's counts
+    int ph = 0, pm = 0;
+    if (lane < cs) {
+      const int* pr = cl.map_shared_rank(pub, lane);
+      ph = pr[2];
+      pm = pr[3];
     }
-    tot[3] = H;
-    tot[4] = Hb;
-    tot[5] = M;
-    tot[6] = Mb;
+    int phb = lane < rank ? ph : 0, pmb = lane < rank ? pm : 0;
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+      ph += __shfl_xor_sync(0xffffffffu, ph, sh);
+      pm += __shfl_xor_sync(0xffffffffu, pm, sh);
+      phb += __shfl_xor_sync(0xffffffffu, phb, sh);
+      pmb += __shfl_xor_sync(0xffffffffu, pmb, sh);
+    }
+    if (lane == 0) {
+      tot[3] = ph;
+      tot[4] = phb;
+      tot[5] = pm;
+      tot[6] = pmb;
+    }
   }
   __syncthreads();
   const int H_tot = tot[3], M_tot = E_tot + tot[5];
