@@ -34,8 +34,7 @@
 
 namespace sfi {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
+constexpr int kConsumerWarps = 4;   // consumer warps of one head group: one per tile of a stage
 constexpr int kBoxBytes = 16 * 128;   // 16 rows x 128 bytes: one column block of a tile
 constexpr long kDenseItemsPerSm = 8;  // dense step: work items per SM
 constexpr long kFastItemTiles = 64;   // fast step: target tiles per work item
@@ -86,9 +85,13 @@ constexpr int kMaxBH = 512;
 // Shared-memory plan.  A tile is 16 rows of K (or V): one TMA box of
 // [D/64 column blocks][16 rows][128 B], 128B-swizzled.  Each consumer warp
 // takes TT tiles of every stage, so a stage holds 4 * TT tiles of K and V.
+// NT head groups of 8: the consumer warps come in NT sets of four, set s
+// taking heads 8s .. 8s + 7 of every tile (the sets read the same tiles).
 // kCps CTAs share an SM; together they keep about 192 KB of copies in flight.
 template <int D, int NT>
 struct Plan {
+  static constexpr int kCW = kConsumerWarps * NT;        // consumer warps
+  static constexpr int kThreads = (kCW + 1) * 32;        // + the producer warp
   static constexpr int kCps = (NT == 1) ? 2 : 1;
   static constexpr int TT = (NT == 1 && kCps == 1) ? 2 : 1;
   static constexpr int kTPS = 4 * TT;
@@ -186,7 +189,7 @@ struct Maps {
 };
 
 template <int D, int NT, int MODE>
-__global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
+__global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
     attn_kernel(const __grid_constant__ Maps maps, const __grid_constant__ AttnArgs a) {
   using S = Smem<D, NT>;
   using P = Plan<D, NT>;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], P::kCW);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -226,13 +229,13 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
   // signal them only at exit), so the copies overlap the previous kernel's
   // tail.  The producer waits before it touches the work counter (reset by
   // the previous combine) or appends the step's token.
-  if (warp != kConsumerWarps) {
+  if (warp != P::kCW) {
     grid_dep_wait();
     if (!a.late_trigger) grid_dep_launch();
   }
 
   // ------------------------------------------------------------ producer warp
-  if (warp == kConsumerWarps) {
+  if (warp == P::kCW) {
     bool waited = false;
     auto ensure_wait = [&]() {
       if (!waited) {
@@ -452,11 +455,14 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
   const int chV = (lane >> 3) & 1;
   const float NEG_INF = -INFINITY;
 
+  // this warp: tile warp % 4 (+ 4 * tt) of every stage, heads hbase .. hbase + 7
+  const int twarp = warp % kConsumerWarps;
+  const int hbase = (warp / kConsumerWarps) * 8;
   int slot = 0;
   uint32_t phase = 0;
-  uint32_t qb[NT][kMT][2];
-  float o[NT][kMT][4];
-  float mrun[NT][2], lrun[NT][2], lcand[NT][2];
+  uint32_t qb[1][kMT][2];
+  float o[1][kMT][4];
+  float mrun[1][2], lrun[1][2], lcand[1][2];
   int cur_b = 0, cur_g = 0;
   for (;;) {
     if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer, a.wait_ns)) {
@@ -477,8 +483,8 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
       cur_g = m.g;
       const uint32_t* q32 = reinterpret_cast<const uint32_t*>(sq + slot * P::kQBytes);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int hh = nt * 8 + r0;
+      for (int nt = 0; nt < 1; ++nt) {
+        const int hh = hbase + nt * 8 + r0;
         const bool hv = hh < a.G;
 #pragma unroll
         for (int ks = 0; ks < kMT; ++ks) {
@@ -505,7 +511,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     bool any = false;
 #pragma unroll
     for (int tt = 0; tt < TT; ++tt) {
-      const int ti = warp + 4 * tt;
+      const int ti = twarp + 4 * tt;
       kind_[tt] = (m.kinds >> (2 * ti)) & 3;
       act[tt] = ti < m.ntiles && kind_[tt] != 2;
       any |= act[tt];
@@ -546,12 +552,12 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
 
     if (any) {
       // S^T = K . Q^T per tile, two independent accumulator chains over D
-      float s[TT][NT][4];
+      float s[TT][1][4];
 #pragma unroll
       for (int tt = 0; tt < TT; ++tt) {
-        float s2[NT][4];
+        float s2[1][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < 1; ++nt)
 #pragma unroll
           for (int i = 0; i < 4; ++i) s[tt][nt][i] = s2[nt][i] = 0.f;
         if (act[tt]) {
@@ -561,28 +567,28 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
             ldmatrix_x4(af, swz(kb_[tt], rowA, ks * 2 + chA));
             ldmatrix_x4(ag, swz(kb_[tt], rowA, (ks + 1) * 2 + chA));
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
+            for (int nt = 0; nt < 1; ++nt) {
               mma_bf16_16816(s[tt][nt], af, qb[nt][ks][0], qb[nt][ks][1]);
               mma_bf16_16816(s2[nt], ag, qb[nt][ks + 1][0], qb[nt][ks + 1][1]);
             }
           }
         }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < 1; ++nt)
 #pragma unroll
           for (int i = 0; i < 4; ++i) s[tt][nt][i] += s2[nt][i];
       }
 
       // mask, scale, online softmax over the warp's TT tiles at once
-      uint32_t pb_hi[TT][NT][2], pb_lo[TT][NT][2];
+      uint32_t pb_hi[TT][1][2], pb_lo[TT][1][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
+      for (int nt = 0; nt < 1; ++nt) {
         float x[TT][4];
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int hh = nt * 8 + cq + (i & 1);
+            const int hh = hbase + nt * 8 + cq + (i & 1);
             const bool v = (rmask[tt][i >> 1] >> hh) & 1u;
             x[tt][i] = (v && hh < a.G) ? s[tt][nt][i] * a.scale_log2 : NEG_INF;
           }
@@ -592,7 +598,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
             if (!act[tt] || kind_[tt] != 0) continue;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int hh = nt * 8 + cq + (i & 1);
+              const int hh = hbase + nt * 8 + cq + (i & 1);
               const int pos = pos0_[tt] + r0 + 8 * (i >> 1);
               if (hh < a.G && pos < a.L)
                 a.logits[((size_t)cur_b * a.Hq + cur_g * a.G + hh) * a.ld + pos] = s[tt][nt][i] * a.scale;
@@ -653,7 +659,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
           uint32_t vf[4];
           ldmatrix_x4_trans(vf, swz(vb_[tt], rowV, mt * 2 + chV));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
+          for (int nt = 0; nt < 1; ++nt) {
             mma_bf16_16816(o[nt][mt], vf, pb_hi[tt][nt][0], pb_hi[tt][nt][1]);
             mma_bf16_16816(o[nt][mt], vf, pb_lo[tt][nt][0], pb_lo[tt][nt][1]);
           }
@@ -672,7 +678,7 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
     // global memory as it is (m, l, l_cand and the unnormalised O of each
     // query head); the combine kernel merges all partials.
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < 1; ++nt)
 #pragma unroll
       for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -680,21 +686,21 @@ __global__ void __launch_bounds__(kAttnThreads, Plan<D, NT>::kCps)
           lrun[nt][j] += __shfl_xor_sync(0xffffffffu, lrun[nt][j], sh);
           if (MODE == kDenseExtras) lcand[nt][j] += __shfl_xor_sync(0xffffffffu, lcand[nt][j], sh);
         }
-    float* part = a.part + ((size_t)item * kConsumerWarps + warp) * a.G * (D + 4);
+    float* part = a.part + ((size_t)item * kConsumerWarps + twarp) * a.G * (D + 4);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int nt = 0; nt < 1; ++nt) {
 #pragma unroll
       for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int hh = nt * 8 + cq + (i & 1);
+          const int hh = hbase + nt * 8 + cq + (i & 1);
           const int d = mt * 16 + r0 + (i >> 1) * 8;
           if (hh < a.G) part[hh * (D + 4) + d] = o[nt][mt][i];
         }
       if (lane < 4) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int hh = nt * 8 + cq + j;
+          const int hh = hbase + nt * 8 + cq + j;
           if (hh < a.G) {
             part[hh * (D + 4) + D] = mrun[nt][j];
             part[hh * (D + 4) + D + 1] = lrun[nt][j];
@@ -954,7 +960,7 @@ sfi_status launch_attn_t(const Maps& maps, const AttnArgs& a, cudaStream_t st) {
     if (!attr.mark(e)) return SFI_ERR_CUDA;
   }
   const int grid = std::min(a.n_items, num_sms() * Plan<D, NT>::kCps);
-  launch_k(kern, dim3(grid), dim3(kAttnThreads), S::kTotal, st, maps, a);
+  launch_k(kern, dim3(grid), dim3(Plan<D, NT>::kThreads), S::kTotal, st, maps, a);
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
