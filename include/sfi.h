@@ -28,6 +28,14 @@
  *    by value and is the same for every sequence of the batch.
  *  - Device pointers handed to TMA (k_pool, v_pool, packed k/v) must be
  *    16-byte aligned.  Nothing here ever aborts or exits the process.
+ *  - Consecutive calls on one stream overlap on the GPU: an attention call
+ *    starts loading its query and cache rows, and a fast call appends its
+ *    token, while the two attention calls before it on the same stream
+ *    finish.  So the query of an attention call must not be the output of
+ *    either of those two calls, and a fast call must not append to a cache
+ *    row that they read or append.  (In a decode loop each layer has its own
+ *    rows and other kernels produce the query.)  Any kernel or copy of the
+ *    caller's in between orders the calls fully.
  */
 #ifndef SFI_H_
 #define SFI_H_
@@ -397,13 +405,16 @@ sfi_status sfi_ctx_join(sfi_ctx* ctx, sfi_stream stream);
 
 /* Per-kernel CUDA-event timing of the attention kernels launched by
  * sfi_decode_step (kind 0 = fast-attention main kernel, 1 = dense main
- * kernel).  sfi_ctx_set_timing(ctx, n): n = 0 off; n > 0 brackets the
- * attention launches of layers 0, n, 2n, ... with an event pair (an event
- * between two launches keeps the second from starting early, so sparse
- * sampling leaves the other layers' launches overlapped).  sfi_ctx_timing
+ * kernel).  A utility of this library, no step of the pages.
+ * sfi_ctx_set_timing_layers(ctx, first, n): n = 0 off; n > 0 brackets the
+ * attention launches of layers first, first + n, first + 2n, ... with an
+ * event pair (an event between two launches keeps the second from starting
+ * early, so sparse sampling leaves the other layers' launches overlapped).
+ * sfi_ctx_set_timing(ctx, n) is the same with first = 0.  sfi_ctx_timing
  * synchronises on the recorded events and returns total milliseconds and
  * launch count since the last reset. */
 sfi_status sfi_ctx_set_timing(sfi_ctx* ctx, int32_t layer_stride);
+sfi_status sfi_ctx_set_timing_layers(sfi_ctx* ctx, int32_t first_layer, int32_t layer_stride);
 sfi_status sfi_ctx_timing(sfi_ctx* ctx, int32_t kind, double* total_ms, int64_t* launches,
                           int32_t reset);
 

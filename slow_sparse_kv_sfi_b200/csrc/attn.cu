@@ -221,16 +221,22 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
     fence_barrier_init();
   }
   __syncthreads();
-  // The consumers wait for the previous kernel of the stream before anything
-  // else (they write the partials, which it may still read).  The producer
-  // issues its first copies at once: the query, the pages, the page table,
-  // the packed buffers and n_rows are written by no kernel of this library
-  // that lets its dependents start early (the append and the compaction
-  // signal them only at exit), so the copies overlap the previous kernel's
-  // tail.  The producer waits before it touches the work counter (reset by
-  // the previous combine) or appends the step's token.
+  // Ordering with the previous kernels of the stream.  The producer issues
+  // its first copies at once: the query, the pages, the page table, the
+  // packed buffers and n_rows are written by no kernel of this library that
+  // lets its dependents start early (the append and the compaction signal
+  // them only at exit), so the copies overlap the previous kernels' tails.
+  // The producer waits before it touches the work counter (reset by the
+  // previous combine).  The dense consumers wait at once (they write logits
+  // from their first tile on).  The fast consumers let the next kernel start
+  // at once; they read shared memory only until the end of their first item
+  // and wait there, before their first partial (the previous combine may
+  // still read the partials).  Every write that a kernel before this one
+  // reads or writes (the partials, the counter) thus follows a wait, and the
+  // waits chain: the previous combine waited for the previous attention,
+  // whose consumers waited for the combine before it.
   if (warp != P::kCW) {
-    grid_dep_wait();
+    if (MODE != kFast) grid_dep_wait();
     if (!a.late_trigger) grid_dep_launch();
   }
 
@@ -321,9 +327,12 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
         nst = max(1, (it.t_end - it.t_begin + kTPS - 1) / kTPS);
         p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
         // the item holding position L - 1 first appends the step's token
-        // there (the whole warp), before any copy of that tile is issued
+        // there (the whole warp), before any copy of that tile is issued.  A
+        // fast step appends without waiting: the kernels still running (the
+        // previous attention launch and its combine) neither read nor write
+        // that row of this cache.
         if (a.k_new && it.t_begin < it.t_end && it.t_end == it.t_total) {
-          ensure_wait();
+          if (MODE != kFast) ensure_wait();
           const int pos = a.L - 1;
           append_row_warp<D>(lane, it.bg, it.g, pos, ptbuf[pos / kPage - p_lo], a.Hkv, a.num_pages, a.k_pool,
                              a.v_pool, a.k_new, a.v_new, a.norms, a.norm_ld, a.err);
@@ -464,15 +473,18 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
   float o[1][kMT][4];
   float mrun[1][2], lrun[1][2], lcand[1][2];
   int cur_b = 0, cur_g = 0;
+  bool waited = MODE != kFast;   // the dense consumers waited at their start
   for (;;) {
     if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer, a.wait_ns)) {
       *abort_flag = 1;
+      if (!waited) grid_dep_wait();
       if (a.late_trigger) grid_dep_launch();
       break;
     }
     const StageMeta& m = smeta[slot];
     const int item = m.item;
     if (item < 0) {
+      if (!waited) grid_dep_wait();
       if (a.late_trigger) grid_dep_launch();
       break;
     }
@@ -686,6 +698,10 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
           lrun[nt][j] += __shfl_xor_sync(0xffffffffu, lrun[nt][j], sh);
           if (MODE == kDenseExtras) lcand[nt][j] += __shfl_xor_sync(0xffffffffu, lcand[nt][j], sh);
         }
+    if (!waited) {
+      grid_dep_wait();
+      waited = true;
+    }
     float* part = a.part + ((size_t)item * kConsumerWarps + twarp) * a.G * (D + 4);
 #pragma unroll
     for (int nt = 0; nt < 1; ++nt) {
@@ -712,23 +728,41 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
   }
 }
 
-// Merge the partials of every (b, query head): one CTA of kCombWarps warps
-// each, one pass.  Warp w folds partials w, w + kCombWarps, ... (eight loads
-// in flight per lane, each partial's m, l, l_C and a 4-column slice of O per
-// lane) into a running (m, l, l_C, O) with online rescaling; the warps' states
-// meet in shared memory, where thread d merges column d.
+// Merge the partials of every (b, query head): one CTA of NW warps each, one
+// pass.  Warp w folds partials w, w + NW, ... (IN loads in flight per lane,
+// each partial's m, l, l_C and a 4-column slice of O per lane) into a running
+// (m, l, l_C, O) with online rescaling; the warps' states meet in shared
+// memory, where thread d merges column d.
+//  - After a dense step: 24 warps, eight loads in flight (the merge is on the
+//    path to the Selector).
+//  - After a fast step whose attention runs one CTA per SM (G > 8;
+//    attn_combine_fast_kernel): 7 warps of at most 64 registers and 4 KB of
+//    shared memory, which fit on an SM beside that CTA.  It lets the next
+//    launch start at once, so the merge runs while the attention finishes
+//    and the next layer's attention starts, instead of holding an SM.  Beside
+//    two attention CTAs per SM (G <= 8) it does not fit, and the fast steps
+//    take the 24-warp merge.
 constexpr int kCombWarps = 24;
+constexpr int kCombWarpsFast = 7;
 
-template <int D>
-__global__ void __launch_bounds__(kCombWarps * 32)
-    attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
-                        float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
-                        const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
-                        const __grid_constant__ RowMap rows) {
-  grid_dep_enter();
+template <int D, int NW>
+__device__ __forceinline__ void combine_body(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv,
+                                             int G, float* __restrict__ out, float* __restrict__ lse,
+                                             float* __restrict__ lse_cand, const int32_t* n_rows, int p_max,
+                                             int rec_tiles, int tps, int* err, int* ctr, int early,
+                                             const RowMap& rows) {
+  // After a fast step the next launch may start before this one has waited:
+  // it is the next layer's attention, whose consumers wait before their
+  // first partial and whose producer waits before it touches the counter.
+  if (early) {
+    grid_dep_launch();
+    grid_dep_wait();
+  } else {
+    grid_dep_enter();
+  }
   constexpr int kPer = D / 32;     // columns of O per lane
   static_assert(kPer == 4 || kPer == 2, "head dim");
-  __shared__ float red[kCombWarps][D + 4];
+  __shared__ float red[NW][D + 4];
   if (blockIdx.x == 0 && threadIdx.x == 0) ctr[0] = 0;   // the attention kernel is done with it
   const int bl = blockIdx.x / Hq, hq = blockIdx.x - bl * Hq;   // logical row of the launch, query head
   const int b = rows.phys(bl);
@@ -754,18 +788,18 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     chunks = (T + ct - 1) / ct;
   }
   const int n = chunks * kConsumerWarps;
+  constexpr int kIn = NW > 8 ? 8 : 6;   // partials in flight per warp
   const float* base = part + (size_t)bgl * n_chunks * kConsumerWarps * stride + (size_t)hh * (D + 4);
   float m = -INFINITY, l = 0.f, lc = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  constexpr int kIn = 8;   // partials in flight per warp
-  for (int c0 = warp; c0 < n; c0 += kIn * kCombWarps) {
+  for (int c0 = warp; c0 < n; c0 += kIn * NW) {
     float st[kIn][3];
     float ov[kIn][kPer];
 #pragma unroll
     for (int u = 0; u < kIn; ++u) {
-      const int c = c0 + u * kCombWarps;
+      const int c = c0 + u * NW;
       if (c < n) {
         const float* pc = base + c * stride;
         st[u][0] = __ldg(pc + D);
@@ -819,11 +853,11 @@ __global__ void __launch_bounds__(kCombWarps * 32)
   if (threadIdx.x < D) {
     float M = -INFINITY;
 #pragma unroll 8
-    for (int w = 0; w < kCombWarps; ++w) M = fmaxf(M, red[w][D]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[w][D]);
     const float mref = (M == -INFINITY) ? 0.f : M;
     float lt = 0.f, lct = 0.f, o = 0.f;
 #pragma unroll 8
-    for (int w = 0; w < kCombWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const float wt = fast_exp2(red[w][D] - mref);
       lt += wt * red[w][D + 1];
       lct += wt * red[w][D + 2];
@@ -835,6 +869,26 @@ __global__ void __launch_bounds__(kCombWarps * 32)
       if (lse_cand) lse_cand[row] = lct > 0.f ? (M + log2f(lct)) * kLn2 : -INFINITY;
     }
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCombWarps * 32)
+    attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
+                        float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
+                        const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
+                        int early, const __grid_constant__ RowMap rows) {
+  combine_body<D, kCombWarps>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles, tps,
+                              err, ctr, early, rows);
+}
+
+template <int D>
+__global__ void __maxnreg__(64)
+    attn_combine_fast_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
+                             float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
+                             const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
+                             int early, const __grid_constant__ RowMap rows) {
+  combine_body<D, kCombWarpsFast>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles,
+                                  tps, err, ctr, early, rows);
 }
 
 __global__ void probs_kernel(int L, int Hq, const float* __restrict__ logits, int64_t ld,
@@ -976,15 +1030,20 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int rec_tiles, int tps,
-                          int* err, int* ctr, cudaStream_t st, const RowMap& rows) {
+                          int* err, int* ctr, cudaStream_t st, const RowMap& rows, int early) {
   const int G = s.Hq / s.Hkv;
   const int grid = rows.count(s.B) * s.Hq;
-  if (D == 128)
-    launch_k(attn_combine_kernel<128>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr, rows);
-  else
-    launch_k(attn_combine_kernel<64>, dim3(grid), dim3(kCombWarps * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G,
-             out, lse, lse_cand, n_rows, p_max, rec_tiles, tps, err, ctr, rows);
+  auto go = [&](auto kern, int nw) {
+    launch_k(kern, dim3(grid), dim3(nw * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse, lse_cand, n_rows,
+             p_max, rec_tiles, tps, err, ctr, early, rows);
+  };
+  if (early) {
+    if (D == 128) go(attn_combine_fast_kernel<128>, kCombWarpsFast);
+    else go(attn_combine_fast_kernel<64>, kCombWarpsFast);
+  } else {
+    if (D == 128) go(attn_combine_kernel<128>, kCombWarps);
+    else go(attn_combine_kernel<64>, kCombWarps);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
@@ -1115,7 +1174,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
   r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0, 0, 1,
-                     kv.err, ctr, st, rmap);
+                     kv.err, ctr, st, rmap, 0);
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
     if (rmap.n) return SFI_ERR_UNSUPPORTED;   // probabilities of the whole batch only
@@ -1164,8 +1223,12 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
   const int rec_tiles = (L - 1) / kPage - a.rec_lo / kPage + 1;
+  // The small merge that lets the next launch start early fits on an SM only
+  // beside an attention grid of one CTA per SM (G > 8); beside two it waits
+  // for an attention CTA to leave, and the 24-warp merge is the faster one.
+  const int early = attn_grid(s.D, G).ctas <= num_sms() ? 1 : 0;
   return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, rec_tiles, nts, kv.err,
-                        ctr, st, rmap);
+                        ctr, st, rmap, early);
 }
 
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,

@@ -69,7 +69,8 @@ struct sfi_ctx {
   std::vector<sfi::AttnMapCache> maps;   // per layer
   // timing of the attention kernels (kind 0 fast, 1 dense) of every
   // timing-th layer (0: off)
-  int timing = 0;
+  int timing = 0;         // layer stride of the timed attention launches (0: off)
+  int timing_first = 0;   // first timed layer
   std::vector<cudaEvent_t> tev[2];
   size_t tused[2] = {0, 0};
 };
@@ -143,7 +144,7 @@ sfi_status cu(cudaError_t e) { return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA; 
 // Event pair for one timed launch, or nulls when timing is off.
 void timing_events(sfi_ctx* c, int kind, int layer, cudaEvent_t* b, cudaEvent_t* e) {
   *b = *e = nullptr;
-  if (c->timing <= 0 || layer % c->timing != 0) return;
+  if (c->timing <= 0 || layer < c->timing_first || (layer - c->timing_first) % c->timing != 0) return;
   auto& v = c->tev[kind];
   if (c->tused[kind] + 2 > v.size()) {
     for (int i = 0; i < 256; ++i) {
@@ -456,8 +457,13 @@ sfi_status sfi_ctx_join(sfi_ctx* c, sfi_stream stream) {
 }
 
 sfi_status sfi_ctx_set_timing(sfi_ctx* c, int32_t layer_stride) {
-  if (!c || layer_stride < 0) return SFI_ERR_INVALID_ARG;
+  return sfi_ctx_set_timing_layers(c, 0, layer_stride);
+}
+
+sfi_status sfi_ctx_set_timing_layers(sfi_ctx* c, int32_t first_layer, int32_t layer_stride) {
+  if (!c || layer_stride < 0 || first_layer < 0) return SFI_ERR_INVALID_ARG;
   c->timing = layer_stride;
+  c->timing_first = first_layer;
   return SFI_OK;
 }
 

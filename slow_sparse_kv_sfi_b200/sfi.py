@@ -99,6 +99,7 @@ def _declare(L):
         "sfi_decode_step_rows": (C.c_int, [P, I32, I32, P, I32, P, P, P, P, P, P, P, P]),
         "sfi_ctx_join": (C.c_int, [P, P]),
         "sfi_ctx_set_timing": (C.c_int, [P, I32]),
+        "sfi_ctx_set_timing_layers": (C.c_int, [P, I32, I32]),
         "sfi_ctx_set_compaction": (C.c_int, [P, I32]),
         "sfi_ctx_timing": (C.c_int, [P, I32, C.POINTER(C.c_double), C.POINTER(I64), I32]),
     }
@@ -115,7 +116,7 @@ EXPORTED = ["sfi_status_str", "sfi_version", "sfi_workspace_size", "sfi_packed_r
             "sfi_compact_incremental", "sfi_poll_error", "sfi_set_wait_limit", "sfi_get_wait_limit",
             "sfi_selftest_wait",
             "sfi_ctx_create", "sfi_ctx_destroy", "sfi_ctx_workspace_size", "sfi_ctx_set_workspace",
-            "sfi_decode_step", "sfi_decode_step_rows", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_compaction",
+            "sfi_decode_step", "sfi_decode_step_rows", "sfi_ctx_join", "sfi_ctx_set_timing", "sfi_ctx_set_timing_layers", "sfi_ctx_set_compaction",
             "sfi_ctx_timing"]
 
 
@@ -343,9 +344,10 @@ class Context:
     def join(self, stream=None):
         _check(lib().sfi_ctx_join(self.h, _stream(stream)), "sfi_ctx_join")
 
-    def set_timing(self, layer_stride: int):
-        """Time the attention launches of layers 0, n, 2n, ... (n = layer_stride; 0 = off)."""
-        _check(lib().sfi_ctx_set_timing(self.h, int(layer_stride)), "sfi_ctx_set_timing")
+    def set_timing(self, layer_stride: int, first_layer: int = 0):
+        """Time the attention launches of layers first, first + n, ... (n = layer_stride; 0 = off)."""
+        _check(lib().sfi_ctx_set_timing_layers(self.h, int(first_layer), int(layer_stride)),
+               "sfi_ctx_set_timing_layers")
 
     def timing(self, kind: int, reset: bool = True):
         ms = C.c_double(0)
