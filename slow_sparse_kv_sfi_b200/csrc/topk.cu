@@ -4,9 +4,12 @@
 //
 // Exact MSB radix select on the order-preserving uint32 image of every fp32
 // score, one thread-block cluster per row.  The row is cut into slices of
-// T * 32 scores, one CTA of T threads each (1, 2, 4 or 8 CTAs, cluster rank
-// = slice), and every thread keeps its 32 keys in registers for the whole
-// kernel, so the scores are read once:
+// T * 32 * KU / 8 scores, one CTA of T threads each (1, 2, 4 or 8 CTAs,
+// cluster rank = slice), and every thread keeps its keys on chip for the
+// whole kernel, so the scores are read once: 32 in registers, and with KU =
+// 16 another 32 in shared memory (a CTA of 1024 threads fills an SM's
+// registers, so the second half halves the CTAs of a row and the waves of a
+// launch):
 //   1. the cluster's smallest and largest key: the passes work on the offset
 //      key - smallest, whose bits above the highest bit of (largest -
 //      smallest) are zero, in as few passes of at most 14 bits as cover the
@@ -40,7 +43,7 @@ namespace sfi {
 
 namespace {
 
-constexpr int kKPT = 32;              // keys per thread: 8 loads of 4
+constexpr int kKPT = 32;              // keys per thread in registers: 8 loads of 4
 constexpr int kMaxCluster = 8;        // portable cluster size
 constexpr int kDigitBits = 14;        // widest digit
 constexpr int kDigitBins = 1 << kDigitBits;
@@ -62,7 +65,8 @@ struct TopkArgs {
 };
 
 // Element e of load u of thread t: score s0 + (u * T + t) * 4 + e, so every
-// warp-wide load reads 512 consecutive bytes.
+// warp-wide load reads 512 consecutive bytes.  Loads 0 .. 7 stay in
+// registers, loads 8 .. 15 (KU = 16) in shared memory.
 template <int T>
 __device__ __forceinline__ int pos_of(int s0, int u, int e) {
   return s0 + (u * T + (int)threadIdx.x) * 4 + e;
@@ -117,10 +121,13 @@ __device__ __forceinline__ uint32_t block_reduce_u32(uint32_t v, bool take_max, 
   return r;
 }
 
-// Dynamic shared memory of the kernel: the digit histogram, then (clusters of
-// more than one CTA) this CTA's range of the cluster-wide histogram.
-__host__ __device__ constexpr size_t topk_smem_bytes(int cs) {
-  return (size_t)kDigitBins * 4 + (cs > 1 ? (size_t)((kDigitBins + cs - 1) / cs) * 4 : 0);
+// Dynamic shared memory of the kernel: the digit histogram (after the passes:
+// the selection and tie words), then (clusters of more than one CTA) this
+// CTA's range of the cluster-wide histogram, then (KU = 16) the keys of loads
+// 8 .. 15, [32][T].
+__host__ __device__ constexpr size_t topk_red_ints(int cs) { return cs > 1 ? (size_t)((kDigitBins + cs - 1) / cs) : 0; }
+__host__ __device__ constexpr size_t topk_smem_bytes(int cs, int t, int ku) {
+  return (size_t)kDigitBins * 4 + topk_red_ints(cs) * 4 + (ku > 8 ? (size_t)32 * t * 4 : 0);
 }
 
 // Reads one int that every CTA of the cluster published at `pub` (lanes c <
@@ -143,18 +150,32 @@ __device__ __forceinline__ int published_before(cg::cluster_group& cl, int* pub,
   return v;
 }
 
-template <int T, int CS>
+// Key of element e of load u: registers for u < 8, shared memory for u >= 8
+// (u and e are constants after unrolling).
+template <int T>
+__device__ __forceinline__ uint32_t& key_at(uint32_t (&key)[8][4], uint32_t* skey, int u, int e) {
+  return u < 8 ? key[u & 7][e] : skey[((u - 8) * 4 + e) * T + threadIdx.x];
+}
+
+template <int T, int CS, int KU>
 __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__ TopkArgs a) {
+  static_assert(KU == 8 || KU == 16, "loads per thread");
+  constexpr int W = KU / 8;         // bitmap words per thread
   grid_dep_enter();
   cg::cluster_group cl = cg::this_cluster();
   const int rank = CS > 1 ? (int)cl.block_rank() : 0;
   const int row = blockIdx.y;
-  const int s0 = rank * T * kKPT;
+  const int s0 = rank * T * KU * 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   extern __shared__ int dyn[];
   int* hist = dyn;                  // [2^nbits] this CTA's digit counts; then a copy of the chosen range
   int* red = dyn + kDigitBins;      // this CTA's range, summed over the cluster (CS > 1)
-  __shared__ uint32_t selw[T], tiew[T];
+  uint32_t* skey = reinterpret_cast<uint32_t*>(dyn + kDigitBins + topk_red_ints(CS));   // KU = 16: [32][T]
+  // after the passes the histogram holds the selection and tie words of the
+  // slice: thread i owns words i, T + i, ... (in position order, word w
+  // covering scores s0 + 32 w .. s0 + 32 w + 31)
+  uint32_t* selw = reinterpret_cast<uint32_t*>(hist);
+  uint32_t* tiew = selw + W * T;
   __shared__ int ws[33];
   __shared__ uint32_t wsu[32];
   __shared__ int pub[3];            // published to the cluster: range total, ties, selected
@@ -165,10 +186,33 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     else __syncthreads();
   };
 
-  // ---- keys
+  // ---- keys (loads 8 .. 15 first, into shared memory)
   const float* srow = a.scores + (size_t)row * a.ld_s;
   uint32_t key[8][4];
-  if (a.vec && s0 + T * kKPT <= a.n) {
+  const bool full = a.vec && s0 + T * KU * 4 <= a.n;
+  if constexpr (KU > 8) {
+    if (full) {
+      float4 f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(srow + pos_of<T>(s0, 8 + u, 0)));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        skey[(u * 4 + 0) * T + threadIdx.x] = float_key(f[u].x);
+        skey[(u * 4 + 1) * T + threadIdx.x] = float_key(f[u].y);
+        skey[(u * 4 + 2) * T + threadIdx.x] = float_key(f[u].z);
+        skey[(u * 4 + 3) * T + threadIdx.x] = float_key(f[u].w);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = pos_of<T>(s0, 8 + u, e);
+          skey[(u * 4 + e) * T + threadIdx.x] = j < a.n ? float_key(__ldg(srow + j)) : 0u;
+        }
+    }
+  }
+  if (full) {
     float4 f[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) f[u] = __ldg(reinterpret_cast<const float4*>(srow + pos_of<T>(s0, u, 0)));
@@ -192,12 +236,13 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   if (a.minmax == nullptr) {
     uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < KU; ++u)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (pos_of<T>(s0, u, e) < a.n) {
-          kmin = min(kmin, key[u][e]);
-          kmax = max(kmax, key[u][e]);
+          const uint32_t v = key_at<T>(key, skey, u, e);
+          kmin = min(kmin, v);
+          kmax = max(kmax, v);
         }
     kmin = block_reduce_u32<T>(kmin, false, wsu);
     kmax = block_reduce_u32<T>(kmax, true, wsu);
@@ -239,9 +284,9 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   uint32_t prefix = 0u;
   int k = a.K;
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
+  for (int u = 0; u < KU; ++u)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) key[u][e] -= gmin;
+    for (int e = 0; e < 4; ++e) key_at<T>(key, skey, u, e) -= gmin;
 
   // ---- 2. digit passes over bits hb .. 0, as few as cover them, balanced
   const int npass = (hb + 1 + kDigitBits - 1) / kDigitBits;
@@ -256,10 +301,10 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     __syncthreads();
     // the keys still matching the prefix, counted by digit
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < KU; ++u)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint32_t off = key[u][e];
+        const uint32_t off = key_at<T>(key, skey, u, e);
         if (pos_of<T>(s0, u, e) < a.n && (off & pmask) == prefix) atomicAdd(&hist[(off >> shift) & dm], 1);
       }
     csync();   // every histogram of the cluster complete
@@ -355,13 +400,13 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   const uint32_t thr = prefix;
   const bool take_all_ties = (hb < 0 ? a.n : s_pick[3]) == k;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
+  for (int u = 0; u < KU; ++u) {
     const int jb = pos_of<T>(s0, u, 0);
     uint32_t up = 0u, eq = 0u;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (jb + e < a.n) {
-        const uint32_t off = key[u][e];
+        const uint32_t off = key_at<T>(key, skey, u, e);
         up |= (off > thr ? 1u : 0u) << e;
         eq |= (off == thr ? 1u : 0u) << e;
       }
@@ -380,52 +425,76 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
     }
   }
   __syncthreads();
-  // thread i owns word i of the slice (words are in position order)
+  // thread i owns words i, T + i, ... of the slice
   const int i = threadIdx.x;
-  const uint32_t tw = tiew[i];
-  uint32_t take = tw;
-  if (!take_all_ties) {   // the same decision in every CTA of the cluster
-    int ties_tot;
-    const int tie_before_local = block_excl<T>(__popc(tw), ws, &ties_tot);
-    if (threadIdx.x == 0) pub[1] = ties_tot;
+  uint32_t sw[W];
+  if (take_all_ties) {
+#pragma unroll
+    for (int j = 0; j < W; ++j) sw[j] = selw[j * T + i] | tiew[j * T + i];
+  } else {   // the same decision in every CTA of the cluster
+    int before[W];
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      int tot;
+      before[j] = base + block_excl<T>(__popc(tiew[j * T + i]), ws, &tot);
+      base += tot;
+    }
+    if (threadIdx.x == 0) pub[1] = base;
     csync();
     if (warp == 0) {
       const int sb = published_before<CS>(cl, pub + 1, lane, rank);
       if (lane == 0) s_pick[1] = sb;
     }
     __syncthreads();
-    int rk = s_pick[1] + tie_before_local;
-    uint32_t t = tw;
-    take = 0u;
-    while (t && rk < k) {
-      const uint32_t lowbit = t & (~t + 1u);
-      take |= lowbit;
-      t ^= lowbit;
-      ++rk;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      int rk = s_pick[1] + before[j];
+      uint32_t t = tiew[j * T + i];
+      uint32_t take = 0u;
+      while (t && rk < k) {
+        const uint32_t lowbit = t & (~t + 1u);
+        take |= lowbit;
+        t ^= lowbit;
+        ++rk;
+      }
+      sw[j] = selw[j * T + i] | take;
     }
   }
-  const uint32_t sw = selw[i] | take;
-  const int word = rank * T + i;
   const int nw = (a.n + 31) / 32;
-  if (a.bits && word < nw) a.bits[(size_t)row * a.ld_b + word] = sw;
+#pragma unroll
+  for (int j = 0; j < W; ++j) {
+    const int word = rank * W * T + j * T + i;
+    if (a.bits && word < nw) a.bits[(size_t)row * a.ld_b + word] = sw[j];
+  }
   if (a.idx) {
-    int sel_tot;
-    const int sel_before_local = block_excl<T>(__popc(sw), ws, &sel_tot);
-    if (threadIdx.x == 0) pub[2] = sel_tot;
+    int before[W];
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      int tot;
+      before[j] = base + block_excl<T>(__popc(sw[j]), ws, &tot);
+      base += tot;
+    }
+    if (threadIdx.x == 0) pub[2] = base;
     csync();
     if (warp == 0) {
       const int sb = published_before<CS>(cl, pub + 2, lane, rank);
       if (lane == 0) s_pick[1] = sb;
     }
     __syncthreads();
-    int at = s_pick[1] + sel_before_local;
     int32_t* out = a.idx + (size_t)row * a.ld_i;
-    uint32_t x = sw;
-    while (x) {
-      const int bpos = __ffs(x) - 1;
-      x &= x - 1u;
-      if (at < a.K) out[at] = a.offset + word * 32 + bpos;
-      ++at;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+      const int word = rank * W * T + j * T + i;
+      int at = s_pick[1] + before[j];
+      uint32_t x = sw[j];
+      while (x) {
+        const int bpos = __ffs(x) - 1;
+        x &= x - 1u;
+        if (at < a.K) out[at] = a.offset + word * 32 + bpos;
+        ++at;
+      }
     }
   }
   if constexpr (CS > 1) cl.sync();   // no CTA leaves while another may still read its shared memory
@@ -436,17 +505,17 @@ __global__ void __launch_bounds__(T) topk_cluster_kernel(const __grid_constant__
   }
 }
 
-template <int T, int CS>
+template <int T, int CS, int KU>
 sfi_status launch_topk(const TopkArgs& a, cudaStream_t st) {
   static DeviceOnce smem_attr;
-  if (!smem_attr.done() && !smem_attr.mark(cudaFuncSetAttribute(topk_cluster_kernel<T, CS>,
+  if (!smem_attr.done() && !smem_attr.mark(cudaFuncSetAttribute(topk_cluster_kernel<T, CS, KU>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      (int)topk_smem_bytes(CS))))
+                                                      (int)topk_smem_bytes(CS, T, KU))))
     return SFI_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, a.rows);
   cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = topk_smem_bytes(CS);
+  cfg.dynamicSmemBytes = topk_smem_bytes(CS, T, KU);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -457,15 +526,15 @@ sfi_status launch_topk(const TopkArgs& a, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T, CS>, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<T, CS, KU>, a);
   return e == cudaSuccess ? SFI_OK : SFI_ERR_CUDA;
 }
 
 template <int CS>
 sfi_status launch_topk_cs(const TopkArgs& a, int threads, cudaStream_t st) {
-  if (threads <= 256) return launch_topk<256, CS>(a, st);
-  if (threads <= 512) return launch_topk<512, CS>(a, st);
-  return launch_topk<1024, CS>(a, st);
+  if (threads <= 256) return launch_topk<256, CS, 8>(a, st);
+  if (threads <= 512) return launch_topk<512, CS, 8>(a, st);
+  return launch_topk<1024, CS, 8>(a, st);
 }
 
 }  // namespace
@@ -497,6 +566,17 @@ sfi_status run_topk(int rows, int n, const float* scores, int64_t ld_s, int K, i
   // many at once as clusters of 8 of 512-thread CTAs.
   int cs = 1;
   while (cs < kMaxCluster && cs * 1024 * kKPT < n) cs *= 2;
+  // With more CTAs than SMs (one CTA of 1024 threads per SM) the rows run in
+  // waves; 32 more keys per thread in shared memory halve the CTAs of a row.
+  // Then every CTA has 1024 threads: cs * 1024 * 32 < n made cs, so the half
+  // needs more than 512 threads.
+  if (cs >= 2 && (long)rows * cs > num_sms()) {
+    switch (cs / 2) {
+      case 1: return launch_topk<1024, 1, 16>(a, st);
+      case 2: return launch_topk<1024, 2, 16>(a, st);
+      default: return launch_topk<1024, 4, 16>(a, st);
+    }
+  }
   const int need = (n + cs * kKPT - 1) / (cs * kKPT);   // threads per slice
   switch (cs) {
     case 1: return launch_topk_cs<1>(a, need, st);

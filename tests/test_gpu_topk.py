@@ -1,10 +1,12 @@
 """sfi_topk against the oracle's top-K (K largest, ties to the lower index,
 ascending) on inputs that reach every path of the cluster kernel: one to
 eight slices per row with a ragged last one and slices holding no score,
-256, 512 and 1024 threads per slice (n up to the 262144 maximum), rows that
-are not 16-byte aligned, exact ties at the threshold, rows whose keys share
-no leading bit or all of them (constant rows), K = 1 and K = n, and calls of
-different sizes in a row."""
+256, 512 and 1024 threads per slice (n up to the 262144 maximum), 32 keys
+per thread in registers or (launches with more 1024-thread CTAs than a B200
+has SMs) 64 with half of them in shared memory, rows that are not 16-byte
+aligned, exact ties at the threshold, rows whose keys share no leading bit
+or all of them (constant rows), K = 1 and K = n, and calls of different
+sizes in a row."""
 import numpy as np
 import pytest
 import torch
@@ -51,6 +53,12 @@ def _check(x, K, **kw):
     (1, 262144, 50000),     # eight slices of 1024 threads, full
     (2, 200001, 7),         # eight slices, ragged
     (3, 70000, 9000),       # four slices, the last ones partly empty
+    # more CTAs than SMs with 32 keys per thread: 64 per thread, half of
+    # them in shared memory, half the slices
+    (64, 130812, 19622),    # two slices, ragged (the 128K layer's rows)
+    (80, 40000, 6000),      # one slice of 1024 threads, ragged
+    (76, 65536, 1000),      # one slice, exactly full
+    (40, 200001, 30000),    # four slices, the last one mostly empty
 ])
 def test_topk_random(rows, n, K):
     rng = np.random.default_rng(n + K)
@@ -68,6 +76,15 @@ def test_topk_ties_at_threshold_go_to_lower_positions():
     rng = np.random.default_rng(9)
     n = 50000
     x = rng.integers(0, 40, size=(4, n)).astype(np.float32)    # few distinct values, many ties
+    _check(x, 12345)
+
+
+def test_topk_ties_and_constant_rows_with_keys_in_shared_memory():
+    rng = np.random.default_rng(17)
+    rows, n = 160, 40000                         # 160 rows x 2 slices > 148 SMs
+    x = rng.integers(0, 40, size=(rows, n)).astype(np.float32)
+    x[3] = 2.0                                   # a constant row
+    x[7, :5] = [1e4, -1e4, 2e4, -2e4, 3e4]       # outliers squeeze the rest into one bin
     _check(x, 12345)
 
 
