@@ -101,6 +101,10 @@ struct Plan {
   static constexpr int kStageBytes = 2 * kKBytes;
   static constexpr int kStages = (192 * 1024 / kCps) / kStageBytes;
   static constexpr int kHeads = NT * 8;
+  // Registers per thread: with two CTAs per SM at most 152 (19 x 256 per
+  // warp), which leaves 16 K registers per SM for the merge kernel that runs
+  // beside them after a fast step.
+  static constexpr int kMaxRegs = kCps == 2 ? 152 : 168;
   static constexpr int kQBytes = kHeads * D * 2;
 };
 
@@ -189,7 +193,7 @@ struct Maps {
 };
 
 template <int D, int NT, int MODE>
-__global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
+__global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
     attn_kernel(const __grid_constant__ Maps maps, const __grid_constant__ AttnArgs a) {
   using S = Smem<D, NT>;
   using P = Plan<D, NT>;
@@ -208,6 +212,10 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  uint64_t* mergebar = empty + kStages + 1;   // the consumer warps' merge at an item's end
+  // Fast steps with one head group (NT = 1): the consumer warps merge their
+  // states of an item in shared memory and write one partial per item.
+  constexpr bool kMerge = MODE == kFast && NT == 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -217,6 +225,7 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], P::kCW);
     }
+    mbar_init(mergebar, P::kCW);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -474,6 +483,15 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
   float mrun[1][2], lrun[1][2], lcand[1][2];
   int cur_b = 0, cur_g = 0;
   bool waited = MODE != kFast;   // the dense consumers waited at their start
+  uint32_t mphase = 0;           // parity of the next merge barrier phase
+  // every consumer warp at the merge barrier (bounded; false: the wait gave up)
+  auto merge_sync = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mergebar);
+    const bool ok = mbar_wait(mergebar, mphase, a.err, kSiteAttnConsumer, a.wait_ns);
+    mphase ^= 1u;
+    return ok;
+  };
   for (;;) {
     if (*abort_flag || !mbar_wait(&full[slot], phase, a.err, kSiteAttnConsumer, a.wait_ns)) {
       *abort_flag = 1;
@@ -679,16 +697,19 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
+    const bool item_end = (flags & 2) != 0;
+    const int done_slot = slot;   // with kMerge the item's last stage is released after the merge
+    if (!(kMerge && item_end) && lane == 0) mbar_arrive(&empty[slot]);
     if (++slot == kStages) {
       slot = 0;
       phase ^= 1;
     }
-    if (!(flags & 2)) continue;
+    if (!item_end) continue;
 
-    // ---- last stage of the item: this warp's partial softmax state goes to
-    // global memory as it is (m, l, l_cand and the unnormalised O of each
-    // query head); the combine kernel merges all partials.
+    // ---- last stage of the item: this warp's partial softmax state (m, l,
+    // l_cand and the unnormalised O of each query head) goes to global memory
+    // as it is, or (kMerge) first through the merge of the CTA's consumer
+    // warps; the combine kernel merges the partials of every item.
 #pragma unroll
     for (int nt = 0; nt < 1; ++nt)
 #pragma unroll
@@ -702,25 +723,85 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
       grid_dep_wait();
       waited = true;
     }
-    float* part = a.part + ((size_t)item * kConsumerWarps + twarp) * a.G * (D + 4);
-#pragma unroll
-    for (int nt = 0; nt < 1; ++nt) {
+    if constexpr (kMerge) {
+      // This warp's state into its own tiles of the stage just consumed (K
+      // tile: O of its 8 head slots, [head][D] with the column rotated by 8 *
+      // head against bank conflicts; V tile: m, l per head), then, after
+      // every consumer warp's, thread t of the 4 warps merges column t % D of
+      // heads t / D, t / D + 128 / D, ...: one partial per item.
+      uint8_t* stage = smem + done_slot * P::kStageBytes;
+      float* so = reinterpret_cast<float*>(stage + twarp * P::kTileBytes);
+      float* sml = reinterpret_cast<float*>(stage + P::kKBytes + twarp * P::kTileBytes);
 #pragma unroll
       for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int hh = hbase + nt * 8 + cq + (i & 1);
+          const int hh = cq + (i & 1);
           const int d = mt * 16 + r0 + (i >> 1) * 8;
-          if (hh < a.G) part[hh * (D + 4) + d] = o[nt][mt][i];
+          so[hh * D + ((d + 8 * hh) & (D - 1))] = o[0][mt][i];
         }
       if (lane < 4) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const int hh = hbase + nt * 8 + cq + j;
-          if (hh < a.G) {
-            part[hh * (D + 4) + D] = mrun[nt][j];
-            part[hh * (D + 4) + D + 1] = lrun[nt][j];
-            part[hh * (D + 4) + D + 2] = lcand[nt][j];
+          sml[(cq + j) * 2] = mrun[0][j];
+          sml[(cq + j) * 2 + 1] = lrun[0][j];
+        }
+      }
+      bool ok = merge_sync();
+      if (ok) {
+        float* part = a.part + (size_t)item * a.G * (D + 4);
+        const int t = twarp * 32 + lane;
+        const int d = t % D;
+        for (int hh = t / D; hh < a.G; hh += (kConsumerWarps * 32) / D) {
+          float mw[kConsumerWarps];
+          float M = NEG_INF;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            mw[w] = reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes)[hh * 2];
+            M = fmaxf(M, mw[w]);
+          }
+          const float mref = (M == NEG_INF) ? 0.f : M;
+          float ov = 0.f, lv = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float sc = fast_exp2(mw[w] - mref);
+            ov += sc * reinterpret_cast<const float*>(stage + w * P::kTileBytes)[hh * D + ((d + 8 * hh) & (D - 1))];
+            lv += sc * reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes)[hh * 2 + 1];
+          }
+          part[hh * (D + 4) + d] = ov;
+          if (d == 0) {
+            part[hh * (D + 4) + D] = M;
+            part[hh * (D + 4) + D + 1] = lv;
+            part[hh * (D + 4) + D + 2] = 0.f;
+          }
+        }
+        ok = merge_sync();   // every warp is done reading the stage
+      }
+      if (!ok) *abort_flag = 1;
+      fence_proxy_async_smem();   // the generic writes above before the stage's next copies
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[done_slot]);
+    } else {
+      float* part = a.part + ((size_t)item * kConsumerWarps + twarp) * a.G * (D + 4);
+#pragma unroll
+      for (int nt = 0; nt < 1; ++nt) {
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int hh = hbase + nt * 8 + cq + (i & 1);
+            const int d = mt * 16 + r0 + (i >> 1) * 8;
+            if (hh < a.G) part[hh * (D + 4) + d] = o[nt][mt][i];
+          }
+        if (lane < 4) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int hh = hbase + nt * 8 + cq + j;
+            if (hh < a.G) {
+              part[hh * (D + 4) + D] = mrun[nt][j];
+              part[hh * (D + 4) + D + 1] = lrun[nt][j];
+              part[hh * (D + 4) + D + 2] = lcand[nt][j];
+            }
           }
         }
       }
@@ -737,19 +818,24 @@ __global__ void __launch_bounds__(Plan<D, NT>::kThreads, Plan<D, NT>::kCps)
 //    path to the Selector).
 //  - After a fast step whose attention runs one CTA per SM (G > 8;
 //    attn_combine_fast_kernel): 7 warps of at most 64 registers and 4 KB of
-//    shared memory, which fit on an SM beside that CTA.  It lets the next
-//    launch start at once, so the merge runs while the attention finishes
-//    and the next layer's attention starts, instead of holding an SM.  Beside
-//    two attention CTAs per SM (G <= 8) it does not fit, and the fast steps
-//    take the 24-warp merge.
+//    shared memory, which fit on an SM beside that CTA.
+//  - After a fast step with two attention CTAs per SM (G <= 8), whose CTAs
+//    wrote one merged partial per item (attn_combine_merged_kernel): 4 warps
+//    of at most 96 registers, ten partials in flight per warp, which fit
+//    beside the two CTAs.
+//  After a fast step the merge lets the next launch start at once, so it
+//  runs while the attention finishes and the next layer's attention starts,
+//  instead of holding an SM.
+//  ppi: partials per work item (one per consumer warp, or 1 when merged).
 constexpr int kCombWarps = 24;
 constexpr int kCombWarpsFast = 7;
+constexpr int kCombWarpsMerged = 4;
 
-template <int D, int NW>
+template <int D, int NW, int KIN>
 __device__ __forceinline__ void combine_body(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv,
                                              int G, float* __restrict__ out, float* __restrict__ lse,
                                              float* __restrict__ lse_cand, const int32_t* n_rows, int p_max,
-                                             int rec_tiles, int tps, int* err, int* ctr, int early,
+                                             int rec_tiles, int tps, int* err, int* ctr, int early, int ppi,
                                              const RowMap& rows) {
   // After a fast step the next launch may start before this one has waited:
   // it is the next layer's attention, whose consumers wait before their
@@ -787,9 +873,9 @@ __device__ __forceinline__ void combine_body(const float* __restrict__ part, int
     ct = (ct + tps - 1) / tps * tps;
     chunks = (T + ct - 1) / ct;
   }
-  const int n = chunks * kConsumerWarps;
-  constexpr int kIn = NW > 8 ? 8 : 6;   // partials in flight per warp
-  const float* base = part + (size_t)bgl * n_chunks * kConsumerWarps * stride + (size_t)hh * (D + 4);
+  const int n = chunks * ppi;
+  constexpr int kIn = KIN;   // partials in flight per warp
+  const float* base = part + (size_t)bgl * n_chunks * ppi * stride + (size_t)hh * (D + 4);
   float m = -INFINITY, l = 0.f, lc = 0.f;
   float acc[kPer];
 #pragma unroll
@@ -876,9 +962,9 @@ __global__ void __launch_bounds__(kCombWarps * 32)
     attn_combine_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
                         float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
                         const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
-                        int early, const __grid_constant__ RowMap rows) {
-  combine_body<D, kCombWarps>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles, tps,
-                              err, ctr, early, rows);
+                        int early, int ppi, const __grid_constant__ RowMap rows) {
+  combine_body<D, kCombWarps, 8>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles, tps,
+                                 err, ctr, early, ppi, rows);
 }
 
 template <int D>
@@ -886,9 +972,19 @@ __global__ void __maxnreg__(64)
     attn_combine_fast_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
                              float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
                              const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
-                             int early, const __grid_constant__ RowMap rows) {
-  combine_body<D, kCombWarpsFast>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles,
-                                  tps, err, ctr, early, rows);
+                             int early, int ppi, const __grid_constant__ RowMap rows) {
+  combine_body<D, kCombWarpsFast, 6>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max, rec_tiles,
+                                     tps, err, ctr, early, ppi, rows);
+}
+
+template <int D>
+__global__ void __maxnreg__(96)
+    attn_combine_merged_kernel(const float* __restrict__ part, int n_chunks, int B, int Hq, int Hkv, int G,
+                               float* __restrict__ out, float* __restrict__ lse, float* __restrict__ lse_cand,
+                               const int32_t* n_rows, int p_max, int rec_tiles, int tps, int* err, int* ctr,
+                               int early, int ppi, const __grid_constant__ RowMap rows) {
+  combine_body<D, kCombWarpsMerged, 10>(part, n_chunks, B, Hq, Hkv, G, out, lse, lse_cand, n_rows, p_max,
+                                        rec_tiles, tps, err, ctr, early, ppi, rows);
 }
 
 __global__ void probs_kernel(int L, int Hq, const float* __restrict__ logits, int64_t ld,
@@ -1028,16 +1124,43 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
   return launch_attn_t<64, 2, MODE>(maps, a, st);
 }
 
+// Which merge follows an attention launch: after a dense step, after a fast
+// step whose CTAs wrote one partial per consumer warp (G > 8), or one per item.
+enum CombKind { kCombDense = 0, kCombFast = 1, kCombMerged = 2 };
+
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
                           float* lse, float* lse_cand, const int32_t* n_rows, int p_max, int rec_tiles, int tps,
-                          int* err, int* ctr, cudaStream_t st, const RowMap& rows, int early) {
+                          int* err, int* ctr, cudaStream_t st, const RowMap& rows, CombKind kind) {
   const int G = s.Hq / s.Hkv;
   const int grid = rows.count(s.B) * s.Hq;
+  const int early = kind == kCombDense ? 0 : 1;
+  const int ppi = kind == kCombMerged ? 1 : kConsumerWarps;
   auto go = [&](auto kern, int nw) {
     launch_k(kern, dim3(grid), dim3(nw * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse, lse_cand, n_rows,
-             p_max, rec_tiles, tps, err, ctr, early, rows);
+             p_max, rec_tiles, tps, err, ctr, early, ppi, rows);
   };
-  if (early) {
+  // The merges after a fast step share SMs with attention CTAs: the same
+  // shared-memory carveout, so an SM that takes a merge CTA first stays able
+  // to take attention CTAs.
+  static DeviceOnce carve;
+  if (kind != kCombDense && !carve.done()) {
+    cudaError_t e = cudaFuncSetAttribute(attn_combine_merged_kernel<128>,
+                                         cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_combine_merged_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_combine_fast_kernel<128>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_combine_fast_kernel<64>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    if (!carve.mark(e)) return SFI_ERR_CUDA;
+  }
+  if (kind == kCombMerged) {
+    if (D == 128) go(attn_combine_merged_kernel<128>, kCombWarpsMerged);
+    else go(attn_combine_merged_kernel<64>, kCombWarpsMerged);
+  } else if (kind == kCombFast) {
     if (D == 128) go(attn_combine_fast_kernel<128>, kCombWarpsFast);
     else go(attn_combine_fast_kernel<64>, kCombWarpsFast);
   } else {
@@ -1174,7 +1297,7 @@ sfi_status run_dense_attn(const sfi_shape& s, const sfi_paged_kv& kv, int L, con
   if (r != SFI_OK) return r;
   float* lse_tmp = ex ? ex->lse : nullptr;
   r = launch_combine(s.D, part, a.n_chunks, s, out, lse_tmp, ex ? ex->lse_cand : nullptr, nullptr, 0, 0, 1,
-                     kv.err, ctr, st, rmap, 0);
+                     kv.err, ctr, st, rmap, kCombDense);
   if (r != SFI_OK) return r;
   if (ex && ex->probs) {
     if (rmap.n) return SFI_ERR_UNSUPPORTED;   // probabilities of the whole batch only
@@ -1223,12 +1346,11 @@ sfi_status run_fast_attn(const sfi_shape& s, const sfi_params& p, const sfi_page
   if (ev_end) cudaEventRecord(ev_end, st);
   if (r != SFI_OK) return r;
   const int rec_tiles = (L - 1) / kPage - a.rec_lo / kPage + 1;
-  // The small merge that lets the next launch start early fits on an SM only
-  // beside an attention grid of one CTA per SM (G > 8); beside two it waits
-  // for an attention CTA to leave, and the 24-warp merge is the faster one.
-  const int early = attn_grid(s.D, G).ctas <= num_sms() ? 1 : 0;
+  // G <= 8: the attention's CTAs merged their warps' states (one partial per
+  // item); G > 8: one partial per consumer warp and item.
+  const CombKind kind = G <= 8 ? kCombMerged : kCombFast;
   return launch_combine(s.D, part, a.n_chunks, s, out, lse, nullptr, pk.n_rows, pk.p_max, rec_tiles, nts, kv.err,
-                        ctr, st, rmap, early);
+                        ctr, st, rmap, kind);
 }
 
 sfi_status run_attn_probs(const sfi_shape& s, int L, const float* logits, int64_t ld, const float* lse,
