@@ -211,27 +211,54 @@ class Bench:
                 S.sfi_dense_attn_append(self.shape, layer.kv, L, self.kn[t, l], self.vn[t, l], self.q[t, l],
                                         self.out[l], self.ws)
 
-    def run_e2e(self, host_q, host_k, host_v, host_out, dq, dk, dv):
+    def run_e2e(self, host_q, host_k, host_v, host_out, dq, dk, dv, dout, copy_stream, evs):
         """Every decode step copies that step's inputs (all layers) from pinned
-        host memory and reads all layers' outputs back."""
+        host memory and reads all layers' outputs back.  The copies run on a
+        second stream into two device buffers: step t + 1's inputs arrive and
+        step t's outputs leave while the next step computes."""
         cfg = self.cfg
         NL = len(self.layers)
-        qs, ks, vs = (dq[0].numel() * dq.element_size(), dk[0].numel() * dk.element_size(),
-                      dv[0].numel() * dv.element_size())
-        os_ = self.out[0].numel() * self.out.element_size()
+        T = cfg.steps
+        qs, ks, vs = (dq[0, 0].numel() * dq.element_size(), dk[0, 0].numel() * dk.element_size(),
+                      dv[0, 0].numel() * dv.element_size())
+        os_ = dout[0, 0].numel() * dout.element_size()
         refs = [(C.byref(layer.kv), C.byref(layer.packed)) for layer in self.layers]
-        stream = torch.cuda.current_stream().cuda_stream
+        main = torch.cuda.current_stream()
+        stream = main.cuda_stream
         step_fn = self.ctx.decode_step_ptr
-        for t in range(cfg.steps):
-            dq.copy_(host_q[t], non_blocking=True)
-            dk.copy_(host_k[t], non_blocking=True)
-            dv.copy_(host_v[t], non_blocking=True)
+        ev_in, ev_done, ev_read = evs
+
+        def fetch(t, b):   # on the copy stream
+            dq[b].copy_(host_q[t], non_blocking=True)
+            dk[b].copy_(host_k[t], non_blocking=True)
+            dv[b].copy_(host_v[t], non_blocking=True)
+            ev_in[b].record(copy_stream)
+
+        copy_stream.wait_stream(main)
+        with torch.cuda.stream(copy_stream):
+            fetch(0, 0)
+        for t in range(T):
+            b = t % 2
+            if t + 1 < T:
+                with torch.cuda.stream(copy_stream):
+                    if t >= 1:
+                        copy_stream.wait_event(ev_done[1 - b])   # step t - 1 is done with buffer 1 - b
+                    fetch(t + 1, 1 - b)
+            main.wait_event(ev_in[b])
+            if t >= 2:
+                main.wait_event(ev_read[b])   # step t - 2's outputs have left buffer b
             L = cfg.seq_len(t)
             bprev = int(self.boundary[t - 1]) if t > 0 else 0
+            qb, kb, vb, ob = dq[b].data_ptr(), dk[b].data_ptr(), dv[b].data_ptr(), dout[b].data_ptr()
             for l in range(NL):
-                step_fn(l, t, bprev, L, refs[l][0], refs[l][1], dq.data_ptr() + l * qs, dk.data_ptr() + l * ks,
-                        dv.data_ptr() + l * vs, self.out.data_ptr() + l * os_, stream)
-            host_out[t].copy_(self.out, non_blocking=True)
+                step_fn(l, t, bprev, L, refs[l][0], refs[l][1], qb + l * qs, kb + l * ks, vb + l * vs,
+                        ob + l * os_, stream)
+            ev_done[b].record(main)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(ev_done[b])
+                host_out[t].copy_(dout[b], non_blocking=True)
+                ev_read[b].record(copy_stream)
+        main.wait_stream(copy_stream)   # every output is on the host before the region ends
         self.ctx.join()
 
 
@@ -502,11 +529,17 @@ def run_sfi(args, cfg, rank, world, dist_on):
     hk = bench.kn.cpu().pin_memory()
     hv = bench.vn.cpu().pin_memory()
     hout = torch.empty((T,) + tuple(bench.out.shape), dtype=torch.float32).pin_memory()
-    dq, dk, dv = torch.empty_like(bench.q[0]), torch.empty_like(bench.kn[0]), torch.empty_like(bench.vn[0])
-    bench.run_e2e(hq, hk, hv, hout, dq, dk, dv)
+    dq = torch.empty((2,) + tuple(bench.q[0].shape), dtype=bench.q.dtype, device=dev)
+    dk = torch.empty((2,) + tuple(bench.kn[0].shape), dtype=bench.kn.dtype, device=dev)
+    dv = torch.empty((2,) + tuple(bench.vn[0].shape), dtype=bench.vn.dtype, device=dev)
+    dout = torch.empty((2,) + tuple(bench.out.shape), dtype=bench.out.dtype, device=dev)
+    copy_stream = torch.cuda.Stream(device=dev)
+    evs = tuple([torch.cuda.Event(), torch.cuda.Event()] for _ in range(3))
+    e2e_args = (hq, hk, hv, hout, dq, dk, dv, dout, copy_stream, evs)
+    bench.run_e2e(*e2e_args)
     clocks = Clocks(torch.cuda.current_device())
     clocks.start()
-    t_e2e = _timed(lambda: bench.run_e2e(hq, hk, hv, hout, dq, dk, dv), args.steps, dist_on)
+    t_e2e = _timed(lambda: bench.run_e2e(*e2e_args), args.steps, dist_on)
     clk_e2e = clocks.stop()
     h2d = (hq[0].numel() * 2 + hk[0].numel() * 2 + hv[0].numel() * 2) * T
     d2h = hout[0].numel() * 4 * T
