@@ -747,7 +747,7 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
           sml[(cq + j) * 2 + 1] = lrun[0][j];
         }
       }
-      bool ok = merge_sync();
+      const bool ok = merge_sync();   // every warp's state is in the stage
       if (ok) {
         float* part = a.part + (size_t)item * a.G * (D + 4);
         const int t = twarp * 32 + lane;
@@ -775,9 +775,10 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
             part[hh * (D + 4) + D + 2] = 0.f;
           }
         }
-        ok = merge_sync();   // every warp is done reading the stage
       }
       if (!ok) *abort_flag = 1;
+      // The stage goes back to the producer once every consumer warp has
+      // arrived on its empty barrier, each after its own reads above.
       fence_proxy_async_smem();   // the generic writes above before the stage's next copies
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[done_slot]);
