@@ -218,9 +218,9 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
   uint64_t* mergebar = empty + kStages + 1;   // the consumer warps' merge at an item's end
-  // Fast steps with one head group (NT = 1): the consumer warps merge their
-  // states of an item in shared memory and write one partial per item.
-  constexpr bool kMerge = MODE == kFast && NT == 1;
+  // One head group (NT = 1): the consumer warps merge their states of an
+  // item in shared memory and write one partial per item.
+  constexpr bool kMerge = NT == 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -731,9 +731,9 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
     if constexpr (kMerge) {
       // This warp's state into its own tiles of the stage just consumed (K
       // tile: O of its 8 head slots, [head][D] with the column rotated by 8 *
-      // head against bank conflicts; V tile: m, l per head), then, after
-      // every consumer warp's, thread t of the 4 warps merges column t % D of
-      // heads t / D, t / D + 128 / D, ...: one partial per item.
+      // head against bank conflicts; V tile: m, l, l_cand per head), then,
+      // after every consumer warp's, thread t of the 4 warps merges column
+      // t % D of heads t / D, t / D + 128 / D, ...: one partial per item.
       uint8_t* stage = smem + done_slot * P::kStageBytes;
       float* so = reinterpret_cast<float*>(stage + twarp * P::kTileBytes);
       float* sml = reinterpret_cast<float*>(stage + P::kKBytes + twarp * P::kTileBytes);
@@ -748,8 +748,9 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
       if (lane < 4) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          sml[(cq + j) * 2] = mrun[0][j];
-          sml[(cq + j) * 2 + 1] = lrun[0][j];
+          sml[(cq + j) * 3] = mrun[0][j];
+          sml[(cq + j) * 3 + 1] = lrun[0][j];
+          sml[(cq + j) * 3 + 2] = lcand[0][j];
         }
       }
       const bool ok = merge_sync();   // every warp's state is in the stage
@@ -762,22 +763,24 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
           float M = NEG_INF;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) {
-            mw[w] = reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes)[hh * 2];
+            mw[w] = reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes)[hh * 3];
             M = fmaxf(M, mw[w]);
           }
           const float mref = (M == NEG_INF) ? 0.f : M;
-          float ov = 0.f, lv = 0.f;
+          float ov = 0.f, lv = 0.f, lcv = 0.f;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) {
             const float sc = fast_exp2(mw[w] - mref);
+            const float* ml = reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes) + hh * 3;
             ov += sc * reinterpret_cast<const float*>(stage + w * P::kTileBytes)[hh * D + ((d + 8 * hh) & (D - 1))];
-            lv += sc * reinterpret_cast<const float*>(stage + P::kKBytes + w * P::kTileBytes)[hh * 2 + 1];
+            lv += sc * ml[1];
+            if (MODE == kDenseExtras) lcv += sc * ml[2];
           }
           part[hh * (D + 4) + d] = ov;
           if (d == 0) {
             part[hh * (D + 4) + D] = M;
             part[hh * (D + 4) + D + 1] = lv;
-            part[hh * (D + 4) + D + 2] = 0.f;
+            part[hh * (D + 4) + D + 2] = lcv;
           }
         }
       }
@@ -1145,7 +1148,8 @@ sfi_status launch_attn(int D, int G, const Maps& maps, const AttnArgs& a, cudaSt
 }
 
 // Which merge follows an attention launch: after a dense step, after a fast
-// step whose CTAs wrote one partial per consumer warp (G > 8), or one per item.
+// step whose CTAs wrote one partial per consumer warp (G > 8), or one per item
+// (G <= 8; a dense step's CTAs also write one per item then).
 enum CombKind { kCombDense = 0, kCombFast = 1, kCombMerged = 2 };
 
 sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shape& s, float* out,
@@ -1154,7 +1158,8 @@ sfi_status launch_combine(int D, const float* part, int n_chunks, const sfi_shap
   const int G = s.Hq / s.Hkv;
   const int grid = rows.count(s.B) * s.Hq;
   const int early = kind == kCombDense ? 0 : 1;
-  const int ppi = kind == kCombMerged ? 1 : kConsumerWarps;
+  // one partial per item where the attention's consumer warps merged (G <= 8)
+  const int ppi = G <= 8 ? 1 : kConsumerWarps;
   auto go = [&](auto kern, int nw) {
     launch_k(kern, dim3(grid), dim3(nw * 32), 0, st, part, n_chunks, s.B, s.Hq, s.Hkv, G, out, lse, lse_cand, n_rows,
              p_max, rec_tiles, tps, err, ctr, early, ppi, rows);
