@@ -30,12 +30,13 @@
  *    16-byte aligned.  Nothing here ever aborts or exits the process.
  *  - Consecutive calls on one stream overlap on the GPU: an attention call
  *    starts loading its query and cache rows, and a fast call appends its
- *    token, while the two attention calls before it on the same stream
- *    finish.  So the query of an attention call must not be the output of
- *    either of those two calls, and a fast call must not append to a cache
- *    row that they read or append.  (In a decode loop each layer has its own
- *    rows and other kernels produce the query.)  Any kernel or copy of the
- *    caller's in between orders the calls fully.
+ *    token, while earlier attention calls on the same stream finish.  So
+ *    the query of an attention call must not be the output of an earlier
+ *    attention call, and a fast call must not append to a cache row that an
+ *    earlier call reads or appends, unless a kernel or copy of the caller's
+ *    lies between the two calls on the stream (that orders them fully).  In
+ *    a decode loop each layer has its own rows and other kernels produce the
+ *    query.
  */
 #ifndef SFI_H_
 #define SFI_H_

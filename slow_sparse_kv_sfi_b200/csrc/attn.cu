@@ -342,9 +342,9 @@ __global__ void __maxnreg__((Plan<D, NT>::kMaxRegs))
         p_lo = item_page(it, max(it.t_begin, it.n_packed_tiles));
         // the item holding position L - 1 first appends the step's token
         // there (the whole warp), before any copy of that tile is issued.  A
-        // fast step appends without waiting: the kernels still running (the
-        // previous attention launch and its combine) neither read nor write
-        // that row of this cache.
+        // fast step appends without waiting: the kernels that may still run
+        // (earlier attention launches and their combines) neither read nor
+        // write that row of this cache (the library's ordering rule).
         if (a.k_new && it.t_begin < it.t_end && it.t_end == it.t_total) {
           if (MODE != kFast) ensure_wait();
           const int pos = a.L - 1;
