@@ -211,11 +211,12 @@ class Bench:
                 S.sfi_dense_attn_append(self.shape, layer.kv, L, self.kn[t, l], self.vn[t, l], self.q[t, l],
                                         self.out[l], self.ws)
 
-    def run_e2e(self, host_q, host_k, host_v, host_out, dq, dk, dv, dout, copy_stream, evs):
-        """Every decode step copies that step's inputs (all layers) from pinned
-        host memory and reads all layers' outputs back.  The copies run on a
-        second stream into two device buffers: step t + 1's inputs arrive and
-        step t's outputs leave while the next step computes."""
+    def run_e2e(self, host_in, host_out, dq, dk, dv, din, dout, copy_stream, evs):
+        """Every decode step copies that step's inputs (q, k and v of all
+        layers, packed in one pinned host row per step) from host memory and
+        reads all layers' outputs back.  The copies run on a second stream
+        into two device buffers: step t + 1's inputs arrive and step t's
+        outputs leave while the next step computes."""
         cfg = self.cfg
         NL = len(self.layers)
         T = cfg.steps
@@ -228,10 +229,8 @@ class Bench:
         step_fn = self.ctx.decode_step_ptr
         ev_in, ev_done, ev_read = evs
 
-        def fetch(t, b):   # on the copy stream
-            dq[b].copy_(host_q[t], non_blocking=True)
-            dk[b].copy_(host_k[t], non_blocking=True)
-            dv[b].copy_(host_v[t], non_blocking=True)
+        def fetch(t, b):   # on the copy stream: one copy per step
+            din[b].copy_(host_in[t], non_blocking=True)
             ev_in[b].record(copy_stream)
 
         copy_stream.wait_stream(main)
@@ -525,17 +524,19 @@ def run_sfi(args, cfg, rank, world, dist_on):
     t_dense = _timed(bench.run_dense, args.steps, dist_on)
     clk_dense = clocks.stop()
     # end to end through host buffers
-    hq = bench.q.cpu().pin_memory()
-    hk = bench.kn.cpu().pin_memory()
-    hv = bench.vn.cpu().pin_memory()
+    hq, hk, hv = bench.q.cpu(), bench.kn.cpu(), bench.vn.cpu()
     hout = torch.empty((T,) + tuple(bench.out.shape), dtype=torch.float32).pin_memory()
-    dq = torch.empty((2,) + tuple(bench.q[0].shape), dtype=bench.q.dtype, device=dev)
-    dk = torch.empty((2,) + tuple(bench.kn[0].shape), dtype=bench.kn.dtype, device=dev)
-    dv = torch.empty((2,) + tuple(bench.vn[0].shape), dtype=bench.vn.dtype, device=dev)
+    # each step's q, k and v side by side in one pinned row, one device row per buffer
+    nq, nk, nv = hq[0].numel(), hk[0].numel(), hv[0].numel()
+    hin = torch.cat([hq.reshape(T, nq), hk.reshape(T, nk), hv.reshape(T, nv)], dim=1).pin_memory()
+    din = torch.empty((2, nq + nk + nv), dtype=bench.q.dtype, device=dev)
+    dq = din[:, :nq].view((2,) + tuple(bench.q[0].shape))
+    dk = din[:, nq:nq + nk].view((2,) + tuple(bench.kn[0].shape))
+    dv = din[:, nq + nk:].view((2,) + tuple(bench.vn[0].shape))
     dout = torch.empty((2,) + tuple(bench.out.shape), dtype=bench.out.dtype, device=dev)
     copy_stream = torch.cuda.Stream(device=dev)
     evs = tuple([torch.cuda.Event(), torch.cuda.Event()] for _ in range(3))
-    e2e_args = (hq, hk, hv, hout, dq, dk, dv, dout, copy_stream, evs)
+    e2e_args = (hin, hout, dq, dk, dv, din, dout, copy_stream, evs)
     bench.run_e2e(*e2e_args)
     clocks = Clocks(torch.cuda.current_device())
     clocks.start()
