@@ -9,10 +9,11 @@
 // layer i run on the context's side stream after an event.  The next step of
 // layer i waits for that refresh before it touches the layer's cache or
 // packed buffer.  A logits buffer is rewritten only after the side stream has
-// finished reading it.  The side stream has the highest priority, and the
-// dense launches let the next kernel be scheduled only when their CTAs run
-// out of work, so the Selector kernels take the SMs freed in the attention's
-// tail instead of queueing behind the next layer's whole grid.
+// finished reading it.  The side stream has the lowest priority: a layer's
+// Selector is needed only at the layer's next step, so its kernels fill the
+// SMs the main stream leaves (the tails of the attention launches) instead
+// of holding the next layer's dense attention back.  The dense launches let
+// the next kernel be scheduled only when their CTAs run out of work.
 #include <algorithm>
 #include <vector>
 
@@ -333,11 +334,13 @@ sfi_status sfi_ctx_create(const sfi_shape* shape, const sfi_params* params, int3
   c->n_layers = n_layers;
   c->overlap = overlap ? 1 : 0;
   cudaGetDevice(&c->device);
-  // the side stream gets the highest priority: its Selector kernels take the
-  // SMs that the main stream's attention frees in its tail
+  // the side stream gets the lowest priority: the Selector kernels run where
+  // the main stream's attention leaves SMs free (measured on the 128K
+  // workload: slow layer-step 269 us with the highest priority, 262 us with
+  // the lowest)
   int least = 0, greatest = 0;
   bool ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
-            cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, greatest) == cudaSuccess;
+            cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, least) == cudaSuccess;
   c->ev_pre.resize(n_layers, nullptr);
   c->ev_dense.resize(n_layers, nullptr);
   c->ev_sel.resize(n_layers, nullptr);
