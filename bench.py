@@ -66,14 +66,17 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def kernel_traffic(kind: str):
+def kernel_traffic(kind: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel source changed since the counters were taken."""
+    kernel source changed since the counters were taken or the summary was
+    taken on another workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         d = json.load(fh)
+    if d.get("workload") != workload:
+        return None
     src = open(os.path.join(ROOT, "slow_sparse_kv_sfi_b200", "csrc", "attn.cu"), "rb").read()
     if d.get("attn_cu_sha256") != hashlib.sha256(src).hexdigest():
         return None
@@ -553,14 +556,14 @@ def run_sfi(args, cfg, rank, world, dist_on):
     if dominant == "fast":
         roof = {"kernel": f"attn_kernel<{D},*,kFast> (fast step)", "bound": "hbm", "achieved": ach_fast,
                 "peak": peak, "unit": "GB/s", "frac": ach_fast / peak,
-                "traffic": kernel_traffic("fast_attn_bytes_per_launch"),
+                "traffic": kernel_traffic("fast_attn_bytes_per_launch", cfg.name),
                 "algorithmic_bytes_per_launch": fast_bytes / max(fast_n / k, 1),
                 "launches": fast_n, "avg_launch_us": 1000 * fast_ms / max(fast_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
     else:
         roof = {"kernel": f"attn_kernel<{D},*,kDenseExtras> (slow step)", "bound": "hbm", "achieved": ach_dense,
                 "peak": peak, "unit": "GB/s", "frac": ach_dense / peak,
-                "traffic": kernel_traffic("dense_attn_bytes_per_launch"),
+                "traffic": kernel_traffic("dense_attn_bytes_per_launch", cfg.name),
                 "algorithmic_bytes_per_launch": dense_bytes_slow / max(dense_n / k, 1),
                 "launches": dense_n, "avg_launch_us": 1000 * dense_ms / max(dense_n, 1),
                 "peak_source": f"{peak_kind} hbm_gbs"}
