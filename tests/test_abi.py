@@ -107,6 +107,10 @@ def test_context_rejects_bad_calls(S):
     h = C.c_void_p()
     st = S.lib().sfi_ctx_create(C.byref(sh), C.byref(p), 0, 1, C.byref(h))
     assert st == 1
+    # kernel timing: no context, a negative stride or first layer
+    lib = S.lib()
+    assert lib.sfi_ctx_set_timing(None, 1) == 1
+    assert lib.sfi_ctx_set_timing_layers(None, 0, 1) == 1
 
 
 @pytest.mark.parametrize("window,code", [(0, 0), (1, 0), (4, 0), (33, 1), (65, 1), (-1, 1)])
