@@ -56,6 +56,15 @@ def timed_layer(n_layers):
     return n_layers // 2
 
 
+# With a single layer the sampled layer is every launch; there only every
+# TIMED_STEP_STRIDE-th step is sampled, so that the events slow the run little.
+TIMED_STEP_STRIDE = 8
+
+
+def timed_step_stride(n_layers):
+    return 1 if n_layers > 1 else TIMED_STEP_STRIDE
+
+
 # ---------------------------------------------------------------- helpers
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -173,7 +182,9 @@ class Bench:
         self.ws = torch.zeros(S.sfi_workspace_size(self.shape, self.params), dtype=torch.uint8, device=device)
         torch.cuda.synchronize()
 
-    def run_sfi(self, step_events=None, probe=None, q=None, kn=None, vn=None, out=None):
+    def run_sfi(self, step_events=None, probe=None, q=None, kn=None, vn=None, out=None, timing=False):
+        """One decode run.  timing: the attention launches of the sampled layer
+        are event-timed on the sampled steps (`timed_layer`, `timed_step_stride`)."""
         cfg = self.cfg
         q = self.q if q is None else q
         kn = self.kn if kn is None else kn
@@ -189,10 +200,13 @@ class Bench:
         refs = [(C.byref(layer.kv), C.byref(layer.packed)) for layer in self.layers]
         stream = torch.cuda.current_stream().cuda_stream
         step_fn = self.ctx.decode_step_ptr
+        every = timed_step_stride(NL)
         for t in range(cfg.steps):
             L = cfg.seq_len(t)
             bprev = int(self.boundary[t - 1]) if t > 0 else 0
             slow = False
+            if timing and every > 1:
+                self.ctx.set_timing(NL if t % every == 0 else 0, first_layer=timed_layer(NL))
             for l in range(NL):
                 i = t * NL + l
                 slow = step_fn(l, t, bprev, L, refs[l][0], refs[l][1], qb + i * qs, kb + i * ks, vb + i * vs,
@@ -468,6 +482,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
     # algorithmic bytes: of the attention launches whose durations are sampled
     # (one layer), and of every layer-step of the run
     sampled = [timed_layer(NL)]
+    every = timed_step_stride(NL)
     fast_bytes = 0.0
     run_fast_bytes = run_slow_bytes = 0.0
     union_rows = []
@@ -487,10 +502,10 @@ def run_sfi(args, cfg, rank, world, dist_on):
             for l in range(NL):
                 b_ = step_bytes(cfg, L, cur[l], False)
                 run_fast_bytes += b_
-                if l in sampled:
+                if l in sampled and t % every == 0:
                     fast_bytes += b_
     dense_bytes_slow = sum(float(B * cfg.Hkv * cfg.seq_len(t) * 4 * D + B * cfg.Hq * cfg.seq_len(t) * 4)
-                           for t in range(T) if slows[t]) * len(sampled)
+                           for t in range(T) if slows[t] and t % every == 0) * len(sampled)
     # timed region: SFI mixed decode, with kernel and step events
     clocks = Clocks(torch.cuda.current_device())
     bench.ctx.set_timing(NL, first_layer=timed_layer(NL))
@@ -504,7 +519,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
     e0.record()
     for k in range(args.steps):
         start_ev[k].record()
-        bench.run_sfi(step_events=step_ev[k])
+        bench.run_sfi(step_events=step_ev[k], timing=True)
     e1.record()
     _sync_barrier(dist_on)
     clk_sfi = clocks.stop()
@@ -613,7 +628,7 @@ def run_sfi(args, cfg, rank, world, dist_on):
             "slow_layer_step_us": 1000 * statistics.mean(st_slow) / NL if st_slow else None,
             "fast_layer_step_us": 1000 * statistics.mean(st_fast) / NL if st_fast else None,
             "fast_attn_GBps": ach_fast, "dense_attn_GBps": ach_dense,
-            "timed_layers": f"layer {timed_layer(NL)} (1 of {NL})",
+            "timed_layers": f"layer {timed_layer(NL)} (1 of {NL}), every {timed_step_stride(NL)} step(s)",
             "fast_attn_ms_sampled": fast_ms, "dense_attn_ms_sampled": dense_ms,
             "mean_packed_rows": float(np.mean(union_rows)) if union_rows else None,
             "fast_frac_of_dense_bytes": None if not union_rows else
