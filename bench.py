@@ -67,11 +67,16 @@ def timed_step_stride(n_layers):
 
 # ---------------------------------------------------------------- helpers
 def peaks():
+    """HBM peak in GB/s: the measured copy bandwidth of MEASURED_PEAKS.json,
+    else the fallback 6650 GB/s (also when the file cannot be read)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
+    try:
         with open(p) as fh:
-            d = json.load(fh)
-        return float(d["hbm_gbs"]), "measured"
+            v = float(json.load(fh)["hbm_gbs"])
+        if v > 0:
+            return v, "measured"
+    except (OSError, ValueError, KeyError, TypeError):
+        pass
     return 6650.0, "fallback"
 
 
