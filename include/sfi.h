@@ -276,7 +276,9 @@ sfi_status sfi_select_scores(const sfi_shape* shape, const sfi_params* params,
  * ws_bytes below the reported size is refused).  Exact radix select over
  * order-preserving 32-bit keys of the scores, one thread-block cluster of 1,
  * 2, 4 or 8 CTAs (of up to 1024 threads) per row, each CTA holding its
- * slice's keys in registers: the digit passes run over key - smallest key,
+ * slice's keys on chip (32 per thread in registers, and 32 more in shared
+ * memory when the rows would otherwise take more CTAs than the GPU has
+ * SMs): the digit passes run over key - smallest key,
  * from the highest bit of (largest - smallest), at most 14 bits per pass; CTA
  * histograms meet in distributed shared memory, and the ties at the
  * threshold are taken in position order.  The pages name the step and give
